@@ -1,0 +1,144 @@
+"""Active-expert-chunked MoE OFT forward (float64 oracle).
+
+TEST INFRASTRUCTURE ONLY -- see the package docstring.
+
+The pages describe it as: the experts that the router selects are grouped into
+fixed-size chunks; each chunk is dequantised transiently, fed to a grouped GEMM,
+and its high-precision copy is released afterwards, so that peak transient
+memory stays bounded by one chunk (m.xxlwj.com 771001, section "技术细节",
+paragraph "Active-expert-chunked dequantization"; chooseai.io news 4086,
+section "对低精度 MoE 模型的专门优化").  The routing itself is not specified; the
+readings taken here are:
+
+  * top-k by logit, descending; ties go to the lower expert index; the slot
+    order k is the rank;
+  * gating weights are a softmax over the k selected logits (they sum to 1);
+  * each expert e has gate and up projections with independent OFT rotations
+    (split-projection applied to the expert's fused gate/up tensor):
+        Y_tk = [ (X_t R_e,gate) W_e,gate  |  (X_t R_e,up) W_e,up ]
+  * the layer output is Y_t = sum_k w_tk Y_tk in slot order (the gate/up linear
+    outputs; no activation and no down projection);
+  * bucket order: entries (t, k) sorted by expert, stable in (t, k); active
+    experts are those with a non-zero count, ascending; chunk c holds
+    active[c*C : (c+1)*C], the last one possibly partial.
+
+Pins (tests/test_oracle_moe.py): top-k against a brute-force Python sort;
+buckets against a dictionary build; chunked order equals the direct per-token
+sum; weights sum to one; a router that sends every token to one expert with
+k = 1 reduces to the split-projection linear of oft_ref.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+from .codecs import bf16_bits_to_f64, dequant
+from .oft_ref import rotate, rotations
+
+
+def topk(logits: np.ndarray, k: int):
+    """logits fp32 [T][E] -> (idx int32 [T][k], w float64 [T][k])."""
+    logits = np.asarray(logits, dtype=np.float32)
+    order = np.argsort(-logits, axis=1, kind="stable")[:, :k]
+    sel = np.take_along_axis(logits, order, axis=1).astype(np.float64)
+    z = np.exp(sel - sel.max(axis=1, keepdims=True))
+    return order.astype(np.int32), z / z.sum(axis=1, keepdims=True)
+
+
+def buckets(idx: np.ndarray, E: int):
+    """idx [T][k] -> (counts [E], offsets [E+1], bucket [T*k]).
+
+    bucket lists the flat entries t*k + slot grouped by expert, each expert's
+    entries in increasing (t, slot)."""
+    flat = np.asarray(idx).reshape(-1)
+    counts = np.bincount(flat, minlength=E).astype(np.int32)
+    offsets = np.zeros(E + 1, dtype=np.int32)
+    offsets[1:] = np.cumsum(counts)
+    bucket = np.argsort(flat, kind="stable").astype(np.int32)
+    return counts, offsets, bucket
+
+
+def chunk_table(counts: np.ndarray, chunk: int, E: int):
+    """Active experts (count > 0) ascending, cut into chunks of `chunk`.
+
+    Returns (n_active, table int32 [ceil(E/chunk)][chunk]) padded with -1."""
+    active = np.nonzero(np.asarray(counts) > 0)[0].astype(np.int32)
+    n_chunks_max = (E + chunk - 1) // chunk
+    table = np.full((n_chunks_max, chunk), -1, dtype=np.int32)
+    for c in range(0, len(active), chunk):
+        part = active[c:c + chunk]
+        table[c // chunk, : len(part)] = part
+    return len(active), table
+
+
+class ExpertBank:
+    """Dequantises expert weights on demand from stored INT4 codes/scales.
+
+    codes uint8 [E][2n][K/2], scales bf16 bits [E][K/G][2n]; rows 0..n-1 are the
+    gate projection, n..2n-1 the up projection."""
+
+    def __init__(self, codes, scales_bits, K: int, group: int, n_proj: int):
+        self.codes, self.scales, self.K, self.group, self.n = codes, scales_bits, K, group, n_proj
+
+    def weight_t(self, e: int, rows=None) -> np.ndarray:
+        return dequant("int4", self.codes[e], self.scales[e], self.K, self.group, rows=rows)
+
+
+def expert_outputs(X: np.ndarray, e: int, bank: ExpertBank, Qe_bits: np.ndarray, b: int, cols=None):
+    """Y_tk for tokens X [m][K] routed to expert e: [m][2n] (or the given columns).
+
+    Qe_bits: packed bf16 bits [2][K/b][b(b-1)/2] for (gate, up)."""
+    n = bank.n
+    R = rotations(Qe_bits, b)                                   # [2][K/b][b][b]
+    cols = np.arange(2 * n) if cols is None else np.asarray(cols)
+    out = np.empty((X.shape[0], len(cols)))
+    for proj in (0, 1):
+        sel = np.nonzero((cols >= proj * n) & (cols < (proj + 1) * n))[0]
+        if len(sel) == 0:
+            continue
+        Wt = bank.weight_t(e, rows=cols[sel])
+        out[:, sel] = rotate(X, R[proj]) @ Wt.T
+    return out
+
+
+def moe_fwd_direct(X_bits, logits, bank: ExpertBank, Q_bits, b: int, top_k: int, tokens=None, cols=None):
+    """Y[t] = sum_k w_tk Y_tk, computed token by token in slot order.
+
+    tokens/cols optionally restrict the rows/columns computed (for sampled
+    checks of large problems)."""
+    X = bf16_bits_to_f64(X_bits)
+    idx, w = topk(logits, top_k)
+    T = X.shape[0]
+    tokens = np.arange(T) if tokens is None else np.asarray(tokens)
+    ncols = 2 * bank.n if cols is None else len(cols)
+    Y = np.zeros((len(tokens), ncols))
+    for i, t in enumerate(tokens):
+        for k in range(top_k):
+            e = int(idx[t, k])
+            Y[i] += w[t, k] * expert_outputs(X[t:t + 1], e, bank, Q_bits[e], b, cols)[0]
+    return Y
+
+
+def moe_fwd_chunked(X_bits, logits, bank: ExpertBank, Q_bits, b: int, top_k: int, chunk: int, E: int):
+    """The same result computed in the method's order: route, bucket, walk the
+    chunks of active experts, compute each expert's bucket rows (its grouped-GEMM
+    rows), then combine per token in slot order.  Returns (Y, routing dict)."""
+    X = bf16_bits_to_f64(X_bits)
+    T = X.shape[0]
+    idx, w = topk(logits, top_k)
+    counts, offsets, bucket = buckets(idx, E)
+    n_active, table = chunk_table(counts, chunk, E)
+    Ytk = np.zeros((T * top_k, 2 * bank.n))
+    for c in range(table.shape[0]):
+        for e in table[c]:
+            if e < 0:
+                continue
+            ent = bucket[offsets[e]:offsets[e + 1]]
+            Ytk[offsets[e]:offsets[e + 1]] = expert_outputs(X[ent // top_k], int(e), bank, Q_bits[e], b)
+    pos = np.empty(T * top_k, dtype=np.int64)
+    pos[bucket] = np.arange(T * top_k)
+    Y = np.zeros((T, 2 * bank.n))
+    for k in range(top_k):
+        Y += w[:, k:k + 1] * Ytk[pos[np.arange(T) * top_k + k]]
+    routing = dict(idx=idx, w=w, counts=counts, offsets=offsets, bucket=bucket, n_active=n_active, table=table)
+    return Y, routing

@@ -1,0 +1,534 @@
+#!/usr/bin/env python
+"""Throughput of the OFT + dequant linear hot path on B200.
+
+A step is one pass of the whole path over one batch: Cayley build of every
+rotation block, the split-projection forward (rotate, dequant, tcgen05 GEMM),
+and for the training workloads the adapter backward (dX' GEMM, dX rotation,
+dR reduction, Cayley backward), plus the dQ all-reduce when several ranks run
+data-parallel replicas.  Default workload: the dense fused-QKV FP8 forward +
+backward (4096 tokens x 2560 -> 4096/1024/1024, b = 32).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c1] [--impl ours|reference]
+
+Prints one JSON line (rank 0).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "OFT+dequant linear fwd/bwd tokens/s, TFLOP/s vs B200 dense tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+WORKLOAD_NAMES = {
+    "c0": "tiny fused-QKV OFT linear fwd: 64 x 256 -> 3x128, INT4 g32, b=32",
+    "c1": "dense fused-QKV OFT linear fwd+bwd: 4096 x 2560 -> 4096/1024/1024, FP8 e4m3 per-channel, b=32",
+    "c2": "gated-MLP gate/up OFT linear fwd: 8192 x 4096 -> 2x12288, INT4 g128, b=64",
+    "c3": "MoE active-expert-chunked OFT fwd: 4096 tok, hidden 7168, 384 experts x (2x2048), INT4 g32, top-8, chunk 16, b=32",
+    "c4": "training-step OFT linear fwd+bwd: 16384 x 7168 -> 12288/3072/3072, MXFP4, b=64",
+}
+
+
+# ----------------------------------------------------------------------------
+# helpers (also used by the multi-process CPU tests)
+# ----------------------------------------------------------------------------
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def init_dist(backend: str):
+    import datetime
+    import torch.distributed as dist
+    rank, world, _ = dist_env()
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world
+
+
+def max_over_ranks(x: float, device) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def allreduce_grad(dQ):
+    """Data-parallel replicas: sum the adapter gradient over ranks (the only
+    exchange the path has; the frozen base has no gradient)."""
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(dQ)
+    return dQ
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def linear_flops(spec, backward: bool):
+    M, K, N, P, b = spec.M, spec.K, spec.N, spec.P, spec.b
+    nblk = P * (K // b)
+    gemm = 2.0 * M * K * N
+    rot = 2.0 * M * K * b * P
+    f = dict(gemm_fwd=gemm, rot_fwd=rot, cayley=2.0 * b ** 3 * nblk)
+    if backward:
+        f.update(gemm_bwd=gemm, rot_dx=rot, rot_dr=rot, cayley_bwd=4.0 * b ** 3 * nblk)
+    return f
+
+
+def weight_bytes(spec):
+    N, K = spec.N, spec.K
+    if spec.fmt == "fp8":
+        return N * K + 4 * N
+    if spec.fmt == "int4":
+        return N * K // 2 + 2 * N * (K // spec.group)
+    return N * K // 2 + N * (K // 32)
+
+
+# ----------------------------------------------------------------------------
+# clocks (NVML, sampled in a thread during the timed region)
+# ----------------------------------------------------------------------------
+
+_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+            0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+            0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    def __init__(self, torch_device, period_s: float = 0.02):
+        self.samples, self.reasons, self.power = [], set(), []
+        self.max_mhz = None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(torch_device).uuid)
+            try:
+                self._h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid) if not uuid.startswith("GPU-") else uuid)
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(torch_device.index or 0)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._nvml = pynvml
+        except Exception as e:  # no NVML: report no samples
+            self.error = repr(e)
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in _REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+                self.power.append(nv.nvmlDeviceGetPowerUsage(self._h) / 1000.0)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._h is not None:
+            self._t.join()
+        return False
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples),
+                "power_w_max": max(self.power) if self.power else None}
+
+
+# ----------------------------------------------------------------------------
+# the oracle as a CPU baseline
+# ----------------------------------------------------------------------------
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 0) for d in threadpool_info() if d.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return "unknown"
+
+
+def oracle_linear_step(case, tokens: int, backward: bool):
+    """One oracle step (float64, numpy) on the first `tokens` tokens: dequant the
+    frozen weight, Cayley build, forward, and the adapter backward."""
+    import numpy as np
+    from oracle import oft_ref
+    from oracle.codecs import bf16_bits_to_f64
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from npcase import linear_np
+    c = linear_np(case)
+    spec = case["spec"]
+    t0 = time.perf_counter()
+    Wt = oft_ref.weight_t(c)
+    R = oft_ref.rotations(c["Q"], spec.b)
+    X = bf16_bits_to_f64(c["X"][:tokens])
+    oft_ref.linear_fwd(X, Wt, spec.splits, R)
+    if backward:
+        dY = bf16_bits_to_f64(c["dY"][:tokens])
+        oft_ref.linear_bwd(dY, X, Wt, spec.splits, R, spec.b)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline_linear(case, backward: bool, budget_s: float = 12.0):
+    spec = case["spec"]
+    tokens = min(spec.M, 128)
+    dt = oracle_linear_step(case, tokens, backward)
+    while dt < budget_s / 3 and tokens < spec.M:
+        tokens = min(spec.M, tokens * 4)
+        dt = oracle_linear_step(case, tokens, backward)
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"first {tokens} of {spec.M} tokens, whole weight dequantised, float64 numpy "
+                      f"({cpu_model()}), {dt:.2f} s"}
+
+
+def cpu_baseline_moe(case, budget_s: float = 12.0):
+    import numpy as np
+    from oracle import moe_ref
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from npcase import raw
+    spec = case["spec"]
+    logits = raw(case["logits"])
+    idx, _ = moe_ref.topk(logits, spec.top_k)
+    t0 = time.perf_counter()
+    done = 0
+    X = raw(case["X"])
+    while time.perf_counter() - t0 < budget_s and done < 8:
+        t = done
+        used = np.unique(idx[t])
+        codes = {int(e): raw(case["codes"][int(e)]) for e in used}
+        scales = {int(e): raw(case["scales"][int(e)]) for e in used}
+        bank = moe_ref.ExpertBank(codes, scales, spec.K, spec.group, spec.n_proj)
+        moe_ref.moe_fwd_direct(X[t:t + 1], logits[t:t + 1], bank, raw(case["Q"]), spec.b, spec.top_k)
+        done += 1
+    dt = time.perf_counter() - t0
+    return {"value": done / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{done} tokens of {spec.T}, direct per-token top-{spec.top_k} sum, float64 numpy "
+                      f"({cpu_model()}), {dt:.2f} s"}
+
+
+# ----------------------------------------------------------------------------
+# our path
+# ----------------------------------------------------------------------------
+
+def gemm_traffic(flops_per_launch_unit):
+    """Per-launch DRAM bytes of the GEMM kernel from the committed ncu summary, if
+    the kernel source is unchanged since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "gemm_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    src = os.path.join(ROOT, "orthogonal_fine_tuning_b200", "csrc", "gemm.cuh")
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    if d.get("gemm_cuh_sha256_16") != h:
+        return None
+    return d.get("bytes_per_launch_by_workload", {}).get(flops_per_launch_unit)
+
+
+def run_ours(args, rank, world):
+    import torch
+    import orthogonal_fine_tuning_b200 as oft
+    from gen import LINEAR_CONFIGS, MOE_CONFIGS, make_linear_case, make_moe_case
+
+    _, _, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    peaks, peak_src = load_peaks()
+    name = args.workload
+    is_moe = name in MOE_CONFIGS
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    if is_moe:
+        spec = MOE_CONFIGS[name]
+        case = make_moe_case(spec, device=dev)
+        W = oft.Weight("int4", case["codes"], case["scales"], spec.K, 2 * spec.n_proj, spec.group, n_experts=spec.E)
+        ws = torch.empty(oft.moe_chunked_oft_workspace(spec.T, spec.E, spec.top_k, spec.chunk, W, spec.b),
+                         dtype=torch.uint8, device=dev)
+        X, logits, Q = case["X"], case["logits"], case["Q"]
+        out = oft.moe_chunked_oft_fwd(X, logits, W, spec.b, Q, spec.top_k, spec.chunk, workspace=ws)
+        tokens = spec.T
+        backward = False
+
+        def step(Xi=X, Li=logits, Qi=Q):
+            oft.moe_chunked_oft_fwd(Xi, Li, W, spec.b, Qi, spec.top_k, spec.chunk, workspace=ws, out=out)
+            return out["Y"]
+
+        inputs = dict(X=X, logits=logits, Q=Q)
+        outputs = dict(Y=out["Y"])
+    else:
+        spec = LINEAR_CONFIGS[name]
+        backward = spec.backward
+        case = make_linear_case(spec)
+        W = oft.Weight(spec.fmt, case["codes"].to(dev), case["scales"].to(dev), spec.K, spec.N, spec.group)
+        X, Q = case["X"].to(dev), case["Q"].to(dev)
+        dY = case["dY"].to(dev) if backward else None
+        nbytes = oft.oft_linear_fwd_workspace(spec.M, W, spec.splits, spec.b)
+        if backward:
+            nbytes = max(nbytes, oft.oft_linear_bwd_workspace(spec.M, W, spec.splits, spec.b))
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        R = torch.empty(spec.P, spec.K // spec.b, spec.b, spec.b, dtype=torch.float32, device=dev)
+        Y = torch.empty(spec.M, spec.N, dtype=torch.bfloat16, device=dev)
+        dX = torch.empty(spec.M, spec.K, dtype=torch.bfloat16, device=dev)
+        dQ = torch.empty(spec.P, spec.K // spec.b, spec.b * (spec.b - 1) // 2, dtype=torch.float32, device=dev)
+        tokens = spec.M
+
+        def step(Xi=X, dYi=dY, Qi=Q):
+            oft.oft_build_rotation(Qi, spec.b, R=R)
+            oft.oft_linear_fwd(Xi, W, spec.splits, spec.b, R, Y=Y, workspace=ws)
+            if backward:
+                oft.oft_linear_bwd(dYi, Xi, W, spec.splits, spec.b, R, dX=dX, dQ=dQ, workspace=ws)
+                allreduce_grad(dQ)
+            return Y
+
+        inputs = dict(X=X, Q=Q) if not backward else dict(X=X, dY=dY, Q=Q)
+        outputs = dict(Y=Y) if not backward else dict(Y=Y, dX=dX, dQ=dQ)
+
+    # ---- device-resident timing ----
+    for _ in range(args.warmup):
+        step()
+    oft.oft_check_device()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    with ClockSampler(dev) as clocks, oft.profile(max_launches=max(4096, 64 * args.steps)) as prof:
+        for i in range(args.steps):
+            flush.zero_()                          # evict L2 between timed steps
+            starts[i].record()
+            step()
+            ends[i].record()
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    oft.oft_check_device()
+    ms_steps = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms_local = sum(ms_steps) / len(ms_steps)
+    ms_per_step = max_over_ranks(ms_local, dev)
+    value = tokens * world / (ms_per_step / 1e3)
+
+    # ---- algorithmic work ----
+    if is_moe:
+        n_active = int(out["n_active"].item())
+        TK = spec.T * spec.top_k
+        gemm_flops = 2.0 * TK * spec.K * 2 * spec.n_proj
+        flops = dict(gemm=gemm_flops, rot=2.0 * TK * spec.K * spec.b * 2,
+                     cayley=2.0 * spec.b ** 3 * n_active * 2 * (spec.K // spec.b))
+        total_flops = sum(flops.values())
+        expert_bytes = spec.K * 2 * spec.n_proj // 2 + 2 * 2 * spec.n_proj * (spec.K // spec.group)
+        chunk_buf_bytes = 2 * (2 * spec.K * 2 * spec.n_proj)      # bf16 write + read
+        alg_bytes = n_active * (expert_bytes + chunk_buf_bytes) + 2 * spec.T * spec.K + 2 * spec.T * 2 * spec.n_proj
+    else:
+        flops = linear_flops(spec, backward)
+        total_flops = sum(flops.values())
+        alg_bytes = weight_bytes(spec) + 2 * spec.M * spec.K + 2 * spec.M * spec.N
+        if backward:
+            alg_bytes += 2 * spec.M * spec.N + 2 * spec.M * spec.K + 4 * dQ.numel() + 2 * dQ.numel()
+    tflops = total_flops / (ms_per_step / 1e3) / 1e12
+
+    # ---- dominant kernel roofline ----
+    g_launch = prof.launches["gemm"]
+    g_ms = prof.ms["gemm"]
+    if is_moe:
+        # HBM-bound: algorithmic bytes of the whole step ÷ the step (chunk dequant + grouped GEMM dominate)
+        bound = "hbm"
+        achieved = alg_bytes / (ms_per_step / 1e3) / 1e9
+        peak = peaks["hbm_gbs"]
+        unit = "GB/s"
+        traffic = None
+        kernel = "whole step (chunk dequant + grouped GEMM), HBM"
+    else:
+        gemm_flops = flops["gemm_fwd"] + flops.get("gemm_bwd", 0.0)
+        per_launch = gemm_flops / (g_launch / args.steps)
+        avg_s = g_ms / g_launch / 1e3
+        bound = "tensor"
+        achieved = per_launch / avg_s / 1e12
+        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        unit = "TFLOP/s"
+        traffic = gemm_traffic(name)
+        kernel = "gemm_bf16_kernel (tcgen05/TMEM)"
+    roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+                "traffic": traffic, "kernel": kernel,
+                "peak_source": f"{peak_src} ({'sustained' if bound == 'tensor' else 'copy'})"}
+
+    # ---- end to end through the public API with host buffers ----
+    host_in = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in inputs.items()}
+    for k, v in inputs.items():
+        host_in[k].copy_(v)
+    host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in outputs.items()}
+    dev_in = {k: torch.empty_like(v) for k, v in inputs.items()}
+
+    def e2e_step():
+        for k in dev_in:
+            dev_in[k].copy_(host_in[k], non_blocking=True)
+        if is_moe:
+            step(dev_in["X"], dev_in["logits"], dev_in["Q"])
+        elif backward:
+            step(dev_in["X"], dev_in["dY"], dev_in["Q"])
+        else:
+            step(dev_in["X"], None, dev_in["Q"])
+        for k in host_out:
+            host_out[k].copy_(outputs[k], non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    es.record()
+    for _ in range(args.steps):
+        e2e_step()
+    ee.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(es.elapsed_time(ee) / args.steps, dev)
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+    d2h = sum(v.numel() * v.element_size() for v in host_out.values())
+    e2e = {"value": tokens * world / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    if rank != 0:
+        return None
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_moe(case) if is_moe else cpu_baseline_linear(case, backward)
+    config = {"workload": WORKLOAD_NAMES[name], "name": name, "tokens_per_gpu": tokens,
+              "global_batch_tokens": tokens * world, "parallelism": f"dp{world}" if world > 1 else "single",
+              "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MB write)",
+              "step": "build_rotation + fwd" + (" + bwd" if backward else "") + (" + dQ all-reduce" if world > 1 and backward else "")}
+    if is_moe:
+        config.update(n_active_experts=n_active)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; shapes and distributions of the workload)",
+        "config": config, "tflops": tflops, "algorithmic_flops_per_step": total_flops,
+        "algorithmic_bytes_per_step": alg_bytes, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": int(sum(prof.launches.values())),
+        "kernel_ms_per_step": {k: v / args.steps for k, v in prof.ms.items()},
+        "kernel_launches_per_step": {k: v / args.steps for k, v in prof.launches.items()},
+        "clocks": clocks.summary(),
+    }
+    return line
+
+
+def run_reference(args, rank, world):
+    """The oracle (float64 numpy, as it stands) timed on the host cores, on a
+    bounded sample of the same workload per step."""
+    if rank != 0:
+        return None
+    from gen import LINEAR_CONFIGS, MOE_CONFIGS, make_linear_case, make_moe_case
+    name = args.workload
+    if name in MOE_CONFIGS:
+        import torch
+        spec = MOE_CONFIGS[name]
+        dev = "cuda" if torch.cuda.is_available() else "cpu"
+        case = make_moe_case(spec, device=dev)
+        per = max(2.0, 150.0 / (args.steps + args.warmup))
+        for _ in range(args.warmup):
+            cpu_baseline_moe(case, budget_s=per / 4)
+        res = [cpu_baseline_moe(case, budget_s=per) for _ in range(args.steps)]
+        value = statistics.mean(r["value"] for r in res)
+        sample = res[-1]["sample"]
+    else:
+        spec = LINEAR_CONFIGS[name]
+        case = make_linear_case(spec)
+        per_budget = 150.0 / (args.steps + args.warmup)
+        tokens = min(spec.M, 64)
+        dt = oracle_linear_step(case, tokens, spec.backward)
+        while dt * 2 < per_budget and tokens < spec.M:
+            tokens = min(spec.M, tokens * 2)
+            dt = oracle_linear_step(case, tokens, spec.backward)
+        for _ in range(args.warmup):
+            oracle_linear_step(case, tokens, spec.backward)
+        times = [oracle_linear_step(case, tokens, spec.backward) for _ in range(args.steps)]
+        ms = 1e3 * statistics.mean(times)
+        value = tokens / (ms / 1e3)
+        sample = f"first {tokens} of {spec.M} tokens per step, float64 numpy ({cpu_model()})"
+    ms_per_step = None if name in MOE_CONFIGS else ms
+    return {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": WORKLOAD_NAMES[name], "name": name},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="c1", choices=sorted(WORKLOAD_NAMES))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        rank, world, _ = dist_env()
+        line = run_reference(args, rank, world)
+    else:
+        rank, world = init_dist("nccl")
+        if world != args.gpus:
+            print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+        line = run_ours(args, rank, world)
+        import torch.distributed as dist
+        if dist.is_initialized():
+            dist.barrier()
+            dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,317 @@
+// Persistent tcgen05 / TMEM grouped GEMM, bf16 x bf16 -> fp32 -> bf16.
+//
+//   C[c_row0 + m][c_col0 + n] = sum_k A[a_row0 + m][k] * B[b_row0 + n][k]
+//
+// for every group (sub-projection p of a fused weight, or (expert, projection)
+// pair of an MoE chunk).  The pages call for one independent adapter per
+// sub-projection of a fused QKV / gate-up tensor (chooseai.io news 4086, item
+// "自定义适配器核函数") and for a grouped GEMM over a chunk of transiently
+// dequantised experts (m.xxlwj.com 771001, section "技术细节"); both map onto
+// this one engine as groups.
+//
+// Roles (192 threads, one CTA per SM):
+//   warp 0      TMA producer: A tile 128x64 and B tile 256x64 per stage, SW128
+//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer (M=128, N=256, K=16)
+//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 32 columns -> bf16 -> global
+// Two 256-column fp32 accumulators in TMEM let the epilogue of tile i overlap
+// the main loop of tile i+1.  Every wait is bounded (see common.cuh).
+#pragma once
+
+#include "common.cuh"
+
+namespace oftk {
+namespace gemm {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;
+constexpr int STAGES = 4;
+constexpr int A_TILE_BYTES = BM * BK * 2;
+constexpr int B_TILE_BYTES = BN * BK * 2;
+constexpr int NUM_THREADS = 192;
+constexpr int MAX_GROUPS = 32;
+constexpr int MAX_MAPS = 4;
+constexpr uint32_t TMEM_COLS = 2 * BN;
+constexpr int GM = 16;  // m-tiles per raster band (L2 reuse of the B tiles)
+
+struct Group {
+  int m, n, k;
+  int a_map, b_map;
+  int a_row0, b_row0;
+  int c_row0, c_col0;
+  int tiles_m, tiles_n, tile0;
+};
+
+// MoE chunk: groups are derived on the device from the routing results.
+struct MoESrc {
+  const int* chunk_table;  // [n_chunks][chunk], -1 padded
+  const int* offsets;      // [E+1]
+  int chunk_idx, chunk, TK, n_proj, K;
+};
+
+struct Params {
+  CUtensorMap tmA[MAX_MAPS];
+  CUtensorMap tmB[MAX_MAPS];
+  void* C;            // bf16 [..][ldc], or fp32 when c_f32 != 0
+  long long ldc;
+  int c_f32;
+  int num_groups;
+  int use_moe;
+  Group groups[MAX_GROUPS];
+  MoESrc moe;
+};
+
+constexpr size_t kBarrierBytes = 256;
+constexpr size_t kGroupBytes = sizeof(Group) * MAX_GROUPS;
+constexpr size_t kSmemBytes = 1024 + STAGES * (A_TILE_BYTES + B_TILE_BYTES) + kBarrierBytes + kGroupBytes;
+
+__device__ __forceinline__ void decode_tile(const Group* sg, int ng, int t, int& g, int& mt, int& nt) {
+  g = 0;
+  while (g + 1 < ng && t >= sg[g + 1].tile0) ++g;
+  const int local = t - sg[g].tile0;
+  const int tm = sg[g].tiles_m, tn = sg[g].tiles_n;
+  const int band = local / (GM * tn);
+  const int rem = local - band * GM * tn;
+  const int rows = min(GM, tm - band * GM);
+  mt = band * GM + rem % rows;
+  nt = rem / rows;
+}
+
+// Waits for a phase ignoring the abort flag (teardown drain); bounded.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  const unsigned long long t0 = globaltimer_ns();
+  while (!mbar_try_wait(a, parity)) {
+    if (globaltimer_ns() - t0 > 200000000ull) {
+      atomicOr(&g_dev_err, kErrWaitDrain);
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ uint32_t pack2(uint32_t lo, uint32_t hi) {
+  return pack_bf16x2(__uint_as_float(lo), __uint_as_float(hi));
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1) gemm_bf16_kernel(const __grid_constant__ Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_TILE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_TILE_BYTES);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* acc_full = bars + 2 * STAGES;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* s_meta = reinterpret_cast<int*>(tmem_slot + 2);  // [0] total tiles, [1] groups
+  Group* sg = reinterpret_cast<Group*>(reinterpret_cast<uint8_t*>(bars) + kBarrierBytes);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    // group table
+    int ng = 0, tile = 0;
+    auto add = [&](const Group& src) {
+      Group g = src;
+      g.tiles_m = (g.m + BM - 1) / BM;
+      g.tiles_n = (g.n + BN - 1) / BN;
+      g.tile0 = tile;
+      tile += g.tiles_m * g.tiles_n;
+      sg[ng++] = g;
+    };
+    if (!p.use_moe) {
+      for (int g = 0; g < p.num_groups; ++g)
+        if (p.groups[g].m > 0 && p.groups[g].n > 0) add(p.groups[g]);
+    } else {
+      const MoESrc& s = p.moe;
+      for (int slot = 0; slot < s.chunk; ++slot) {
+        const int e = s.chunk_table[s.chunk_idx * s.chunk + slot];
+        if (e < 0) continue;
+        const int cnt = s.offsets[e + 1] - s.offsets[e];
+        if (cnt <= 0) continue;
+        for (int proj = 0; proj < 2; ++proj) {
+          Group g{};
+          g.m = cnt;
+          g.n = s.n_proj;
+          g.k = s.K;
+          g.a_map = 0;
+          g.b_map = 0;
+          g.a_row0 = proj * s.TK + s.offsets[e];
+          g.b_row0 = (slot * 2 + proj) * s.n_proj;
+          g.c_row0 = s.offsets[e];
+          g.c_col0 = proj * s.n_proj;
+          add(g);
+        }
+      }
+    }
+    s_meta[0] = tile;
+    s_meta[1] = ng;
+  }
+  if (warp == 0 && lane == 0) {
+    for (int i = 0; i < MAX_MAPS; ++i) {
+      tma_prefetch_desc(&p.tmA[i]);
+      tma_prefetch_desc(&p.tmB[i]);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = s_meta[0];
+  const int ng = s_meta[1];
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t ph = 0;
+      long long issued = 0;
+      for (int t = blockIdx.x; t < total; t += gridDim.x) {
+        int g, mt, nt;
+        decode_tile(sg, ng, t, g, mt, nt);
+        const Group& G = sg[g];
+        const int nk = (G.k + BK - 1) / BK;
+        bool ok = true;
+        for (int kt = 0; kt < nk; ++kt) {
+          if (!mbar_wait(&empty[stage], ph ^ 1, abort_flag, kErrWaitEmpty)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], A_TILE_BYTES + B_TILE_BYTES);
+          tma_load_2d(sA + stage * A_TILE_BYTES, &p.tmA[G.a_map], &full[stage], kt * BK, G.a_row0 + mt * BM);
+          tma_load_2d(sB + stage * B_TILE_BYTES, &p.tmB[G.b_map], &full[stage], kt * BK, G.b_row0 + nt * BN);
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            ph ^= 1;
+          }
+        }
+        if (!ok) break;
+      }
+      if (*abort_flag) {  // let the copies already in flight land before the CTA exits
+        for (long long i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
+          mbar_wait_drain(&full[i % STAGES], static_cast<uint32_t>((i / STAGES) & 1));
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t ph = 0;
+      int acc = 0;
+      uint32_t acc_ph = 0;
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+      for (int t = blockIdx.x; t < total; t += gridDim.x) {
+        int g, mt, nt;
+        decode_tile(sg, ng, t, g, mt, nt);
+        const int nk = (sg[g].k + BK - 1) / BK;
+        if (!mbar_wait(&acc_empty[acc], acc_ph ^ 1, abort_flag, kErrWaitAccEmpty)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + static_cast<uint32_t>(acc * BN);
+        bool ok = true;
+        for (int kt = 0; kt < nk; ++kt) {
+          if (!mbar_wait(&full[stage], ph, abort_flag, kErrWaitFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t ad = sdesc_kmajor_sw128(smem_u32(sA + stage * A_TILE_BYTES));
+          const uint64_t bd = sdesc_kmajor_sw128(smem_u32(sB + stage * B_TILE_BYTES));
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            mma_bf16_ss(d, ad + static_cast<uint64_t>(kk * 2), bd + static_cast<uint64_t>(kk * 2), idesc,
+                        (kt | kk) ? 1u : 0u);
+          mma_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            ph ^= 1;
+          }
+        }
+        if (!ok) break;
+        mma_commit(&acc_full[acc]);
+        acc ^= 1;
+        if (acc == 0) acc_ph ^= 1;
+      }
+      // all MMAs issued by this thread have completed once `drain` flips
+      mma_commit(drain);
+      mbar_wait_drain(drain, 0);
+    }
+  } else {
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    int acc = 0;
+    uint32_t acc_ph = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      int g, mt, nt;
+      decode_tile(sg, ng, t, g, mt, nt);
+      const Group& G = sg[g];
+      bool ok = false;
+      if (lane == 0) ok = mbar_wait(&acc_full[acc], acc_ph, abort_flag, kErrWaitAccFull);
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      const int row = mt * BM + q * 32 + lane;
+      const bool row_ok = row < G.m;
+      const long long crow_off = static_cast<long long>(G.c_row0 + (row_ok ? row : 0)) * p.ldc + G.c_col0;
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t r[32];
+        __syncwarp();
+        tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN + c), r);
+        tmem_ld_wait();
+        const int col = nt * BN + c;
+        if (row_ok && col < G.n) {
+          if (p.c_f32) {
+            float* crow = static_cast<float*>(p.C) + crow_off;
+            if (col + 32 <= G.n) {
+              uint4* dst = reinterpret_cast<uint4*>(crow + col);
+#pragma unroll
+              for (int v = 0; v < 8; ++v) dst[v] = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+            } else {
+              for (int i = 0; i < 32 && col + i < G.n; ++i) crow[col + i] = __uint_as_float(r[i]);
+            }
+          } else {
+            uint16_t* crow = static_cast<uint16_t*>(p.C) + crow_off;
+            if (col + 32 <= G.n) {
+              uint4* dst = reinterpret_cast<uint4*>(crow + col);
+#pragma unroll
+              for (int v = 0; v < 4; ++v)
+                dst[v] = make_uint4(pack2(r[8 * v + 0], r[8 * v + 1]), pack2(r[8 * v + 2], r[8 * v + 3]),
+                                    pack2(r[8 * v + 4], r[8 * v + 5]), pack2(r[8 * v + 6], r[8 * v + 7]));
+            } else {
+              for (int i = 0; i < 32 && col + i < G.n; ++i) crow[col + i] = f32_to_bf16_bits(__uint_as_float(r[i]));
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[acc]);
+      acc ^= 1;
+      if (acc == 0) acc_ph ^= 1;
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace gemm
+}  // namespace oftk

@@ -1,0 +1,241 @@
+// Routing, bucketing, chunking, rotated gather and combine for the
+// active-expert-chunked MoE OFT forward.
+//
+// The pages: the experts the router selects are grouped into fixed-size chunks,
+// each chunk is dequantised transiently and fed to a grouped GEMM, after which
+// its high-precision copy is released, so peak transient memory stays bounded by
+// one chunk (m.xxlwj.com 771001, section "技术细节", paragraph
+// "Active-expert-chunked dequantization"; chooseai.io news 4086, section
+// "对低精度 MoE 模型的专门优化").  Readings for what the pages leave open: top-k by
+// logit with ties to the lower expert id, softmax over the selected logits,
+// buckets stable in (token, slot), active experts ascending, combine in slot order.
+#pragma once
+
+#include "common.cuh"
+#include "rotate.cuh"
+
+namespace oftk {
+
+constexpr int kMaxExperts = 512;
+constexpr int kMaxTopK = 8;
+
+// One warp per token: top_k by (logit desc, expert id asc), then softmax over
+// the selected logits (fp32).
+__global__ void __launch_bounds__(256) moe_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                       int* __restrict__ idx_out, float* __restrict__ w_out) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) / 32;
+  const int lane = threadIdx.x % 32;
+  if (warp >= T) return;
+  constexpr int PER = kMaxExperts / 32;
+  float v[PER];
+  uint32_t taken = 0;
+  const float* row = logits + static_cast<size_t>(warp) * E;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int e = lane + 32 * i;
+    v[i] = e < E ? row[e] : -INFINITY;
+    if (e >= E) taken |= 1u << i;
+  }
+  float sel_v[kMaxTopK];
+  int sel_e[kMaxTopK];
+  for (int s = 0; s < k; ++s) {
+    float bv = -INFINITY;
+    int be = 0x7FFFFFFF;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int e = lane + 32 * i;
+      if (!(taken & (1u << i)) && (v[i] > bv || (v[i] == bv && e < be))) {
+        bv = v[i];
+        be = e;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
+      const int oe = __shfl_xor_sync(0xFFFFFFFFu, be, off);
+      if (ov > bv || (ov == bv && oe < be)) {
+        bv = ov;
+        be = oe;
+      }
+    }
+    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+    sel_v[s] = bv;
+    sel_e[s] = be;
+  }
+  if (lane == 0) {
+    const float mx = sel_v[0];
+    float ex[kMaxTopK];
+    float sum = 0.f;
+    for (int s = 0; s < k; ++s) {
+      ex[s] = expf(sel_v[s] - mx);
+      sum += ex[s];
+    }
+    for (int s = 0; s < k; ++s) {
+      idx_out[static_cast<size_t>(warp) * k + s] = sel_e[s];
+      w_out[static_cast<size_t>(warp) * k + s] = ex[s] / sum;
+    }
+  }
+}
+
+// Single CTA of 1024 threads (32 warps).  Each warp owns a contiguous range of
+// the T*k entries; warp-private histograms give every (warp, expert) a base
+// offset, and each warp then places its entries in order (match_any ranks
+// equal experts within a 32-entry step), so the bucket is stable in (t, slot)
+// and independent of scheduling.
+// Outputs: offsets[E+1], bucket[TK], inv_pos[TK] (entry -> bucket position),
+// pos_expert[TK], chunk_table[n_chunks_max * chunk] (-1 padded), n_active[1].
+__global__ void __launch_bounds__(1024) moe_route_kernel(const int* __restrict__ idx, int TK, int E, int chunk,
+                                                         int n_chunks_max, int* __restrict__ offsets,
+                                                         int* __restrict__ bucket, int* __restrict__ inv_pos,
+                                                         int* __restrict__ pos_expert, int* __restrict__ chunk_table,
+                                                         int* __restrict__ n_active) {
+  extern __shared__ int rsm[];
+  int* hist = rsm;                // [32][E]
+  int* off = rsm + 32 * E;        // [E + 1]
+  int* act = off + E + 1;         // [E] exclusive rank among active experts
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int per = (TK + 31) / 32;
+  const int beg = min(TK, warp * per), end = min(TK, beg + per);
+  for (int i = threadIdx.x; i < 32 * E; i += 1024) hist[i] = 0;
+  __syncthreads();
+  for (int j = beg + lane; j < end; j += 32) atomicAdd(&hist[warp * E + idx[j]], 1);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += 1024) {
+    int run = 0;
+    for (int w = 0; w < 32; ++w) {
+      const int c = hist[w * E + e];
+      hist[w * E + e] = run;
+      run += c;
+    }
+    off[e] = run;  // total count for now
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int acc = 0, na = 0;
+    for (int e = 0; e < E; ++e) {
+      const int c = off[e];
+      off[e] = acc;
+      acc += c;
+      act[e] = c > 0 ? na++ : -1;
+    }
+    off[E] = acc;
+    *n_active = na;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e <= E; e += 1024) offsets[e] = off[e];
+  for (int i = threadIdx.x; i < n_chunks_max * chunk; i += 1024) chunk_table[i] = -1;
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += 1024)
+    if (act[e] >= 0) chunk_table[act[e]] = e;
+  // stable fill
+  for (int j0 = beg; j0 < end; j0 += 32) {
+    const int j = j0 + lane;
+    const bool valid = j < end;
+    const int e = valid ? idx[j] : -1 - lane;  // distinct dummies for idle lanes
+    const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    int base = 0;
+    if (valid) base = hist[warp * E + e];
+    __syncwarp();
+    if (valid) {
+      const int pos = off[e] + base + rank;
+      bucket[pos] = j;
+      inv_pos[j] = pos;
+      pos_expert[pos] = e;
+      if (rank == 0) hist[warp * E + e] = base + __popc(peers);
+    }
+    __syncwarp();
+  }
+}
+
+// Xg[proj][pos][:] = X[bucket[pos] / k] R_{e(pos), proj}   (bucket order)
+// grid = (K/B, ceil(TK/64), 2).  Rows of one tile may belong to several experts;
+// the tile walks its expert segments and stages each segment's R block.
+template <int B>
+__global__ void __launch_bounds__(kRotThreads) moe_gather_rotate_kernel(
+    const uint16_t* __restrict__ X, int K, int TK, int top_k, const int* __restrict__ bucket,
+    const int* __restrict__ pos_expert, const float* __restrict__ Rex, uint16_t* __restrict__ Xg) {
+  constexpr int LD = RotCfg<B>::LD, TPT = RotCfg<B>::TPT;
+  __shared__ __align__(16) float xs[kRotTokens * LD];
+  __shared__ __align__(16) float rs[B * B];
+  __shared__ int s_exp[kRotTokens];
+  const int j = blockIdx.x, p0 = blockIdx.y * kRotTokens, proj = blockIdx.z, nb = K / B;
+  const int c = threadIdx.x % B, tg = threadIdx.x / B;
+  constexpr int CH = B / 8;
+  for (int it = threadIdx.x; it < kRotTokens * CH; it += kRotThreads) {
+    const int r = it / CH, ch = it % CH;
+    const int pos = p0 + r;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (pos < TK) {
+      const int t = bucket[pos] / top_k;
+      v = *reinterpret_cast<const uint4*>(X + static_cast<size_t>(t) * K + j * B + ch * 8);
+    }
+    float* d = xs + r * LD + ch * 8;
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      d[2 * i] = __uint_as_float(w[i] << 16);
+      d[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  }
+  for (int r = threadIdx.x; r < kRotTokens; r += kRotThreads) s_exp[r] = (p0 + r < TK) ? pos_expert[p0 + r] : -1;
+  __syncthreads();
+  int s0 = 0;
+  while (s0 < kRotTokens && s_exp[s0] >= 0) {
+    const int e = s_exp[s0];
+    int s1 = s0 + 1;
+    while (s1 < kRotTokens && s_exp[s1] == e) ++s1;
+    const float* Rb = Rex + ((static_cast<size_t>(e) * 2 + proj) * nb + j) * B * B;
+    for (int idx = threadIdx.x; idx < B * B / 4; idx += kRotThreads)
+      reinterpret_cast<float4*>(rs)[idx] = reinterpret_cast<const float4*>(Rb)[idx];
+    __syncthreads();
+#pragma unroll
+    for (int t = 0; t < TPT; ++t) {
+      const int r = tg * TPT + t;
+      if (r < s0 || r >= s1) continue;
+      float acc = 0.f;
+#pragma unroll 8
+      for (int i = 0; i < B; i += 4) {
+        const float4 x = *reinterpret_cast<const float4*>(xs + r * LD + i);
+        acc = fmaf(x.x, rs[(i + 0) * B + c], acc);
+        acc = fmaf(x.y, rs[(i + 1) * B + c], acc);
+        acc = fmaf(x.z, rs[(i + 2) * B + c], acc);
+        acc = fmaf(x.w, rs[(i + 3) * B + c], acc);
+      }
+      Xg[(static_cast<size_t>(proj) * TK + p0 + r) * K + j * B + c] = f32_to_bf16_bits(acc);
+    }
+    __syncthreads();
+    s0 = s1;
+  }
+}
+
+// Y[t][n] = sum_{s < k} w[t][s] * Ytk[inv_pos[t*k + s]][n], fp32 in slot order (Ytk kept in fp32).
+__global__ void __launch_bounds__(256) moe_combine_kernel(const float* __restrict__ Ytk, const float* __restrict__ w,
+                                                          const int* __restrict__ inv_pos, int T, int N, int k,
+                                                          uint16_t* __restrict__ Y) {
+  const long long units = static_cast<long long>(T) * (N / 8);
+  for (long long u = blockIdx.x * 256ll + threadIdx.x; u < units; u += static_cast<long long>(gridDim.x) * 256) {
+    const int t = static_cast<int>(u / (N / 8));
+    const int n = static_cast<int>(u % (N / 8)) * 8;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int s = 0; s < k; ++s) {
+      const float ws = w[static_cast<size_t>(t) * k + s];
+      const int pos = inv_pos[static_cast<size_t>(t) * k + s];
+      const float4 a = *reinterpret_cast<const float4*>(Ytk + static_cast<size_t>(pos) * N + n);
+      const float4 b = *reinterpret_cast<const float4*>(Ytk + static_cast<size_t>(pos) * N + n + 4);
+      acc[0] = fmaf(ws, a.x, acc[0]);
+      acc[1] = fmaf(ws, a.y, acc[1]);
+      acc[2] = fmaf(ws, a.z, acc[2]);
+      acc[3] = fmaf(ws, a.w, acc[3]);
+      acc[4] = fmaf(ws, b.x, acc[4]);
+      acc[5] = fmaf(ws, b.y, acc[5]);
+      acc[6] = fmaf(ws, b.z, acc[6]);
+      acc[7] = fmaf(ws, b.w, acc[7]);
+    }
+    *reinterpret_cast<uint4*>(Y + static_cast<size_t>(t) * N + n) =
+        make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
+                   pack_bf16x2(acc[6], acc[7]));
+  }
+}
+
+}  // namespace oftk

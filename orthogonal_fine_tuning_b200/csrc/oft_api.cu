@@ -1,0 +1,667 @@
+// C ABI of the OFT hot path (declared in include/oft.h): argument checks,
+// workspace carving, TMA descriptor encoding and kernel launches.  All the
+// arithmetic runs in the kernels included below.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "oft.h"
+
+#include "common.cuh"
+#include "dequant.cuh"
+#include "cayley.cuh"
+#include "rotate.cuh"
+#include "gemm.cuh"
+#include "moe.cuh"
+
+using namespace oftk;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+#define OFT_CUDA(call)                                                                      \
+  do {                                                                                      \
+    cudaError_t e_ = (call);                                                                \
+    if (e_ != cudaSuccess) return fail(OFT_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+  } while (0)
+
+#define OFT_LAUNCHED(what)                                                                     \
+  do {                                                                                         \
+    cudaError_t e_ = cudaGetLastError();                                                       \
+    if (e_ != cudaSuccess) return fail(OFT_ERR_CUDA, "launch %s: %s", what, cudaGetErrorString(e_)); \
+  } while (0)
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+// ---- launch profiler: CUDA event pairs around launches, per kernel class ----
+struct ProfState {
+  bool on = false;
+  int cap = 0, n = 0, dropped = 0;
+  cudaEvent_t* ev = nullptr;  // 2 per slot
+  int* kind = nullptr;
+  int counts[OFT_K_NUM] = {0};
+};
+ProfState g_prof;
+
+struct ProfScope {
+  int idx = -1;
+  cudaStream_t st;
+  ProfScope(int k, cudaStream_t s) : st(s) {
+    if (!g_prof.on) return;
+    g_prof.counts[k]++;
+    if (g_prof.n < g_prof.cap) {
+      idx = g_prof.n++;
+      g_prof.kind[idx] = k;
+      cudaEventRecord(g_prof.ev[2 * idx], st);
+    } else {
+      g_prof.dropped++;
+    }
+  }
+  ~ProfScope() {
+    if (idx >= 0) cudaEventRecord(g_prof.ev[2 * idx + 1], st);
+  }
+};
+
+// ---- driver entry point for TMA descriptors (no link-time libcuda dependency) ----
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor [outer][inner] with row pitch `pitch_elems`, box {64, box_rows}, 128B swizzle.
+int make_map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t pitch_elems,
+                  uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return fail(OFT_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {pitch_elems * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(OFT_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d): inner=%llu outer=%llu pitch=%llu", int(r),
+                (unsigned long long)inner, (unsigned long long)outer, (unsigned long long)pitch_elems);
+  return OFT_OK;
+}
+
+// ---- argument checks ----
+int check_weight(const oft_weight* W, bool bank_ok) {
+  if (W == nullptr) return fail(OFT_ERR_INVALID_ARG, "weight descriptor is NULL");
+  if (W->codes == nullptr || W->scales == nullptr) return fail(OFT_ERR_INVALID_ARG, "weight codes/scales NULL");
+  if (!aligned16(W->codes) || !aligned16(W->scales))
+    return fail(OFT_ERR_INVALID_ARG, "weight codes/scales must be 16-byte aligned");
+  if (W->d_in <= 0 || W->d_out <= 0) return fail(OFT_ERR_INVALID_ARG, "d_in/d_out must be positive");
+  if (W->d_in % 32 != 0) return fail(OFT_ERR_UNSUPPORTED, "d_in must be a multiple of 32 (got %d)", W->d_in);
+  if (W->d_out % 8 != 0) return fail(OFT_ERR_UNSUPPORTED, "d_out must be a multiple of 8 (got %d)", W->d_out);
+  if (!bank_ok && W->n_experts > 1) return fail(OFT_ERR_INVALID_ARG, "an expert bank is not accepted here");
+  switch (W->fmt) {
+    case OFT_W_INT4:
+      if (W->group != 32 && W->group != 64 && W->group != 128)
+        return fail(OFT_ERR_UNSUPPORTED, "INT4 group must be 32, 64 or 128 (got %d)", W->group);
+      if (W->d_in % W->group != 0) return fail(OFT_ERR_UNSUPPORTED, "d_in %% group != 0");
+      break;
+    case OFT_W_FP8:
+      break;
+    case OFT_W_MXFP4:
+      if (W->group != 32 && W->group != 0) return fail(OFT_ERR_UNSUPPORTED, "MXFP4 blocks are 32 wide");
+      break;
+    default:
+      return fail(OFT_ERR_UNSUPPORTED, "unknown weight format %d", W->fmt);
+  }
+  return OFT_OK;
+}
+
+int check_b(int b, int K) {
+  if (b != 16 && b != 32 && b != 64) return fail(OFT_ERR_UNSUPPORTED, "block size b must be 16, 32 or 64 (got %d)", b);
+  if (K % b != 0) return fail(OFT_ERR_UNSUPPORTED, "d_in %d is not a multiple of b %d", K, b);
+  return OFT_OK;
+}
+
+int check_split(const oft_split* S, int N) {
+  if (S == nullptr) return fail(OFT_ERR_INVALID_ARG, "split descriptor is NULL");
+  if (S->n < 1 || S->n > 4) return fail(OFT_ERR_UNSUPPORTED, "1..4 sub-projections supported (got %d)", S->n);
+  int sum = 0;
+  for (int i = 0; i < S->n; ++i) {
+    if (S->sizes[i] <= 0 || S->sizes[i] % 8 != 0)
+      return fail(OFT_ERR_UNSUPPORTED, "sub-projection sizes must be positive multiples of 8");
+    sum += S->sizes[i];
+  }
+  if (sum != N) return fail(OFT_ERR_INVALID_ARG, "sub-projection sizes sum to %d, d_out is %d", sum, N);
+  return OFT_OK;
+}
+
+WeightView view_of(const oft_weight* W) {
+  WeightView v{};
+  v.fmt = W->fmt;
+  v.codes = static_cast<const uint8_t*>(W->codes);
+  v.scales = W->scales;
+  v.N = W->d_out;
+  v.K = W->d_in;
+  v.group = W->fmt == OFT_W_INT4 ? W->group : 32;
+  const long long code_bytes = W->fmt == OFT_W_FP8 ? 1ll * W->d_out * W->d_in : 1ll * W->d_out * W->d_in / 2;
+  long long scale_bytes = 0;
+  if (W->fmt == OFT_W_INT4) scale_bytes = 2ll * (W->d_in / W->group) * W->d_out;
+  if (W->fmt == OFT_W_FP8) scale_bytes = 4ll * W->d_out;
+  if (W->fmt == OFT_W_MXFP4) scale_bytes = 1ll * (W->d_in / 32) * W->d_out;
+  v.codes_expert_stride = code_bytes;
+  v.scales_expert_stride = scale_bytes;
+  return v;
+}
+
+int launch_dequant(const WeightView& v, uint16_t* out, bool transpose, cudaStream_t st) {
+  if (!transpose) {
+    const long long units = 1ll * v.N * (v.K / 8);
+    const int grid = static_cast<int>(std::min<long long>((units + 255) / 256, 148ll * 16));
+    ProfScope ps(OFT_K_DEQUANT, st);
+    dequant_rows_kernel<<<grid, 256, 0, st>>>(v, out);
+    OFT_LAUNCHED("dequant_rows_kernel");
+  } else {
+    dim3 grid((v.K + 63) / 64, (v.N + 63) / 64);
+    ProfScope ps(OFT_K_DEQUANT, st);
+    dequant_transposed_kernel<<<grid, 256, 0, st>>>(v, out);
+    OFT_LAUNCHED("dequant_transposed_kernel");
+  }
+  return OFT_OK;
+}
+
+int launch_cayley(const uint16_t* Q, int nblocks, int b, float* R, const int* offsets, int blocks_per_expert,
+                  cudaStream_t st) {
+  const size_t smem = (2 * b * (b + 1) + b) * sizeof(float);
+  const int grid = std::min(nblocks, sm_count() * 8);
+  OFT_CUDA(cudaFuncSetAttribute(cayley_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024));
+  ProfScope ps(OFT_K_CAYLEY, st);
+  cayley_fwd_kernel<<<grid, kCayleyThreads, smem, st>>>(Q, nblocks, b, R, offsets, blocks_per_expert);
+  OFT_LAUNCHED("cayley_fwd_kernel");
+  return OFT_OK;
+}
+
+int launch_rotate_fwd(const uint16_t* X, int M, int K, int P, int b, const float* R, uint16_t* Xr, cudaStream_t st) {
+  dim3 grid(K / b, (M + kRotTokens - 1) / kRotTokens);
+  ProfScope ps(OFT_K_ROTATE, st);
+  if (b == 16) rotate_fwd_kernel<16><<<grid, kRotThreads, 0, st>>>(X, M, K, P, R, Xr);
+  if (b == 32) rotate_fwd_kernel<32><<<grid, kRotThreads, 0, st>>>(X, M, K, P, R, Xr);
+  if (b == 64) rotate_fwd_kernel<64><<<grid, kRotThreads, 0, st>>>(X, M, K, P, R, Xr);
+  OFT_LAUNCHED("rotate_fwd_kernel");
+  return OFT_OK;
+}
+
+int launch_gemm(const gemm::Params& prm, int total_tiles_hint, cudaStream_t st) {
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    OFT_CUDA(cudaFuncSetAttribute(gemm::gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(gemm::kSmemBytes)));
+    attr_set[dev] = true;
+  }
+  int grid = sm_count();
+  if (total_tiles_hint > 0 && total_tiles_hint < grid) grid = total_tiles_hint;
+  ProfScope ps(OFT_K_GEMM, st);
+  gemm::gemm_bf16_kernel<<<grid, gemm::NUM_THREADS, gemm::kSmemBytes, st>>>(prm);
+  OFT_LAUNCHED("gemm_bf16_kernel");
+  return OFT_OK;
+}
+
+int tiles_of(int m, int n) { return ((m + gemm::BM - 1) / gemm::BM) * ((n + gemm::BN - 1) / gemm::BN); }
+
+// number of token partitions for the dR reduction (deterministic in the shape)
+int grad_parts(int M, int P, int nb) {
+  const int want = (600 + P * nb - 1) / (P * nb);
+  const int maxp = (M + kGTok - 1) / kGTok;
+  return std::max(1, std::min(want, maxp));
+}
+
+struct FwdLayout {
+  size_t xr, wdq, total;
+};
+FwdLayout fwd_layout(int M, int K, int N, int P) {
+  FwdLayout L{};
+  L.xr = 0;
+  L.wdq = round_up(L.xr + 2ull * P * M * K, 256);
+  L.total = round_up(L.wdq + 2ull * N * K, 256);
+  return L;
+}
+
+struct BwdLayout {
+  size_t dxr, wdqt, gpart, total;
+  int nparts;
+};
+BwdLayout bwd_layout(int M, int K, int N, int P, int b) {
+  BwdLayout L{};
+  L.nparts = grad_parts(M, P, K / b);
+  L.dxr = 0;
+  L.wdqt = round_up(L.dxr + 4ull * P * M * K, 256);  // dX' kept in fp32
+  L.gpart = round_up(L.wdqt + 2ull * N * K, 256);
+  L.total = round_up(L.gpart + 4ull * P * (K / b) * L.nparts * b * b, 256);
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* oft_version(void) { return "oft-b200 0.1 (sm_100a, tcgen05)"; }
+
+const char* oft_last_error(void) { return g_last_error.c_str(); }
+
+int oft_check_device(void* stream) {
+  OFT_CUDA(cudaStreamSynchronize(as_stream(stream)));
+  unsigned int word = 0, zero = 0;
+  OFT_CUDA(cudaMemcpyFromSymbol(&word, g_dev_err, sizeof(word)));
+  if (word != 0) {
+    OFT_CUDA(cudaMemcpyToSymbol(g_dev_err, &zero, sizeof(zero)));
+    return fail(OFT_ERR_TIMEOUT, "a bounded device wait ran out (error bits 0x%x)", word);
+  }
+  return OFT_OK;
+}
+
+int oft_build_rotation(const uint16_t* Q, int n_blocks, int b, float* R, void* stream) {
+  if (n_blocks < 0) return fail(OFT_ERR_INVALID_ARG, "n_blocks < 0");
+  if (n_blocks == 0) return OFT_OK;
+  if (Q == nullptr || R == nullptr) return fail(OFT_ERR_INVALID_ARG, "Q/R NULL");
+  if (!aligned16(Q) || !aligned16(R)) return fail(OFT_ERR_INVALID_ARG, "Q/R must be 16-byte aligned");
+  if (int rc = check_b(b, b)) return rc;
+  return launch_cayley(Q, n_blocks, b, R, nullptr, 1, as_stream(stream));
+}
+
+int oft_cayley_backward(const float* R, const float* G, int n_blocks, int b, float* dQ, void* stream) {
+  if (n_blocks < 0) return fail(OFT_ERR_INVALID_ARG, "n_blocks < 0");
+  if (n_blocks == 0) return OFT_OK;
+  if (!R || !G || !dQ) return fail(OFT_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(R) || !aligned16(G) || !aligned16(dQ)) return fail(OFT_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (int rc = check_b(b, b)) return rc;
+  const size_t smem = 3 * b * (b + 1) * sizeof(float);
+  const int grid = std::min(n_blocks, sm_count() * 8);
+  OFT_CUDA(cudaFuncSetAttribute(cayley_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024));
+  ProfScope ps(OFT_K_CAYLEY, as_stream(stream));
+  cayley_bwd_kernel<<<grid, kCayleyThreads, smem, as_stream(stream)>>>(R, G, 1, n_blocks, b, dQ);
+  OFT_LAUNCHED("cayley_bwd_kernel");
+  return OFT_OK;
+}
+
+int oft_dequant_weight(const oft_weight* W, uint16_t* out, int transpose, void* stream) {
+  if (int rc = check_weight(W, false)) return rc;
+  if (out == nullptr || !aligned16(out)) return fail(OFT_ERR_INVALID_ARG, "out NULL or misaligned");
+  return launch_dequant(view_of(W), out, transpose != 0, as_stream(stream));
+}
+
+int oft_rotate(const uint16_t* X, int M, int K, int P, int b, const float* R, uint16_t* Xr, void* stream) {
+  if (M < 0 || K <= 0 || P < 1) return fail(OFT_ERR_INVALID_ARG, "bad sizes");
+  if (M == 0) return OFT_OK;
+  if (!X || !R || !Xr || !aligned16(X) || !aligned16(R) || !aligned16(Xr))
+    return fail(OFT_ERR_INVALID_ARG, "NULL or misaligned pointer");
+  if (int rc = check_b(b, K)) return rc;
+  if (K % 8 != 0) return fail(OFT_ERR_UNSUPPORTED, "K must be a multiple of 8");
+  return launch_rotate_fwd(X, M, K, P, b, R, Xr, as_stream(stream));
+}
+
+size_t oft_linear_fwd_workspace(int M, const oft_weight* W, const oft_split* S, int b) {
+  if (W == nullptr || S == nullptr || M <= 0) return 0;
+  (void)b;
+  return fwd_layout(M, W->d_in, W->d_out, S->n).total;
+}
+
+int oft_linear_fwd(const uint16_t* X, int M, const oft_weight* W, const oft_split* S, int b, const float* R,
+                   uint16_t* Y, void* ws, size_t ws_bytes, void* stream) {
+  if (int rc = check_weight(W, false)) return rc;
+  if (int rc = check_split(S, W->d_out)) return rc;
+  const int K = W->d_in, N = W->d_out, P = S->n;
+  if (int rc = check_b(b, K)) return rc;
+  if (M < 0) return fail(OFT_ERR_INVALID_ARG, "M < 0");
+  if (M == 0) return OFT_OK;
+  if (!X || !R || !Y || !ws) return fail(OFT_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(X) || !aligned16(R) || !aligned16(Y) || !aligned16(ws))
+    return fail(OFT_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  const FwdLayout L = fwd_layout(M, K, N, P);
+  if (ws_bytes < L.total) return fail(OFT_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
+  cudaStream_t st = as_stream(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  uint16_t* Xr = reinterpret_cast<uint16_t*>(wsb + L.xr);
+  uint16_t* Wdq = reinterpret_cast<uint16_t*>(wsb + L.wdq);
+
+  if (int rc = launch_rotate_fwd(X, M, K, P, b, R, Xr, st)) return rc;
+  if (int rc = launch_dequant(view_of(W), Wdq, false, st)) return rc;
+
+  gemm::Params prm;
+  memset(&prm, 0, sizeof(prm));
+  if (int rc = make_map_bf16(&prm.tmA[0], Xr, K, 1ull * P * M, K, gemm::BM)) return rc;
+  if (int rc = make_map_bf16(&prm.tmB[0], Wdq, K, N, K, gemm::BN)) return rc;
+  for (int i = 1; i < gemm::MAX_MAPS; ++i) {
+    prm.tmA[i] = prm.tmA[0];
+    prm.tmB[i] = prm.tmB[0];
+  }
+  prm.C = Y;
+  prm.ldc = N;
+  prm.num_groups = P;
+  int off = 0, tiles = 0;
+  for (int p = 0; p < P; ++p) {
+    gemm::Group& g = prm.groups[p];
+    g.m = M;
+    g.n = S->sizes[p];
+    g.k = K;
+    g.a_map = 0;
+    g.b_map = 0;
+    g.a_row0 = p * M;
+    g.b_row0 = off;
+    g.c_row0 = 0;
+    g.c_col0 = off;
+    off += S->sizes[p];
+    tiles += tiles_of(M, g.n);
+  }
+  return launch_gemm(prm, tiles, st);
+}
+
+size_t oft_linear_bwd_workspace(int M, const oft_weight* W, const oft_split* S, int b) {
+  if (W == nullptr || S == nullptr || M <= 0 || b <= 0) return 0;
+  return bwd_layout(M, W->d_in, W->d_out, S->n, b).total;
+}
+
+int oft_linear_bwd(const uint16_t* dY, const uint16_t* X, int M, const oft_weight* W, const oft_split* S, int b,
+                   const float* R, uint16_t* dX, float* dQ, void* ws, size_t ws_bytes, void* stream) {
+  if (int rc = check_weight(W, false)) return rc;
+  if (int rc = check_split(S, W->d_out)) return rc;
+  const int K = W->d_in, N = W->d_out, P = S->n, nb = K / (b > 0 ? b : 1);
+  if (int rc = check_b(b, K)) return rc;
+  if (M < 0) return fail(OFT_ERR_INVALID_ARG, "M < 0");
+  if (!dQ || !R) return fail(OFT_ERR_INVALID_ARG, "NULL pointer");
+  cudaStream_t st = as_stream(stream);
+  if (M == 0) {  // no tokens: dX is empty and dQ is zero
+    OFT_CUDA(cudaMemsetAsync(dQ, 0, sizeof(float) * P * nb * (b * (b - 1) / 2), st));
+    return OFT_OK;
+  }
+  if (!dY || !X || !dX || !ws) return fail(OFT_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(dY) || !aligned16(X) || !aligned16(R) || !aligned16(dX) || !aligned16(dQ) || !aligned16(ws))
+    return fail(OFT_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  const BwdLayout L = bwd_layout(M, K, N, P, b);
+  if (ws_bytes < L.total) return fail(OFT_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  float* dXr = reinterpret_cast<float*>(wsb + L.dxr);
+  uint16_t* WdqT = reinterpret_cast<uint16_t*>(wsb + L.wdqt);
+  float* Gp = reinterpret_cast<float*>(wsb + L.gpart);
+
+  if (int rc = launch_dequant(view_of(W), WdqT, true, st)) return rc;
+
+  // dX'_p = dY_p deq(W_p)^T : A = dY columns of p (reduction over N_p), B = deq(W)^T columns of p
+  gemm::Params prm;
+  memset(&prm, 0, sizeof(prm));
+  int off = 0, tiles = 0;
+  for (int p = 0; p < P; ++p) {
+    const int Np = S->sizes[p];
+    if (int rc = make_map_bf16(&prm.tmA[p], dY + off, Np, M, N, gemm::BM)) return rc;
+    if (int rc = make_map_bf16(&prm.tmB[p], WdqT + off, Np, K, N, gemm::BN)) return rc;
+    gemm::Group& g = prm.groups[p];
+    g.m = M;
+    g.n = K;
+    g.k = Np;
+    g.a_map = p;
+    g.b_map = p;
+    g.a_row0 = 0;
+    g.b_row0 = 0;
+    g.c_row0 = p * M;
+    g.c_col0 = 0;
+    off += Np;
+    tiles += tiles_of(M, K);
+  }
+  for (int p = P; p < gemm::MAX_MAPS; ++p) {
+    prm.tmA[p] = prm.tmA[0];
+    prm.tmB[p] = prm.tmB[0];
+  }
+  prm.C = dXr;
+  prm.c_f32 = 1;
+  prm.ldc = K;
+  prm.num_groups = P;
+  if (int rc = launch_gemm(prm, tiles, st)) return rc;
+
+  dim3 rgrid(nb, (M + kRotTokens - 1) / kRotTokens);
+  {
+  ProfScope ps(OFT_K_ROTATE, st);
+  if (b == 16) rotate_bwd_kernel<16><<<rgrid, kRotThreads, 0, st>>>(dXr, M, K, P, R, dX);
+  if (b == 32) rotate_bwd_kernel<32><<<rgrid, kRotThreads, 0, st>>>(dXr, M, K, P, R, dX);
+  if (b == 64) rotate_bwd_kernel<64><<<rgrid, kRotThreads, 0, st>>>(dXr, M, K, P, R, dX);
+  OFT_LAUNCHED("rotate_bwd_kernel");
+  }
+
+  const int tpp = ((M + L.nparts - 1) / L.nparts + kGTok - 1) / kGTok * kGTok;
+  dim3 ggrid(nb, P, L.nparts);
+  {
+  ProfScope ps(OFT_K_GRAD, st);
+  if (b == 16) rot_grad_partial_kernel<16><<<ggrid, kRotThreads, 0, st>>>(X, dXr, M, K, tpp, Gp);
+  if (b == 32) rot_grad_partial_kernel<32><<<ggrid, kRotThreads, 0, st>>>(X, dXr, M, K, tpp, Gp);
+  if (b == 64) rot_grad_partial_kernel<64><<<ggrid, kRotThreads, 0, st>>>(X, dXr, M, K, tpp, Gp);
+  OFT_LAUNCHED("rot_grad_partial_kernel");
+  }
+
+  const size_t smem = 3 * b * (b + 1) * sizeof(float);
+  const int cgrid = std::min(P * nb, sm_count() * 8);
+  OFT_CUDA(cudaFuncSetAttribute(cayley_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024));
+  ProfScope ps(OFT_K_CAYLEY, st);
+  cayley_bwd_kernel<<<cgrid, kCayleyThreads, smem, st>>>(R, Gp, L.nparts, P * nb, b, dQ);
+  OFT_LAUNCHED("cayley_bwd_kernel");
+  return OFT_OK;
+}
+
+// ---------------------------------------------------------------------------
+// MoE
+// ---------------------------------------------------------------------------
+namespace {
+struct MoeLayout {
+  size_t rex, xg, buf, ytk, inv, pexp, total;
+};
+MoeLayout moe_layout(int T, int E, int top_k, int chunk, int K, int N, int b) {
+  MoeLayout L{};
+  const size_t TK = 1ull * T * top_k;
+  L.rex = 0;
+  L.xg = round_up(L.rex + 4ull * E * 2 * (K / b) * b * b, 256);
+  L.buf = round_up(L.xg + 2ull * 2 * TK * K, 256);
+  L.ytk = round_up(L.buf + 2ull * chunk * N * K, 256);
+  L.inv = round_up(L.ytk + 4ull * TK * N, 256);  // per-slot expert outputs kept in fp32
+  L.pexp = round_up(L.inv + 4ull * TK, 256);
+  L.total = round_up(L.pexp + 4ull * TK, 256);
+  return L;
+}
+}  // namespace
+
+size_t moe_chunked_oft_workspace(int T, int E, int top_k, int chunk, const oft_weight* W, int b) {
+  if (W == nullptr || T <= 0 || E <= 0 || top_k <= 0 || chunk <= 0 || b <= 0) return 0;
+  return moe_layout(T, E, top_k, chunk, W->d_in, W->d_out, b).total;
+}
+
+int moe_chunked_oft_fwd(const uint16_t* X, int T, const float* logits, int E, int top_k, int chunk,
+                        const oft_weight* W, int b, const uint16_t* Q, uint16_t* Y, int32_t* topk_idx, float* topk_w,
+                        int32_t* offsets, int32_t* bucket, int32_t* chunk_table, int32_t* n_active, void* ws,
+                        size_t ws_bytes, void* stream) {
+  if (int rc = check_weight(W, true)) return rc;
+  if (W->fmt != OFT_W_INT4) return fail(OFT_ERR_UNSUPPORTED, "the MoE expert bank must be INT4");
+  const int K = W->d_in, N = W->d_out;
+  if (int rc = check_b(b, K)) return rc;
+  if (T <= 0) return fail(OFT_ERR_INVALID_ARG, "T must be positive");
+  if (E < 1 || E > kMaxExperts || W->n_experts != E)
+    return fail(OFT_ERR_UNSUPPORTED, "E must be 1..%d and match the bank's n_experts", kMaxExperts);
+  if (top_k < 1 || top_k > kMaxTopK || top_k > E) return fail(OFT_ERR_UNSUPPORTED, "top_k must be 1..%d", kMaxTopK);
+  if (chunk < 1 || chunk > gemm::MAX_GROUPS / 2) return fail(OFT_ERR_UNSUPPORTED, "chunk must be 1..%d", gemm::MAX_GROUPS / 2);
+  if (N % 16 != 0) return fail(OFT_ERR_UNSUPPORTED, "expert d_out (gate+up) must be a multiple of 16");
+  if (1ll * T * top_k * 2 > (1ll << 31) - 1) return fail(OFT_ERR_UNSUPPORTED, "too many routed rows");
+  const void* ptrs[] = {X, logits, Q, Y, topk_idx, topk_w, offsets, bucket, chunk_table, n_active, ws};
+  for (const void* q : ptrs)
+    if (q == nullptr || !aligned16(q)) return fail(OFT_ERR_INVALID_ARG, "NULL or misaligned pointer");
+  const int n_proj = N / 2, TK = T * top_k, nb = K / b;
+  const int n_chunks_max = (E + chunk - 1) / chunk;
+  const MoeLayout L = moe_layout(T, E, top_k, chunk, K, N, b);
+  if (ws_bytes < L.total) return fail(OFT_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
+  cudaStream_t st = as_stream(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  float* Rex = reinterpret_cast<float*>(wsb + L.rex);
+  uint16_t* Xg = reinterpret_cast<uint16_t*>(wsb + L.xg);
+  uint16_t* buf = reinterpret_cast<uint16_t*>(wsb + L.buf);
+  float* Ytk = reinterpret_cast<float*>(wsb + L.ytk);
+  int* inv = reinterpret_cast<int*>(wsb + L.inv);
+  int* pexp = reinterpret_cast<int*>(wsb + L.pexp);
+
+  // 1. top-k + gating
+  {
+    ProfScope ps(OFT_K_ROUTE, st);
+    moe_topk_kernel<<<(T * 32 + 255) / 256, 256, 0, st>>>(logits, T, E, top_k, topk_idx, topk_w);
+    OFT_LAUNCHED("moe_topk_kernel");
+  }
+  // 2. buckets, active experts, chunk table
+  const size_t rsmem = sizeof(int) * (32 * E + 2 * E + 1);
+  OFT_CUDA(cudaFuncSetAttribute(moe_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(rsmem)));
+  {
+    ProfScope ps(OFT_K_ROUTE, st);
+    moe_route_kernel<<<1, 1024, rsmem, st>>>(topk_idx, TK, E, chunk, n_chunks_max, offsets, bucket, inv, pexp,
+                                            chunk_table, n_active);
+    OFT_LAUNCHED("moe_route_kernel");
+  }
+  // 3. rotations of the active experts (gate and up)
+  if (int rc = launch_cayley(Q, E * 2 * nb, b, Rex, offsets, 2 * nb, st)) return rc;
+  // 4. rotated gather in bucket order: Xg[proj][pos] = X[t] R_{e,proj}
+  dim3 ggrid(nb, (TK + kRotTokens - 1) / kRotTokens, 2);
+  {
+  ProfScope ps(OFT_K_ROTATE, st);
+  if (b == 16) moe_gather_rotate_kernel<16><<<ggrid, kRotThreads, 0, st>>>(X, K, TK, top_k, bucket, pexp, Rex, Xg);
+  if (b == 32) moe_gather_rotate_kernel<32><<<ggrid, kRotThreads, 0, st>>>(X, K, TK, top_k, bucket, pexp, Rex, Xg);
+  if (b == 64) moe_gather_rotate_kernel<64><<<ggrid, kRotThreads, 0, st>>>(X, K, TK, top_k, bucket, pexp, Rex, Xg);
+  OFT_LAUNCHED("moe_gather_rotate_kernel");
+  }
+  // 5. chunks: transient dequant of the chunk's experts, then one grouped GEMM
+  gemm::Params prm;
+  memset(&prm, 0, sizeof(prm));
+  if (int rc = make_map_bf16(&prm.tmA[0], Xg, K, 2ull * TK, K, gemm::BM)) return rc;
+  if (int rc = make_map_bf16(&prm.tmB[0], buf, K, 1ull * chunk * N, K, gemm::BN)) return rc;
+  for (int i = 1; i < gemm::MAX_MAPS; ++i) {
+    prm.tmA[i] = prm.tmA[0];
+    prm.tmB[i] = prm.tmB[0];
+  }
+  prm.C = Ytk;
+  prm.c_f32 = 1;
+  prm.ldc = N;
+  prm.use_moe = 1;
+  prm.moe.chunk_table = chunk_table;
+  prm.moe.offsets = offsets;
+  prm.moe.chunk = chunk;
+  prm.moe.TK = TK;
+  prm.moe.n_proj = n_proj;
+  prm.moe.K = K;
+  WeightView bank = view_of(W);
+  const long long units = 1ll * N * (K / 8);
+  const int dq_blocks = static_cast<int>(std::min<long long>((units + 255) / 256, std::max(1, sm_count() * 8 / chunk)));
+  for (int c = 0; c < n_chunks_max; ++c) {
+    {
+      ProfScope ps(OFT_K_DEQUANT, st);
+      moe_chunk_dequant_kernel<<<dim3(dq_blocks, chunk), 256, 0, st>>>(bank, chunk_table, c, chunk, buf);
+      OFT_LAUNCHED("moe_chunk_dequant_kernel");
+    }
+    prm.moe.chunk_idx = c;
+    if (int rc = launch_gemm(prm, 0, st)) return rc;
+  }
+  // 6. weighted combine in slot order
+  const long long cunits = 1ll * T * (N / 8);
+  const int cgrid = static_cast<int>(std::min<long long>((cunits + 255) / 256, 148ll * 16));
+  ProfScope ps(OFT_K_ROUTE, st);
+  moe_combine_kernel<<<cgrid, 256, 0, st>>>(Ytk, topk_w, inv, T, N, top_k, Y);
+  OFT_LAUNCHED("moe_combine_kernel");
+  return OFT_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// bounded-wait self test
+// ---------------------------------------------------------------------------
+namespace {
+__global__ void debug_bounded_wait_kernel(unsigned long long timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, kErrWaitDebug, timeout_ns);  // nothing ever arrives
+  __syncthreads();
+}
+}  // namespace
+
+extern "C" int oft_debug_bounded_wait(int timeout_us, void* stream) {
+  if (timeout_us <= 0 || timeout_us > 2000000) return fail(OFT_ERR_INVALID_ARG, "timeout_us must be 1..2000000");
+  debug_bounded_wait_kernel<<<1, 32, 0, as_stream(stream)>>>(1000ull * timeout_us);
+  OFT_LAUNCHED("debug_bounded_wait_kernel");
+  return OFT_OK;
+}
+
+extern "C" int oft_profile_begin(int max_launches) {
+  if (max_launches < 1 || max_launches > (1 << 20)) return fail(OFT_ERR_INVALID_ARG, "max_launches must be 1..2^20");
+  if (g_prof.cap < max_launches) {
+    for (int i = 0; i < 2 * g_prof.cap; ++i) cudaEventDestroy(g_prof.ev[i]);
+    delete[] g_prof.ev;
+    delete[] g_prof.kind;
+    g_prof.ev = new cudaEvent_t[2 * max_launches];
+    g_prof.kind = new int[max_launches];
+    g_prof.cap = 0;
+    for (int i = 0; i < 2 * max_launches; ++i) OFT_CUDA(cudaEventCreate(&g_prof.ev[i]));
+    g_prof.cap = max_launches;
+  }
+  g_prof.n = 0;
+  g_prof.dropped = 0;
+  for (int k = 0; k < OFT_K_NUM; ++k) g_prof.counts[k] = 0;
+  g_prof.on = true;
+  return OFT_OK;
+}
+
+extern "C" int oft_profile_end(double* ms_by_kind, int* launches_by_kind, int n_kinds, int* dropped) {
+  if (!g_prof.on) return fail(OFT_ERR_INVALID_ARG, "profiling was not started");
+  g_prof.on = false;
+  if (n_kinds < 0 || n_kinds > OFT_K_NUM) return fail(OFT_ERR_INVALID_ARG, "n_kinds must be 0..%d", OFT_K_NUM);
+  double ms[OFT_K_NUM] = {0};
+  for (int i = 0; i < g_prof.n; ++i) {
+    OFT_CUDA(cudaEventSynchronize(g_prof.ev[2 * i + 1]));
+    float t = 0.f;
+    OFT_CUDA(cudaEventElapsedTime(&t, g_prof.ev[2 * i], g_prof.ev[2 * i + 1]));
+    ms[g_prof.kind[i]] += t;
+  }
+  for (int k = 0; k < n_kinds; ++k) {
+    if (ms_by_kind) ms_by_kind[k] = ms[k];
+    if (launches_by_kind) launches_by_kind[k] = g_prof.counts[k];
+  }
+  if (dropped) *dropped = g_prof.dropped;
+  return OFT_OK;
+}

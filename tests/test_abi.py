@@ -1,0 +1,120 @@
+"""The C ABI without a GPU: every symbol the header declares is exported, the
+host-side argument checks return the documented codes, and no call that is
+checked here launches a kernel."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "oft.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from orthogonal_fine_tuning_b200 import _lib
+    return _lib.load()
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_]\w*\s*\*?\s+\*?([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_path(lib):
+    names = _declared()
+    for required in ("oft_build_rotation", "oft_linear_fwd", "oft_linear_bwd", "moe_chunked_oft_fwd"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    from orthogonal_fine_tuning_b200 import _lib
+    names = _declared()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) <= set(_lib.EXPORTS)
+
+
+def test_version(lib):
+    assert b"sm_100a" in lib.oft_version()
+
+
+def _w(lib, fmt=1, codes=0x1000, scales=0x2000, d_in=256, d_out=384, group=32, n=0):
+    from orthogonal_fine_tuning_b200 import _lib
+    return _lib.CWeight(fmt, codes, scales, d_in, d_out, group, n)
+
+
+def _s(sizes):
+    from orthogonal_fine_tuning_b200 import _lib
+    s = _lib.CSplit()
+    s.n = len(sizes)
+    for i, v in enumerate(sizes):
+        s.sizes[i] = v
+    return s
+
+
+def _fwd(lib, w, s, b=32, X=0x3000, R=0x4000, Y=0x5000, ws=0x6000, nbytes=1 << 40, M=64):
+    return lib.oft_linear_fwd(X, M, ctypes.byref(w), ctypes.byref(s), b, R, Y, ws, nbytes, None)
+
+
+def test_argument_checks(lib):
+    from orthogonal_fine_tuning_b200 import _lib as L
+    s = _s([128, 128, 128])
+    assert _fwd(lib, _w(lib, codes=0), s) == L.OFT_ERR_INVALID_ARG                  # NULL codes
+    assert _fwd(lib, _w(lib, codes=0x1001), s) == L.OFT_ERR_INVALID_ARG             # misaligned
+    assert _fwd(lib, _w(lib), s, b=48) == L.OFT_ERR_UNSUPPORTED                     # b not supported
+    assert _fwd(lib, _w(lib, d_in=160), s, b=64) == L.OFT_ERR_UNSUPPORTED                # K % b
+    assert _fwd(lib, _w(lib, group=48), s) == L.OFT_ERR_UNSUPPORTED                 # INT4 group
+    assert _fwd(lib, _w(lib, fmt=9), s) == L.OFT_ERR_UNSUPPORTED                    # format
+    assert _fwd(lib, _w(lib, d_in=250), s) == L.OFT_ERR_UNSUPPORTED                 # K % 32
+    assert _fwd(lib, _w(lib), _s([128, 128, 120])) == L.OFT_ERR_INVALID_ARG         # sizes != d_out
+    assert _fwd(lib, _w(lib), _s([128, 128, 124, 4])) == L.OFT_ERR_UNSUPPORTED      # size % 8
+    s5 = _s([128] * 4)
+    s5.n = 5
+    assert _fwd(lib, _w(lib, d_out=640), s5) == L.OFT_ERR_UNSUPPORTED               # > 4 splits
+    assert _fwd(lib, _w(lib), s, X=0) == L.OFT_ERR_INVALID_ARG                      # NULL X
+    assert _fwd(lib, _w(lib), s, Y=0x5008) == L.OFT_ERR_INVALID_ARG                 # misaligned Y
+    assert _fwd(lib, _w(lib), s, nbytes=16) == L.OFT_ERR_WORKSPACE                  # workspace too small
+    assert _fwd(lib, _w(lib), s, M=-1) == L.OFT_ERR_INVALID_ARG
+    assert _fwd(lib, _w(lib), s, M=0) == L.OFT_OK                                   # nothing to do
+    assert lib.oft_last_error() != b""
+
+
+def test_workspace_sizes(lib):
+    w, s = _w(lib, d_in=2560, d_out=6144, group=0, fmt=2), _s([4096, 1024, 1024])
+    fwd = lib.oft_linear_fwd_workspace(4096, ctypes.byref(w), ctypes.byref(s), 32)
+    # rotated activations for 3 sub-projections + one bf16 copy of the weight
+    assert fwd >= 2 * (3 * 4096 * 2560 + 6144 * 2560)
+    bwd = lib.oft_linear_bwd_workspace(4096, ctypes.byref(w), ctypes.byref(s), 32)
+    assert bwd >= 2 * (3 * 4096 * 2560 + 6144 * 2560)
+    assert lib.oft_linear_fwd_workspace(0, ctypes.byref(w), ctypes.byref(s), 32) == 0
+
+
+def test_moe_argument_checks(lib):
+    from orthogonal_fine_tuning_b200 import _lib as L
+    w = _w(lib, d_in=256, d_out=64, group=32, n=16)
+    p = [0x10000 * (i + 1) for i in range(11)]
+
+    def call(E=16, top_k=4, chunk=4, b=32, w=w):
+        args = [p[0], 32, p[1], E, top_k, chunk, ctypes.byref(w), b, p[2], p[3], p[4], p[5], p[6], p[7], p[8],
+                p[9], p[10], 1 << 40, None]
+        return lib.moe_chunked_oft_fwd(*args)
+
+    assert call(E=600, w=_w(lib, d_in=256, d_out=64, n=600)) == L.OFT_ERR_UNSUPPORTED
+    assert call(top_k=9) == L.OFT_ERR_UNSUPPORTED
+    assert call(chunk=17) == L.OFT_ERR_UNSUPPORTED
+    assert call(E=8) == L.OFT_ERR_UNSUPPORTED                       # bank size mismatch
+    assert call(w=_w(lib, fmt=2, d_in=256, d_out=64, n=16)) == L.OFT_ERR_UNSUPPORTED
+
+
+def test_rotation_and_debug_checks(lib):
+    from orthogonal_fine_tuning_b200 import _lib as L
+    assert lib.oft_build_rotation(0x1000, 4, 24, 0x2000, None) == L.OFT_ERR_UNSUPPORTED
+    assert lib.oft_build_rotation(0, 4, 32, 0x2000, None) == L.OFT_ERR_INVALID_ARG
+    assert lib.oft_build_rotation(0x1000, 0, 32, 0x2000, None) == L.OFT_OK
+    assert lib.oft_debug_bounded_wait(0, None) == L.OFT_ERR_INVALID_ARG

@@ -171,6 +171,31 @@ int oft_cayley_backward(const float* R, const float* G, int n_blocks, int b, flo
  * word.  Exercises the timeout path without faulting or hanging the GPU. */
 int oft_debug_bounded_wait(int timeout_us, void* stream);
 
+/* ---- forward without a caller workspace ----
+ * The pages have no counterpart to this entry point; it exists for callers that
+ * cannot allocate device memory or pass a workspace: for example a runtime
+ * whose memory pool already owns all free HBM (a serving engine that reserves
+ * the card for its KV cache, where cudaMalloc would fail), or a plugin
+ * interface whose signature carries only inputs and outputs.
+ *
+ * Same result as oft_linear_fwd (same kernels, same launch sequence), but the
+ * scratch (rotated activations and the bf16 copy of the weight) lives in a
+ * fixed file-scope device array of OFT_NOALLOC_SCRATCH_BYTES (32 MiB) that every
+ * GPU loading this library holds until the process exits.  Allocates nothing:
+ * no cudaMalloc/cudaFree and no allocating library call.
+ *   - Shapes whose oft_linear_fwd_workspace() exceeds OFT_NOALLOC_SCRATCH_BYTES
+ *     are rejected with OFT_ERR_WORKSPACE and a message giving both sizes.
+ *   - The first call on a device (with that device current) looks up the
+ *     array's device address; make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents.
+ *     Every scratch byte a call reads is written earlier in the same call, so
+ *     nothing needs clearing, but calls whose kernels overlap on the GPU (two
+ *     streams, or two host threads) race on the array: serialise them. */
+#define OFT_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+int oft_linear_fwd_noalloc(const uint16_t* X, int M, const oft_weight* W, const oft_split* S, int b,
+                           const float* R, uint16_t* Y, void* stream);
+
 /* ---- profiling hooks (measurement plumbing, not part of the method) ---- */
 
 /* Kernel classes reported by oft_profile_end(). */

@@ -17,6 +17,7 @@ from .binding import (  # noqa: F401
     oft_linear_bwd,
     oft_linear_bwd_workspace,
     oft_linear_fwd,
+    oft_linear_fwd_noalloc,
     oft_linear_fwd_workspace,
     oft_rotate,
     profile,

@@ -18,11 +18,14 @@ OFT_W_INT4 = 1
 OFT_W_FP8 = 2
 OFT_W_MXFP4 = 3
 
+OFT_NOALLOC_SCRATCH_BYTES = 32 << 20
+
 EXPORTS = (
     "oft_version", "oft_last_error", "oft_check_device", "oft_build_rotation",
     "oft_linear_fwd_workspace", "oft_linear_fwd", "oft_linear_bwd_workspace", "oft_linear_bwd",
     "moe_chunked_oft_workspace", "moe_chunked_oft_fwd", "oft_dequant_weight", "oft_rotate",
     "oft_cayley_backward", "oft_debug_bounded_wait", "oft_profile_begin", "oft_profile_end",
+    "oft_linear_fwd_noalloc",
 )
 
 
@@ -57,6 +60,7 @@ _SIGS = {
     "oft_rotate": (_I, [_P, _I, _I, _I, _I, _P, _P, _P]),
     "oft_cayley_backward": (_I, [_P, _P, _I, _I, _P, _P]),
     "oft_debug_bounded_wait": (_I, [_I, _P]),
+    "oft_linear_fwd_noalloc": (_I, [_P, _I, _WP, _SP, _I, _P, _P, _P]),
     "oft_profile_begin": (_I, [_I]),
     "oft_profile_end": (_I, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int), _I,
                             ctypes.POINTER(ctypes.c_int)]),

@@ -106,6 +106,17 @@ def oft_linear_fwd_workspace(M: int, W: Weight, splits: Sequence[int], b: int) -
     return int(_L.oft_linear_fwd_workspace(M, ctypes.byref(cw), ctypes.byref(cs), b))
 
 
+def oft_linear_fwd_noalloc(X: torch.Tensor, W: Weight, splits: Sequence[int], b: int, R: torch.Tensor,
+                           Y: torch.Tensor, stream=None) -> torch.Tensor:
+    """oft_linear_fwd without a workspace: scratch lives in the library's fixed
+    device array (OFT_NOALLOC_SCRATCH_BYTES).  Y must be preallocated; nothing
+    is allocated by this call."""
+    cw, cs = W.c(), _split(splits)
+    _check(_L.oft_linear_fwd_noalloc(_ptr(_bits(X)), X.shape[0], ctypes.byref(cw), ctypes.byref(cs), b, _ptr(R),
+                                     _ptr(Y), _stream(stream)))
+    return Y
+
+
 def oft_linear_bwd_workspace(M: int, W: Weight, splits: Sequence[int], b: int) -> int:
     cw, cs = W.c(), _split(splits)
     return int(_L.oft_linear_bwd_workspace(M, ctypes.byref(cw), ctypes.byref(cs), b))

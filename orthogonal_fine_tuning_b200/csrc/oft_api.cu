@@ -7,6 +7,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include "oft.h"
@@ -664,4 +665,50 @@ extern "C" int oft_profile_end(double* ms_by_kind, int* launches_by_kind, int n_
   }
   if (dropped) *dropped = g_prof.dropped;
   return OFT_OK;
+}
+
+// ---------------------------------------------------------------------------
+// forward without a caller workspace: the scratch is a fixed device array
+// ---------------------------------------------------------------------------
+namespace {
+// Scratch of oft_linear_fwd_noalloc.  A __device__ symbol: in host code its
+// name is only a host-side stand-in, so the kernels get the device address that
+// cudaGetSymbolAddress returns for the current device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[OFT_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {nullptr};
+
+// Once per device, with that device current: look up the array's device address.
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  OFT_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(OFT_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    OFT_CUDA(cudaGetSymbolAddress(&ptr, g_noalloc_scratch));
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return OFT_OK;
+}
+}  // namespace
+
+extern "C" int oft_linear_fwd_noalloc(const uint16_t* X, int M, const oft_weight* W, const oft_split* S, int b,
+                                      const float* R, uint16_t* Y, void* stream) {
+  if (int rc = check_weight(W, false)) return rc;
+  if (int rc = check_split(S, W->d_out)) return rc;
+  if (int rc = check_b(b, W->d_in)) return rc;
+  if (M < 0) return fail(OFT_ERR_INVALID_ARG, "M < 0");
+  if (M == 0) return OFT_OK;
+  const size_t need = oft_linear_fwd_workspace(M, W, S, b);
+  if (need > OFT_NOALLOC_SCRATCH_BYTES)
+    return fail(OFT_ERR_WORKSPACE,
+                "oft_linear_fwd_noalloc: this shape needs %zu bytes of scratch, more than the fixed %u-byte "
+                "array; use oft_linear_fwd with a caller workspace",
+                need, (unsigned)OFT_NOALLOC_SCRATCH_BYTES);
+  void* scratch = nullptr;
+  if (int rc = noalloc_scratch(&scratch)) return rc;
+  return oft_linear_fwd(X, M, W, S, b, R, Y, scratch, OFT_NOALLOC_SCRATCH_BYTES, stream);
 }

@@ -77,19 +77,6 @@ __device__ __forceinline__ void decode_tile(const Group* sg, int ng, int t, int&
   nt = rem / rows;
 }
 
-// Waits for a phase ignoring the abort flag (teardown drain); bounded.
-__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
-  const uint32_t a = smem_u32(bar);
-  const unsigned long long t0 = globaltimer_ns();
-  while (!mbar_try_wait(a, parity)) {
-    if (globaltimer_ns() - t0 > 200000000ull) {
-      atomicOr(&g_dev_err, kErrWaitDrain);
-      return false;
-    }
-  }
-  return true;
-}
-
 __device__ __forceinline__ uint32_t pack2(uint32_t lo, uint32_t hi) {
   return pack_bf16x2(__uint_as_float(lo), __uint_as_float(hi));
 }
@@ -208,7 +195,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_bf16_kernel(const __grid_
       }
       if (*abort_flag) {  // let the copies already in flight land before the CTA exits
         for (long long i = (issued > STAGES ? issued - STAGES : 0); i < issued; ++i)
-          mbar_wait_drain(&full[i % STAGES], static_cast<uint32_t>((i / STAGES) & 1));
+          gemm_drain_wait(&full[i % STAGES], static_cast<uint32_t>((i / STAGES) & 1));
       }
     }
   } else if (warp == 1) {
@@ -251,7 +238,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_bf16_kernel(const __grid_
       }
       // all MMAs issued by this thread have completed once `drain` flips
       mma_commit(drain);
-      mbar_wait_drain(drain, 0);
+      gemm_drain_wait(drain, 0);
     }
   } else {
     const int q = warp & 3;  // TMEM lane quarter this warp may access

@@ -18,6 +18,7 @@
 #include "rotate.cuh"
 #include "gemm.cuh"
 #include "moe.cuh"
+#include "rot_tc.cuh"
 
 using namespace oftk;
 
@@ -123,6 +124,23 @@ int make_map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t out
   return OFT_OK;
 }
 
+// 3-D fp32 tensor [P][M][K] (dX'), box {32, 128, 1}; rows past M read as zero.  `swizzle` is the
+// 128B swizzle (K-major operands) or its 32-byte-atom variant (MN-major tf32 operands).
+int make_map_f32_3d(CUtensorMap* m, const void* base, uint64_t K, uint64_t M, uint64_t P,
+                    CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return fail(OFT_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[3] = {K, M, P};
+  cuuint64_t strides[2] = {K * 4, M * K * 4};
+  cuuint32_t box[3] = {32, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(OFT_ERR_CUDA, "cuTensorMapEncodeTiled (fp32 3-D) failed (%d)", int(r));
+  return OFT_OK;
+}
+
 // ---- argument checks ----
 int check_weight(const oft_weight* W, bool bank_ok) {
   if (W == nullptr) return fail(OFT_ERR_INVALID_ARG, "weight descriptor is NULL");
@@ -214,13 +232,89 @@ int launch_cayley(const uint16_t* Q, int nblocks, int b, float* R, const int* of
   return OFT_OK;
 }
 
+template <typename KernelT>
+int set_smem(KernelT kernel, size_t bytes) {
+  OFT_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)));
+  return OFT_OK;
+}
+
+// X'_p = X R_p on the tensor cores (all P sub-projections in one pass).
 int launch_rotate_fwd(const uint16_t* X, int M, int K, int P, int b, const float* R, uint16_t* Xr, cudaStream_t st) {
-  dim3 grid(K / b, (M + kRotTokens - 1) / kRotTokens);
+  rtc::FwdParams prm;
+  memset(&prm, 0, sizeof(prm));
+  if (int rc = make_map_bf16(&prm.tmX, X, K, M, K, rtc::TM)) return rc;
+  prm.R = R;
+  prm.Xr = Xr;
+  prm.M = M;
+  prm.K = K;
+  prm.P = P;
+  prm.b = b;
+  prm.nb = K / b;
+  prm.groups = (K + 63) / 64;
+  prm.tiles_m = (M + rtc::TM - 1) / rtc::TM;
+  if (int rc = set_smem(rtc::rot_fwd_tc_kernel, rtc::kFwdSmem)) return rc;
+  const int grid = std::min(sm_count(), prm.groups * prm.tiles_m);
   ProfScope ps(OFT_K_ROTATE, st);
-  if (b == 16) rotate_fwd_kernel<16><<<grid, kRotThreads, 0, st>>>(X, M, K, P, R, Xr);
-  if (b == 32) rotate_fwd_kernel<32><<<grid, kRotThreads, 0, st>>>(X, M, K, P, R, Xr);
-  if (b == 64) rotate_fwd_kernel<64><<<grid, kRotThreads, 0, st>>>(X, M, K, P, R, Xr);
-  OFT_LAUNCHED("rotate_fwd_kernel");
+  rtc::rot_fwd_tc_kernel<<<grid, rtc::NUM_THREADS, rtc::kFwdSmem, st>>>(prm);
+  OFT_LAUNCHED("rot_fwd_tc_kernel");
+  return OFT_OK;
+}
+
+// dX = sum_p dX'_p R_p^T on the tensor cores (tf32).
+int launch_rotate_bwd(const float* dXr, int M, int K, int P, int b, const float* R, uint16_t* dX, cudaStream_t st) {
+  rtc::BwdParams prm;
+  memset(&prm, 0, sizeof(prm));
+  if (int rc = make_map_f32_3d(&prm.tmD, dXr, K, M, P)) return rc;
+  prm.R = R;
+  prm.dX = dX;
+  prm.M = M;
+  prm.K = K;
+  prm.P = P;
+  prm.b = b;
+  prm.nb = K / b;
+  prm.groups = (K + 63) / 64;
+  prm.tiles_m = (M + rtc::TM - 1) / rtc::TM;
+  if (int rc = set_smem(rtc::rot_bwd_tc_kernel, rtc::kBwdSmem)) return rc;
+  const int grid = std::min(sm_count(), prm.groups * prm.tiles_m);
+  ProfScope ps(OFT_K_ROTATE, st);
+  rtc::rot_bwd_tc_kernel<<<grid, rtc::NUM_THREADS, rtc::kBwdSmem, st>>>(prm);
+  OFT_LAUNCHED("rot_bwd_tc_kernel");
+  return OFT_OK;
+}
+
+// Token chunking of the dR reduction (deterministic in the shape): about one
+// (128-column group, chunk) unit per SM of a 148-SM part.
+struct GradChunks {
+  int chunks, tiles_per_chunk;
+};
+GradChunks grad_chunks(int M, int K) {
+  const int groups = (K + 127) / 128, tiles_m = (M + 127) / 128;
+  const int want = std::max(1, std::min(tiles_m, 148 / groups));
+  const int tpc = (tiles_m + want - 1) / want;
+  return GradChunks{(tiles_m + tpc - 1) / tpc, tpc};
+}
+
+int launch_grad(const uint16_t* X, const float* dXr, int M, int K, int P, int b, float* Gp, cudaStream_t st) {
+  rtc::GradParams prm;
+  memset(&prm, 0, sizeof(prm));
+  if (int rc = make_map_f32_3d(&prm.tmD, dXr, K, M, P, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B)) return rc;
+  const GradChunks gc = grad_chunks(M, K);
+  prm.X = X;
+  prm.Gp = Gp;
+  prm.M = M;
+  prm.K = K;
+  prm.P = P;
+  prm.b = b;
+  prm.nb = K / b;
+  prm.groups = (K + 127) / 128;
+  prm.chunks = gc.chunks;
+  prm.tiles_per_chunk = gc.tiles_per_chunk;
+  prm.tiles_m = (M + rtc::TM - 1) / rtc::TM;
+  if (int rc = set_smem(rtc::grad_tc_kernel, rtc::kGradSmem)) return rc;
+  const int grid = std::min(sm_count(), prm.groups * prm.chunks);
+  ProfScope ps(OFT_K_GRAD, st);
+  rtc::grad_tc_kernel<<<grid, rtc::NUM_THREADS, rtc::kGradSmem, st>>>(prm);
+  OFT_LAUNCHED("grad_tc_kernel");
   return OFT_OK;
 }
 
@@ -243,13 +337,6 @@ int launch_gemm(const gemm::Params& prm, int total_tiles_hint, cudaStream_t st) 
 
 int tiles_of(int m, int n) { return ((m + gemm::BM - 1) / gemm::BM) * ((n + gemm::BN - 1) / gemm::BN); }
 
-// number of token partitions for the dR reduction (deterministic in the shape)
-int grad_parts(int M, int P, int nb) {
-  const int want = (600 + P * nb - 1) / (P * nb);
-  const int maxp = (M + kGTok - 1) / kGTok;
-  return std::max(1, std::min(want, maxp));
-}
-
 struct FwdLayout {
   size_t xr, wdq, total;
 };
@@ -267,7 +354,7 @@ struct BwdLayout {
 };
 BwdLayout bwd_layout(int M, int K, int N, int P, int b) {
   BwdLayout L{};
-  L.nparts = grad_parts(M, P, K / b);
+  L.nparts = grad_chunks(M, K).chunks;
   L.dxr = 0;
   L.wdqt = round_up(L.dxr + 4ull * P * M * K, 256);  // dX' kept in fp32
   L.gpart = round_up(L.wdqt + 2ull * N * K, 256);
@@ -326,11 +413,12 @@ int oft_dequant_weight(const oft_weight* W, uint16_t* out, int transpose, void* 
 
 int oft_rotate(const uint16_t* X, int M, int K, int P, int b, const float* R, uint16_t* Xr, void* stream) {
   if (M < 0 || K <= 0 || P < 1) return fail(OFT_ERR_INVALID_ARG, "bad sizes");
+  if (P > 4) return fail(OFT_ERR_UNSUPPORTED, "1..4 sub-projections supported (got %d)", P);
   if (M == 0) return OFT_OK;
   if (!X || !R || !Xr || !aligned16(X) || !aligned16(R) || !aligned16(Xr))
     return fail(OFT_ERR_INVALID_ARG, "NULL or misaligned pointer");
   if (int rc = check_b(b, K)) return rc;
-  if (K % 8 != 0) return fail(OFT_ERR_UNSUPPORTED, "K must be a multiple of 8");
+  if (K % 32 != 0) return fail(OFT_ERR_UNSUPPORTED, "K must be a multiple of 32");
   return launch_rotate_fwd(X, M, K, P, b, R, Xr, as_stream(stream));
 }
 
@@ -451,24 +539,8 @@ int oft_linear_bwd(const uint16_t* dY, const uint16_t* X, int M, const oft_weigh
   prm.num_groups = P;
   if (int rc = launch_gemm(prm, tiles, st)) return rc;
 
-  dim3 rgrid(nb, (M + kRotTokens - 1) / kRotTokens);
-  {
-  ProfScope ps(OFT_K_ROTATE, st);
-  if (b == 16) rotate_bwd_kernel<16><<<rgrid, kRotThreads, 0, st>>>(dXr, M, K, P, R, dX);
-  if (b == 32) rotate_bwd_kernel<32><<<rgrid, kRotThreads, 0, st>>>(dXr, M, K, P, R, dX);
-  if (b == 64) rotate_bwd_kernel<64><<<rgrid, kRotThreads, 0, st>>>(dXr, M, K, P, R, dX);
-  OFT_LAUNCHED("rotate_bwd_kernel");
-  }
-
-  const int tpp = ((M + L.nparts - 1) / L.nparts + kGTok - 1) / kGTok * kGTok;
-  dim3 ggrid(nb, P, L.nparts);
-  {
-  ProfScope ps(OFT_K_GRAD, st);
-  if (b == 16) rot_grad_partial_kernel<16><<<ggrid, kRotThreads, 0, st>>>(X, dXr, M, K, tpp, Gp);
-  if (b == 32) rot_grad_partial_kernel<32><<<ggrid, kRotThreads, 0, st>>>(X, dXr, M, K, tpp, Gp);
-  if (b == 64) rot_grad_partial_kernel<64><<<ggrid, kRotThreads, 0, st>>>(X, dXr, M, K, tpp, Gp);
-  OFT_LAUNCHED("rot_grad_partial_kernel");
-  }
+  if (int rc = launch_rotate_bwd(dXr, M, K, P, b, R, dX, st)) return rc;
+  if (int rc = launch_grad(X, dXr, M, K, P, b, Gp, st)) return rc;
 
   const size_t smem = 3 * b * (b + 1) * sizeof(float);
   const int cgrid = std::min(P * nb, sm_count() * 8);

@@ -1,13 +1,13 @@
-// Cayley map of the OFT adapter and its backward, one CTA per b x b block.
+// Cayley map of the OFT adapter and its backward.
 //
 // OFT parameterises each block of the orthogonal rotation by a skew-symmetric Q
 // (the pages name OFT as Orbit's default adapter: chooseai.io news 4086, section
 // "技术原理：低精度基座 + BF16 适配器 + OFT"):
 //     R = (I + Q)(I - Q)^-1 = (I - Q)^-1 (I + Q)
-// Forward: solve (I - Q) R = (I + Q) by Gauss-Jordan elimination in shared
-// memory, fp32, without pivoting.  I - Q has symmetric part I, so x^T (I-Q) x =
-// |x|^2 > 0: every leading minor is non-zero, every pivot stays >= 1 in exact
-// arithmetic, and sigma_min(I - Q) >= 1 (the solve is well conditioned for any Q).
+// Forward: solve (I - Q) R = (I + Q) by Gauss-Jordan elimination in fp32
+// without pivoting.  I - Q has symmetric part I, so x^T (I-Q) x = |x|^2 > 0:
+// every leading minor is non-zero, every pivot stays >= 1 in exact arithmetic,
+// and sigma_min(I - Q) >= 1 (the solve is well conditioned for any Q).
 // Backward: with G = dL/dR, dL/dQ = 1/2 (I + R)^T G (I + R)^T, projected onto the
 // packed strict-upper parameters as dq_ij = D_ij - D_ji.
 #pragma once
@@ -18,104 +18,204 @@ namespace oftk {
 
 constexpr int kCayleyThreads = 256;
 
-__device__ __forceinline__ int tri_index(int i, int j, int b) {  // i < j, row-major strict upper
+__host__ __device__ __forceinline__ int tri_index(int i, int j, int b) {  // i < j, row-major strict upper
   return i * b - i * (i + 1) / 2 + (j - i - 1);
 }
 
-// Q: bf16 [nblocks][b(b-1)/2]; R: fp32 [nblocks][b][b].
-// Optional MoE filter: when `counts` is given, block `blk` belongs to expert
-// blk / blocks_per_expert and is skipped when that expert has no tokens.
-__global__ void __launch_bounds__(kCayleyThreads) cayley_fwd_kernel(const uint16_t* __restrict__ Q, int nblocks, int b,
-                                                                    float* __restrict__ R, const int* __restrict__ offsets,
-                                                                    int blocks_per_expert) {
-  extern __shared__ float sm[];
-  const int ld = b + 1;
-  float* A = sm;               // I - Q, reduced to I
-  float* B = sm + b * ld;      // I + Q, becomes R
-  float* f = sm + 2 * b * ld;  // elimination factors of the current pivot column
-  const int tid = threadIdx.x;
-  for (int blk = blockIdx.x; blk < nblocks; blk += gridDim.x) {
-    if (offsets != nullptr) {
-      const int e = blk / blocks_per_expert;
-      if (offsets[e + 1] == offsets[e]) continue;
+// Forward, one thread per matrix row: thread r keeps row r of A = I - Q and of
+// the right-hand side I + Q in registers.  A is held as a sliding window of its
+// not-yet-eliminated columns (a[k] = A[r][c + k] at pivot c): after pivot c,
+// column c of A is a unit column and is dropped by shifting the window, so the
+// pivot element is always a[0] and every register index is static while the
+// pivot loop itself stays rolled (small code).  Each pivot row is broadcast
+// through shared memory.  CTAs are one warp (B = 16: two blocks; B = 32: one)
+// or two warps (B = 64, synchronised with a named barrier), so the serial pivot
+// chains of different blocks spread over every SM.
+// Q: bf16 [nblocks][B(B-1)/2]; R: fp32 [nblocks][B][B].  Optional MoE filter:
+// block `blk` belongs to expert blk / blocks_per_expert and is skipped when that
+// expert has no tokens (offsets[e+1] == offsets[e]).
+template <int B>
+struct CayleyFwdCfg {
+  static constexpr int THREADS = B < 32 ? 32 : B;
+  static constexpr int BPC = THREADS / B;  // blocks per CTA
+};
+
+template <int B>
+__global__ void __launch_bounds__(CayleyFwdCfg<B>::THREADS) cayley_fwd_kernel(const uint16_t* __restrict__ Q,
+                                                                               int nblocks, float* __restrict__ R,
+                                                                               const int* __restrict__ offsets,
+                                                                               int blocks_per_expert) {
+  constexpr int BPC = CayleyFwdCfg<B>::BPC;
+  __shared__ __align__(16) float piv[BPC][2 * B];
+  const int sub = threadIdx.x / B, r = threadIdx.x % B;
+  const int blk = blockIdx.x * BPC + sub;
+  bool active = blk < nblocks;
+  if (active && offsets != nullptr) {
+    const int e = blk / blocks_per_expert;
+    active = offsets[e + 1] > offsets[e];
+  }
+  auto block_sync = [&]() {
+    if constexpr (B <= 32) {
+      __syncwarp();
+    } else {
+      __syncthreads();  // one block per CTA
     }
-    const uint16_t* q = Q + static_cast<size_t>(blk) * (b * (b - 1) / 2);
-    for (int idx = tid; idx < b * b; idx += kCayleyThreads) {
-      const int i = idx / b, j = idx % b;
-      float v = 0.f;
-      if (i < j) v = bf16_bits_to_f32(q[tri_index(i, j, b)]);
-      else if (i > j) v = -bf16_bits_to_f32(q[tri_index(j, i, b)]);
-      const float d = (i == j) ? 1.f : 0.f;
-      A[i * ld + j] = d - v;
-      B[i * ld + j] = d + v;
+  };
+
+  float a[B], rhs[B];
+  const uint16_t* q = Q + static_cast<size_t>(active ? blk : 0) * (B * (B - 1) / 2);
+#pragma unroll
+  for (int j = 0; j < B; ++j) {
+    float v = 0.f;
+    if (active && j != r) {
+      const float t = bf16_bits_to_f32(q[j > r ? tri_index(r, j, B) : tri_index(j, r, B)]);
+      v = j > r ? t : -t;  // Q[r][j]
     }
-    __syncthreads();
-    for (int c = 0; c < b; ++c) {
-      const float inv = 1.0f / A[c * ld + c];
-      __syncthreads();
-      for (int j = tid; j < b; j += kCayleyThreads) {
-        A[c * ld + j] *= inv;
-        B[c * ld + j] *= inv;
+    const float d = (j == r) ? 1.f : 0.f;
+    a[j] = d - v;
+    rhs[j] = d + v;
+  }
+
+#pragma unroll 1
+  for (int c = 0; c < B; ++c) {
+    if (r == c) {
+      const float inv = 1.0f / a[0];
+#pragma unroll
+      for (int k = 0; k < B; ++k) {
+        a[k] *= inv;
+        rhs[k] *= inv;
       }
-      for (int r = tid; r < b; r += kCayleyThreads) f[r] = (r == c) ? 0.f : A[r * ld + c];
-      __syncthreads();
-      for (int idx = tid; idx < b * b; idx += kCayleyThreads) {
-        const int r = idx / b, j = idx % b;
-        const float fr = f[r];
-        if (fr != 0.f) {
-          A[r * ld + j] -= fr * A[c * ld + j];
-          B[r * ld + j] -= fr * B[c * ld + j];
-        }
+#pragma unroll
+      for (int k = 0; k < B; k += 4) {
+        *reinterpret_cast<float4*>(&piv[sub][k]) = make_float4(a[k], a[k + 1], a[k + 2], a[k + 3]);
+        *reinterpret_cast<float4*>(&piv[sub][B + k]) = make_float4(rhs[k], rhs[k + 1], rhs[k + 2], rhs[k + 3]);
       }
-      __syncthreads();
     }
-    float* out = R + static_cast<size_t>(blk) * b * b;
-    for (int idx = tid; idx < b * b; idx += kCayleyThreads) out[idx] = B[(idx / b) * ld + idx % b];
-    __syncthreads();
+    block_sync();
+    const float f = (r == c) ? 0.f : a[0];
+#pragma unroll
+    for (int k = 0; k < B; k += 4) {
+      const float4 pa = *reinterpret_cast<const float4*>(&piv[sub][k]);
+      const float4 pr = *reinterpret_cast<const float4*>(&piv[sub][B + k]);
+      a[k] = fmaf(-f, pa.x, a[k]);
+      a[k + 1] = fmaf(-f, pa.y, a[k + 1]);
+      a[k + 2] = fmaf(-f, pa.z, a[k + 2]);
+      a[k + 3] = fmaf(-f, pa.w, a[k + 3]);
+      rhs[k] = fmaf(-f, pr.x, rhs[k]);
+      rhs[k + 1] = fmaf(-f, pr.y, rhs[k + 1]);
+      rhs[k + 2] = fmaf(-f, pr.z, rhs[k + 2]);
+      rhs[k + 3] = fmaf(-f, pr.w, rhs[k + 3]);
+    }
+    // drop the eliminated column c: the window moves one column right
+#pragma unroll
+    for (int k = 0; k < B - 1; ++k) a[k] = a[k + 1];
+    a[B - 1] = 0.f;
+    block_sync();
+  }
+  if (active) {
+    float* out = R + (static_cast<size_t>(blk) * B + r) * B;
+#pragma unroll
+    for (int j = 0; j < B; j += 4)
+      *reinterpret_cast<float4*>(out + j) = make_float4(rhs[j], rhs[j + 1], rhs[j + 2], rhs[j + 3]);
   }
 }
 
 // dQ[blk] = pack(D - D^T), D = 1/2 (I+R)^T G (I+R)^T.
-// G is read either directly ([nblocks][b][b]) or as `nparts` partial sums laid
-// out [nblocks][nparts][b][b], summed in part order (deterministic).
+// G is read either directly ([nblocks][b][b], nparts = 1) or as `nparts` partial
+// sums laid out [nblocks][nparts][b][b], summed in part order (deterministic).
+// One CTA per block; each thread owns a TI x TI tile of the two b x b products.
+// Dynamic shared memory: 3 * B * (B + 1) floats.
+template <int B>
 __global__ void __launch_bounds__(kCayleyThreads) cayley_bwd_kernel(const float* __restrict__ R,
                                                                     const float* __restrict__ G, int nparts,
-                                                                    int nblocks, int b, float* __restrict__ dQ) {
-  extern __shared__ float sm[];
-  const int ld = b + 1;
-  float* T = sm;               // (I + R)^T, stored as T[i][j] = (I+R)[j][i]
-  float* Gs = sm + b * ld;     // G
-  float* U = sm + 2 * b * ld;  // T G, then D
+                                                                    int nblocks, float* __restrict__ dQ) {
+  constexpr int TI = (B == 64) ? 4 : (B == 32 ? 2 : 1);
+  constexpr int NT = B / TI;  // threads per output row of tiles
+  static_assert(NT * NT == kCayleyThreads, "tile grid must cover the CTA");
+  constexpr int LD = B + 1;
+  extern __shared__ float csm[];
+  float* T = csm;               // (I + R)^T
+  float* Gs = csm + B * LD;     // G, then D * 2
+  float* U = csm + 2 * B * LD;  // T G
   const int tid = threadIdx.x;
+  const int ti = (tid / NT) * TI, tj = (tid % NT) * TI;
   for (int blk = blockIdx.x; blk < nblocks; blk += gridDim.x) {
-    const float* r = R + static_cast<size_t>(blk) * b * b;
-    for (int idx = tid; idx < b * b; idx += kCayleyThreads) {
-      const int i = idx / b, j = idx % b;
-      T[j * ld + i] = r[idx] + (i == j ? 1.f : 0.f);
-      const float* g = G + static_cast<size_t>(blk) * nparts * b * b + idx;
-      float acc = 0.f;
-      for (int p = 0; p < nparts; ++p) acc += g[static_cast<size_t>(p) * b * b];
-      Gs[i * ld + j] = acc;
+    const float* rb = R + static_cast<size_t>(blk) * B * B;
+    const float* gb = G + static_cast<size_t>(blk) * nparts * B * B;
+    constexpr int EPT = B * B / kCayleyThreads;  // elements per thread
+    float acc[EPT], rv[EPT];
+#pragma unroll
+    for (int k = 0; k < EPT; ++k) {
+      rv[k] = rb[tid + k * kCayleyThreads];
+      acc[k] = 0.f;
+    }
+    for (int p = 0; p < nparts; p += 4) {  // 4 * EPT independent loads in flight, summed in part order
+      float t[4][EPT];
+#pragma unroll
+      for (int pp = 0; pp < 4; ++pp)
+#pragma unroll
+        for (int k = 0; k < EPT; ++k)
+          t[pp][k] = (p + pp < nparts) ? gb[static_cast<size_t>(p + pp) * B * B + tid + k * kCayleyThreads] : 0.f;
+#pragma unroll
+      for (int pp = 0; pp < 4; ++pp)
+#pragma unroll
+        for (int k = 0; k < EPT; ++k) acc[k] += t[pp][k];
+    }
+#pragma unroll
+    for (int k = 0; k < EPT; ++k) {
+      const int idx = tid + k * kCayleyThreads;
+      const int i = idx / B, j = idx % B;
+      T[j * LD + i] = rv[k] + (i == j ? 1.f : 0.f);
+      Gs[i * LD + j] = acc[k];
     }
     __syncthreads();
-    for (int idx = tid; idx < b * b; idx += kCayleyThreads) {  // U = T G
-      const int i = idx / b, j = idx % b;
-      float acc = 0.f;
-      for (int l = 0; l < b; ++l) acc = fmaf(T[i * ld + l], Gs[l * ld + j], acc);
-      U[i * ld + j] = acc;
+    float o[TI][TI];
+#pragma unroll
+    for (int x = 0; x < TI; ++x)
+#pragma unroll
+      for (int y = 0; y < TI; ++y) o[x][y] = 0.f;
+#pragma unroll 4
+    for (int l = 0; l < B; ++l) {  // U = T G
+      float tv[TI], gv[TI];
+#pragma unroll
+      for (int x = 0; x < TI; ++x) tv[x] = T[(ti + x) * LD + l];
+#pragma unroll
+      for (int y = 0; y < TI; ++y) gv[y] = Gs[l * LD + tj + y];
+#pragma unroll
+      for (int x = 0; x < TI; ++x)
+#pragma unroll
+        for (int y = 0; y < TI; ++y) o[x][y] = fmaf(tv[x], gv[y], o[x][y]);
     }
+#pragma unroll
+    for (int x = 0; x < TI; ++x)
+#pragma unroll
+      for (int y = 0; y < TI; ++y) U[(ti + x) * LD + tj + y] = o[x][y];
     __syncthreads();
-    for (int idx = tid; idx < b * b; idx += kCayleyThreads) {  // Gs = U T = D * 2
-      const int i = idx / b, j = idx % b;
-      float acc = 0.f;
-      for (int l = 0; l < b; ++l) acc = fmaf(U[i * ld + l], T[l * ld + j], acc);
-      Gs[i * ld + j] = acc;
+#pragma unroll
+    for (int x = 0; x < TI; ++x)
+#pragma unroll
+      for (int y = 0; y < TI; ++y) o[x][y] = 0.f;
+#pragma unroll 4
+    for (int l = 0; l < B; ++l) {  // 2D = U T
+      float uv[TI], tv[TI];
+#pragma unroll
+      for (int x = 0; x < TI; ++x) uv[x] = U[(ti + x) * LD + l];
+#pragma unroll
+      for (int y = 0; y < TI; ++y) tv[y] = T[l * LD + tj + y];
+#pragma unroll
+      for (int x = 0; x < TI; ++x)
+#pragma unroll
+        for (int y = 0; y < TI; ++y) o[x][y] = fmaf(uv[x], tv[y], o[x][y]);
     }
+#pragma unroll
+    for (int x = 0; x < TI; ++x)
+#pragma unroll
+      for (int y = 0; y < TI; ++y) Gs[(ti + x) * LD + tj + y] = o[x][y];
     __syncthreads();
-    float* out = dQ + static_cast<size_t>(blk) * (b * (b - 1) / 2);
-    for (int idx = tid; idx < b * b; idx += kCayleyThreads) {
-      const int i = idx / b, j = idx % b;
-      if (i < j) out[tri_index(i, j, b)] = 0.5f * (Gs[i * ld + j] - Gs[j * ld + i]);
+    float* out = dQ + static_cast<size_t>(blk) * (B * (B - 1) / 2);
+    for (int idx = tid; idx < B * B; idx += kCayleyThreads) {
+      const int i = idx / B, j = idx % B;
+      if (i < j) out[tri_index(i, j, B)] = 0.5f * (Gs[i * LD + j] - Gs[j * LD + i]);
     }
     __syncthreads();
   }

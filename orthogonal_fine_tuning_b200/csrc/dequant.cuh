@@ -11,6 +11,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "dq_pack.cuh"
 
 namespace oftk {
 
@@ -25,78 +26,30 @@ struct WeightView {
   long long scales_expert_stride;  // bytes between experts (bank only)
 };
 
-// OCP e4m3fn -> fp32, from the format definition (bias 7, subnormal m * 2^-9,
-// S.1111.111 = NaN).  Exact.
-__device__ __forceinline__ float e4m3_to_f32(uint32_t c) {
-  const uint32_t s = (c & 0x80u) << 24;
-  const uint32_t e = (c >> 3) & 0xFu;
-  const uint32_t m = c & 0x7u;
-  if (e == 0xFu && m == 0x7u) return __uint_as_float(s | 0x7FC00000u);
-  if (e == 0u) {
-    const float v = static_cast<float>(m) * 0.001953125f;  // m * 2^-9, exact
-    return s ? -v : v;
-  }
-  return __uint_as_float(s | ((e + 120u) << 23) | (m << 20));
-}
-
-// OCP e2m1 -> fp32 (bias 1, subnormal m * 0.5).  Exact.
-__device__ __forceinline__ float e2m1_to_f32(uint32_t c) {
-  const uint32_t s = (c & 0x8u) << 28;
-  const uint32_t e = (c >> 1) & 0x3u;
-  const uint32_t m = c & 0x1u;
-  if (e == 0u) return __uint_as_float(s | (m ? 0x3F000000u : 0u));
-  return __uint_as_float(s | ((e + 126u) << 23) | (m << 22));
-}
-
-// OCP e8m0 -> fp32: 2^(e-127); 0 is the subnormal 2^-127; 255 is NaN.
-__device__ __forceinline__ float e8m0_to_f32(uint32_t e) {
-  if (e == 255u) return __uint_as_float(0x7FC00000u);
-  if (e == 0u) return __uint_as_float(0x00400000u);
-  return __uint_as_float(e << 23);
-}
-
-__device__ __forceinline__ float int4_to_f32(uint32_t nib) {
-  return static_cast<float>(static_cast<int>(nib ^ 8u) - 8);
-}
-
 // Dequantise 8 consecutive elements k0..k0+7 (k0 % 8 == 0) of stored row n into
-// four packed bf16x2 words (element k0 in the low half of out[0]).
+// four packed bf16x2 words (element k0 in the low half of out[0]), with the same
+// packed decoders the fused GEMM's producer warps use (dq_pack.cuh).
 __device__ __forceinline__ void dequant8(const WeightView& w, const uint8_t* codes, const void* scales, int n, int k0,
                                          uint32_t out[4]) {
   if (w.fmt == kFmtFp8) {
     const uint2 c = *reinterpret_cast<const uint2*>(codes + static_cast<size_t>(n) * w.K + k0);
     const float s = static_cast<const float*>(scales)[n];
+    uint32_t v[4];
+    dq::e4m3x4(c.x, v);      // exact bf16 codes
+    dq::e4m3x4(c.y, v + 2);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t word = i < 2 ? c.x : c.y;
-      const uint32_t sh = (i & 1) * 16;
-      const float a = __fmul_rn(e4m3_to_f32((word >> sh) & 0xFFu), s);
-      const float b = __fmul_rn(e4m3_to_f32((word >> (sh + 8)) & 0xFFu), s);
-      out[i] = pack_bf16x2(a, b);
-    }
+    for (int i = 0; i < 4; ++i)  // canonical chain: fp32 product, then bf16
+      out[i] = pack_bf16x2(__fmul_rn(__uint_as_float(v[i] << 16), s), __fmul_rn(__uint_as_float(v[i] & 0xFFFF0000u), s));
     return;
   }
   const uint32_t word = *reinterpret_cast<const uint32_t*>(codes + static_cast<size_t>(n) * (w.K / 2) + k0 / 2);
   if (w.fmt == kFmtInt4) {
     const uint16_t sb = static_cast<const uint16_t*>(scales)[static_cast<size_t>(k0 / w.group) * w.N + n];
-    const float s = bf16_bits_to_f32(sb);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float a = __fmul_rn(int4_to_f32((word >> (8 * i)) & 0xFu), s);  // exact in fp32
-      const float b = __fmul_rn(int4_to_f32((word >> (8 * i + 4)) & 0xFu), s);
-      out[i] = pack_bf16x2(a, b);
-    }
+    dq::int4x8(word, dq::bf2_splat(sb), out);
     return;
   }
-  // MXFP4
   const uint8_t eb = static_cast<const uint8_t*>(scales)[static_cast<size_t>(k0 / 32) * w.N + n];
-  const float x = e8m0_to_f32(eb);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float a = e2m1_to_f32((word >> (8 * i)) & 0xFu) * x;          // exact
-    const float b = e2m1_to_f32((word >> (8 * i + 4)) & 0xFu) * x;
-    out[i] = pack_bf16x2(a, b);
-  }
+  dq::mxfp4x8(word, eb, out);
 }
 
 // out[n][k] = deq(W)[n][k] for all n < N, k < K.  One thread per 8 elements.
@@ -164,6 +117,59 @@ __global__ void __launch_bounds__(256) moe_chunk_dequant_kernel(WeightView bank,
     uint32_t v[4];
     dequant8(bank, codes, scales, n, k0, v);
     *reinterpret_cast<uint4*>(out + static_cast<size_t>(n) * bank.K + k0) = make_uint4(v[0], v[1], v[2], v[3]);
+  }
+}
+
+// MXFP4 e8m0 scales -> bf16 factors 2^(e-127) (exact: e = 0 is the bf16 subnormal
+// 2^-127, e = 255 is NaN), so the backward's producers apply a per-element scale
+// with one multiply.
+__global__ void e8m0_factor_kernel(const uint8_t* __restrict__ e, long long n, uint16_t* __restrict__ out) {
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const uint32_t v = e[i];
+  out[i] = static_cast<uint16_t>(v == 255u ? 0x7FC0u : (v == 0u ? 0x0040u : (v << 7)));
+}
+
+// Transposed copy of the codes for the backward's dequant producers:
+// nibbles [N][K/2] -> [K][N/2] (NIB), or bytes [N][K] -> [K][N].  64 x 64 code tiles.
+template <bool NIB>
+__global__ void __launch_bounds__(256) transpose_codes_kernel(const uint8_t* __restrict__ in, int N, int K,
+                                                              uint8_t* __restrict__ out) {
+  __shared__ uint8_t t[64][64 + 4];  // [n][k], one code per byte
+  const int n0 = blockIdx.y * 64, k0 = blockIdx.x * 64;
+  const int kv = min(64, K - k0);
+  constexpr int WPR = NIB ? 8 : 16;  // 32-bit words per 64 codes of a row
+  for (int it = threadIdx.x; it < 64 * WPR; it += 256) {
+    const int r = it / WPR, wi = it % WPR;
+    const int n = n0 + r;
+    uint32_t w = 0;
+    if (n < N && wi * (NIB ? 8 : 4) < kv)
+      w = NIB ? *reinterpret_cast<const uint32_t*>(in + static_cast<size_t>(n) * (K / 2) + k0 / 2 + 4 * wi)
+              : *reinterpret_cast<const uint32_t*>(in + static_cast<size_t>(n) * K + k0 + 4 * wi);
+    if (NIB) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) t[r][8 * wi + i] = (w >> (4 * i)) & 0xFu;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) t[r][4 * wi + i] = (w >> (8 * i)) & 0xFFu;
+    }
+  }
+  __syncthreads();
+  const int nv = min(64, N - n0);
+  for (int it = threadIdx.x; it < 64 * WPR; it += 256) {
+    const int kk = it / WPR, wi = it % WPR;
+    const int k = k0 + kk;
+    if (kk >= kv || wi * (NIB ? 8 : 4) >= nv) continue;
+    uint32_t w = 0;
+    if (NIB) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w |= static_cast<uint32_t>(t[8 * wi + i][kk]) << (4 * i);
+      *reinterpret_cast<uint32_t*>(out + static_cast<size_t>(k) * (N / 2) + n0 / 2 + 4 * wi) = w;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) w |= static_cast<uint32_t>(t[4 * wi + i][kk]) << (8 * i);
+      *reinterpret_cast<uint32_t*>(out + static_cast<size_t>(k) * N + n0 + 4 * wi) = w;
+    }
   }
 }
 

@@ -19,6 +19,7 @@
 #include "gemm.cuh"
 #include "moe.cuh"
 #include "rot_tc.cuh"
+#include "gemm_dq.cuh"
 
 using namespace oftk;
 
@@ -141,6 +142,21 @@ int make_map_f32_3d(CUtensorMap* m, const void* base, uint64_t K, uint64_t M, ui
   return OFT_OK;
 }
 
+// Generic 2-D map without swizzle (scale tiles of the backward's dequant producers).
+int make_map_plain_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+                      uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return fail(OFT_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {pitch_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(OFT_ERR_CUDA, "cuTensorMapEncodeTiled (plain 2-D) failed (%d)", int(r));
+  return OFT_OK;
+}
+
 // ---- argument checks ----
 int check_weight(const oft_weight* W, bool bank_ok) {
   if (W == nullptr) return fail(OFT_ERR_INVALID_ARG, "weight descriptor is NULL");
@@ -223,12 +239,26 @@ int launch_dequant(const WeightView& v, uint16_t* out, bool transpose, cudaStrea
 
 int launch_cayley(const uint16_t* Q, int nblocks, int b, float* R, const int* offsets, int blocks_per_expert,
                   cudaStream_t st) {
-  const size_t smem = (2 * b * (b + 1) + b) * sizeof(float);
-  const int grid = std::min(nblocks, sm_count() * 8);
-  OFT_CUDA(cudaFuncSetAttribute(cayley_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024));
   ProfScope ps(OFT_K_CAYLEY, st);
-  cayley_fwd_kernel<<<grid, kCayleyThreads, smem, st>>>(Q, nblocks, b, R, offsets, blocks_per_expert);
+  if (b == 16)
+    cayley_fwd_kernel<16><<<(nblocks + 1) / 2, 32, 0, st>>>(Q, nblocks, R, offsets, blocks_per_expert);
+  if (b == 32) cayley_fwd_kernel<32><<<nblocks, 32, 0, st>>>(Q, nblocks, R, offsets, blocks_per_expert);
+  if (b == 64) cayley_fwd_kernel<64><<<nblocks, 64, 0, st>>>(Q, nblocks, R, offsets, blocks_per_expert);
   OFT_LAUNCHED("cayley_fwd_kernel");
+  return OFT_OK;
+}
+
+int launch_cayley_bwd(const float* R, const float* G, int nparts, int nblocks, int b, float* dQ, cudaStream_t st) {
+  const size_t smem = 3ull * b * (b + 1) * sizeof(float);
+  const int grid = std::min(nblocks, sm_count() * 8);
+  if (b == 16) OFT_CUDA(cudaFuncSetAttribute(cayley_bwd_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  if (b == 32) OFT_CUDA(cudaFuncSetAttribute(cayley_bwd_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  if (b == 64) OFT_CUDA(cudaFuncSetAttribute(cayley_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  ProfScope ps(OFT_K_CAYLEY, st);
+  if (b == 16) cayley_bwd_kernel<16><<<grid, kCayleyThreads, smem, st>>>(R, G, nparts, nblocks, dQ);
+  if (b == 32) cayley_bwd_kernel<32><<<grid, kCayleyThreads, smem, st>>>(R, G, nparts, nblocks, dQ);
+  if (b == 64) cayley_bwd_kernel<64><<<grid, kCayleyThreads, smem, st>>>(R, G, nparts, nblocks, dQ);
+  OFT_LAUNCHED("cayley_bwd_kernel");
   return OFT_OK;
 }
 
@@ -298,6 +328,7 @@ int launch_grad(const uint16_t* X, const float* dXr, int M, int K, int P, int b,
   rtc::GradParams prm;
   memset(&prm, 0, sizeof(prm));
   if (int rc = make_map_f32_3d(&prm.tmD, dXr, K, M, P, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B)) return rc;
+  if (int rc = make_map_bf16(&prm.tmX, X, K, M, K, rtc::TM)) return rc;
   const GradChunks gc = grad_chunks(M, K);
   prm.X = X;
   prm.Gp = Gp;
@@ -335,30 +366,63 @@ int launch_gemm(const gemm::Params& prm, int total_tiles_hint, cudaStream_t st) 
   return OFT_OK;
 }
 
-int tiles_of(int m, int n) { return ((m + gemm::BM - 1) / gemm::BM) * ((n + gemm::BN - 1) / gemm::BN); }
+template <int FMT, bool BWD>
+int launch_gemm_dq_t(const gdq::Params& prm, int tiles, cudaStream_t st) {
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    OFT_CUDA(cudaFuncSetAttribute(gdq::gemm_dq_kernel<FMT, BWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(gdq::kSmemBytes)));
+    attr_set[dev] = true;
+  }
+  const int grid = std::max(1, std::min(sm_count(), tiles));
+  ProfScope ps(OFT_K_GEMM, st);
+  gdq::gemm_dq_kernel<FMT, BWD><<<grid, gdq::NUM_THREADS, gdq::kSmemBytes, st>>>(prm);
+  OFT_LAUNCHED("gemm_dq_kernel");
+  return OFT_OK;
+}
+
+int launch_gemm_dq(int fmt, bool bwd, const gdq::Params& prm, int tiles, cudaStream_t st) {
+  if (fmt == OFT_W_INT4) return bwd ? launch_gemm_dq_t<gdq::kInt4, true>(prm, tiles, st)
+                                    : launch_gemm_dq_t<gdq::kInt4, false>(prm, tiles, st);
+  if (fmt == OFT_W_FP8) return bwd ? launch_gemm_dq_t<gdq::kFp8, true>(prm, tiles, st)
+                                   : launch_gemm_dq_t<gdq::kFp8, false>(prm, tiles, st);
+  return bwd ? launch_gemm_dq_t<gdq::kMxfp4, true>(prm, tiles, st) : launch_gemm_dq_t<gdq::kMxfp4, false>(prm, tiles, st);
+}
+
+int dq_tiles(int rows, int tokens) {
+  return ((rows + gdq::WM - 1) / gdq::WM) * (((tokens + gdq::TN - 1) / gdq::TN + gdq::TP - 1) / gdq::TP);
+}
+
 
 struct FwdLayout {
-  size_t xr, wdq, total;
+  size_t xr, total;
 };
 FwdLayout fwd_layout(int M, int K, int N, int P) {
+  (void)N;
   FwdLayout L{};
   L.xr = 0;
-  L.wdq = round_up(L.xr + 2ull * P * M * K, 256);
-  L.total = round_up(L.wdq + 2ull * N * K, 256);
+  L.total = round_up(L.xr + 2ull * P * M * K, 256);
   return L;
 }
 
+size_t code_bytes(int fmt, int N, int K) { return fmt == OFT_W_FP8 ? 1ull * N * K : 1ull * N * K / 2; }
+
 struct BwdLayout {
-  size_t dxr, wdqt, gpart, total;
+  size_t dxr, codes_t, gpart, factors, total;
   int nparts;
 };
-BwdLayout bwd_layout(int M, int K, int N, int P, int b) {
+BwdLayout bwd_layout(int M, int K, int N, int P, int b, int fmt) {
   BwdLayout L{};
   L.nparts = grad_chunks(M, K).chunks;
   L.dxr = 0;
-  L.wdqt = round_up(L.dxr + 4ull * P * M * K, 256);  // dX' kept in fp32
-  L.gpart = round_up(L.wdqt + 2ull * N * K, 256);
-  L.total = round_up(L.gpart + 4ull * P * (K / b) * L.nparts * b * b, 256);
+  L.codes_t = round_up(L.dxr + 4ull * P * M * K, 256);  // dX' kept in fp32
+  L.gpart = round_up(L.codes_t + code_bytes(fmt, N, K), 256);
+  L.factors = round_up(L.gpart + 4ull * P * (K / b) * L.nparts * b * b, 256);
+  // MXFP4: one bf16 factor per e8m0 scale
+  const size_t sbytes = fmt == OFT_W_MXFP4 ? 2ull * (K / 32) * N : 0ull;
+  L.total = round_up(L.factors + sbytes, 256);
   return L;
 }
 
@@ -396,13 +460,7 @@ int oft_cayley_backward(const float* R, const float* G, int n_blocks, int b, flo
   if (!R || !G || !dQ) return fail(OFT_ERR_INVALID_ARG, "NULL pointer");
   if (!aligned16(R) || !aligned16(G) || !aligned16(dQ)) return fail(OFT_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
   if (int rc = check_b(b, b)) return rc;
-  const size_t smem = 3 * b * (b + 1) * sizeof(float);
-  const int grid = std::min(n_blocks, sm_count() * 8);
-  OFT_CUDA(cudaFuncSetAttribute(cayley_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024));
-  ProfScope ps(OFT_K_CAYLEY, as_stream(stream));
-  cayley_bwd_kernel<<<grid, kCayleyThreads, smem, as_stream(stream)>>>(R, G, 1, n_blocks, b, dQ);
-  OFT_LAUNCHED("cayley_bwd_kernel");
-  return OFT_OK;
+  return launch_cayley_bwd(R, G, 1, n_blocks, b, dQ, as_stream(stream));
 }
 
 int oft_dequant_weight(const oft_weight* W, uint16_t* out, int transpose, void* stream) {
@@ -444,43 +502,45 @@ int oft_linear_fwd(const uint16_t* X, int M, const oft_weight* W, const oft_spli
   cudaStream_t st = as_stream(stream);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   uint16_t* Xr = reinterpret_cast<uint16_t*>(wsb + L.xr);
-  uint16_t* Wdq = reinterpret_cast<uint16_t*>(wsb + L.wdq);
 
   if (int rc = launch_rotate_fwd(X, M, K, P, b, R, Xr, st)) return rc;
-  if (int rc = launch_dequant(view_of(W), Wdq, false, st)) return rc;
 
-  gemm::Params prm;
+  // Y[:, cols of p] = X'_p deq(W_p): dequant fused into the GEMM's weight operand
+  gdq::Params prm;
   memset(&prm, 0, sizeof(prm));
-  if (int rc = make_map_bf16(&prm.tmA[0], Xr, K, 1ull * P * M, K, gemm::BM)) return rc;
-  if (int rc = make_map_bf16(&prm.tmB[0], Wdq, K, N, K, gemm::BN)) return rc;
-  for (int i = 1; i < gemm::MAX_MAPS; ++i) {
-    prm.tmA[i] = prm.tmA[0];
-    prm.tmB[i] = prm.tmB[0];
-  }
-  prm.C = Y;
-  prm.ldc = N;
+  if (int rc = make_map_bf16(&prm.tmB[0], Xr, K, 1ull * P * M, K, gdq::TN)) return rc;
+  for (int i = 1; i < gdq::MAX_GROUPS; ++i) prm.tmB[i] = prm.tmB[0];
+  prm.codes = static_cast<const uint8_t*>(W->codes);
+  prm.code_row_bytes = W->fmt == OFT_W_FP8 ? K : K / 2;
+  prm.scales = W->scales;
+  prm.N = N;
+  prm.K = K;
+  prm.group = W->fmt == OFT_W_INT4 ? W->group : 32;
   prm.num_groups = P;
   int off = 0, tiles = 0;
   for (int p = 0; p < P; ++p) {
-    gemm::Group& g = prm.groups[p];
-    g.m = M;
-    g.n = S->sizes[p];
-    g.k = K;
-    g.a_map = 0;
+    gdq::Group& g = prm.groups[p];
+    g.rows = S->sizes[p];
+    g.tokens = M;
+    g.kred = K;
     g.b_map = 0;
-    g.a_row0 = p * M;
-    g.b_row0 = off;
-    g.c_row0 = 0;
-    g.c_col0 = off;
+    g.b_row0 = p * M;
+    g.w_row0 = off;
+    g.w_k0 = 0;
+    g.y_map = p;
+    // Y[:, off : off + N_p] as its own tensor, so stores clip at the sub-projection's edge
+    if (int rc = make_map_plain_2d(&prm.tmY[p], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y + off, S->sizes[p], M, 2ull * N,
+                                   32, 32))
+      return rc;
     off += S->sizes[p];
-    tiles += tiles_of(M, g.n);
+    tiles += dq_tiles(g.rows, M);
   }
-  return launch_gemm(prm, tiles, st);
+  return launch_gemm_dq(W->fmt, false, prm, tiles, st);
 }
 
 size_t oft_linear_bwd_workspace(int M, const oft_weight* W, const oft_split* S, int b) {
   if (W == nullptr || S == nullptr || M <= 0 || b <= 0) return 0;
-  return bwd_layout(M, W->d_in, W->d_out, S->n, b).total;
+  return bwd_layout(M, W->d_in, W->d_out, S->n, b, W->fmt).total;
 }
 
 int oft_linear_bwd(const uint16_t* dY, const uint16_t* X, int M, const oft_weight* W, const oft_split* S, int b,
@@ -499,55 +559,82 @@ int oft_linear_bwd(const uint16_t* dY, const uint16_t* X, int M, const oft_weigh
   if (!dY || !X || !dX || !ws) return fail(OFT_ERR_INVALID_ARG, "NULL pointer");
   if (!aligned16(dY) || !aligned16(X) || !aligned16(R) || !aligned16(dX) || !aligned16(dQ) || !aligned16(ws))
     return fail(OFT_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
-  const BwdLayout L = bwd_layout(M, K, N, P, b);
+  const BwdLayout L = bwd_layout(M, K, N, P, b, W->fmt);
   if (ws_bytes < L.total) return fail(OFT_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   float* dXr = reinterpret_cast<float*>(wsb + L.dxr);
-  uint16_t* WdqT = reinterpret_cast<uint16_t*>(wsb + L.wdqt);
+  uint8_t* codes_t = wsb + L.codes_t;
   float* Gp = reinterpret_cast<float*>(wsb + L.gpart);
 
-  if (int rc = launch_dequant(view_of(W), WdqT, true, st)) return rc;
+  // transposed codes: one contiguous row per input feature for the dequant producers
+  {
+    dim3 grid((K + 63) / 64, (N + 63) / 64);
+    ProfScope ps(OFT_K_DEQUANT, st);
+    if (W->fmt == OFT_W_FP8)
+      transpose_codes_kernel<false><<<grid, 256, 0, st>>>(static_cast<const uint8_t*>(W->codes), N, K, codes_t);
+    else
+      transpose_codes_kernel<true><<<grid, 256, 0, st>>>(static_cast<const uint8_t*>(W->codes), N, K, codes_t);
+    OFT_LAUNCHED("transpose_codes_kernel");
+  }
 
-  // dX'_p = dY_p deq(W_p)^T : A = dY columns of p (reduction over N_p), B = deq(W)^T columns of p
-  gemm::Params prm;
+  // dX'_p = dY_p deq(W_p)^T, dequant fused into the GEMM's weight operand, fp32 out
+  gdq::Params prm;
   memset(&prm, 0, sizeof(prm));
+  const int G = W->fmt == OFT_W_INT4 ? W->group : 32;
+  if (W->fmt == OFT_W_INT4) {
+    if (int rc = make_map_plain_2d(&prm.tmS, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W->scales, N, K / G, 2ull * N, 64,
+                                   gdq::WM / G))
+      return rc;
+  } else if (W->fmt == OFT_W_MXFP4) {
+    uint16_t* fac = reinterpret_cast<uint16_t*>(wsb + L.factors);
+    const long long n = 1ll * (K / 32) * N;
+    {
+      ProfScope ps(OFT_K_DEQUANT, st);
+      e8m0_factor_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
+          static_cast<const uint8_t*>(W->scales), n, fac);
+      OFT_LAUNCHED("e8m0_factor_kernel");
+    }
+    if (int rc = make_map_plain_2d(&prm.tmS, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, fac, N, K / 32, 2ull * N, 64,
+                                   gdq::WM / 32))
+      return rc;
+  } else {
+    // fp32 channel scales, one row
+    if (int rc = make_map_plain_2d(&prm.tmS, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, W->scales, N, 1, 4ull * N, 64, 1))
+      return rc;
+  }
   int off = 0, tiles = 0;
   for (int p = 0; p < P; ++p) {
     const int Np = S->sizes[p];
-    if (int rc = make_map_bf16(&prm.tmA[p], dY + off, Np, M, N, gemm::BM)) return rc;
-    if (int rc = make_map_bf16(&prm.tmB[p], WdqT + off, Np, K, N, gemm::BN)) return rc;
-    gemm::Group& g = prm.groups[p];
-    g.m = M;
-    g.n = K;
-    g.k = Np;
-    g.a_map = p;
+    if (int rc = make_map_bf16(&prm.tmB[p], dY + off, Np, M, N, gdq::TN)) return rc;
+    gdq::Group& g = prm.groups[p];
+    g.rows = K;
+    g.tokens = M;
+    g.kred = Np;
     g.b_map = p;
-    g.a_row0 = 0;
     g.b_row0 = 0;
-    g.c_row0 = p * M;
-    g.c_col0 = 0;
+    g.w_row0 = 0;
+    g.w_k0 = off;
+    g.y_map = p;
+    if (int rc = make_map_plain_2d(&prm.tmY[p], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, dXr + 1ull * p * M * K, K, M,
+                                   4ull * K, 32, 32))
+      return rc;
     off += Np;
-    tiles += tiles_of(M, K);
+    tiles += dq_tiles(K, M);
   }
-  for (int p = P; p < gemm::MAX_MAPS; ++p) {
-    prm.tmA[p] = prm.tmA[0];
-    prm.tmB[p] = prm.tmB[0];
-  }
-  prm.C = dXr;
-  prm.c_f32 = 1;
-  prm.ldc = K;
+  for (int p = P; p < gdq::MAX_GROUPS; ++p) prm.tmB[p] = prm.tmB[0];
+  prm.codes = codes_t;
+  prm.code_row_bytes = W->fmt == OFT_W_FP8 ? N : N / 2;
+  prm.scales = W->scales;
+  prm.N = N;
+  prm.K = K;
+  prm.group = G;
   prm.num_groups = P;
-  if (int rc = launch_gemm(prm, tiles, st)) return rc;
+  if (int rc = launch_gemm_dq(W->fmt, true, prm, tiles, st)) return rc;
 
   if (int rc = launch_rotate_bwd(dXr, M, K, P, b, R, dX, st)) return rc;
   if (int rc = launch_grad(X, dXr, M, K, P, b, Gp, st)) return rc;
 
-  const size_t smem = 3 * b * (b + 1) * sizeof(float);
-  const int cgrid = std::min(P * nb, sm_count() * 8);
-  OFT_CUDA(cudaFuncSetAttribute(cayley_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024));
-  ProfScope ps(OFT_K_CAYLEY, st);
-  cayley_bwd_kernel<<<cgrid, kCayleyThreads, smem, st>>>(R, Gp, L.nparts, P * nb, b, dQ);
-  OFT_LAUNCHED("cayley_bwd_kernel");
+  if (int rc = launch_cayley_bwd(R, Gp, L.nparts, P * nb, b, dQ, st)) return rc;
   return OFT_OK;
 }
 

@@ -44,9 +44,7 @@ __device__ __forceinline__ void unit_range(int total, int& beg, int& end) {
 }
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, unsigned err) {
-  bool ok = false;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, err);
-  return __shfl_sync(0xFFFFFFFFu, ok, 0);
+  return warp_wait_bounded(bar, parity, abort, err);
 }
 
 // Offset of 16-byte chunk `c` of row `r` in a 128B-swizzled region of 128-byte rows.
@@ -73,36 +71,54 @@ constexpr int FWD_A_BYTES = TM * 64 * 2;           // 16 KB
 constexpr int FWD_BP_BYTES = 64 * 64 * 2;          // one 64x64 bf16 tile
 constexpr size_t kFwdSmem = 1024 + A_STAGES * FWD_A_BYTES + 2 * MAX_P * FWD_BP_BYTES + 256;
 
-// B[r = p*64 + c][i] = R_p[i][c] restricted to group g (block-diagonal), split hi/lo.
+// Named barrier over the 128 builder/epilogue threads (warps 2..5).
+__device__ __forceinline__ void builders_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// B[r = p*64 + c][i] = R_p[i][c] restricted to group g (block-diagonal), split
+// hi/lo.  Zero the tiles, then stream each diagonal R block in with coalesced
+// float4 loads (eight in flight per thread) and scatter it transposed.
 __device__ void build_fwd_b(const FwdParams& p, int g, uint8_t* sBhi, uint8_t* sBlo, int tid) {
   const int b = p.b;
-  for (int item = tid; item < p.P * 64 * 8; item += 128) {
-    const int r = item >> 3, ch = item & 7;
-    const int sp = r >> 6, c = r & 63;
-    const int col_c = g * 64 + c;
-    uint32_t hi[4], lo[4];
+  for (int v = tid; v < p.P * FWD_BP_BYTES / 16; v += 128) {
+    reinterpret_cast<uint4*>(sBhi)[v] = make_uint4(0, 0, 0, 0);
+    reinterpret_cast<uint4*>(sBlo)[v] = make_uint4(0, 0, 0, 0);
+  }
+  builders_sync();
+  const int per_split = 16 * b;             // float4s of the group's diagonal blocks: (64/b) * b * b / 4
+  const int total = p.P * per_split;
+  for (int base = 0; base < total; base += 128 * 8) {
+    float4 v[8];
+    int meta[8];
 #pragma unroll
-    for (int e2 = 0; e2 < 4; ++e2) {
-      float v2[2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int i = ch * 8 + e2 * 2 + h;
-        const int col_i = g * 64 + i;
-        float v = 0.f;
-        if (col_c < p.K && col_i < p.K && (c / b) == (i / b)) {
-          const int j = col_c / b;
-          v = p.R[((static_cast<size_t>(sp) * p.nb + j) * b + (i % b)) * b + (c % b)];
+    for (int u = 0; u < 8; ++u) {
+      const int f = base + u * 128 + tid;
+      meta[u] = -1;
+      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (f < total) {
+        const int sp = f / per_split, rem = f % per_split;
+        const int jb = rem / (b * b / 4), w = rem % (b * b / 4);
+        const int i = w / (b / 4), c4 = (w % (b / 4)) * 4;
+        const int j = (g * 64) / b + jb;
+        if ((j + 1) * b <= p.K) {
+          v[u] = *reinterpret_cast<const float4*>(p.R + ((static_cast<size_t>(sp) * p.nb + j) * b + i) * b + c4);
+          meta[u] = (sp << 16) | ((jb * b + i) << 8) | (jb * b + c4);  // split, k (= i in group), first c in group
         }
-        v2[h] = v;
       }
-      const uint16_t h0 = bf16_rn(v2[0]), h1 = bf16_rn(v2[1]);
-      const uint16_t l0 = bf16_rn(v2[0] - bf16_bits_to_f32(h0)), l1 = bf16_rn(v2[1] - bf16_bits_to_f32(h1));
-      hi[e2] = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
-      lo[e2] = static_cast<uint32_t>(l0) | (static_cast<uint32_t>(l1) << 16);
     }
-    const uint32_t off = swz(r, ch);
-    *reinterpret_cast<uint4*>(sBhi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-    *reinterpret_cast<uint4*>(sBlo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (meta[u] < 0) continue;
+      const int sp = meta[u] >> 16, k = (meta[u] >> 8) & 255, c0 = meta[u] & 255;
+      const float e[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int r = sp * 64 + c0 + t;
+        const uint32_t off = swz(r, k >> 3) + (k & 7) * 2;
+        const uint16_t h = bf16_rn(e[t]);
+        *reinterpret_cast<uint16_t*>(sBhi + off) = h;
+        *reinterpret_cast<uint16_t*>(sBlo + off) = bf16_rn(e[t] - bf16_bits_to_f32(h));
+      }
+    }
   }
 }
 
@@ -266,26 +282,40 @@ constexpr int BWD_A_BYTES = TM * 64 * 4;           // 32 KB: two 128 x 32 fp32 b
 constexpr int BWD_BP_BYTES = 64 * 64 * 4;          // 16 KB: one 64 x 64 fp32 tile (two K chunks)
 constexpr size_t kBwdSmem = 1024 + A_STAGES * BWD_A_BYTES + MAX_P * BWD_BP_BYTES + 256;
 
-// B_p[i][l] = R_p[i][l] restricted to group g (block-diagonal), fp32, K-major in two 32-wide chunks.
+// B_p[i][l] = R_p[i][l] restricted to group g (block-diagonal), fp32, K-major in
+// two 32-wide chunks.  Zero the tiles, then stream the diagonal blocks in with
+// coalesced float4 loads (eight in flight per thread).
 __device__ void build_bwd_b(const BwdParams& p, int g, uint8_t* sB, int tid) {
   const int b = p.b;
-  for (int item = tid; item < p.P * 64 * 16; item += 128) {
-    const int sp = item / (64 * 16);
-    const int r = (item / 16) & 63, ch = item & 15;
-    const int h = ch >> 3, cc = ch & 7;
-    const int col_i = g * 64 + r;
-    float v[4];
+  for (int v = tid; v < p.P * BWD_BP_BYTES / 16; v += 128) reinterpret_cast<uint4*>(sB)[v] = make_uint4(0, 0, 0, 0);
+  builders_sync();
+  const int per_split = 16 * b;
+  const int total = p.P * per_split;
+  for (int base = 0; base < total; base += 128 * 8) {
+    float4 v[8];
+    int meta[8];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int l = h * 32 + cc * 4 + e;
-      const int col_l = g * 64 + l;
-      v[e] = 0.f;
-      if (col_i < p.K && col_l < p.K && (r / b) == (l / b)) {
-        const int j = col_i / b;
-        v[e] = p.R[((static_cast<size_t>(sp) * p.nb + j) * b + (r % b)) * b + (l % b)];
+    for (int u = 0; u < 8; ++u) {
+      const int f = base + u * 128 + tid;
+      meta[u] = -1;
+      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (f < total) {
+        const int sp = f / per_split, rem = f % per_split;
+        const int jb = rem / (b * b / 4), w = rem % (b * b / 4);
+        const int i = w / (b / 4), l4 = (w % (b / 4)) * 4;
+        const int j = (g * 64) / b + jb;
+        if ((j + 1) * b <= p.K) {
+          v[u] = *reinterpret_cast<const float4*>(p.R + ((static_cast<size_t>(sp) * p.nb + j) * b + i) * b + l4);
+          meta[u] = (sp << 16) | ((jb * b + i) << 8) | (jb * b + l4);  // split, row i in group, first l in group
+        }
       }
     }
-    *reinterpret_cast<float4*>(sB + sp * BWD_BP_BYTES + h * 8192 + swz(r, cc)) = make_float4(v[0], v[1], v[2], v[3]);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (meta[u] < 0) continue;
+      const int sp = meta[u] >> 16, r = (meta[u] >> 8) & 255, k = meta[u] & 255;
+      *reinterpret_cast<float4*>(sB + sp * BWD_BP_BYTES + (k >> 5) * 8192 + swz(r, (k & 31) >> 2)) = v[u];
+    }
   }
 }
 
@@ -456,27 +486,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) rot_bwd_tc_kernel(const __grid
 // ===========================================================================
 struct GradParams {
   CUtensorMap tmD;      // dX' fp32, 3-D {K, M, P}, box {32, 128, 1}, 128B swizzle with 32-byte atoms
+  CUtensorMap tmX;      // X bf16 [M][K], box {64, 128}, 128B swizzle
   const uint16_t* X;    // [M][K]
   float* Gp;            // [(p*nb + j)][chunks][b][b]
   int M, K, P, b, nb, groups, chunks, tiles_per_chunk, tiles_m;
 };
 
 constexpr int GR_X_BYTES = 4 * 16384;   // 128 tokens x 128 columns fp32, MN-major (4 atom columns)
-constexpr int GR_B_BYTES = 4 * 16384;   // one dX' tile, same layout
+constexpr int GR_XS_BYTES = 2 * 16384;  // the same tile as staged by TMA: bf16, two 64-column boxes
+constexpr int GR_B_BYTES = 4 * 16384;   // one dX' tile, same layout as the fp32 X tile
 constexpr int GR_STAGES = 2;
-constexpr size_t kGradSmem = 1024 + GR_X_BYTES + GR_STAGES * GR_B_BYTES + 256;
+constexpr size_t kGradSmem = 1024 + GR_X_BYTES + GR_XS_BYTES + GR_STAGES * GR_B_BYTES + 256;
 
 __global__ void __launch_bounds__(NUM_THREADS, 1) grad_tc_kernel(const __grid_constant__ GradParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sX = smem;
-  uint8_t* sB = sX + GR_X_BYTES;
+  uint8_t* sXs = sX + GR_X_BYTES;
+  uint8_t* sB = sXs + GR_XS_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sB + GR_STAGES * GR_B_BYTES);
   uint64_t* full = bars;
   uint64_t* empty = bars + GR_STAGES;
   uint64_t* x_full = bars + 2 * GR_STAGES;
   uint64_t* x_empty = x_full + 1;
-  uint64_t* acc_full = x_empty + 1;
+  uint64_t* xs_full = x_empty + 1;
+  uint64_t* xs_empty = xs_full + 1;
+  uint64_t* acc_full = xs_empty + 1;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* drain = acc_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -490,13 +525,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grad_tc_kernel(const __grid_co
     }
     mbar_init(x_full, 128);
     mbar_init(x_empty, 1);
+    mbar_init(xs_full, 1);
+    mbar_init(xs_empty, 128);
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 128);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) tma_prefetch_desc(&p.tmD);
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&p.tmD);
+    tma_prefetch_desc(&p.tmX);
+  }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
@@ -511,13 +551,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grad_tc_kernel(const __grid_co
   if (warp == 0) {
     if (lane == 0) {
       int stage = 0;
-      uint32_t ph = 0;
-      long long issued = 0;
+      uint32_t ph = 0, xs_ph = 0;
+      long long issued = 0, xs_issued = 0;
       bool ok = true;
       for (int u = ubeg; u < uend && ok; ++u) {
         const int g = u / p.chunks, c = u % p.chunks;
         const int mt0 = c * p.tiles_per_chunk, mt1 = min(p.tiles_m, mt0 + p.tiles_per_chunk);
-        for (int mt = mt0; mt < mt1 && ok; ++mt)
+        for (int mt = mt0; mt < mt1 && ok; ++mt) {
+          if (!mbar_wait(xs_empty, xs_ph ^ 1, abort_flag, kErrWaitEmpty)) {
+            ok = false;
+            break;
+          }
+          xs_ph ^= 1;
+          mbar_arrive_expect_tx(xs_full, GR_XS_BYTES);
+          tma_load_2d(sXs, &p.tmX, xs_full, g * 128, mt * TM);
+          tma_load_2d(sXs + 16384, &p.tmX, xs_full, g * 128 + 64, mt * TM);
+          ++xs_issued;
           for (int sp = 0; sp < p.P; ++sp) {
             if (!mbar_wait(&empty[stage], ph ^ 1, abort_flag, kErrWaitEmpty)) {
               ok = false;
@@ -533,10 +582,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grad_tc_kernel(const __grid_co
               ph ^= 1;
             }
           }
+        }
       }
-      if (*abort_flag)
+      if (*abort_flag) {
         for (long long i = (issued > GR_STAGES ? issued - GR_STAGES : 0); i < issued; ++i)
           gemm_drain_wait(&full[i % GR_STAGES], static_cast<uint32_t>((i / GR_STAGES) & 1));
+        if (xs_issued > 0) gemm_drain_wait(xs_full, static_cast<uint32_t>((xs_issued - 1) & 1));
+      }
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -586,7 +638,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grad_tc_kernel(const __grid_co
     }
   } else {
     const int q = warp & 3, tid = threadIdx.x - 64;
-    uint32_t x_ph = 0, acc_ph = 0;
+    uint32_t x_ph = 0, xs_ph = 0, acc_ph = 0;
     const int b = p.b;
     for (int u = ubeg; u < uend; ++u) {
       const int g = u / p.chunks, c = u % p.chunks;
@@ -599,14 +651,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grad_tc_kernel(const __grid_co
           break;
         }
         x_ph ^= 1;
-        // X tile (128 tokens x 128 columns, bf16) -> fp32, MN-major, 128B rows with 32-byte atoms
+        if (!warp_wait(xs_full, xs_ph, abort_flag, kErrWaitFull)) {
+          ok = false;
+          break;
+        }
+        xs_ph ^= 1;
+        // staged X tile (bf16, K-major 128B-swizzled) -> fp32, MN-major, 128B rows with 32-byte atoms
 #pragma unroll 4
         for (int it = 0; it < 16; ++it) {
           const int k = tid + 128 * it;
           const int t = k >> 4, ci = k & 15;
-          const int row = mt * TM + t, col = g * 128 + ci * 8;
-          uint4 v = make_uint4(0, 0, 0, 0);
-          if (row < p.M && col < p.K) v = *reinterpret_cast<const uint4*>(p.X + static_cast<size_t>(row) * p.K + col);
+          const uint4 v = *reinterpret_cast<const uint4*>(sXs + (ci >> 3) * 16384 + swz(t, ci & 7));
           uint8_t* base = sX + (ci >> 2) * 16384;
           const uint32_t c16 = (ci & 3) * 2;
           *reinterpret_cast<uint4*>(base + swz32(t, c16)) =
@@ -614,6 +669,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grad_tc_kernel(const __grid_co
           *reinterpret_cast<uint4*>(base + swz32(t, c16 + 1)) =
               make_uint4(v.z << 16, v.z & 0xFFFF0000u, v.w << 16, v.w & 0xFFFF0000u);
         }
+        mbar_arrive(xs_empty);
         fence_proxy_async_smem();
         mbar_arrive(x_full);
       }
@@ -652,11 +708,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grad_tc_kernel(const __grid_co
           if (gcol < p.K) {
             const int j = gcol / 16;
             float* dst = p.Gp + ((static_cast<size_t>(sp) * p.nb + j) * p.chunks + c) * 256 + (lane & 15) * 16;
+            uint32_t hv[16];
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              const int e = half * 16 + 4 * v;
-              reinterpret_cast<uint4*>(dst)[v] = make_uint4(r[e], r[e + 1], r[e + 2], r[e + 3]);
-            }
+            for (int e = 0; e < 16; ++e) hv[e] = half ? r[16 + e] : r[e];
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              reinterpret_cast<uint4*>(dst)[v] = make_uint4(hv[4 * v], hv[4 * v + 1], hv[4 * v + 2], hv[4 * v + 3]);
           }
         }
       }

@@ -101,3 +101,55 @@ def test_bounded_wait_reports_timeout_and_context_survives(oft):
     Q = torch.zeros(2, 32 * 31 // 2, dtype=torch.bfloat16, device="cuda")
     R = oft.oft_build_rotation(Q, 32)         # the context is still usable
     assert torch.equal(R.cpu(), torch.eye(32).expand(2, 32, 32))
+
+
+# The fused GEMM decodes the weight inside its producer warps, so its decode is
+# checked through the GEMM itself: with Q = 0 (R = I exactly) and one-hot
+# activations, every output is a single product 1 * w accumulated with exact
+# zeros, so the forward returns deq(W)^T and the backward's dX returns deq(W)
+# value for value.  Scales cover the decode's special paths: FP8 channel scales
+# too large to carry the 2^120 of the bit-pattern decode (and negative ones),
+# MXFP4 exponents on both sides of the two-step factor (kept where every value
+# and product stays finite and normal).
+FUSED_DQ_CASES = [
+    ("int4", 32, 256, (136, 120)),
+    ("int4", 128, 384, (200, 56)),
+    ("fp8", 0, 256, (136, 64, 40)),
+    ("mxfp4", 32, 256, (264, 8)),
+]
+
+
+def _extreme_scales(fmt, scales, seed):
+    g = torch.Generator().manual_seed(seed)
+    if fmt == "fp8":
+        s = scales.clone()
+        big = torch.tensor([200.0, -1000.0, 3.0e4, 128.0, -0.75])
+        idx = torch.arange(0, s.numel(), 5)
+        s[idx] = big[torch.arange(idx.numel()) % big.numel()]
+        s[1::11] = -s[1::11]
+        return s
+    if fmt == "mxfp4":
+        return torch.randint(2, 253, scales.shape, generator=g).to(torch.uint8)
+    s = scales.clone()
+    s[1::7] = -s[1::7]
+    return s
+
+
+@pytest.mark.parametrize("fmt,group,K,splits", FUSED_DQ_CASES, ids=[f"{c[0]}-{c[2]}" for c in FUSED_DQ_CASES])
+def test_fused_decode_exact_through_gemm(oft, fmt, group, K, splits):
+    N = sum(splits)
+    spec = LinearSpec("fdq", M=K, K=K, splits=splits, fmt=fmt, group=group, b=32, q_sigma=0.0, w_mode="normal",
+                      seed=K + N)
+    case = make_linear_case(spec, q_zero=True)
+    case["scales"] = _extreme_scales(fmt, case["scales"], N)
+    W = device_weight(case, "cuda")
+    ref = codecs.dequant(fmt, raw(case["codes"]), raw(case["scales"]), K, group)  # [N][K] float64
+    assert np.all(np.isfinite(ref))
+    R = oft.oft_build_rotation(case["Q"].cuda(), spec.b)
+    eye_k = torch.eye(K, dtype=torch.bfloat16, device="cuda")
+    Y = oft.oft_linear_fwd(eye_k, W, splits, spec.b, R)
+    dX, _ = oft.oft_linear_bwd(torch.eye(N, dtype=torch.bfloat16, device="cuda"),
+                               torch.zeros(N, K, dtype=torch.bfloat16, device="cuda"), W, splits, spec.b, R)
+    oft.oft_check_device()
+    np.testing.assert_array_equal(f64(Y), ref.T)
+    np.testing.assert_array_equal(f64(dX), ref)

@@ -10,6 +10,8 @@
 // reproduce the canonical bf16 dequantised value bit for bit.
 #pragma once
 
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 
 namespace oftk {
@@ -82,6 +84,17 @@ __device__ __forceinline__ uint32_t e4m3x2_hi_lanes(uint32_t u) {
 // The same pair without the final multiply: bf16 bits of v * 2^-120 (exact).
 __device__ __forceinline__ uint32_t e4m3x2_bits(uint32_t u) {
   return ((u >> 4) & 0x07F007F0u) | (u & 0x80008000u);
+}
+
+// FP8 e4m3, four codes (byte i = element i) -> four exact fp32 values.  e4m3 is a
+// subset of f16 (subnormals included), so the hardware pair conversion is exact.
+__device__ __forceinline__ void e4m3x4_f32(uint32_t w, float (&out)[4]) {
+  uint32_t h0, h1;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h0) : "h"(static_cast<uint16_t>(w & 0xFFFFu)));
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h1) : "h"(static_cast<uint16_t>(w >> 16)));
+  const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&h0));
+  const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&h1));
+  out[0] = a.x, out[1] = a.y, out[2] = b.x, out[3] = b.y;
 }
 
 // FP8 e4m3, four codes (byte i = element i) -> 2 exact bf16 pairs (no scale).

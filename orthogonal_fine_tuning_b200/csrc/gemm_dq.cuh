@@ -95,7 +95,6 @@ __device__ __forceinline__ void decode(const Group* sg, int ng, int u, int& g, i
 struct Raw {
   uint32_t c[16];  // INT4 / MXFP4: 8 words (64 codes); FP8: 16 words
   uint32_t sc;     // forward: INT4 two bf16 group scales; MXFP4 two e8m0 exponents; FP8 the row's fp32 scale
-  uint32_t big;    // forward FP8: the scale is too large to carry the decode's 2^120
 };
 
 template <int FMT, bool BWD>
@@ -106,7 +105,6 @@ __device__ __forceinline__ void load_raw(const Params& p, const Group& G, int ro
 #pragma unroll
   for (int i = 0; i < NW; ++i) raw.c[i] = 0;
   raw.sc = 0;
-  raw.big = 0;
   if (row >= G.rows || k0 >= G.kred) return;
   const int valid = min(BK, G.kred - k0);      // reduction elements present in this k-step
   const long long rbase = static_cast<long long>(G.w_row0 + row) * p.code_row_bytes;
@@ -123,12 +121,7 @@ __device__ __forceinline__ void load_raw(const Params& p, const Group& G, int ro
       }
     }
     if (FMT == kFp8) {
-      // this row's fp32 channel scale, times 2^120 (which the bit-pattern decode leaves
-      // out: it yields v * 2^-120) unless that would overflow
-      float sv = static_cast<const float*>(p.scales)[G.w_row0 + row];
-      raw.big = fabsf(sv) < 128.f ? 0u : 1u;
-      if (!raw.big) sv *= 1.329227995784916e36f;  // 2^120, exact
-      raw.sc = __float_as_uint(sv);
+      raw.sc = __float_as_uint(static_cast<const float*>(p.scales)[G.w_row0 + row]);  // fp32 channel scale
     } else {
       const int n = G.w_row0 + row;
       const bool second = valid > 32;
@@ -185,28 +178,14 @@ __device__ __forceinline__ void convert(const Raw& raw, const uint8_t* sS, int s
         o[4 * w] = t[0], o[4 * w + 1] = t[1], o[4 * w + 2] = t[2], o[4 * w + 3] = t[3];
       }
     } else {
-      // FP8: w = bf16(fp32(v * s)).  The bit pattern gives v * 2^-120 exactly; widened to
-      // fp32 and multiplied by s * 2^120 it yields the same real product v * s, so the one
-      // fp32 rounding is the canonical one, followed by the bf16 rounding.
+      // FP8: w = bf16(fp32(v * s)): exact v, one fp32 product, then the bf16 rounding
       const float sv = __uint_as_float(raw.sc);
-      if (__any_sync(0xFFFFFFFFu, raw.big)) {
-        // some row's scale did not take the 2^120: restore it on the decoded value (exact)
-        const float up = raw.big ? 1.329227995784916e36f : 1.f;
 #pragma unroll
-        for (int w = 0; w < 16; ++w) {
-          const uint32_t t0 = dq::e4m3x2_bits(dq::prmt(raw.c[w], 0u, 0x1404u));
-          const uint32_t t1 = dq::e4m3x2_bits(dq::prmt(raw.c[w], 0u, 0x3424u));
-          o[2 * w] = pack_bf16x2(__uint_as_float(t0 << 16) * up * sv, __uint_as_float(t0 & 0xFFFF0000u) * up * sv);
-          o[2 * w + 1] = pack_bf16x2(__uint_as_float(t1 << 16) * up * sv, __uint_as_float(t1 & 0xFFFF0000u) * up * sv);
-        }
-      } else {
-#pragma unroll
-        for (int w = 0; w < 16; ++w) {
-          const uint32_t t0 = dq::e4m3x2_bits(dq::prmt(raw.c[w], 0u, 0x1404u));
-          const uint32_t t1 = dq::e4m3x2_bits(dq::prmt(raw.c[w], 0u, 0x3424u));
-          o[2 * w] = pack_bf16x2(__uint_as_float(t0 << 16) * sv, __uint_as_float(t0 & 0xFFFF0000u) * sv);
-          o[2 * w + 1] = pack_bf16x2(__uint_as_float(t1 << 16) * sv, __uint_as_float(t1 & 0xFFFF0000u) * sv);
-        }
+      for (int w = 0; w < 16; ++w) {
+        float f[4];
+        dq::e4m3x4_f32(raw.c[w], f);
+        o[2 * w] = pack_bf16x2(f[0] * sv, f[1] * sv);
+        o[2 * w + 1] = pack_bf16x2(f[2] * sv, f[3] * sv);
       }
     }
   } else {
@@ -231,17 +210,15 @@ __device__ __forceinline__ void convert(const Raw& raw, const uint8_t* sS, int s
         for (int i = 0; i < 4; ++i) o[4 * w + i] = dq::bf2_mul(t[i], S[4 * w + i]);
       }
     } else {
-      // FP8: per-element fp32 channel scales; the decoded v * 2^-120 is widened to fp32
-      // and restored to v exactly, then one fp32 product and the bf16 rounding
-      const float* Sf = reinterpret_cast<const float*>(sS);
+      // FP8: per-element fp32 channel scales; exact v, one fp32 product, the bf16 rounding
+      const float4* S4 = reinterpret_cast<const float4*>(sS);
 #pragma unroll
       for (int w = 0; w < 16; ++w) {
-        const uint32_t t0 = dq::e4m3x2_bits(dq::prmt(raw.c[w], 0u, 0x1404u));
-        const uint32_t t1 = dq::e4m3x2_bits(dq::prmt(raw.c[w], 0u, 0x3424u));
-        const float4 s4 = reinterpret_cast<const float4*>(Sf)[w];
-        const float k = 1.329227995784916e36f;  // 2^120
-        o[2 * w] = pack_bf16x2(__uint_as_float(t0 << 16) * k * s4.x, __uint_as_float(t0 & 0xFFFF0000u) * k * s4.y);
-        o[2 * w + 1] = pack_bf16x2(__uint_as_float(t1 << 16) * k * s4.z, __uint_as_float(t1 & 0xFFFF0000u) * k * s4.w);
+        float f[4];
+        dq::e4m3x4_f32(raw.c[w], f);
+        const float4 s4 = S4[w];
+        o[2 * w] = pack_bf16x2(f[0] * s4.x, f[1] * s4.y);
+        o[2 * w + 1] = pack_bf16x2(f[2] * s4.z, f[3] * s4.w);
       }
     }
   }
@@ -258,8 +235,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_co
   uint64_t* full_b = bars;
   uint64_t* full_a = bars + STAGES;
   uint64_t* empty = bars + 2 * STAGES;
-  uint64_t* acc_full = bars + 3 * STAGES;
-  uint64_t* acc_empty = acc_full + 1;  // one per 192-column half
+  uint64_t* acc_full = bars + 3 * STAGES;  // one per 192-column accumulator half
+  uint64_t* acc_empty = acc_full + TP;
   uint64_t* drain = acc_empty + TP;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -273,8 +250,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_co
       mbar_init(&full_a[s], 128);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(acc_full, 1);
-    for (int h = 0; h < TP; ++h) mbar_init(&acc_empty[h], 128);
+    for (int h = 0; h < TP; ++h) {
+      mbar_init(&acc_full[h], 1);
+      mbar_init(&acc_empty[h], 128);
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -351,67 +330,85 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_co
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      int stage = 0;
-      uint32_t ph = 0, acc_ph = 0;
+      uint32_t acc_ph = 0;
       constexpr uint32_t idesc = idesc_bf16_f32(WM, TN);
       bool ok = true;
+      long long gk = 0;  // k-steps of this CTA's earlier units
       for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
         int g, tw, tt;
         decode(sg, ng, u, g, tw, tt);
         const int nk = (sg[g].kred + BK - 1) / BK;
-        // The first D k-steps feed only accumulator half 0 while the epilogue may still be
-        // reading half 1 of the previous unit; their half-1 products follow once it is free.
+        // Accumulator halves overlap with the epilogue at both ends of a unit: the first D
+        // k-steps feed half 0 only while the epilogue still reads half 1 of the previous
+        // unit, and the last D k-steps finish half 0 first, so the epilogue can drain it
+        // while their half-1 products run.  Each A slot and B stage is released after its
+        // half-1 products.
         const int D = nk < STAGES ? nk : STAGES;
-        auto issue = [&](int h, int ks, int st) {
+        const int T0 = nk - D > D ? nk - D : D;  // tail [T0, nk); empty when nk <= D
+        auto st_of = [&](int j) { return static_cast<int>((gk + j) % STAGES); };
+        auto issue = [&](int h, int j) {
+          const int st = st_of(j);
           const uint32_t a0 = tmem + A_COL0 + static_cast<uint32_t>(st * 32);
           const uint32_t b0 = smem_u32(sB + st * B_BYTES + h * BT_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
             mma_bf16_ts(tmem + static_cast<uint32_t>(h * TN), a0 + kk * 8, sdesc_sw128(b0 + kk * 32, 16, 1024), idesc,
-                        (ks | kk) ? 1u : 0u);
+                        (j | kk) ? 1u : 0u);
         };
-        for (int h = 0; h < TP && ok; ++h) {
-          if (!mbar_wait(&acc_empty[h], acc_ph ^ 1, abort_flag, kErrWaitAccEmpty)) {
-            ok = false;
-            break;
-          }
+        auto wait_full = [&](int j) {
+          const int st = st_of(j);
+          const uint32_t pj = static_cast<uint32_t>(((gk + j) / STAGES) & 1);
+          if (!mbar_wait(&full_a[st], pj, abort_flag, kErrWaitDequant) ||
+              !mbar_wait(&full_b[st], pj, abort_flag, kErrWaitFull))
+            return false;
           tc_fence_after();
+          return true;
+        };
+        auto wait_acc = [&](int h) {
+          if (!mbar_wait(&acc_empty[h], acc_ph ^ 1, abort_flag, kErrWaitAccEmpty)) return false;
+          tc_fence_after();
+          return true;
+        };
+        auto release = [&](int j) { mma_commit(&empty[st_of(j)]); };
+        if (!wait_acc(0)) break;
+        for (int j = 0; j < D && ok; ++j) {
+          ok = wait_full(j);
+          if (ok) issue(0, j);
+        }
+        if (!ok) break;
+        if (nk <= D) {
+          mma_commit(&acc_full[0]);
+          if (!wait_acc(1)) break;
           for (int j = 0; j < D; ++j) {
-            const int st = (stage + j) % STAGES;
-            const uint32_t pj = ph ^ static_cast<uint32_t>(stage + j >= STAGES);
-            if (h == 0 && (!mbar_wait(&full_a[st], pj, abort_flag, kErrWaitDequant) ||
-                           !mbar_wait(&full_b[st], pj, abort_flag, kErrWaitFull))) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            issue(h, j, st);
-            if (h == TP - 1) mma_commit(&empty[st]);
+            issue(1, j);
+            release(j);
+          }
+        } else {
+          if (!wait_acc(1)) break;
+          for (int j = 0; j < D; ++j) {
+            issue(1, j);
+            release(j);
+          }
+          for (int j = D; j < T0 && ok; ++j) {
+            ok = wait_full(j);
+            if (!ok) break;
+            issue(0, j);
+            issue(1, j);
+            release(j);
+          }
+          for (int j = T0; j < nk && ok; ++j) {
+            ok = wait_full(j);
+            if (ok) issue(0, j);
+          }
+          if (!ok) break;
+          mma_commit(&acc_full[0]);
+          for (int j = T0; j < nk; ++j) {
+            issue(1, j);
+            release(j);
           }
         }
-        if (!ok) break;
-        stage += D;
-        if (stage >= STAGES) {
-          stage -= STAGES;
-          ph ^= 1;
-        }
-        for (int ks = D; ks < nk; ++ks) {
-          if (!mbar_wait(&full_a[stage], ph, abort_flag, kErrWaitDequant) ||
-              !mbar_wait(&full_b[stage], ph, abort_flag, kErrWaitFull)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-#pragma unroll
-          for (int h = 0; h < TP; ++h) issue(h, ks, stage);
-          mma_commit(&empty[stage]);
-          if (++stage == STAGES) {
-            stage = 0;
-            ph ^= 1;
-          }
-        }
-        if (!ok) break;
-        mma_commit(acc_full);
+        mma_commit(&acc_full[1]);
+        gk += nk;
         acc_ph ^= 1;
       }
       mma_commit(drain);
@@ -437,9 +434,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_co
       int g, tw, tt;
       decode(sg, ng, u, g, tw, tt);
       const Group& G = sg[g];
-      if (!warp_wait_bounded(acc_full, acc_ph, abort_flag, kErrWaitAccFull)) break;
-      acc_ph ^= 1;
-      tc_fence_after();
       const int n0 = tw * WM + q * 32;  // first weight row of this warp's blocks
       const int m_base = tt * TP * TN;
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
@@ -468,24 +462,37 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_co
         }
         slot = (slot + 1) % SLOTS;
       };
-      __syncwarp();
-      tmem_ld_32x32b_x32(taddr, ra);
-      tmem_ld_wait();
-#pragma unroll 1
-      for (int c = 0; c < NCH; c += 2) {
-        // chunk c is in ra; fetch c + 1 into rb while ra is staged
-        tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>((c + 1) * 32), rb);
-        stage_chunk(ra, c);
-        tmem_ld_wait();
-        if (c + 1 == NCH / 2 - 1 || c + 1 == NCH - 1) {
-          // every column of this half has been read into registers
-          tc_fence_before();
-          mbar_arrive(&acc_empty[(c + 1) / (NCH / 2)]);
+      constexpr int HCH = NCH / TP;  // chunks per half
+      static_assert(HCH % 2 == 0, "chunks are drained in pairs");
+      bool ok = true;
+      for (int h = 0; h < TP; ++h) {
+        if (!warp_wait_bounded(&acc_full[h], acc_ph, abort_flag, kErrWaitAccFull)) {
+          ok = false;
+          break;
         }
-        if (c + 2 < NCH) tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>((c + 2) * 32), ra);
-        stage_chunk(rb, c + 1);
+        tc_fence_after();
+        const int c0 = h * HCH;
+        __syncwarp();
+        tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(c0 * 32), ra);
         tmem_ld_wait();
+#pragma unroll 1
+        for (int c = c0; c < c0 + HCH; c += 2) {
+          // chunk c is in ra; fetch c + 1 into rb while ra is staged
+          tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>((c + 1) * 32), rb);
+          stage_chunk(ra, c);
+          tmem_ld_wait();
+          if (c + 1 == c0 + HCH - 1) {
+            // every column of this half has been read into registers
+            tc_fence_before();
+            mbar_arrive(&acc_empty[h]);
+          }
+          if (c + 2 < c0 + HCH) tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>((c + 2) * 32), ra);
+          stage_chunk(rb, c + 1);
+          tmem_ld_wait();
+        }
       }
+      if (!ok) break;
+      acc_ph ^= 1;
     }
     if (lane == 0) bulk_wait_all();
     __syncwarp();

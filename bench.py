@@ -264,11 +264,18 @@ def gemm_traffic(flops_per_launch_unit):
         return None
     with open(path) as f:
         d = json.load(f)
-    src = os.path.join(ROOT, "orthogonal_fine_tuning_b200", "csrc", "gemm.cuh")
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    if d.get("gemm_cuh_sha256_16") != h:
+    if d.get("kernel_sha256_16") != gemm_kernel_hash():
         return None
     return d.get("bytes_per_launch_by_workload", {}).get(flops_per_launch_unit)
+
+
+def gemm_kernel_hash() -> str:
+    """Hash of the fused-dequant GEMM's device sources (the kernel and its decoders)."""
+    h = hashlib.sha256()
+    for f in ("gemm_dq.cuh", "dq_pack.cuh"):
+        with open(os.path.join(ROOT, "orthogonal_fine_tuning_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
 
 
 def run_ours(args, rank, world):
@@ -394,7 +401,7 @@ def run_ours(args, rank, world):
         peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
         unit = "TFLOP/s"
         traffic = gemm_traffic(name)
-        kernel = "gemm_bf16_kernel (tcgen05/TMEM)"
+        kernel = "gemm_dq_kernel (fused dequant, tcgen05/TMEM)"
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
                 "traffic": traffic, "kernel": kernel,
                 "peak_source": f"{peak_src} ({'sustained' if bound == 'tensor' else 'copy'})"}

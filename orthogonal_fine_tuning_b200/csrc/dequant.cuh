@@ -130,46 +130,64 @@ __global__ void e8m0_factor_kernel(const uint8_t* __restrict__ e, long long n, u
   out[i] = static_cast<uint16_t>(v == 255u ? 0x7FC0u : (v == 0u ? 0x0040u : (v << 7)));
 }
 
-// Transposed copy of the codes for the backward's dequant producers:
-// nibbles [N][K/2] -> [K][N/2] (NIB), or bytes [N][K] -> [K][N].  64 x 64 code tiles.
+// Code layout for the backward's dequant producers.  In the dX' product the weight
+// rows are input features k and the reduction runs over the output channels n of
+// one sub-projection.  For sub-projection g, row tile tw (128 features) and k-step
+// ks (64 channels from the sub-projection's first), one block holds 128 rows x 64
+// codes as [16-byte vector v][row r]: the 32 rows of a warp read 512 contiguous
+// bytes per load.  Features past K and channels past the sub-projection's end
+// are zero codes, so the producers never test bounds.
+struct PackBwdParams {
+  int num_groups;
+  int blk0[5];          // first CTA (block) of each group; blk0[num_groups] = total
+  int n0[4], np[4];     // channel range of each group
+  int nk[4];            // k-steps of each group: ceil(np / 64)
+  long long off[4];     // byte offset of each group's first block
+};
+
 template <bool NIB>
-__global__ void __launch_bounds__(256) transpose_codes_kernel(const uint8_t* __restrict__ in, int N, int K,
-                                                              uint8_t* __restrict__ out) {
-  __shared__ uint8_t t[64][64 + 4];  // [n][k], one code per byte
-  const int n0 = blockIdx.y * 64, k0 = blockIdx.x * 64;
-  const int kv = min(64, K - k0);
-  constexpr int WPR = NIB ? 8 : 16;  // 32-bit words per 64 codes of a row
+__global__ void __launch_bounds__(256) pack_codes_bwd_kernel(const uint8_t* __restrict__ in, int N, int K,
+                                                             PackBwdParams pp, uint8_t* __restrict__ out) {
+  __shared__ uint8_t t[64][128 + 4];  // [channel][feature], one code per byte
+  int g = 0;
+  while (g + 1 < pp.num_groups && static_cast<int>(blockIdx.x) >= pp.blk0[g + 1]) ++g;
+  const int local = static_cast<int>(blockIdx.x) - pp.blk0[g];
+  const int tw = local / pp.nk[g], ks = local % pp.nk[g];
+  const int k0 = tw * 128;
+  const int nbeg = pp.n0[g] + ks * 64;
+  const int nv = min(64, pp.n0[g] + pp.np[g] - nbeg);  // channels present
+  const int kv = min(128, K - k0);                      // features present
+  constexpr int WPR = NIB ? 16 : 32;                    // 32-bit input words per 128 features
+  constexpr int CPW = NIB ? 8 : 4;                      // codes per word
   for (int it = threadIdx.x; it < 64 * WPR; it += 256) {
     const int r = it / WPR, wi = it % WPR;
-    const int n = n0 + r;
     uint32_t w = 0;
-    if (n < N && wi * (NIB ? 8 : 4) < kv)
-      w = NIB ? *reinterpret_cast<const uint32_t*>(in + static_cast<size_t>(n) * (K / 2) + k0 / 2 + 4 * wi)
-              : *reinterpret_cast<const uint32_t*>(in + static_cast<size_t>(n) * K + k0 + 4 * wi);
-    if (NIB) {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) t[r][8 * wi + i] = (w >> (4 * i)) & 0xFu;
-    } else {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) t[r][4 * wi + i] = (w >> (8 * i)) & 0xFFu;
+    if (r < nv && wi * CPW < kv) {
+      const size_t row = static_cast<size_t>(nbeg + r);
+      w = NIB ? *reinterpret_cast<const uint32_t*>(in + row * (K / 2) + k0 / 2 + 4 * wi)
+              : *reinterpret_cast<const uint32_t*>(in + row * K + k0 + 4 * wi);
     }
+#pragma unroll
+    for (int i = 0; i < CPW; ++i) t[r][CPW * wi + i] = NIB ? ((w >> (4 * i)) & 0xFu) : ((w >> (8 * i)) & 0xFFu);
   }
   __syncthreads();
-  const int nv = min(64, N - n0);
-  for (int it = threadIdx.x; it < 64 * WPR; it += 256) {
-    const int kk = it / WPR, wi = it % WPR;
-    const int k = k0 + kk;
-    if (kk >= kv || wi * (NIB ? 8 : 4) >= nv) continue;
-    uint32_t w = 0;
-    if (NIB) {
+  constexpr int NV4 = NIB ? 2 : 4;   // 16-byte vectors per row (64 codes)
+  constexpr int CPV = 64 / NV4;      // codes per vector
+  uint4* dst = reinterpret_cast<uint4*>(out + pp.off[g] + static_cast<size_t>(local) * (NV4 * 128 * 16));
+  for (int it = threadIdx.x; it < NV4 * 128; it += 256) {
+    const int v = it / 128, r = it % 128;
+    uint32_t w[4];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) w |= static_cast<uint32_t>(t[8 * wi + i][kk]) << (4 * i);
-      *reinterpret_cast<uint32_t*>(out + static_cast<size_t>(k) * (N / 2) + n0 / 2 + 4 * wi) = w;
-    } else {
+    for (int q = 0; q < 4; ++q) {
+      uint32_t x = 0;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) w |= static_cast<uint32_t>(t[4 * wi + i][kk]) << (8 * i);
-      *reinterpret_cast<uint32_t*>(out + static_cast<size_t>(k) * N + n0 + 4 * wi) = w;
+      for (int i = 0; i < CPW; ++i) {
+        const uint32_t c = t[v * CPV + q * CPW + i][r];
+        x |= NIB ? (c << (4 * i)) : (c << (8 * i));
+      }
+      w[q] = x;
     }
+    dst[v * 128 + r] = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 

@@ -65,14 +65,15 @@ struct Group {
   int w_k0;      // first reduction index within a codes row
   int y_map;     // output tensor map (rows: tokens, columns: this group's weight rows)
   int tiles_w, tiles_t, tile0;
+  long long code_off;  // backward: byte offset of this group's blocks in the packed codes
 };
 
 struct Params {
   CUtensorMap tmB[MAX_GROUPS];  // activations, bf16, box {64, 192}, 128B swizzle
   CUtensorMap tmS;              // backward only: bf16 scales (INT4), bf16 factors (MXFP4), fp32 scales (FP8); box {64, rows}
   CUtensorMap tmY[MAX_GROUPS];  // outputs, box {32, 32}, no swizzle: forward Y_p bf16, backward dX'_p fp32
-  const uint8_t* codes;         // forward: [N][K] codes; backward: transposed [K][N]
-  long long code_row_bytes;
+  const uint8_t* codes;         // forward: [N][K] codes; backward: blocks packed by pack_codes_bwd_kernel
+  long long code_row_bytes;     // forward only
   const void* scales;           // INT4 bf16 [K/G][N]; FP8 fp32 [N]; MXFP4 e8m0 [K/32][N]
   int N, K, group;
   int num_groups;
@@ -98,10 +99,26 @@ struct Raw {
 };
 
 template <int FMT, bool BWD>
-__device__ __forceinline__ void load_raw(const Params& p, const Group& G, int row, int ks, Raw& raw) {
+__device__ __forceinline__ void load_raw(const Params& p, const Group& G, int tw, int r, int ks, Raw& raw) {
   constexpr int NW = (FMT == kFp8) ? 16 : 8;   // 32-bit words per k-step
   constexpr int PER = (FMT == kFp8) ? 4 : 8;   // codes per word
   const int k0 = ks * BK;
+  if (BWD) {
+    // packed blocks: zero codes pad every row and k-step, so no bounds tests; the
+    // warp's 32 rows read 512 contiguous bytes per vector
+    constexpr int NV4 = NW / 4;
+    const int nk = (G.kred + BK - 1) / BK;
+    const uint4* src = reinterpret_cast<const uint4*>(p.codes + G.code_off) +
+                       (static_cast<size_t>(tw) * nk + ks) * (NV4 * WM) + r;
+#pragma unroll
+    for (int i = 0; i < NV4; ++i) {
+      const uint4 v = src[i * WM];
+      raw.c[4 * i] = v.x, raw.c[4 * i + 1] = v.y, raw.c[4 * i + 2] = v.z, raw.c[4 * i + 3] = v.w;
+    }
+    raw.sc = 0;
+    return;
+  }
+  const int row = tw * WM + r;
 #pragma unroll
   for (int i = 0; i < NW; ++i) raw.c[i] = 0;
   raw.sc = 0;
@@ -109,50 +126,31 @@ __device__ __forceinline__ void load_raw(const Params& p, const Group& G, int ro
   const int valid = min(BK, G.kred - k0);      // reduction elements present in this k-step
   const long long rbase = static_cast<long long>(G.w_row0 + row) * p.code_row_bytes;
   const int kk = G.w_k0 + k0;                  // first reduction index in the codes row
-  if (!BWD) {
-    // forward rows are 32/64-byte aligned; the reduction (d_in) is a multiple of 32
-    const uint4* src = reinterpret_cast<const uint4*>(p.codes + rbase + (FMT == kFp8 ? kk : kk / 2));
-    constexpr int NV = NW / 4;
+  // forward rows are 32/64-byte aligned; the reduction (d_in) is a multiple of 32
+  const uint4* src = reinterpret_cast<const uint4*>(p.codes + rbase + (FMT == kFp8 ? kk : kk / 2));
+  constexpr int NV = NW / 4;
 #pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      if (i * 4 * PER < valid) {
-        const uint4 v = src[i];
-        raw.c[4 * i] = v.x, raw.c[4 * i + 1] = v.y, raw.c[4 * i + 2] = v.z, raw.c[4 * i + 3] = v.w;
-      }
+  for (int i = 0; i < NV; ++i) {
+    if (i * 4 * PER < valid) {
+      const uint4 v = src[i];
+      raw.c[4 * i] = v.x, raw.c[4 * i + 1] = v.y, raw.c[4 * i + 2] = v.z, raw.c[4 * i + 3] = v.w;
     }
-    if (FMT == kFp8) {
-      raw.sc = __float_as_uint(static_cast<const float*>(p.scales)[G.w_row0 + row]);  // fp32 channel scale
-    } else {
-      const int n = G.w_row0 + row;
-      const bool second = valid > 32;
-      if (FMT == kInt4) {
-        const uint16_t* S = static_cast<const uint16_t*>(p.scales);
-        const uint32_t s0 = S[static_cast<size_t>(kk / p.group) * p.N + n];
-        const uint32_t s1 = second ? S[static_cast<size_t>((kk + 32) / p.group) * p.N + n] : 0u;
-        raw.sc = s0 | (s1 << 16);
-      } else {
-        const uint8_t* E = static_cast<const uint8_t*>(p.scales);
-        const uint32_t e0 = E[static_cast<size_t>(kk / 32) * p.N + n];
-        const uint32_t e1 = second ? E[static_cast<size_t>(kk / 32 + 1) * p.N + n] : 127u;
-        raw.sc = e0 | (e1 << 8);
-      }
-    }
+  }
+  if (FMT == kFp8) {
+    raw.sc = __float_as_uint(static_cast<const float*>(p.scales)[G.w_row0 + row]);  // fp32 channel scale
   } else {
-    // transposed codes: row segments are 8-byte (FP8) / 4-byte (FP4, INT4) aligned
-    if (FMT == kFp8) {
-      const uint2* src = reinterpret_cast<const uint2*>(p.codes + rbase + kk);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        if (i * 8 < valid) {
-          const uint2 v = src[i];
-          raw.c[2 * i] = v.x, raw.c[2 * i + 1] = v.y;
-        }
-      }
+    const int n = G.w_row0 + row;
+    const bool second = valid > 32;
+    if (FMT == kInt4) {
+      const uint16_t* S = static_cast<const uint16_t*>(p.scales);
+      const uint32_t s0 = S[static_cast<size_t>(kk / p.group) * p.N + n];
+      const uint32_t s1 = second ? S[static_cast<size_t>((kk + 32) / p.group) * p.N + n] : 0u;
+      raw.sc = s0 | (s1 << 16);
     } else {
-      const uint32_t* src = reinterpret_cast<const uint32_t*>(p.codes + rbase + kk / 2);
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        if (i * 8 < valid) raw.c[i] = src[i];
+      const uint8_t* E = static_cast<const uint8_t*>(p.scales);
+      const uint32_t e0 = E[static_cast<size_t>(kk / 32) * p.N + n];
+      const uint32_t e1 = second ? E[static_cast<size_t>(kk / 32 + 1) * p.N + n] : 127u;
+      raw.sc = e0 | (e1 << 8);
     }
   }
 }
@@ -529,7 +527,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_co
     auto fetch = [&](Raw& raw) {
       to_parity(ld);
       if (ld.u < total) {
-        load_raw<FMT, BWD>(p, sg[ld.g], ld.tw * WM + r, ld.ks, raw);
+        load_raw<FMT, BWD>(p, sg[ld.g], ld.tw, r, ld.ks, raw);
         advance(ld);
       }
     };

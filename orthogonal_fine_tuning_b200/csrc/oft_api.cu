@@ -407,18 +407,26 @@ FwdLayout fwd_layout(int M, int K, int N, int P) {
   return L;
 }
 
-size_t code_bytes(int fmt, int N, int K) { return fmt == OFT_W_FP8 ? 1ull * N * K : 1ull * N * K / 2; }
 
 struct BwdLayout {
   size_t dxr, codes_t, gpart, factors, total;
   int nparts;
 };
-BwdLayout bwd_layout(int M, int K, int N, int P, int b, int fmt) {
+// Bytes of the backward's packed code blocks: per sub-projection, ceil(K/128) row
+// tiles x ceil(N_p/64) k-steps of 128 x 64 codes.
+size_t packed_bwd_code_bytes(int fmt, int K, const oft_split* S) {
+  size_t blocks = 0;
+  for (int p = 0; p < S->n; ++p) blocks += 1ull * ((K + 127) / 128) * ((S->sizes[p] + 63) / 64);
+  return blocks * (fmt == OFT_W_FP8 ? 8192ull : 4096ull);
+}
+
+BwdLayout bwd_layout(int M, int K, int N, const oft_split* S, int b, int fmt) {
   BwdLayout L{};
+  const int P = S->n;
   L.nparts = grad_chunks(M, K).chunks;
   L.dxr = 0;
   L.codes_t = round_up(L.dxr + 4ull * P * M * K, 256);  // dX' kept in fp32
-  L.gpart = round_up(L.codes_t + code_bytes(fmt, N, K), 256);
+  L.gpart = round_up(L.codes_t + packed_bwd_code_bytes(fmt, K, S), 256);
   L.factors = round_up(L.gpart + 4ull * P * (K / b) * L.nparts * b * b, 256);
   // MXFP4: one bf16 factor per e8m0 scale
   const size_t sbytes = fmt == OFT_W_MXFP4 ? 2ull * (K / 32) * N : 0ull;
@@ -540,7 +548,7 @@ int oft_linear_fwd(const uint16_t* X, int M, const oft_weight* W, const oft_spli
 
 size_t oft_linear_bwd_workspace(int M, const oft_weight* W, const oft_split* S, int b) {
   if (W == nullptr || S == nullptr || M <= 0 || b <= 0) return 0;
-  return bwd_layout(M, W->d_in, W->d_out, S->n, b, W->fmt).total;
+  return bwd_layout(M, W->d_in, W->d_out, S, b, W->fmt).total;
 }
 
 int oft_linear_bwd(const uint16_t* dY, const uint16_t* X, int M, const oft_weight* W, const oft_split* S, int b,
@@ -559,22 +567,42 @@ int oft_linear_bwd(const uint16_t* dY, const uint16_t* X, int M, const oft_weigh
   if (!dY || !X || !dX || !ws) return fail(OFT_ERR_INVALID_ARG, "NULL pointer");
   if (!aligned16(dY) || !aligned16(X) || !aligned16(R) || !aligned16(dX) || !aligned16(dQ) || !aligned16(ws))
     return fail(OFT_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
-  const BwdLayout L = bwd_layout(M, K, N, P, b, W->fmt);
+  const BwdLayout L = bwd_layout(M, K, N, S, b, W->fmt);
   if (ws_bytes < L.total) return fail(OFT_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   float* dXr = reinterpret_cast<float*>(wsb + L.dxr);
   uint8_t* codes_t = wsb + L.codes_t;
   float* Gp = reinterpret_cast<float*>(wsb + L.gpart);
 
-  // transposed codes: one contiguous row per input feature for the dequant producers
+  // codes re-laid out per (sub-projection, 128 input features, 64 channels) block for
+  // the dequant producers: one row per input feature, coalesced across a warp
+  long long code_off[gdq::MAX_GROUPS] = {0};
   {
-    dim3 grid((K + 63) / 64, (N + 63) / 64);
+    PackBwdParams pp;
+    memset(&pp, 0, sizeof(pp));
+    pp.num_groups = P;
+    int blk = 0, n0 = 0;
+    long long off = 0;
+    const long long blk_bytes = W->fmt == OFT_W_FP8 ? 8192 : 4096;
+    for (int p = 0; p < P; ++p) {
+      pp.blk0[p] = blk;
+      pp.n0[p] = n0;
+      pp.np[p] = S->sizes[p];
+      pp.nk[p] = (S->sizes[p] + 63) / 64;
+      pp.off[p] = off;
+      code_off[p] = off;
+      const int nblk = ((K + 127) / 128) * pp.nk[p];
+      blk += nblk;
+      off += nblk * blk_bytes;
+      n0 += S->sizes[p];
+    }
+    pp.blk0[P] = blk;
     ProfScope ps(OFT_K_DEQUANT, st);
     if (W->fmt == OFT_W_FP8)
-      transpose_codes_kernel<false><<<grid, 256, 0, st>>>(static_cast<const uint8_t*>(W->codes), N, K, codes_t);
+      pack_codes_bwd_kernel<false><<<blk, 256, 0, st>>>(static_cast<const uint8_t*>(W->codes), N, K, pp, codes_t);
     else
-      transpose_codes_kernel<true><<<grid, 256, 0, st>>>(static_cast<const uint8_t*>(W->codes), N, K, codes_t);
-    OFT_LAUNCHED("transpose_codes_kernel");
+      pack_codes_bwd_kernel<true><<<blk, 256, 0, st>>>(static_cast<const uint8_t*>(W->codes), N, K, pp, codes_t);
+    OFT_LAUNCHED("pack_codes_bwd_kernel");
   }
 
   // dX'_p = dY_p deq(W_p)^T, dequant fused into the GEMM's weight operand, fp32 out
@@ -615,6 +643,7 @@ int oft_linear_bwd(const uint16_t* dY, const uint16_t* X, int M, const oft_weigh
     g.w_row0 = 0;
     g.w_k0 = off;
     g.y_map = p;
+    g.code_off = code_off[p];
     if (int rc = make_map_plain_2d(&prm.tmY[p], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, dXr + 1ull * p * M * K, K, M,
                                    4ull * K, 32, 32))
       return rc;
@@ -623,7 +652,7 @@ int oft_linear_bwd(const uint16_t* dY, const uint16_t* X, int M, const oft_weigh
   }
   for (int p = P; p < gdq::MAX_GROUPS; ++p) prm.tmB[p] = prm.tmB[0];
   prm.codes = codes_t;
-  prm.code_row_bytes = W->fmt == OFT_W_FP8 ? N : N / 2;
+  prm.code_row_bytes = 0;
   prm.scales = W->scales;
   prm.N = N;
   prm.K = K;

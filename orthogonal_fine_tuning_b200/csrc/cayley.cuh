@@ -17,48 +17,50 @@
 namespace oftk {
 
 constexpr int kCayleyThreads = 256;
+constexpr int kCayleyUnrollBlocks = 4096;  // forward launches at least this large use the unrolled pivots
 
 __host__ __device__ __forceinline__ int tri_index(int i, int j, int b) {  // i < j, row-major strict upper
   return i * b - i * (i + 1) / 2 + (j - i - 1);
 }
 
 // Forward, one thread per matrix row: thread r keeps row r of A = I - Q and of
-// the right-hand side I + Q in registers.  A is held as a sliding window of its
-// not-yet-eliminated columns (a[k] = A[r][c + k] at pivot c): after pivot c,
-// column c of A is a unit column and is dropped by shifting the window, so the
-// pivot element is always a[0] and every register index is static while the
-// pivot loop itself stays rolled (small code).  Each pivot row is broadcast
-// through shared memory.  CTAs are one warp (B = 16: two blocks; B = 32: one)
-// or two warps (B = 64, synchronised with a named barrier), so the serial pivot
-// chains of different blocks spread over every SM.
-// Q: bf16 [nblocks][B(B-1)/2]; R: fp32 [nblocks][B][B].  Optional MoE filter:
-// block `blk` belongs to expert blk / blocks_per_expert and is skipped when that
-// expert has no tokens (offsets[e+1] == offsets[e]).
+// the right-hand side I + Q in registers.  At pivot c the pivot row is published
+// through shared memory (double-buffered, so one barrier per pivot).  UNROLL = true unrolls the pivot loop, so every register index is
+// static and only the columns right of c are updated: the fastest form when
+// many blocks share each SM's instruction cache (the MoE build of every active
+// expert).  UNROLL = false keeps a small rolled loop over a sliding window of
+// the uneliminated columns, for launches of a few hundred blocks, where the
+// unrolled code would mostly miss in the instruction cache.  CTAs are one warp (B = 16: two blocks; B = 32: one) or two warps
+// (B = 64, one block, block-wide barrier), so the serial pivot chains of many
+// blocks interleave on every SM.
+// Q: bf16 [nblocks][B(B-1)/2]; R: fp32 [nblocks][B][B].  The grid is persistent:
+// each CTA walks blocks with a stride of the whole grid.  With an active-expert
+// list (MoE), only the blocks of the first *n_active experts of `active` are
+// built: linear block i is block i % blocks_per_expert of expert
+// active[i / blocks_per_expert].
 template <int B>
 struct CayleyFwdCfg {
   static constexpr int THREADS = B < 32 ? 32 : B;
   static constexpr int BPC = THREADS / B;  // blocks per CTA
+  static constexpr int MIN_CTAS = B == 64 ? 4 : 16;  // resident CTAs per SM the register budget allows
 };
 
-template <int B>
-__global__ void __launch_bounds__(CayleyFwdCfg<B>::THREADS) cayley_fwd_kernel(const uint16_t* __restrict__ Q,
-                                                                               int nblocks, float* __restrict__ R,
-                                                                               const int* __restrict__ offsets,
-                                                                               int blocks_per_expert) {
+template <int B, bool UNROLL>
+__device__ __forceinline__ void cayley_fwd_block(const uint16_t* __restrict__ Q, float* __restrict__ R, int lin,
+                                                 int total, const int* __restrict__ active_list,
+                                                 int blocks_per_expert) {
   constexpr int BPC = CayleyFwdCfg<B>::BPC;
-  __shared__ __align__(16) float piv[BPC][2 * B];
+  __shared__ __align__(16) float piv[2][BPC][2 * B + 4];  // pivot row, right-hand side, 1 / pivot
   const int sub = threadIdx.x / B, r = threadIdx.x % B;
-  const int blk = blockIdx.x * BPC + sub;
-  bool active = blk < nblocks;
-  if (active && offsets != nullptr) {
-    const int e = blk / blocks_per_expert;
-    active = offsets[e + 1] > offsets[e];
-  }
+  const bool active = lin < total;  // B = 16: the CTA's second block may run past the end
+  int blk = lin;
+  if (active && active_list != nullptr)
+    blk = active_list[lin / blocks_per_expert] * blocks_per_expert + lin % blocks_per_expert;
   auto block_sync = [&]() {
     if constexpr (B <= 32) {
       __syncwarp();
     } else {
-      __syncthreads();  // one block per CTA
+      __syncthreads();
     }
   };
 
@@ -76,48 +78,103 @@ __global__ void __launch_bounds__(CayleyFwdCfg<B>::THREADS) cayley_fwd_kernel(co
     rhs[j] = d + v;
   }
 
-#pragma unroll 1
-  for (int c = 0; c < B; ++c) {
-    if (r == c) {
-      const float inv = 1.0f / a[0];
+  // Rows are never normalised during the sweep: the pivot row stays as it is and
+  // every other row subtracts f = A[r][c] / A[c][c] times it, so all threads run
+  // the same instructions (the pivot row with f = 0).  The pivot thread computes
+  // 1 / A[c][c] once and publishes it with its row; at the end each row divides
+  // by its own pivot.
+  float my_inv = 1.f;
+  if constexpr (UNROLL) {
 #pragma unroll
-      for (int k = 0; k < B; ++k) {
-        a[k] *= inv;
-        rhs[k] *= inv;
+    for (int c = 0; c < B; ++c) {
+      float* pr = piv[c & 1][sub];
+      const int k0 = c & ~3;  // first float4 holding a column >= c
+      if (r == c) {
+        my_inv = 1.0f / a[c];  // >= 1 in exact arithmetic, so never a zero pivot
+        pr[2 * B] = my_inv;
+#pragma unroll
+        for (int k = k0; k < B; k += 4)
+          *reinterpret_cast<float4*>(pr + k) = make_float4(a[k], a[k + 1], a[k + 2], a[k + 3]);
+#pragma unroll
+        for (int k = 0; k < B; k += 4)
+          *reinterpret_cast<float4*>(pr + B + k) = make_float4(rhs[k], rhs[k + 1], rhs[k + 2], rhs[k + 3]);
+      }
+      block_sync();
+      const float f = (r == c) ? 0.f : a[c] * pr[2 * B];
+#pragma unroll
+      for (int k = k0; k < B; k += 4) {
+        if (k + 3 <= c) continue;
+        const float4 v = *reinterpret_cast<const float4*>(pr + k);
+        if (k + 0 > c) a[k + 0] = fmaf(-f, v.x, a[k + 0]);
+        if (k + 1 > c) a[k + 1] = fmaf(-f, v.y, a[k + 1]);
+        if (k + 2 > c) a[k + 2] = fmaf(-f, v.z, a[k + 2]);
+        a[k + 3] = fmaf(-f, v.w, a[k + 3]);
       }
 #pragma unroll
       for (int k = 0; k < B; k += 4) {
-        *reinterpret_cast<float4*>(&piv[sub][k]) = make_float4(a[k], a[k + 1], a[k + 2], a[k + 3]);
-        *reinterpret_cast<float4*>(&piv[sub][B + k]) = make_float4(rhs[k], rhs[k + 1], rhs[k + 2], rhs[k + 3]);
+        const float4 v = *reinterpret_cast<const float4*>(pr + B + k);
+        rhs[k] = fmaf(-f, v.x, rhs[k]);
+        rhs[k + 1] = fmaf(-f, v.y, rhs[k + 1]);
+        rhs[k + 2] = fmaf(-f, v.z, rhs[k + 2]);
+        rhs[k + 3] = fmaf(-f, v.w, rhs[k + 3]);
       }
     }
-    block_sync();
-    const float f = (r == c) ? 0.f : a[0];
+  } else {
+    // rolled: a[k] = A[r][c + k] is a window over the columns not yet eliminated,
+    // shifted left after each pivot, so the pivot element is always a[0]
+#pragma unroll 1
+    for (int c = 0; c < B; ++c) {
+      float* pr = piv[c & 1][sub];
+      if (r == c) {
+        my_inv = 1.0f / a[0];
+        pr[2 * B] = my_inv;
 #pragma unroll
-    for (int k = 0; k < B; k += 4) {
-      const float4 pa = *reinterpret_cast<const float4*>(&piv[sub][k]);
-      const float4 pr = *reinterpret_cast<const float4*>(&piv[sub][B + k]);
-      a[k] = fmaf(-f, pa.x, a[k]);
-      a[k + 1] = fmaf(-f, pa.y, a[k + 1]);
-      a[k + 2] = fmaf(-f, pa.z, a[k + 2]);
-      a[k + 3] = fmaf(-f, pa.w, a[k + 3]);
-      rhs[k] = fmaf(-f, pr.x, rhs[k]);
-      rhs[k + 1] = fmaf(-f, pr.y, rhs[k + 1]);
-      rhs[k + 2] = fmaf(-f, pr.z, rhs[k + 2]);
-      rhs[k + 3] = fmaf(-f, pr.w, rhs[k + 3]);
+        for (int k = 0; k < B; k += 4) {
+          *reinterpret_cast<float4*>(pr + k) = make_float4(a[k], a[k + 1], a[k + 2], a[k + 3]);
+          *reinterpret_cast<float4*>(pr + B + k) = make_float4(rhs[k], rhs[k + 1], rhs[k + 2], rhs[k + 3]);
+        }
+      }
+      block_sync();
+      const float f = (r == c) ? 0.f : a[0] * pr[2 * B];
+#pragma unroll
+      for (int k = 0; k < B; k += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(pr + k);
+        const float4 w = *reinterpret_cast<const float4*>(pr + B + k);
+        a[k] = fmaf(-f, v.x, a[k]);
+        a[k + 1] = fmaf(-f, v.y, a[k + 1]);
+        a[k + 2] = fmaf(-f, v.z, a[k + 2]);
+        a[k + 3] = fmaf(-f, v.w, a[k + 3]);
+        rhs[k] = fmaf(-f, w.x, rhs[k]);
+        rhs[k + 1] = fmaf(-f, w.y, rhs[k + 1]);
+        rhs[k + 2] = fmaf(-f, w.z, rhs[k + 2]);
+        rhs[k + 3] = fmaf(-f, w.w, rhs[k + 3]);
+      }
+      // drop the eliminated column c: the window moves one column right
+#pragma unroll
+      for (int k = 0; k < B - 1; ++k) a[k] = a[k + 1];
+      a[B - 1] = 0.f;
     }
-    // drop the eliminated column c: the window moves one column right
-#pragma unroll
-    for (int k = 0; k < B - 1; ++k) a[k] = a[k + 1];
-    a[B - 1] = 0.f;
-    block_sync();
   }
+#pragma unroll
+  for (int k = 0; k < B; ++k) rhs[k] *= my_inv;
   if (active) {
     float* out = R + (static_cast<size_t>(blk) * B + r) * B;
 #pragma unroll
     for (int j = 0; j < B; j += 4)
       *reinterpret_cast<float4*>(out + j) = make_float4(rhs[j], rhs[j + 1], rhs[j + 2], rhs[j + 3]);
   }
+}
+
+template <int B, bool UNROLL>
+__global__ void __launch_bounds__(CayleyFwdCfg<B>::THREADS, CayleyFwdCfg<B>::MIN_CTAS) cayley_fwd_kernel(const uint16_t* __restrict__ Q,
+                                                                               int nblocks, float* __restrict__ R,
+                                                                               const int* __restrict__ active_list,
+                                                                               const int* __restrict__ n_active,
+                                                                               int blocks_per_expert) {
+  constexpr int BPC = CayleyFwdCfg<B>::BPC;
+  const int total = active_list != nullptr ? min(nblocks, *n_active * blocks_per_expert) : nblocks;
+  for (int base = blockIdx.x * BPC; base < total; base += gridDim.x * BPC)
+    cayley_fwd_block<B, UNROLL>(Q, R, base + threadIdx.x / B, total, active_list, blocks_per_expert);
 }
 
 // dQ[blk] = pack(D - D^T), D = 1/2 (I+R)^T G (I+R)^T.

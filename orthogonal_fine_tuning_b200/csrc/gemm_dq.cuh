@@ -531,8 +531,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_co
         advance(ld);
       }
     };
-    // decode the k-step at `cv` from `cur`, store it to TMEM, refill `cur` while the
-    // store lands, then publish the A slot
+    // decode the k-step at `cv` from `cur`, store it to TMEM, publish the A slot, then
+    // refill `cur`: the next loads stay off the path from a freed slot to a full one
     auto step_one = [&](Raw& cur) -> bool {
       to_parity(cv);
       if (cv.u >= total) return false;
@@ -546,10 +546,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_co
       convert<FMT, BWD>(cur, sS + stage * S_BYTES, srow, o);
       __syncwarp();
       tmem_st_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + A_COL0 + static_cast<uint32_t>(stage * 32), o);
-      fetch(cur);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&full_a[stage]);
+      fetch(cur);
       advance(cv);
       return true;
     };

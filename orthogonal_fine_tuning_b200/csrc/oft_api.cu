@@ -15,7 +15,6 @@
 #include "common.cuh"
 #include "dequant.cuh"
 #include "cayley.cuh"
-#include "rotate.cuh"
 #include "gemm.cuh"
 #include "moe.cuh"
 #include "rot_tc.cuh"
@@ -237,13 +236,24 @@ int launch_dequant(const WeightView& v, uint16_t* out, bool transpose, cudaStrea
   return OFT_OK;
 }
 
-int launch_cayley(const uint16_t* Q, int nblocks, int b, float* R, const int* offsets, int blocks_per_expert,
-                  cudaStream_t st) {
+// active_list / n_active (device): build only the blocks of the active experts.
+int launch_cayley(const uint16_t* Q, int nblocks, int b, float* R, const int* active_list, const int* n_active,
+                  int blocks_per_expert, cudaStream_t st) {
   ProfScope ps(OFT_K_CAYLEY, st);
-  if (b == 16)
-    cayley_fwd_kernel<16><<<(nblocks + 1) / 2, 32, 0, st>>>(Q, nblocks, R, offsets, blocks_per_expert);
-  if (b == 32) cayley_fwd_kernel<32><<<nblocks, 32, 0, st>>>(Q, nblocks, R, offsets, blocks_per_expert);
-  if (b == 64) cayley_fwd_kernel<64><<<nblocks, 64, 0, st>>>(Q, nblocks, R, offsets, blocks_per_expert);
+  // unrolled pivots pay off once many blocks run from a warm instruction cache;
+  // persistent grid of about 32 resident warps per SM
+  const int bpc = b == 16 ? 2 : 1, warps = b == 64 ? 2 : 1;
+  const int grid = std::max(1, std::min((nblocks + bpc - 1) / bpc, sm_count() * 32 / warps));
+  const int* al = active_list;
+  if (nblocks >= kCayleyUnrollBlocks) {
+    if (b == 16) cayley_fwd_kernel<16, true><<<grid, 32, 0, st>>>(Q, nblocks, R, al, n_active, blocks_per_expert);
+    if (b == 32) cayley_fwd_kernel<32, true><<<grid, 32, 0, st>>>(Q, nblocks, R, al, n_active, blocks_per_expert);
+    if (b == 64) cayley_fwd_kernel<64, true><<<grid, 64, 0, st>>>(Q, nblocks, R, al, n_active, blocks_per_expert);
+  } else {
+    if (b == 16) cayley_fwd_kernel<16, false><<<grid, 32, 0, st>>>(Q, nblocks, R, al, n_active, blocks_per_expert);
+    if (b == 32) cayley_fwd_kernel<32, false><<<grid, 32, 0, st>>>(Q, nblocks, R, al, n_active, blocks_per_expert);
+    if (b == 64) cayley_fwd_kernel<64, false><<<grid, 64, 0, st>>>(Q, nblocks, R, al, n_active, blocks_per_expert);
+  }
   OFT_LAUNCHED("cayley_fwd_kernel");
   return OFT_OK;
 }
@@ -459,7 +469,7 @@ int oft_build_rotation(const uint16_t* Q, int n_blocks, int b, float* R, void* s
   if (Q == nullptr || R == nullptr) return fail(OFT_ERR_INVALID_ARG, "Q/R NULL");
   if (!aligned16(Q) || !aligned16(R)) return fail(OFT_ERR_INVALID_ARG, "Q/R must be 16-byte aligned");
   if (int rc = check_b(b, b)) return rc;
-  return launch_cayley(Q, n_blocks, b, R, nullptr, 1, as_stream(stream));
+  return launch_cayley(Q, n_blocks, b, R, nullptr, nullptr, 1, as_stream(stream));
 }
 
 int oft_cayley_backward(const float* R, const float* G, int n_blocks, int b, float* dQ, void* stream) {
@@ -740,15 +750,15 @@ int moe_chunked_oft_fwd(const uint16_t* X, int T, const float* logits, int E, in
     OFT_LAUNCHED("moe_route_kernel");
   }
   // 3. rotations of the active experts (gate and up)
-  if (int rc = launch_cayley(Q, E * 2 * nb, b, Rex, offsets, 2 * nb, st)) return rc;
+  if (int rc = launch_cayley(Q, E * 2 * nb, b, Rex, chunk_table, n_active, 2 * nb, st)) return rc;
   // 4. rotated gather in bucket order: Xg[proj][pos] = X[t] R_{e,proj}
-  dim3 ggrid(nb, (TK + kRotTokens - 1) / kRotTokens, 2);
+  dim3 ggrid((K + 63) / 64, (TK + kGatherRows - 1) / kGatherRows);
   {
-  ProfScope ps(OFT_K_ROTATE, st);
-  if (b == 16) moe_gather_rotate_kernel<16><<<ggrid, kRotThreads, 0, st>>>(X, K, TK, top_k, bucket, pexp, Rex, Xg);
-  if (b == 32) moe_gather_rotate_kernel<32><<<ggrid, kRotThreads, 0, st>>>(X, K, TK, top_k, bucket, pexp, Rex, Xg);
-  if (b == 64) moe_gather_rotate_kernel<64><<<ggrid, kRotThreads, 0, st>>>(X, K, TK, top_k, bucket, pexp, Rex, Xg);
-  OFT_LAUNCHED("moe_gather_rotate_kernel");
+    ProfScope ps(OFT_K_ROTATE, st);
+    if (b == 16) moe_gather_rotate_kernel<16><<<ggrid, kGatherThreads, 0, st>>>(X, K, TK, top_k, bucket, pexp, Rex, Xg);
+    if (b == 32) moe_gather_rotate_kernel<32><<<ggrid, kGatherThreads, 0, st>>>(X, K, TK, top_k, bucket, pexp, Rex, Xg);
+    if (b == 64) moe_gather_rotate_kernel<64><<<ggrid, kGatherThreads, 0, st>>>(X, K, TK, top_k, bucket, pexp, Rex, Xg);
+    OFT_LAUNCHED("moe_gather_rotate_kernel");
   }
   // 5. chunks: transient dequant of the chunk's experts, then one grouped GEMM
   gemm::Params prm;

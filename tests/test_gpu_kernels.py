@@ -59,6 +59,19 @@ def test_cayley_forward(oft, b, sigma):
     assert np.abs(np.swapaxes(got, -1, -2) @ got - I).max() < 1e-4
 
 
+@pytest.mark.parametrize("b", [16, 32, 64])
+def test_cayley_forward_many_blocks(oft, b):
+    """Launches of many blocks take the unrolled pivot loop; same result bar."""
+    g = torch.Generator().manual_seed(100 + b)
+    Q = (torch.randn(4101, b * (b - 1) // 2, generator=g) * 0.05).to(torch.bfloat16)
+    R = oft.oft_build_rotation(Q.cuda(), b)
+    ref = oft_ref.rotations(raw(Q), b)
+    got = f64(R)
+    assert np.abs(got - ref).max() < 2e-5 * max(1.0, 0.05 * b)
+    I = np.eye(b)
+    assert np.abs(np.swapaxes(got, -1, -2) @ got - I).max() < 1e-4
+
+
 def test_cayley_zero_is_identity(oft):
     Q = torch.zeros(5, 32 * 31 // 2, dtype=torch.bfloat16, device="cuda")
     R = oft.oft_build_rotation(Q, 32)

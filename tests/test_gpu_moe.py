@@ -47,9 +47,10 @@ def _to(case, dev):
     return {k: (v.to(dev) if torch.is_tensor(v) else v) for k, v in case.items()}
 
 
-@pytest.mark.parametrize("T,E,top_k,chunk,b", [(200, 24, 4, 4, 32), (77, 9, 3, 2, 16), (64, 5, 1, 3, 64)])
-def test_small_moe(oft, T, E, top_k, chunk, b):
-    spec = MoESpec("s", T=T, K=256, E=E, n_proj=48, top_k=top_k, chunk=chunk, group=32, b=b, q_sigma=0.05,
+@pytest.mark.parametrize("T,E,top_k,chunk,b,K", [(200, 24, 4, 4, 32, 256), (77, 9, 3, 2, 16, 256), (64, 5, 1, 3, 64, 256),
+                                                  (50, 7, 2, 3, 32, 160)])
+def test_small_moe(oft, T, E, top_k, chunk, b, K):
+    spec = MoESpec("s", T=T, K=K, E=E, n_proj=48, top_k=top_k, chunk=chunk, group=32, b=b, q_sigma=0.05,
                    seed=T + E)
     case = make_moe_case(spec)
     out = _run(oft, _to(case, "cuda"))

@@ -100,23 +100,58 @@ __global__ void __launch_bounds__(256) dequant_transposed_kernel(WeightView w, u
   }
 }
 
-// MoE: dequantise the experts of chunk `chunk_idx` into buf[slot][N][K].
-// grid = (blocks per expert, chunk slots).  Slots without an expert (-1) do nothing.
+// MoE: dequantise the experts of chunk `chunk_idx` into buf[slot][N][K] (INT4 bank).
+// grid = (ceil(N / 64) row tiles, chunk slots); slots without an expert (-1) do
+// nothing.  A CTA takes 64 rows of one expert: their K/G group scales are staged
+// in shared memory row-major, then each warp walks whole rows, lane l decoding
+// the 8 codes of word l + 32 i, so every load and store instruction of a warp
+// covers contiguous memory (128 B of codes in, 512 B of bf16 out).
+constexpr int kChunkRows = 64;
+
+__host__ __device__ constexpr int chunk_scale_ld(int groups) { return groups + 2; }
+
 __global__ void __launch_bounds__(256) moe_chunk_dequant_kernel(WeightView bank, const int* __restrict__ chunk_table,
                                                                 int chunk_idx, int chunk, uint16_t* __restrict__ buf) {
+  extern __shared__ uint16_t s_scale[];  // [kChunkRows][K/G + 2]
   const int slot = blockIdx.y;
   const int e = chunk_table[chunk_idx * chunk + slot];
   if (e < 0) return;
-  const uint8_t* codes = bank.codes + static_cast<long long>(e) * bank.codes_expert_stride;
-  const void* scales = static_cast<const uint8_t*>(bank.scales) + static_cast<long long>(e) * bank.scales_expert_stride;
-  uint16_t* out = buf + static_cast<size_t>(slot) * bank.N * bank.K;
-  const long long units = static_cast<long long>(bank.N) * (bank.K / 8);
-  for (long long u = blockIdx.x * 256ll + threadIdx.x; u < units; u += static_cast<long long>(gridDim.x) * 256) {
-    const int n = static_cast<int>(u / (bank.K / 8));
-    const int k0 = static_cast<int>(u % (bank.K / 8)) * 8;
-    uint32_t v[4];
-    dequant8(bank, codes, scales, n, k0, v);
-    *reinterpret_cast<uint4*>(out + static_cast<size_t>(n) * bank.K + k0) = make_uint4(v[0], v[1], v[2], v[3]);
+  const int N = bank.N, K = bank.K, G = bank.group;
+  const int ng = K / G, ld = chunk_scale_ld(ng);
+  const int n0 = blockIdx.x * kChunkRows, rows = min(kChunkRows, N - n0);
+  const uint32_t* codes = reinterpret_cast<const uint32_t*>(bank.codes + static_cast<long long>(e) * bank.codes_expert_stride);
+  const uint16_t* S = reinterpret_cast<const uint16_t*>(static_cast<const uint8_t*>(bank.scales) +
+                                                        static_cast<long long>(e) * bank.scales_expert_stride);
+  for (int it = threadIdx.x; it < ng * kChunkRows; it += 256) {
+    const int j = it / kChunkRows, r = it % kChunkRows;
+    if (r < rows) s_scale[r * ld + j] = S[static_cast<size_t>(j) * N + n0 + r];
+  }
+  __syncthreads();
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int words = K / 8;  // 8 codes per 32-bit word
+  uint16_t* out = buf + (static_cast<size_t>(slot) * N + n0) * K;
+  for (int r = warp; r < rows; r += 8) {
+    const uint32_t* crow = codes + static_cast<size_t>(n0 + r) * words;
+    const uint16_t* srow = s_scale + r * ld;
+    uint4* orow = reinterpret_cast<uint4*>(out + static_cast<size_t>(r) * K);
+    int w = lane;
+    for (; w + 96 < words; w += 128) {  // four independent loads in flight per lane
+      uint32_t c[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) c[u] = crow[w + 32 * u];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int wu = w + 32 * u;
+        uint32_t v[4];
+        dq::int4x8(c[u], dq::bf2_splat(srow[(wu * 8) / G]), v);
+        orow[wu] = make_uint4(v[0], v[1], v[2], v[3]);
+      }
+    }
+    for (; w < words; w += 32) {
+      uint32_t v[4];
+      dq::int4x8(crow[w], dq::bf2_splat(srow[(w * 8) / G]), v);
+      orow[w] = make_uint4(v[0], v[1], v[2], v[3]);
+    }
   }
 }
 

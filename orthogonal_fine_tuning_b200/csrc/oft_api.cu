@@ -54,6 +54,34 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Per-device side stream and events for the MoE chunk pipeline (dequant of chunk
+// c + 1 overlaps the grouped GEMM of chunk c).  Created on first use, kept until
+// exit; they hold no device memory.
+struct SidePipe {
+  bool ready = false;
+  cudaStream_t side = nullptr;
+  cudaEvent_t start = nullptr, dq_done[2] = {nullptr, nullptr}, gemm_done[2] = {nullptr, nullptr};
+};
+SidePipe g_side[64];
+
+int side_pipe(SidePipe** out) {
+  int dev = 0;
+  OFT_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(OFT_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  SidePipe& sp = g_side[dev];
+  if (!sp.ready) {
+    OFT_CUDA(cudaStreamCreateWithFlags(&sp.side, cudaStreamNonBlocking));
+    OFT_CUDA(cudaEventCreateWithFlags(&sp.start, cudaEventDisableTiming));
+    for (int i = 0; i < 2; ++i) {
+      OFT_CUDA(cudaEventCreateWithFlags(&sp.dq_done[i], cudaEventDisableTiming));
+      OFT_CUDA(cudaEventCreateWithFlags(&sp.gemm_done[i], cudaEventDisableTiming));
+    }
+    sp.ready = true;
+  }
+  *out = &sp;
+  return OFT_OK;
+}
+
 int sm_count() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -690,7 +718,7 @@ MoeLayout moe_layout(int T, int E, int top_k, int chunk, int K, int N, int b) {
   L.rex = 0;
   L.xg = round_up(L.rex + 4ull * E * 2 * (K / b) * b * b, 256);
   L.buf = round_up(L.xg + 2ull * 2 * TK * K, 256);
-  L.ytk = round_up(L.buf + 2ull * chunk * N * K, 256);
+  L.ytk = round_up(L.buf + 2ull * 2 * chunk * N * K, 256);  // two chunk buffers (double-buffered)
   L.inv = round_up(L.ytk + 4ull * TK * N, 256);  // per-slot expert outputs kept in fp32
   L.pexp = round_up(L.inv + 4ull * TK, 256);
   L.total = round_up(L.pexp + 4ull * TK, 256);
@@ -764,11 +792,7 @@ int moe_chunked_oft_fwd(const uint16_t* X, int T, const float* logits, int E, in
   gemm::Params prm;
   memset(&prm, 0, sizeof(prm));
   if (int rc = make_map_bf16(&prm.tmA[0], Xg, K, 2ull * TK, K, gemm::BM)) return rc;
-  if (int rc = make_map_bf16(&prm.tmB[0], buf, K, 1ull * chunk * N, K, gemm::BN)) return rc;
-  for (int i = 1; i < gemm::MAX_MAPS; ++i) {
-    prm.tmA[i] = prm.tmA[0];
-    prm.tmB[i] = prm.tmB[0];
-  }
+  for (int i = 1; i < gemm::MAX_MAPS; ++i) prm.tmA[i] = prm.tmA[0];  // B maps: per chunk buffer, below
   prm.C = Ytk;
   prm.c_f32 = 1;
   prm.ldc = N;
@@ -780,16 +804,35 @@ int moe_chunked_oft_fwd(const uint16_t* X, int T, const float* logits, int E, in
   prm.moe.n_proj = n_proj;
   prm.moe.K = K;
   WeightView bank = view_of(W);
-  const long long units = 1ll * N * (K / 8);
-  const int dq_blocks = static_cast<int>(std::min<long long>((units + 255) / 256, std::max(1, sm_count() * 8 / chunk)));
+  const size_t dq_smem = sizeof(uint16_t) * kChunkRows * chunk_scale_ld(K / W->group);
+  if (dq_smem > 227 * 1024) return fail(OFT_ERR_UNSUPPORTED, "d_in / group too large for the chunk dequant");
+  OFT_CUDA(cudaFuncSetAttribute(moe_chunk_dequant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(dq_smem)));
+  // Chunk c is dequantised into buffer c % 2 on the side stream while the grouped
+  // GEMM of chunk c - 1 runs on the caller's stream; the dequant of chunk c waits
+  // for the GEMM of chunk c - 2 (the last reader of its buffer).
+  SidePipe* sp = nullptr;
+  if (int rc = side_pipe(&sp)) return rc;
+  OFT_CUDA(cudaEventRecord(sp->start, st));
+  OFT_CUDA(cudaStreamWaitEvent(sp->side, sp->start, 0));
+  const size_t buf_elems = 1ull * chunk * N * K;
   for (int c = 0; c < n_chunks_max; ++c) {
+    const int h = c & 1;
+    uint16_t* bufc = buf + h * buf_elems;
+    if (c >= 2) OFT_CUDA(cudaStreamWaitEvent(sp->side, sp->gemm_done[h], 0));
     {
-      ProfScope ps(OFT_K_DEQUANT, st);
-      moe_chunk_dequant_kernel<<<dim3(dq_blocks, chunk), 256, 0, st>>>(bank, chunk_table, c, chunk, buf);
+      ProfScope ps(OFT_K_DEQUANT, sp->side);
+      moe_chunk_dequant_kernel<<<dim3((N + kChunkRows - 1) / kChunkRows, chunk), 256, dq_smem, sp->side>>>(
+          bank, chunk_table, c, chunk, bufc);
       OFT_LAUNCHED("moe_chunk_dequant_kernel");
     }
+    OFT_CUDA(cudaEventRecord(sp->dq_done[h], sp->side));
+    OFT_CUDA(cudaStreamWaitEvent(st, sp->dq_done[h], 0));
     prm.moe.chunk_idx = c;
+    if (int rc = make_map_bf16(&prm.tmB[0], bufc, K, 1ull * chunk * N, K, gemm::BN)) return rc;
+    for (int i = 1; i < gemm::MAX_MAPS; ++i) prm.tmB[i] = prm.tmB[0];
     if (int rc = launch_gemm(prm, 0, st)) return rc;
+    OFT_CUDA(cudaEventRecord(sp->gemm_done[h], st));
   }
   // 6. weighted combine in slot order
   const long long cunits = 1ll * T * (N / 8);

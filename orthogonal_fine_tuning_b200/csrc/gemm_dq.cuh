@@ -80,6 +80,27 @@ struct Params {
   Group groups[MAX_GROUPS];
 };
 
+// Balanced static schedule for launches whose groups have different reduction
+// lengths (the backward of a fused weight with unequal sub-projections): the host
+// assigns units longest-first to the least-loaded CTA, and CTA b runs
+// list[off[b] .. off[b+1]) in order.  Without it, CTA b runs units b, b + grid, ...
+constexpr int kMaxSchedCtas = 160;
+constexpr int kMaxSchedUnits = 12000;
+struct Sched {
+  uint16_t off[kMaxSchedCtas + 1];
+  uint16_t list[kMaxSchedUnits];
+};
+
+template <bool SCHED>
+struct KParams {
+  Params p;
+};
+template <>
+struct KParams<true> {
+  Params p;
+  Sched s;
+};
+
 constexpr size_t kBarBytes = 256;
 constexpr int EP_BYTES = 16384;  // epilogue staging: 4 warps x 4 KB (two bf16 or one fp32 32 x 32 block)
 constexpr size_t kSmemBytes = 1024 + STAGES * (B_BYTES + S_BYTES) + EP_BYTES + kBarBytes + sizeof(Group) * MAX_GROUPS;
@@ -222,8 +243,9 @@ __device__ __forceinline__ void convert(const Raw& raw, const uint8_t* sS, int s
   }
 }
 
-template <int FMT, bool BWD>
-__global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_constant__ Params p) {
+template <int FMT, bool BWD, bool SCHED>
+__global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_constant__ KParams<SCHED> kp) {
+  const Params& p = kp.p;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sB = smem;
@@ -284,6 +306,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_co
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int total = s_meta[0], ng = s_meta[1];
+  // this CTA's units: count, and the i-th one
+  int nu;
+  if constexpr (SCHED) {
+    nu = kp.s.off[blockIdx.x + 1] - kp.s.off[blockIdx.x];
+  } else {
+    nu = static_cast<int>(blockIdx.x) < total ? (total - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1 : 0;
+  }
+  auto unit_at = [&](int i) -> int {
+    if constexpr (SCHED) {
+      return kp.s.list[kp.s.off[blockIdx.x] + i];
+    } else {
+      return static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
+    }
+  };
   const int scale_rows = BWD ? (FMT == kFp8 ? 1 : (FMT == kInt4 ? WM / p.group : WM / 32)) : 0;
   const uint32_t s_tx = BWD ? static_cast<uint32_t>(FMT == kFp8 ? 64 * 4 : 64 * 2 * scale_rows) : 0u;
 
@@ -294,9 +330,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_co
       uint32_t ph = 0;
       long long issued = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+      for (int i = 0; i < nu && ok; ++i) {
         int g, tw, tt;
-        decode(sg, ng, u, g, tw, tt);
+        decode(sg, ng, unit_at(i), g, tw, tt);
         const Group& G = sg[g];
         const int nk = (G.kred + BK - 1) / BK;
         for (int ks = 0; ks < nk; ++ks) {
@@ -332,9 +368,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_co
       constexpr uint32_t idesc = idesc_bf16_f32(WM, TN);
       bool ok = true;
       long long gk = 0;  // k-steps of this CTA's earlier units
-      for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
+      for (int i = 0; i < nu && ok; ++i) {
         int g, tw, tt;
-        decode(sg, ng, u, g, tw, tt);
+        decode(sg, ng, unit_at(i), g, tw, tt);
         const int nk = (sg[g].kred + BK - 1) / BK;
         // Accumulator halves overlap with the epilogue at both ends of a unit: the first D
         // k-steps feed half 0 only while the epilogue still reads half 1 of the previous
@@ -428,9 +464,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_co
     uint8_t* ebuf = sE + q * (EP_BYTES / 4);
     int slot = 0;
     uint32_t acc_ph = 0;
-    for (int u = blockIdx.x; u < total; u += gridDim.x) {
+    for (int i = 0; i < nu; ++i) {
       int g, tw, tt;
-      decode(sg, ng, u, g, tw, tt);
+      decode(sg, ng, unit_at(i), g, tw, tt);
       const Group& G = sg[g];
       const int n0 = tw * WM + q * 32;  // first weight row of this warp's blocks
       const int m_base = tt * TP * TN;
@@ -502,11 +538,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_co
     // a cursor over this CTA's flattened (unit, k-step) sequence; the load cursor
     // runs PREFETCH of this warp's k-steps ahead of the decode cursor
     struct Cursor {
-      int u, ks, step, g, tw, tt, nk;
+      int i, ks, step, g, tw, tt, nk;  // i: index into this CTA's units
     };
     auto set_unit = [&](Cursor& c) {
-      if (c.u < total) {
-        decode(sg, ng, c.u, c.g, c.tw, c.tt);
+      if (c.i < nu) {
+        decode(sg, ng, unit_at(c.i), c.g, c.tw, c.tt);
         c.nk = (sg[c.g].kred + BK - 1) / BK;
       }
     };
@@ -514,19 +550,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_co
       ++c.step;
       if (++c.ks >= c.nk) {
         c.ks = 0;
-        c.u += gridDim.x;
+        ++c.i;
         set_unit(c);
       }
     };
     auto to_parity = [&](Cursor& c) {
-      if (c.u < total && (c.step & 1) != par) advance(c);
+      if (c.i < nu && (c.step & 1) != par) advance(c);
     };
-    Cursor ld{static_cast<int>(blockIdx.x), 0, 0, 0, 0, 0, 1};
+    Cursor ld{0, 0, 0, 0, 0, 0, 1};
     set_unit(ld);
     Cursor cv = ld;
     auto fetch = [&](Raw& raw) {
       to_parity(ld);
-      if (ld.u < total) {
+      if (ld.i < nu) {
         load_raw<FMT, BWD>(p, sg[ld.g], ld.tw, r, ld.ks, raw);
         advance(ld);
       }
@@ -535,7 +571,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_co
     // refill `cur`: the next loads stay off the path from a freed slot to a full one
     auto step_one = [&](Raw& cur) -> bool {
       to_parity(cv);
-      if (cv.u >= total) return false;
+      if (cv.i >= nu) return false;
       const int stage = cv.step % STAGES;
       const uint32_t ph = static_cast<uint32_t>((cv.step / STAGES) & 1);
       // the MMA that last read this A slot has completed

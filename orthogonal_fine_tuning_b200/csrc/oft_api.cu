@@ -7,7 +7,10 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
+#include <queue>
+#include <vector>
 #include <string>
 
 #include "oft.h"
@@ -404,21 +407,99 @@ int launch_gemm(const gemm::Params& prm, int total_tiles_hint, cudaStream_t st) 
   return OFT_OK;
 }
 
-template <int FMT, bool BWD>
-int launch_gemm_dq_t(const gdq::Params& prm, int tiles, cudaStream_t st) {
+int dq_tiles(int rows, int tokens) {
+  return ((rows + gdq::WM - 1) / gdq::WM) * (((tokens + gdq::TN - 1) / gdq::TN + gdq::TP - 1) / gdq::TP);
+}
+
+template <int FMT, bool BWD, bool SCHED>
+int launch_gemm_dq_k(const gdq::KParams<SCHED>& kp, int grid, cudaStream_t st) {
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    OFT_CUDA(cudaFuncSetAttribute(gdq::gemm_dq_kernel<FMT, BWD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    OFT_CUDA(cudaFuncSetAttribute(gdq::gemm_dq_kernel<FMT, BWD, SCHED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   static_cast<int>(gdq::kSmemBytes)));
     attr_set[dev] = true;
   }
-  const int grid = std::max(1, std::min(sm_count(), tiles));
   ProfScope ps(OFT_K_GEMM, st);
-  gdq::gemm_dq_kernel<FMT, BWD><<<grid, gdq::NUM_THREADS, gdq::kSmemBytes, st>>>(prm);
+  gdq::gemm_dq_kernel<FMT, BWD, SCHED><<<grid, gdq::NUM_THREADS, gdq::kSmemBytes, st>>>(kp);
   OFT_LAUNCHED("gemm_dq_kernel");
   return OFT_OK;
+}
+
+// Longest-first assignment of the launch's units to `grid` CTAs, each unit to the
+// least-loaded CTA (ties: lowest index); a CTA runs its units in ascending order.
+// Units are numbered as the kernel numbers them (groups in order, a group's units
+// token-pair-major).  Returns false when the launch does not need or fit one.
+bool build_schedule(const gdq::Params& prm, int grid, gdq::Sched& s) {
+  struct Cls {
+    int first, count, len;
+  };
+  std::vector<Cls> cls;
+  int u0 = 0;
+  bool mixed = false;
+  for (int g = 0; g < prm.num_groups; ++g) {
+    const gdq::Group& G = prm.groups[g];
+    if (G.rows <= 0 || G.tokens <= 0) continue;
+    const int n = dq_tiles(G.rows, G.tokens), len = (G.kred + gdq::BK - 1) / gdq::BK;
+    if (!cls.empty() && cls.back().len != len) mixed = true;
+    cls.push_back({u0, n, len});
+    u0 += n;
+  }
+  if (!mixed || u0 > gdq::kMaxSchedUnits || grid > gdq::kMaxSchedCtas) return false;
+  std::stable_sort(cls.begin(), cls.end(), [](const Cls& a, const Cls& b) { return a.len > b.len; });
+  using Load = std::pair<long long, int>;  // (k-steps, cta)
+  std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+  for (int b = 0; b < grid; ++b) heap.push({0ll, b});
+  std::vector<std::vector<int>> per(grid);
+  for (const Cls& c : cls)
+    for (int k = 0; k < c.count; ++k) {
+      Load l = heap.top();
+      heap.pop();
+      per[l.second].push_back(c.first + k);
+      l.first += c.len;
+      heap.push(l);
+    }
+  // keep round-robin (better L2 locality: all CTAs sweep the units together) unless
+  // the balanced schedule shortens the longest CTA by more than 5 %
+  long long lpt_max = 0;
+  while (!heap.empty()) {
+    lpt_max = std::max(lpt_max, heap.top().first);
+    heap.pop();
+  }
+  std::vector<int> len_of(u0);
+  for (const Cls& c : cls)
+    for (int k = 0; k < c.count; ++k) len_of[c.first + k] = c.len;
+  long long rr_max = 0;
+  for (int b = 0; b < grid; ++b) {
+    long long l = 0;
+    for (int u = b; u < u0; u += grid) l += len_of[u];
+    rr_max = std::max(rr_max, l);
+  }
+  if (lpt_max * 100 > rr_max * 95) return false;
+  int pos = 0;
+  for (int b = 0; b < grid; ++b) {
+    s.off[b] = static_cast<uint16_t>(pos);
+    std::sort(per[b].begin(), per[b].end());
+    for (int u : per[b]) s.list[pos++] = static_cast<uint16_t>(u);
+  }
+  s.off[grid] = static_cast<uint16_t>(pos);
+  return true;
+}
+
+template <int FMT, bool BWD>
+int launch_gemm_dq_t(const gdq::Params& prm, int tiles, cudaStream_t st) {
+  const int grid = std::max(1, std::min(sm_count(), tiles));
+  if (BWD) {
+    static thread_local gdq::KParams<true> kps;  // 25 KB: kept off the stack
+    if (build_schedule(prm, grid, kps.s)) {
+      kps.p = prm;
+      return launch_gemm_dq_k<FMT, BWD, true>(kps, grid, st);
+    }
+  }
+  gdq::KParams<false> kp;
+  kp.p = prm;
+  return launch_gemm_dq_k<FMT, BWD, false>(kp, grid, st);
 }
 
 int launch_gemm_dq(int fmt, bool bwd, const gdq::Params& prm, int tiles, cudaStream_t st) {
@@ -429,9 +510,6 @@ int launch_gemm_dq(int fmt, bool bwd, const gdq::Params& prm, int tiles, cudaStr
   return bwd ? launch_gemm_dq_t<gdq::kMxfp4, true>(prm, tiles, st) : launch_gemm_dq_t<gdq::kMxfp4, false>(prm, tiles, st);
 }
 
-int dq_tiles(int rows, int tokens) {
-  return ((rows + gdq::WM - 1) / gdq::WM) * (((tokens + gdq::TN - 1) / gdq::TN + gdq::TP - 1) / gdq::TP);
-}
 
 
 struct FwdLayout {

@@ -172,6 +172,21 @@ int make_map_f32_3d(CUtensorMap* m, const void* base, uint64_t K, uint64_t M, ui
   return OFT_OK;
 }
 
+// 3-D bf16 tensor [P][M][K] for TMA stores of 32-row x 64-column boxes, 128B swizzle:
+// stores clip at M within each split and at K.
+int make_map_bf16_3d_store(CUtensorMap* m, void* base, uint64_t K, uint64_t M, uint64_t P) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return fail(OFT_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[3] = {K, M, P};
+  cuuint64_t strides[2] = {K * 2, M * K * 2};
+  cuuint32_t box[3] = {64, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(OFT_ERR_CUDA, "cuTensorMapEncodeTiled (bf16 3-D store) failed (%d)", int(r));
+  return OFT_OK;
+}
+
 // Generic 2-D map without swizzle (scale tiles of the backward's dequant producers).
 int make_map_plain_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
                       uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer) {
@@ -314,6 +329,7 @@ int launch_rotate_fwd(const uint16_t* X, int M, int K, int P, int b, const float
   rtc::FwdParams prm;
   memset(&prm, 0, sizeof(prm));
   if (int rc = make_map_bf16(&prm.tmX, X, K, M, K, rtc::TM)) return rc;
+  if (int rc = make_map_bf16_3d_store(&prm.tmY, Xr, K, M, P)) return rc;
   prm.R = R;
   prm.Xr = Xr;
   prm.M = M;

@@ -62,6 +62,7 @@ __device__ __forceinline__ uint16_t bf16_rn(float v) { return f32_to_bf16_bits(v
 // ===========================================================================
 struct FwdParams {
   CUtensorMap tmX;  // X bf16 [M][K], box {64, 128}
+  CUtensorMap tmY;  // X' bf16 3-D {K, M, P}, box {64, 32, 1}, 128B swizzle (stores clip at M and K)
   const float* R;   // [P][nb][b][b]
   uint16_t* Xr;     // [P][M][K]
   int M, K, P, b, nb, groups, tiles_m;
@@ -69,7 +70,9 @@ struct FwdParams {
 
 constexpr int FWD_A_BYTES = TM * 64 * 2;           // 16 KB
 constexpr int FWD_BP_BYTES = 64 * 64 * 2;          // one 64x64 bf16 tile
-constexpr size_t kFwdSmem = 1024 + A_STAGES * FWD_A_BYTES + 2 * MAX_P * FWD_BP_BYTES + 256;
+constexpr int FWD_OUT_BYTES = 32 * 64 * 2;           // one staged 32-token x 64-column bf16 box
+constexpr int FWD_OUT_SLOTS = 2;                     // per epilogue warp
+constexpr size_t kFwdSmem = 1024 + A_STAGES * FWD_A_BYTES + 2 * MAX_P * FWD_BP_BYTES + 4 * FWD_OUT_SLOTS * FWD_OUT_BYTES + 256;
 
 // Named barrier over the 128 builder/epilogue threads (warps 2..5).
 __device__ __forceinline__ void builders_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
@@ -128,7 +131,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) rot_fwd_tc_kernel(const __grid
   uint8_t* sA = smem;
   uint8_t* sBhi = sA + A_STAGES * FWD_A_BYTES;
   uint8_t* sBlo = sBhi + MAX_P * FWD_BP_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sBlo + MAX_P * FWD_BP_BYTES);
+  uint8_t* sOut = sBlo + MAX_P * FWD_BP_BYTES;  // 1024-byte aligned: the store boxes are 128B-swizzled
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + 4 * FWD_OUT_SLOTS * FWD_OUT_BYTES);
   uint64_t* full = bars;
   uint64_t* empty = bars + A_STAGES;
   uint64_t* acc_full = bars + 2 * A_STAGES;
@@ -153,7 +157,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) rot_fwd_tc_kernel(const __grid
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) tma_prefetch_desc(&p.tmX);
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&p.tmX);
+    tma_prefetch_desc(&p.tmY);
+  }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
@@ -222,7 +229,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) rot_fwd_tc_kernel(const __grid
     }
   } else {
     const int q = warp & 3, tid = threadIdx.x - 64;
-    int acc = 0, cur_g = -1;
+    int acc = 0, cur_g = -1, out_slot = 0;
     uint32_t acc_ph = 0;
     for (int u = ubeg; u < uend; ++u) {
       const int g = u / p.tiles_m, mt = u % p.tiles_m;
@@ -234,8 +241,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) rot_fwd_tc_kernel(const __grid
       }
       if (!warp_wait(&acc_full[acc], acc_ph, abort_flag, kErrWaitAccFull)) break;
       tc_fence_after();
-      const int t = mt * TM + q * 32 + lane;
+      // Each warp owns 32 tokens: per split, its 32 x 64 bf16 block is staged in a
+      // 128B-swizzled slot (row = token, lane-private, conflict-free) and leaves by one
+      // TMA store, which clips tokens past M and columns past K.
       for (int sp = 0; sp < p.P; ++sp) {
+        uint8_t* slot = sOut + (q * FWD_OUT_SLOTS + out_slot) * FWD_OUT_BYTES;
+        if (lane == 0) bulk_wait_read<FWD_OUT_SLOTS - 1>();  // the store that last read this slot is done
+        __syncwarp();
 #pragma unroll 1
         for (int h = 0; h < 2; ++h) {
           uint32_t r[32];
@@ -243,23 +255,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) rot_fwd_tc_kernel(const __grid
           tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) +
                                  static_cast<uint32_t>(acc * 256 + sp * 64 + h * 32), r);
           tmem_ld_wait();
-          const int col = g * 64 + h * 32;
-          if (t < p.M && col < p.K) {
-            uint4* dst = reinterpret_cast<uint4*>(p.Xr + (static_cast<size_t>(sp) * p.M + t) * p.K + col);
 #pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * v]), __uint_as_float(r[8 * v + 1])),
-                                  pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3])),
-                                  pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5])),
-                                  pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7])));
-          }
+          for (int v = 0; v < 4; ++v)
+            *reinterpret_cast<uint4*>(slot + swz(lane, h * 4 + v)) =
+                make_uint4(pack_bf16x2(__uint_as_float(r[8 * v]), __uint_as_float(r[8 * v + 1])),
+                           pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3])),
+                           pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5])),
+                           pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7])));
         }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&p.tmY, slot, g * 64, mt * TM + q * 32, sp);
+          bulk_commit();
+        }
+        out_slot = (out_slot + 1) % FWD_OUT_SLOTS;
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[acc]);
       acc ^= 1;
       if (acc == 0) acc_ph ^= 1;
     }
+    if (lane == 0) bulk_wait_all();  // the staged blocks are read (and written) before the CTA exits
+    __syncwarp();
   }
   __syncthreads();
   if (warp == 1) {

@@ -166,6 +166,14 @@ int oft_rotate(const uint16_t* X, int M, int K, int P, int b, const float* R, ui
  * R, G fp32 [n_blocks][b][b]; dQ fp32 [n_blocks][b(b-1)/2]. */
 int oft_cayley_backward(const float* R, const float* G, int n_blocks, int b, float* dQ, void* stream);
 
+/* Selects the kernel of the fused-dequant GEMM inside oft_linear_fwd / oft_linear_bwd
+ * (test and benchmarking hook; process-wide, not thread-safe against concurrent
+ * calls): 0 = by problem size (default: the 2-SM pair kernel for launches of at
+ * least two waves of one-CTA tiles), 1 = always the one-CTA kernel, 2 = always the
+ * 2-SM pair kernel.  Both compute the same product.  Returns OFT_ERR_INVALID_ARG
+ * for any other value. */
+int oft_set_gemm_mode(int mode);
+
 /* Launches a kernel that waits on a barrier nothing will complete, bounded by
  * timeout_us microseconds; it must return on its own and set the device error
  * word.  Exercises the timeout path without faulting or hanging the GPU. */

@@ -20,6 +20,7 @@ from .binding import (  # noqa: F401
     oft_linear_fwd_noalloc,
     oft_linear_fwd_workspace,
     oft_rotate,
+    oft_set_gemm_mode,
     profile,
     version,
 )

@@ -25,7 +25,7 @@ EXPORTS = (
     "oft_linear_fwd_workspace", "oft_linear_fwd", "oft_linear_bwd_workspace", "oft_linear_bwd",
     "moe_chunked_oft_workspace", "moe_chunked_oft_fwd", "oft_dequant_weight", "oft_rotate",
     "oft_cayley_backward", "oft_debug_bounded_wait", "oft_profile_begin", "oft_profile_end",
-    "oft_linear_fwd_noalloc",
+    "oft_linear_fwd_noalloc", "oft_set_gemm_mode",
 )
 
 
@@ -60,6 +60,7 @@ _SIGS = {
     "oft_rotate": (_I, [_P, _I, _I, _I, _I, _P, _P, _P]),
     "oft_cayley_backward": (_I, [_P, _P, _I, _I, _P, _P]),
     "oft_debug_bounded_wait": (_I, [_I, _P]),
+    "oft_set_gemm_mode": (_I, [_I]),
     "oft_linear_fwd_noalloc": (_I, [_P, _I, _WP, _SP, _I, _P, _P, _P]),
     "oft_profile_begin": (_I, [_I]),
     "oft_profile_end": (_I, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int), _I,

@@ -219,6 +219,12 @@ def oft_cayley_backward(R: torch.Tensor, G: torch.Tensor, b: int, out: Optional[
     return out
 
 
+def oft_set_gemm_mode(mode: int) -> None:
+    """Fused-dequant GEMM kernel inside the linear calls: 0 by size (default),
+    1 the one-CTA kernel, 2 the 2-SM pair kernel (same product)."""
+    _check(_L.oft_set_gemm_mode(int(mode)))
+
+
 def oft_debug_bounded_wait(timeout_us: int, stream=None) -> None:
     _check(_L.oft_debug_bounded_wait(int(timeout_us), _stream(stream)))
 

@@ -125,9 +125,16 @@ __device__ __forceinline__ void load_raw(const Params& p, const Group& G, int tw
   constexpr int PER = (FMT == kFp8) ? 4 : 8;   // codes per word
   const int k0 = ks * BK;
   if (BWD) {
-    // packed blocks: zero codes pad every row and k-step, so no bounds tests; the
-    // warp's 32 rows read 512 contiguous bytes per vector
+    // packed blocks: zero codes pad every row and k-step of the existing row tiles;
+    // the warp's 32 rows read 512 contiguous bytes per vector.  A 256-row pair unit
+    // may reach one 128-row tile past the last: it decodes zeros.
     constexpr int NV4 = NW / 4;
+    if (tw * WM >= G.rows) {
+#pragma unroll
+      for (int i = 0; i < NW; ++i) raw.c[i] = 0;
+      raw.sc = 0;
+      return;
+    }
     const int nk = (G.kred + BK - 1) / BK;
     const uint4* src = reinterpret_cast<const uint4*>(p.codes + G.code_off) +
                        (static_cast<size_t>(tw) * nk + ks) * (NV4 * WM) + r;
@@ -574,12 +581,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_co
       if (cv.i >= nu) return false;
       const int stage = cv.step % STAGES;
       const uint32_t ph = static_cast<uint32_t>((cv.step / STAGES) & 1);
-      // the MMA that last read this A slot has completed
-      if (!warp_wait_bounded(&empty[stage], ph ^ 1, abort_flag, kErrWaitEmpty)) return false;
-      if (BWD && !warp_wait_bounded(&full_b[stage], ph, abort_flag, kErrWaitFull)) return false;
+      // Forward: decode first, then wait for the MMA that last read this A slot and only
+      // store.  Backward: the scale tile of this step lands after the slot is free
+      // (same stage), so wait for it, then decode.
       uint32_t o[32];
       const int srow = BWD ? ((FMT == kFp8) ? 0 : r / (FMT == kInt4 ? p.group : 32)) : 0;
-      convert<FMT, BWD>(cur, sS + stage * S_BYTES, srow, o);
+      if (BWD) {
+        if (!warp_wait_bounded(&empty[stage], ph ^ 1, abort_flag, kErrWaitEmpty)) return false;
+        if (!warp_wait_bounded(&full_b[stage], ph, abort_flag, kErrWaitFull)) return false;
+        convert<FMT, BWD>(cur, sS + stage * S_BYTES, srow, o);
+      } else {
+        convert<FMT, BWD>(cur, sS + stage * S_BYTES, srow, o);
+        if (!warp_wait_bounded(&empty[stage], ph ^ 1, abort_flag, kErrWaitEmpty)) return false;
+      }
       __syncwarp();
       tmem_st_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + A_COL0 + static_cast<uint32_t>(stage * 32), o);
       tmem_st_wait();

@@ -22,6 +22,7 @@
 #include "moe.cuh"
 #include "rot_tc.cuh"
 #include "gemm_dq.cuh"
+#include "gemm_dq2.cuh"
 
 using namespace oftk;
 
@@ -423,9 +424,15 @@ int launch_gemm(const gemm::Params& prm, int total_tiles_hint, cudaStream_t st) 
   return OFT_OK;
 }
 
-int dq_tiles(int rows, int tokens) {
-  return ((rows + gdq::WM - 1) / gdq::WM) * (((tokens + gdq::TN - 1) / gdq::TN + gdq::TP - 1) / gdq::TP);
+// Work units of the fused-dequant GEMM for one group: weight-row tiles (128 rows for the
+// one-CTA kernel, 256 for the 2-SM pair) x token-tile pairs (2 x 192 tokens; 2 x 160 for the pair).
+int dq_tiles(int rows, int tokens, int unit_rows = gdq::WM) {
+  const int tn = unit_rows == gdq2::UROWS ? gdq2::TN : gdq::TN;
+  return ((rows + unit_rows - 1) / unit_rows) * (((tokens + tn - 1) / tn + gdq::TP - 1) / gdq::TP);
 }
+
+// 0: choose by size; 1: always the one-CTA kernel; 2: always the 2-SM pair kernel.
+int g_gemm_mode = 0;
 
 template <int FMT, bool BWD, bool SCHED>
 int launch_gemm_dq_k(const gdq::KParams<SCHED>& kp, int grid, cudaStream_t st) {
@@ -447,7 +454,7 @@ int launch_gemm_dq_k(const gdq::KParams<SCHED>& kp, int grid, cudaStream_t st) {
 // least-loaded CTA (ties: lowest index); a CTA runs its units in ascending order.
 // Units are numbered as the kernel numbers them (groups in order, a group's units
 // token-pair-major).  Returns false when the launch does not need or fit one.
-bool build_schedule(const gdq::Params& prm, int grid, gdq::Sched& s) {
+bool build_schedule(const gdq::Params& prm, int grid, gdq::Sched& s, int unit_rows = gdq::WM) {
   struct Cls {
     int first, count, len;
   };
@@ -457,7 +464,7 @@ bool build_schedule(const gdq::Params& prm, int grid, gdq::Sched& s) {
   for (int g = 0; g < prm.num_groups; ++g) {
     const gdq::Group& G = prm.groups[g];
     if (G.rows <= 0 || G.tokens <= 0) continue;
-    const int n = dq_tiles(G.rows, G.tokens), len = (G.kred + gdq::BK - 1) / gdq::BK;
+    const int n = dq_tiles(G.rows, G.tokens, unit_rows), len = (G.kred + gdq::BK - 1) / gdq::BK;
     if (!cls.empty() && cls.back().len != len) mixed = true;
     cls.push_back({u0, n, len});
     u0 += n;
@@ -518,6 +525,80 @@ int launch_gemm_dq_t(const gdq::Params& prm, int tiles, cudaStream_t st) {
   return launch_gemm_dq_k<FMT, BWD, false>(kp, grid, st);
 }
 
+template <int FMT, bool BWD, bool SCHED>
+int launch_gemm_dq2_k(const gdq::KParams<SCHED>& kp, int clusters, cudaStream_t st) {
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    OFT_CUDA(cudaFuncSetAttribute(gdq2::gemm_dq2_kernel<FMT, BWD, SCHED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(gdq2::kSmemBytes)));
+    attr_set[dev] = true;
+  }
+  ProfScope ps(OFT_K_GEMM, st);
+  gdq2::gemm_dq2_kernel<FMT, BWD, SCHED><<<2 * clusters, gdq2::NUM_THREADS, gdq2::kSmemBytes, st>>>(kp);
+  OFT_LAUNCHED("gemm_dq2_kernel");
+  return OFT_OK;
+}
+
+// Number of 2-CTA clusters of the pair kernel that fit on the device at once (cached).
+int pair_clusters_resident() {
+  static int cached[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+  int n = 0;
+  cudaFuncSetAttribute(gdq2::gemm_dq2_kernel<gdq::kInt4, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       static_cast<int>(gdq2::kSmemBytes));
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(2 * sm_count());
+  cfg.blockDim = dim3(gdq2::NUM_THREADS);
+  cfg.dynamicSmemBytes = gdq2::kSmemBytes;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = 2;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  if (cudaOccupancyMaxActiveClusters(&n, gdq2::gemm_dq2_kernel<gdq::kInt4, false, false>, &cfg) != cudaSuccess || n <= 0)
+    n = sm_count() / 2;
+  cudaGetLastError();
+  if (dev >= 0 && dev < 64) cached[dev] = n;
+  return n;
+}
+
+template <int FMT, bool BWD>
+int launch_gemm_dq2_t(const gdq::Params& prm, int units, cudaStream_t st) {
+  const int clusters = std::max(1, std::min(pair_clusters_resident(), units));
+  if (BWD) {
+    static thread_local gdq::KParams<true> kps;
+    if (build_schedule(prm, clusters, kps.s, gdq2::UROWS)) {
+      kps.p = prm;
+      return launch_gemm_dq2_k<FMT, BWD, true>(kps, clusters, st);
+    }
+  }
+  gdq::KParams<false> kp;
+  kp.p = prm;
+  return launch_gemm_dq2_k<FMT, BWD, false>(kp, clusters, st);
+}
+
+// Pair kernel for launches of at least two one-CTA waves (unless forced).
+bool use_pair(int tiles_one_cta) {
+  if (g_gemm_mode == 1) return false;
+  if (g_gemm_mode == 2) return true;
+  return tiles_one_cta >= 2 * sm_count();
+}
+
+int launch_gemm_dq2(int fmt, bool bwd, const gdq::Params& prm, int units, cudaStream_t st) {
+  if (fmt == OFT_W_INT4) return bwd ? launch_gemm_dq2_t<gdq::kInt4, true>(prm, units, st)
+                                    : launch_gemm_dq2_t<gdq::kInt4, false>(prm, units, st);
+  if (fmt == OFT_W_FP8) return bwd ? launch_gemm_dq2_t<gdq::kFp8, true>(prm, units, st)
+                                   : launch_gemm_dq2_t<gdq::kFp8, false>(prm, units, st);
+  return bwd ? launch_gemm_dq2_t<gdq::kMxfp4, true>(prm, units, st) : launch_gemm_dq2_t<gdq::kMxfp4, false>(prm, units, st);
+}
+
 int launch_gemm_dq(int fmt, bool bwd, const gdq::Params& prm, int tiles, cudaStream_t st) {
   if (fmt == OFT_W_INT4) return bwd ? launch_gemm_dq_t<gdq::kInt4, true>(prm, tiles, st)
                                     : launch_gemm_dq_t<gdq::kInt4, false>(prm, tiles, st);
@@ -573,6 +654,12 @@ extern "C" {
 const char* oft_version(void) { return "oft-b200 0.1 (sm_100a, tcgen05)"; }
 
 const char* oft_last_error(void) { return g_last_error.c_str(); }
+
+int oft_set_gemm_mode(int mode) {
+  if (mode < 0 || mode > 2) return fail(OFT_ERR_INVALID_ARG, "gemm mode must be 0, 1 or 2");
+  g_gemm_mode = mode;
+  return OFT_OK;
+}
 
 int oft_check_device(void* stream) {
   OFT_CUDA(cudaStreamSynchronize(as_stream(stream)));
@@ -646,9 +733,15 @@ int oft_linear_fwd(const uint16_t* X, int M, const oft_weight* W, const oft_spli
   if (int rc = launch_rotate_fwd(X, M, K, P, b, R, Xr, st)) return rc;
 
   // Y[:, cols of p] = X'_p deq(W_p): dequant fused into the GEMM's weight operand
+  int tiles1 = 0, units2 = 0;
+  for (int p = 0; p < P; ++p) {
+    tiles1 += dq_tiles(S->sizes[p], M);
+    units2 += dq_tiles(S->sizes[p], M, gdq2::UROWS);
+  }
+  const bool pair = use_pair(tiles1);
   gdq::Params prm;
   memset(&prm, 0, sizeof(prm));
-  if (int rc = make_map_bf16(&prm.tmB[0], Xr, K, 1ull * P * M, K, gdq::TN)) return rc;
+  if (int rc = make_map_bf16(&prm.tmB[0], Xr, K, 1ull * P * M, K, pair ? gdq2::TNC : gdq::TN)) return rc;
   for (int i = 1; i < gdq::MAX_GROUPS; ++i) prm.tmB[i] = prm.tmB[0];
   prm.codes = static_cast<const uint8_t*>(W->codes);
   prm.code_row_bytes = W->fmt == OFT_W_FP8 ? K : K / 2;
@@ -657,7 +750,7 @@ int oft_linear_fwd(const uint16_t* X, int M, const oft_weight* W, const oft_spli
   prm.K = K;
   prm.group = W->fmt == OFT_W_INT4 ? W->group : 32;
   prm.num_groups = P;
-  int off = 0, tiles = 0;
+  int off = 0;
   for (int p = 0; p < P; ++p) {
     gdq::Group& g = prm.groups[p];
     g.rows = S->sizes[p];
@@ -673,9 +766,8 @@ int oft_linear_fwd(const uint16_t* X, int M, const oft_weight* W, const oft_spli
                                    32, 32))
       return rc;
     off += S->sizes[p];
-    tiles += dq_tiles(g.rows, M);
   }
-  return launch_gemm_dq(W->fmt, false, prm, tiles, st);
+  return pair ? launch_gemm_dq2(W->fmt, false, prm, units2, st) : launch_gemm_dq(W->fmt, false, prm, tiles1, st);
 }
 
 size_t oft_linear_bwd_workspace(int M, const oft_weight* W, const oft_split* S, int b) {
@@ -762,10 +854,12 @@ int oft_linear_bwd(const uint16_t* dY, const uint16_t* X, int M, const oft_weigh
     if (int rc = make_map_plain_2d(&prm.tmS, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, W->scales, N, 1, 4ull * N, 64, 1))
       return rc;
   }
-  int off = 0, tiles = 0;
+  const int tiles1 = P * dq_tiles(K, M), units2 = P * dq_tiles(K, M, gdq2::UROWS);
+  const bool pair = use_pair(tiles1);
+  int off = 0;
   for (int p = 0; p < P; ++p) {
     const int Np = S->sizes[p];
-    if (int rc = make_map_bf16(&prm.tmB[p], dY + off, Np, M, N, gdq::TN)) return rc;
+    if (int rc = make_map_bf16(&prm.tmB[p], dY + off, Np, M, N, pair ? gdq2::TNC : gdq::TN)) return rc;
     gdq::Group& g = prm.groups[p];
     g.rows = K;
     g.tokens = M;
@@ -780,7 +874,6 @@ int oft_linear_bwd(const uint16_t* dY, const uint16_t* X, int M, const oft_weigh
                                    4ull * K, 32, 32))
       return rc;
     off += Np;
-    tiles += dq_tiles(K, M);
   }
   for (int p = P; p < gdq::MAX_GROUPS; ++p) prm.tmB[p] = prm.tmB[0];
   prm.codes = codes_t;
@@ -790,7 +883,8 @@ int oft_linear_bwd(const uint16_t* dY, const uint16_t* X, int M, const oft_weigh
   prm.K = K;
   prm.group = G;
   prm.num_groups = P;
-  if (int rc = launch_gemm_dq(W->fmt, true, prm, tiles, st)) return rc;
+  if (int rc = pair ? launch_gemm_dq2(W->fmt, true, prm, units2, st) : launch_gemm_dq(W->fmt, true, prm, tiles1, st))
+    return rc;
 
   if (int rc = launch_rotate_bwd(dXr, M, K, P, b, R, dX, st)) return rc;
   if (int rc = launch_grad(X, dXr, M, K, P, b, Gp, st)) return rc;

@@ -45,8 +45,16 @@ SMALL = [
 ]
 
 
+@pytest.fixture(params=[1, 2], ids=["one-cta", "pair"])
+def gemm_mode(oft, request):
+    """Both fused-dequant GEMM kernels: the one-CTA kernel and the 2-SM pair."""
+    oft.oft_set_gemm_mode(request.param)
+    yield request.param
+    oft.oft_set_gemm_mode(0)
+
+
 @pytest.mark.parametrize("name,M,K,splits,fmt,group,b", SMALL, ids=[s[0] for s in SMALL])
-def test_small_fwd_bwd(oft, name, M, K, splits, fmt, group, b):
+def test_small_fwd_bwd(oft, gemm_mode, name, M, K, splits, fmt, group, b):
     spec = LinearSpec(name, M=M, K=K, splits=splits, fmt=fmt, group=group, b=b, q_sigma=0.05,
                       w_mode="codes" if name == "c0" else "normal", backward=True, seed=len(name) + M)
     case = make_linear_case(spec)

@@ -270,9 +270,9 @@ def gemm_traffic(flops_per_launch_unit):
 
 
 def gemm_kernel_hash() -> str:
-    """Hash of the fused-dequant GEMM's device sources (the kernel and its decoders)."""
+    """Hash of the fused-dequant GEMMs' device sources (both kernels and their decoders)."""
     h = hashlib.sha256()
-    for f in ("gemm_dq.cuh", "dq_pack.cuh"):
+    for f in ("gemm_dq.cuh", "gemm_dq2.cuh", "dq_pack.cuh"):
         with open(os.path.join(ROOT, "orthogonal_fine_tuning_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -401,7 +401,10 @@ def run_ours(args, rank, world):
         peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
         unit = "TFLOP/s"
         traffic = gemm_traffic(name)
-        kernel = "gemm_dq_kernel (fused dequant, tcgen05/TMEM)"
+        # the library picks the 2-SM pair kernel for launches of two or more one-CTA waves
+        tiles1 = sum(-(-n // 128) for n in spec.splits) * (-(-(-(-spec.M // 192)) // 2))
+        kernel = ("gemm_dq2_kernel (fused dequant, 2-SM pair, tcgen05 cta_group::2)" if tiles1 >= 2 * 148
+                  else "gemm_dq_kernel (fused dequant, tcgen05/TMEM)")
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
                 "traffic": traffic, "kernel": kernel,
                 "peak_source": f"{peak_src} ({'sustained' if bound == 'tensor' else 'copy'})"}

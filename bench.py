@@ -302,12 +302,18 @@ def run_ours(args, rank, world):
         tokens = spec.T
         backward = False
 
-        def step(Xi=X, Li=logits, Qi=Q):
-            oft.moe_chunked_oft_fwd(Xi, Li, W, spec.b, Qi, spec.top_k, spec.chunk, workspace=ws, out=out)
-            return out["Y"]
+        def new_outputs():
+            o = oft.moe_chunked_oft_fwd(X, logits, W, spec.b, Q, spec.top_k, spec.chunk, workspace=ws)
+            return o
+
+        def step(Xi=X, Li=logits, Qi=Q, o=None):
+            o = out if o is None else o
+            oft.moe_chunked_oft_fwd(Xi, Li, W, spec.b, Qi, spec.top_k, spec.chunk, workspace=ws, out=o)
+            return o["Y"]
 
         inputs = dict(X=X, logits=logits, Q=Q)
         outputs = dict(Y=out["Y"])
+        result_keys = ("Y",)
     else:
         spec = LINEAR_CONFIGS[name]
         backward = spec.backward
@@ -325,16 +331,21 @@ def run_ours(args, rank, world):
         dQ = torch.empty(spec.P, spec.K // spec.b, spec.b * (spec.b - 1) // 2, dtype=torch.float32, device=dev)
         tokens = spec.M
 
-        def step(Xi=X, dYi=dY, Qi=Q):
+        def new_outputs():
+            return dict(Y=torch.empty_like(Y), dX=torch.empty_like(dX), dQ=torch.empty_like(dQ))
+
+        def step(Xi=X, dYi=dY, Qi=Q, o=None):
+            o = dict(Y=Y, dX=dX, dQ=dQ) if o is None else o
             oft.oft_build_rotation(Qi, spec.b, R=R)
-            oft.oft_linear_fwd(Xi, W, spec.splits, spec.b, R, Y=Y, workspace=ws)
+            oft.oft_linear_fwd(Xi, W, spec.splits, spec.b, R, Y=o["Y"], workspace=ws)
             if backward:
-                oft.oft_linear_bwd(dYi, Xi, W, spec.splits, spec.b, R, dX=dX, dQ=dQ, workspace=ws)
-                allreduce_grad(dQ)
-            return Y
+                oft.oft_linear_bwd(dYi, Xi, W, spec.splits, spec.b, R, dX=o["dX"], dQ=o["dQ"], workspace=ws)
+                allreduce_grad(o["dQ"])
+            return o["Y"]
 
         inputs = dict(X=X, Q=Q) if not backward else dict(X=X, dY=dY, Q=Q)
         outputs = dict(Y=Y) if not backward else dict(Y=Y, dX=dX, dQ=dQ)
+        result_keys = tuple(outputs)
 
     # ---- device-resident timing ----
     for _ in range(args.warmup):
@@ -410,40 +421,69 @@ def run_ours(args, rank, world):
                 "peak_source": f"{peak_src} ({'sustained' if bound == 'tensor' else 'copy'})"}
 
     # ---- end to end through the public API with host buffers ----
+    # Every step copies its own inputs from pinned host memory and reads all of its
+    # outputs back into pinned host memory.  Copies in, compute and copies out run on
+    # three streams, double-buffered, so step i's read-back and step i+1's upload
+    # overlap step i+1's / step i's compute (one step in flight on each engine).
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
     host_in = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in inputs.items()}
     for k, v in inputs.items():
         host_in[k].copy_(v)
-    host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in outputs.items()}
-    dev_in = {k: torch.empty_like(v) for k, v in inputs.items()}
+    dev_in = [{k: torch.empty_like(v) for k, v in inputs.items()} for _ in range(2)]
+    dev_out = [new_outputs() for _ in range(2)]
+    host_out = [{k: torch.empty(dev_out[b][k].shape, dtype=dev_out[b][k].dtype, pin_memory=True)
+                 for k in result_keys} for b in range(2)]
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    for b in range(2):  # all buffers free at the start
+        ev_comp[b].record(comp)
+        ev_out[b].record(comp)
 
-    def e2e_step():
-        for k in dev_in:
-            dev_in[k].copy_(host_in[k], non_blocking=True)
+    def e2e_step(i):
+        b = i % 2
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(ev_comp[b])          # compute of step i-2 is done with dev_in[b]
+            for k in dev_in[b]:
+                dev_in[b][k].copy_(host_in[k], non_blocking=True)
+            ev_in[b].record(s_in)
+        comp.wait_event(ev_in[b])
+        comp.wait_event(ev_out[b])               # read-back of step i-2 is done with dev_out[b]
+        d = dev_in[b]
         if is_moe:
-            step(dev_in["X"], dev_in["logits"], dev_in["Q"])
+            step(d["X"], d["logits"], d["Q"], o=dev_out[b])
         elif backward:
-            step(dev_in["X"], dev_in["dY"], dev_in["Q"])
+            step(d["X"], d["dY"], d["Q"], o=dev_out[b])
         else:
-            step(dev_in["X"], None, dev_in["Q"])
-        for k in host_out:
-            host_out[k].copy_(outputs[k], non_blocking=True)
+            step(d["X"], None, d["Q"], o=dev_out[b])
+        ev_comp[b].record(comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_comp[b])
+            for k in result_keys:
+                host_out[b][k].copy_(dev_out[b][k], non_blocking=True)
+            ev_out[b].record(s_out)
 
-    for _ in range(args.warmup):
-        e2e_step()
+    for i in range(args.warmup):
+        e2e_step(i)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    es.record()
-    for _ in range(args.steps):
-        e2e_step()
-    ee.record()
+    es.record(comp)
+    s_in.wait_event(es)
+    for i in range(args.steps):
+        e2e_step(i)
+    for b in range(2):
+        comp.wait_event(ev_out[b])
+    ee.record(comp)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(es.elapsed_time(ee) / args.steps, dev)
     h2d = sum(v.numel() * v.element_size() for v in host_in.values())
-    d2h = sum(v.numel() * v.element_size() for v in host_out.values())
+    d2h = sum(v.numel() * v.element_size() for v in host_out[0].values())
     e2e = {"value": tokens * world / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+           "pipelining": "double-buffered: upload, compute and read-back on three streams"}
 
     if rank != 0:
         return None

@@ -223,6 +223,198 @@ __global__ void __launch_bounds__(kGatherThreads) moe_gather_rotate_kernel(
   }
 }
 
+// Rotated gather on the tensor cores: Xg[proj][pos][:] = X[bucket[pos] / k] R_{e,proj}.
+// Units are (active expert, 64-column group, 128-position tile of that expert's
+// bucket rows), in that order with the tile fastest, so a tile never mixes experts
+// and consecutive units of a CTA share the expert's rotation tiles.  A CTA (128
+// threads, four resident per SM) walks a contiguous range of units:
+//   gather the tile's 128 activation rows (64 bf16 columns) into a 128B-swizzled
+//   K-major tile; on an (expert, group) change rebuild B[p*64 + c][i] =
+//   R_{e,p}[i][c] over the group's diagonal blocks for p = gate, up, split into
+//   bf16 hi + lo; one thread issues 8 tcgen05.mma (M = 128, N = 128, K = 64 as
+//   4 x 16, hi and lo) into TMEM; the epilogue writes the tile's valid rows.
+// The rotation of activations in front of the frozen weight is the OFT adapter
+// ("Orbit", chooseai.io news 4086, section "技术原理：低精度基座 + BF16 适配器 + OFT");
+// the per-expert split into gate and up is its split-projection form (item
+// "自定义适配器核函数").
+constexpr int kMoeRotThreads = 128;
+constexpr size_t kMoeRotSmem = 1024 + 3 * 16384 + 64;
+
+template <int B>
+__global__ void __launch_bounds__(kMoeRotThreads) moe_rot_tc_kernel(
+    const uint16_t* __restrict__ X, int K, int top_k, const int* __restrict__ bucket,
+    const int* __restrict__ offsets, const int* __restrict__ active, const int* __restrict__ n_active_p,
+    const float* __restrict__ Rex, int TK, uint16_t* __restrict__ Xg) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;                 // 128 positions x 64 columns, bf16, 128B swizzle
+  uint8_t* sBhi = sA + 16384;         // 128 (gate|up output columns) x 64, bf16 hi
+  uint8_t* sBlo = sBhi + 16384;       // lo
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sBlo + 16384);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  __shared__ int s_pref[kMaxExperts + 1];  // units before active expert a
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int G = (K + 63) / 64, nb = K / B;
+  const int na = *n_active_p;
+  if (warp == 0) {
+    // prefix over active experts of (position tiles x column groups), one warp
+    int carry = 0;
+    for (int a0 = 0; a0 < na; a0 += 32) {
+      const int a = a0 + lane;
+      int v = 0;
+      if (a < na) {
+        const int e = active[a];
+        v = ((offsets[e + 1] - offsets[e] + 127) / 128) * G;
+      }
+      int x = v;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, x, d);
+        if (lane >= d) x += y;
+      }
+      if (a < na) s_pref[a + 1] = carry + x;
+      carry += __shfl_sync(0xFFFFFFFFu, x, 31);
+    }
+    if (lane == 0) s_pref[0] = 0;
+  }
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int total = s_pref[na];
+  const int per = total / static_cast<int>(gridDim.x), rem = total % static_cast<int>(gridDim.x);
+  const int ubeg = static_cast<int>(blockIdx.x) * per + min(static_cast<int>(blockIdx.x), rem);
+  const int uend = ubeg + per + (static_cast<int>(blockIdx.x) < rem ? 1 : 0);
+  constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
+  int cur_e = -1, cur_g = -1, a = 0;
+  uint32_t phase = 0;
+  for (int u = ubeg; u < uend; ++u) {
+    while (a + 1 < na && s_pref[a + 1] <= u) ++a;  // units are visited in increasing order
+    const int e = active[a];
+    const int pos_beg = offsets[e], n_e = offsets[e + 1] - pos_beg;
+    const int tiles = (n_e + 127) / 128;
+    const int local = u - s_pref[a];
+    const int g = local / tiles, rt = local % tiles;
+    const int pos0 = pos_beg + rt * 128, nrows = min(128, n_e - rt * 128);
+    // 1. rotation tiles of (e, g), when they change (the previous unit's MMAs have completed)
+    if (e != cur_e || g != cur_g) {
+      for (int v = tid; v < 16384 / 16; v += kMoeRotThreads) {  // each tile is 16 KB
+        reinterpret_cast<uint4*>(sBhi)[v] = make_uint4(0, 0, 0, 0);
+        reinterpret_cast<uint4*>(sBlo)[v] = make_uint4(0, 0, 0, 0);
+      }
+      __syncthreads();
+      constexpr int PER = 16 * B;  // float4s of one projection's diagonal blocks in the group
+      constexpr int NIT = 2 * PER / kMoeRotThreads;  // b / 4 per thread: all loads in flight first
+      float4 rv[NIT];
+#pragma unroll
+      for (int q = 0; q < NIT; ++q) {
+        const int f = tid + q * kMoeRotThreads;
+        const int pr = f / PER, rem4 = f % PER;
+        const int jb = rem4 / (B * B / 4), w = rem4 % (B * B / 4);
+        const int i = w / (B / 4), c4 = (w % (B / 4)) * 4;
+        const int j = (g * 64) / B + jb;
+        rv[q] = (j + 1) * B <= K ? *reinterpret_cast<const float4*>(
+                                       Rex + (((static_cast<size_t>(e) * 2 + pr) * nb + j) * B + i) * B + c4)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int q = 0; q < NIT; ++q) {
+        const int f = tid + q * kMoeRotThreads;
+        const int pr = f / PER, rem4 = f % PER;
+        const int jb = rem4 / (B * B / 4), w = rem4 % (B * B / 4);
+        const int i = w / (B / 4), c4 = (w % (B / 4)) * 4;
+        const float ev[4] = {rv[q].x, rv[q].y, rv[q].z, rv[q].w};
+        const int k = jb * B + i;  // reduction index within the group
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int r = pr * 64 + jb * B + c4 + t;  // output column (gate 0..63, up 64..127)
+          const uint32_t off = sw128_offset(static_cast<uint32_t>(r), static_cast<uint32_t>(k >> 3)) + (k & 7) * 2;
+          const uint16_t h = f32_to_bf16_bits(ev[t]);
+          *reinterpret_cast<uint16_t*>(sBhi + off) = h;
+          *reinterpret_cast<uint16_t*>(sBlo + off) = f32_to_bf16_bits(ev[t] - bf16_bits_to_f32(h));
+        }
+      }
+      cur_e = e;
+      cur_g = g;
+    }
+    // 2. gather the tile's activation rows: the 8 loads of each thread are all in flight
+    //    before any of them is stored
+    {
+      constexpr int NIT = 128 * 8 / kMoeRotThreads;
+      uint4 xv[NIT];
+#pragma unroll
+      for (int q = 0; q < NIT; ++q) {
+        const int it = tid + q * kMoeRotThreads, r = it >> 3, col = g * 64 + (it & 7) * 8;
+        xv[q] = make_uint4(0, 0, 0, 0);
+        if (r < nrows && col < K)
+          xv[q] = *reinterpret_cast<const uint4*>(X + static_cast<size_t>(bucket[pos0 + r] / top_k) * K + col);
+      }
+#pragma unroll
+      for (int q = 0; q < NIT; ++q) {
+        const int it = tid + q * kMoeRotThreads;
+        *reinterpret_cast<uint4*>(sA + sw128_offset(static_cast<uint32_t>(it >> 3), static_cast<uint32_t>(it & 7))) = xv[q];
+      }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    // 3. the product
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t a0 = smem_u32(sA), bh = smem_u32(sBhi), bl = smem_u32(sBlo);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t ad = sdesc_sw128(a0 + kk * 32, 16, 1024);
+        mma_bf16_ss(tmem, ad, sdesc_sw128(bh + kk * 32, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+        mma_bf16_ss(tmem, ad, sdesc_sw128(bl + kk * 32, 16, 1024), idesc, 1u);
+      }
+      mma_commit(bar);
+    }
+    if (!warp_wait_bounded(bar, phase, abort_flag, kErrWaitAccFull)) break;
+    phase ^= 1;
+    tc_fence_after();
+    // 4. epilogue: TMEM lane = position row, 64 columns per projection
+    const int r = warp * 32 + lane;
+#pragma unroll 1
+    for (int pr = 0; pr < 2; ++pr) {
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        uint32_t v[32];
+        __syncwarp();
+        tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(pr * 64 + h * 32), v);
+        tmem_ld_wait();
+        const int col = g * 64 + h * 32;
+        if (r < nrows) {
+          uint4* dst = reinterpret_cast<uint4*>(Xg + (static_cast<size_t>(pr) * TK + pos0 + r) * K + col);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (col + 8 * q < K)  // K is a multiple of 16: 8-column chunks are whole
+            dst[q] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * q]), __uint_as_float(v[8 * q + 1])),
+                                pack_bf16x2(__uint_as_float(v[8 * q + 2]), __uint_as_float(v[8 * q + 3])),
+                                pack_bf16x2(__uint_as_float(v[8 * q + 4]), __uint_as_float(v[8 * q + 5])),
+                                pack_bf16x2(__uint_as_float(v[8 * q + 6]), __uint_as_float(v[8 * q + 7])));
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();  // TMEM and the shared tiles are free for the next unit
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
 // Y[t][n] = sum_{s < k} w[t][s] * Ytk[inv_pos[t*k + s]][n], fp32 in slot order (Ytk kept in fp32).
 __global__ void __launch_bounds__(256) moe_combine_kernel(const float* __restrict__ Ytk, const float* __restrict__ w,
                                                           const int* __restrict__ inv_pos, int T, int N, int k,

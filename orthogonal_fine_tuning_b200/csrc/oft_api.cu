@@ -968,13 +968,26 @@ int moe_chunked_oft_fwd(const uint16_t* X, int T, const float* logits, int E, in
   // 3. rotations of the active experts (gate and up)
   if (int rc = launch_cayley(Q, E * 2 * nb, b, Rex, chunk_table, n_active, 2 * nb, st)) return rc;
   // 4. rotated gather in bucket order: Xg[proj][pos] = X[t] R_{e,proj}
-  dim3 ggrid((K + 63) / 64, (TK + kGatherRows - 1) / kGatherRows);
+  //    on the tensor cores, units (active expert, 64-column group, 128-position tile)
   {
+    const int rgrid = sm_count() * 4;  // four 128-thread CTAs per SM, persistent
     ProfScope ps(OFT_K_ROTATE, st);
-    if (b == 16) moe_gather_rotate_kernel<16><<<ggrid, kGatherThreads, 0, st>>>(X, K, TK, top_k, bucket, pexp, Rex, Xg);
-    if (b == 32) moe_gather_rotate_kernel<32><<<ggrid, kGatherThreads, 0, st>>>(X, K, TK, top_k, bucket, pexp, Rex, Xg);
-    if (b == 64) moe_gather_rotate_kernel<64><<<ggrid, kGatherThreads, 0, st>>>(X, K, TK, top_k, bucket, pexp, Rex, Xg);
-    OFT_LAUNCHED("moe_gather_rotate_kernel");
+    if (b == 16) {
+      if (int rc = set_smem(moe_rot_tc_kernel<16>, kMoeRotSmem)) return rc;
+      moe_rot_tc_kernel<16><<<rgrid, kMoeRotThreads, kMoeRotSmem, st>>>(X, K, top_k, bucket, offsets, chunk_table,
+                                                                         n_active, Rex, TK, Xg);
+    }
+    if (b == 32) {
+      if (int rc = set_smem(moe_rot_tc_kernel<32>, kMoeRotSmem)) return rc;
+      moe_rot_tc_kernel<32><<<rgrid, kMoeRotThreads, kMoeRotSmem, st>>>(X, K, top_k, bucket, offsets, chunk_table,
+                                                                         n_active, Rex, TK, Xg);
+    }
+    if (b == 64) {
+      if (int rc = set_smem(moe_rot_tc_kernel<64>, kMoeRotSmem)) return rc;
+      moe_rot_tc_kernel<64><<<rgrid, kMoeRotThreads, kMoeRotSmem, st>>>(X, K, top_k, bucket, offsets, chunk_table,
+                                                                         n_active, Rex, TK, Xg);
+    }
+    OFT_LAUNCHED("moe_rot_tc_kernel");
   }
   // 5. chunks: transient dequant of the chunk's experts, then one grouped GEMM
   gemm::Params prm;

@@ -101,12 +101,12 @@ __global__ void __launch_bounds__(256) dequant_transposed_kernel(WeightView w, u
 }
 
 // MoE: dequantise the experts of chunk `chunk_idx` into buf[slot][N][K] (INT4 bank).
-// grid = (ceil(N / 64) row tiles, chunk slots); slots without an expert (-1) do
-// nothing.  A CTA takes 64 rows of one expert: their K/G group scales are staged
+// grid = (ceil(N / 32) row tiles, chunk slots); slots without an expert (-1) do
+// nothing.  A CTA takes 32 rows of one expert: their K/G group scales are staged
 // in shared memory row-major, then each warp walks whole rows, lane l decoding
 // the 8 codes of word l + 32 i, so every load and store instruction of a warp
 // covers contiguous memory (128 B of codes in, 512 B of bf16 out).
-constexpr int kChunkRows = 64;
+constexpr int kChunkRows = 32;  // small enough (staged scales ~14 KB) to co-reside with the grouped GEMM
 
 __host__ __device__ constexpr int chunk_scale_ld(int groups) { return groups + 2; }
 

@@ -295,20 +295,21 @@ def run_ours(args, rank, world):
         spec = MOE_CONFIGS[name]
         case = make_moe_case(spec, device=dev)
         W = oft.Weight("int4", case["codes"], case["scales"], spec.K, 2 * spec.n_proj, spec.group, n_experts=spec.E)
-        ws = torch.empty(oft.moe_chunked_oft_workspace(spec.T, spec.E, spec.top_k, spec.chunk, W, spec.b),
-                         dtype=torch.uint8, device=dev)
+        fused = args.moe == "fused"
+        moe_ws = oft.moe_fused_oft_workspace if fused else oft.moe_chunked_oft_workspace
+        moe_fwd = oft.moe_fused_oft_fwd if fused else oft.moe_chunked_oft_fwd
+        ws = torch.empty(moe_ws(spec.T, spec.E, spec.top_k, spec.chunk, W, spec.b), dtype=torch.uint8, device=dev)
         X, logits, Q = case["X"], case["logits"], case["Q"]
-        out = oft.moe_chunked_oft_fwd(X, logits, W, spec.b, Q, spec.top_k, spec.chunk, workspace=ws)
+        out = moe_fwd(X, logits, W, spec.b, Q, spec.top_k, spec.chunk, workspace=ws)
         tokens = spec.T
         backward = False
 
         def new_outputs():
-            o = oft.moe_chunked_oft_fwd(X, logits, W, spec.b, Q, spec.top_k, spec.chunk, workspace=ws)
-            return o
+            return moe_fwd(X, logits, W, spec.b, Q, spec.top_k, spec.chunk, workspace=ws)
 
         def step(Xi=X, Li=logits, Qi=Q, o=None):
             o = out if o is None else o
-            oft.moe_chunked_oft_fwd(Xi, Li, W, spec.b, Qi, spec.top_k, spec.chunk, workspace=ws, out=o)
+            moe_fwd(Xi, Li, W, spec.b, Qi, spec.top_k, spec.chunk, workspace=ws, out=o)
             return o["Y"]
 
         inputs = dict(X=X, logits=logits, Q=Q)
@@ -382,7 +383,8 @@ def run_ours(args, rank, world):
                      cayley=2.0 * spec.b ** 3 * n_active * 2 * (spec.K // spec.b))
         total_flops = sum(flops.values())
         expert_bytes = spec.K * 2 * spec.n_proj // 2 + 2 * 2 * spec.n_proj * (spec.K // spec.group)
-        chunk_buf_bytes = 2 * (2 * spec.K * 2 * spec.n_proj)      # bf16 write + read
+        # the chunked variant materialises each active expert in bf16 (write + read), as the pages do
+        chunk_buf_bytes = 0 if args.moe == "fused" else 2 * (2 * spec.K * 2 * spec.n_proj)
         alg_bytes = n_active * (expert_bytes + chunk_buf_bytes) + 2 * spec.T * spec.K + 2 * spec.T * 2 * spec.n_proj
     else:
         flops = linear_flops(spec, backward)
@@ -395,7 +397,15 @@ def run_ours(args, rank, world):
     # ---- dominant kernel roofline ----
     g_launch = prof.launches["gemm"]
     g_ms = prof.ms["gemm"]
-    if is_moe:
+    if is_moe and args.moe == "fused":
+        # the grouped fused-dequant GEMM against the tensor peak (no chunk buffer: compute-bound)
+        bound = "tensor"
+        achieved = flops["gemm"] / (g_ms / args.steps / 1e3) / 1e12
+        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        unit = "TFLOP/s"
+        traffic = None
+        kernel = "gemm_dq_kernel, MoE mode (grouped over active experts x gate/up, fused INT4 dequant)"
+    elif is_moe:
         # HBM-bound: algorithmic bytes of the whole step ÷ the step (chunk dequant + grouped GEMM dominate)
         bound = "hbm"
         achieved = alg_bytes / (ms_per_step / 1e3) / 1e9
@@ -495,7 +505,7 @@ def run_ours(args, rank, world):
               "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MB write)",
               "step": "build_rotation + fwd" + (" + bwd" if backward else "") + (" + dQ all-reduce" if world > 1 and backward else "")}
     if is_moe:
-        config.update(n_active_experts=n_active)
+        config.update(n_active_experts=n_active, moe_variant=args.moe)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -561,6 +571,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="c1", choices=sorted(WORKLOAD_NAMES))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--moe", default="chunked", choices=["chunked", "fused"],
+                    help="MoE workload: the pages' chunked dequant (default) or the fused-dequant grouped GEMM")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

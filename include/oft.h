@@ -154,6 +154,21 @@ int moe_chunked_oft_fwd(const uint16_t* X, int T, const float* logits, int E, in
                         int32_t* topk_idx, float* topk_w, int32_t* offsets, int32_t* bucket, int32_t* chunk_table,
                         int32_t* n_active, void* ws, size_t ws_bytes, void* stream);
 
+/* Bytes of scratch moe_fused_oft_fwd needs (no chunk buffers). */
+size_t moe_fused_oft_workspace(int T, int E, int top_k, int chunk, const oft_weight* W_experts, int b);
+
+/* MoE OFT forward with the dequant fused into the grouped GEMM: the next step after
+ * the chunked variant above (the chunk dequantisation is the pages' design: "技术细节"
+ * of m.xxlwj.com 771001).  Same arguments, same routing outputs (chunk_table still
+ * lists the active experts in chunks of `chunk`) and the same result Y.  There is no
+ * bf16 chunk buffer: one launch covers every (active expert, projection) group and
+ * decodes the INT4 codes straight into the tensor-core operand, so each active
+ * expert's weight crosses HBM once, as 4-bit codes.  Same limits. */
+int moe_fused_oft_fwd(const uint16_t* X, int T, const float* logits, int E, int top_k, int chunk,
+                      const oft_weight* W_experts, int b, const uint16_t* Q_experts, uint16_t* Y,
+                      int32_t* topk_idx, float* topk_w, int32_t* offsets, int32_t* bucket, int32_t* chunk_table,
+                      int32_t* n_active, void* ws, size_t ws_bytes, void* stream);
+
 /* ---- test hooks: single steps of the path, same kernels ---- */
 
 /* Dequantise a single weight to bf16: out [N][K] (transpose = 0) or [K][N]. */

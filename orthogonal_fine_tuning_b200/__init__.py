@@ -9,6 +9,8 @@ from .binding import (  # noqa: F401
     library_path,
     moe_chunked_oft_fwd,
     moe_chunked_oft_workspace,
+    moe_fused_oft_fwd,
+    moe_fused_oft_workspace,
     oft_build_rotation,
     oft_cayley_backward,
     oft_check_device,

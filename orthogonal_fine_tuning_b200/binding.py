@@ -164,9 +164,12 @@ def moe_chunked_oft_workspace(T: int, E: int, top_k: int, chunk: int, W: Weight,
     return int(_L.moe_chunked_oft_workspace(T, E, top_k, chunk, ctypes.byref(cw), b))
 
 
-def moe_chunked_oft_fwd(X: torch.Tensor, logits: torch.Tensor, W: Weight, b: int, Q: torch.Tensor, top_k: int,
-                        chunk: int, workspace: Optional[torch.Tensor] = None, out: Optional[dict] = None,
-                        stream=None) -> dict:
+def moe_fused_oft_workspace(T: int, E: int, top_k: int, chunk: int, W: Weight, b: int) -> int:
+    cw = W.c()
+    return int(_L.moe_fused_oft_workspace(T, E, top_k, chunk, ctypes.byref(cw), b))
+
+
+def _moe_fwd(fused: bool, X, logits, W, b, Q, top_k, chunk, workspace, out, stream) -> dict:
     T, E = logits.shape
     dev = X.device
     n_chunks = (E + chunk - 1) // chunk
@@ -180,13 +183,30 @@ def moe_chunked_oft_fwd(X: torch.Tensor, logits: torch.Tensor, W: Weight, b: int
         n_active=torch.empty(4, dtype=torch.int32, device=dev)[:1],
     )
     cw = W.c()
-    nbytes = int(_L.moe_chunked_oft_workspace(T, E, top_k, chunk, ctypes.byref(cw), b))
+    size_fn = _L.moe_fused_oft_workspace if fused else _L.moe_chunked_oft_workspace
+    run_fn = _L.moe_fused_oft_fwd if fused else _L.moe_chunked_oft_fwd
+    nbytes = int(size_fn(T, E, top_k, chunk, ctypes.byref(cw), b))
     ws = _ws(nbytes, dev, workspace)
-    _check(_L.moe_chunked_oft_fwd(
+    _check(run_fn(
         _ptr(_bits(X)), T, _ptr(logits), E, top_k, chunk, ctypes.byref(cw), b, _ptr(_bits(Q)), _ptr(o["Y"]),
         _ptr(o["topk_idx"]), _ptr(o["topk_w"]), _ptr(o["offsets"]), _ptr(o["bucket"]), _ptr(o["chunk_table"]),
         _ptr(o["n_active"]), _ptr(ws), ws.numel(), _stream(stream)))
     return o
+
+
+def moe_chunked_oft_fwd(X: torch.Tensor, logits: torch.Tensor, W: Weight, b: int, Q: torch.Tensor, top_k: int,
+                        chunk: int, workspace: Optional[torch.Tensor] = None, out: Optional[dict] = None,
+                        stream=None) -> dict:
+    """Chunked MoE forward: each chunk of active experts is dequantised to a bf16
+    buffer, then one grouped GEMM."""
+    return _moe_fwd(False, X, logits, W, b, Q, top_k, chunk, workspace, out, stream)
+
+
+def moe_fused_oft_fwd(X: torch.Tensor, logits: torch.Tensor, W: Weight, b: int, Q: torch.Tensor, top_k: int,
+                      chunk: int, workspace: Optional[torch.Tensor] = None, out: Optional[dict] = None,
+                      stream=None) -> dict:
+    """The same MoE forward with the dequant fused into the grouped GEMM (no chunk buffer)."""
+    return _moe_fwd(True, X, logits, W, b, Q, top_k, chunk, workspace, out, stream)
 
 
 def oft_dequant_weight(W: Weight, transpose: bool = False, out: Optional[torch.Tensor] = None,

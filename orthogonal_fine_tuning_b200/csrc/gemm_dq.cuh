@@ -65,13 +65,20 @@ struct Group {
   int w_k0;      // first reduction index within a codes row
   int y_map;     // output tensor map (rows: tokens, columns: this group's weight rows)
   int tiles_w, tiles_t, tile0;
-  long long code_off;  // backward: byte offset of this group's blocks in the packed codes
+  long long code_off;   // byte offset of this group's codes (backward: packed blocks; MoE: the expert's codes)
+  long long scale_off;  // byte offset of this group's scales (MoE: the expert's scales)
+  int out_row0, out_col0;  // MoE: output row of the group's first token, column of its first weight row
 };
 
 struct Params {
   CUtensorMap tmB[MAX_GROUPS];  // activations, bf16, box {64, 192}, 128B swizzle
   CUtensorMap tmS;              // backward only: bf16 scales (INT4), bf16 factors (MXFP4), fp32 scales (FP8); box {64, rows}
   CUtensorMap tmY[MAX_GROUPS];  // outputs, box {32, 32}, no swizzle: forward Y_p bf16, backward dX'_p fp32
+  // MoE mode: groups built on the device (one per active expert and projection), fp32 output
+  const Group* moe_groups;      // [n_groups], tile0 ascending
+  const int* moe_meta;          // [0] total units, [1] n_groups
+  float* moe_out;               // [token slots][moe_ldo]: row out_row0 + token, column out_col0 + weight row
+  int moe_ldo;
   const uint8_t* codes;         // forward: [N][K] codes; backward: blocks packed by pack_codes_bwd_kernel
   long long code_row_bytes;     // forward only
   const void* scales;           // INT4 bf16 [K/G][N]; FP8 fp32 [N]; MXFP4 e8m0 [K/32][N]
@@ -106,8 +113,17 @@ constexpr int EP_BYTES = 16384;  // epilogue staging: 4 warps x 4 KB (two bf16 o
 constexpr size_t kSmemBytes = 1024 + STAGES * (B_BYTES + S_BYTES) + EP_BYTES + kBarBytes + sizeof(Group) * MAX_GROUPS;
 
 __device__ __forceinline__ void decode(const Group* sg, int ng, int u, int& g, int& tw, int& tt) {
-  g = 0;
-  while (g + 1 < ng && u >= sg[g + 1].tile0) ++g;
+  if (ng > 8) {  // many groups (MoE, built on the device): binary search on tile0
+    int lo = 0, hi = ng - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (sg[mid].tile0 <= u) lo = mid; else hi = mid - 1;
+    }
+    g = lo;
+  } else {
+    g = 0;
+    while (g + 1 < ng && u >= sg[g + 1].tile0) ++g;
+  }
   const int local = u - sg[g].tile0;
   tt = local / sg[g].tiles_w;
   tw = local % sg[g].tiles_w;
@@ -152,10 +168,11 @@ __device__ __forceinline__ void load_raw(const Params& p, const Group& G, int tw
   raw.sc = 0;
   if (row >= G.rows || k0 >= G.kred) return;
   const int valid = min(BK, G.kred - k0);      // reduction elements present in this k-step
-  const long long rbase = static_cast<long long>(G.w_row0 + row) * p.code_row_bytes;
+  const long long rbase = G.code_off + static_cast<long long>(G.w_row0 + row) * p.code_row_bytes;
   const int kk = G.w_k0 + k0;                  // first reduction index in the codes row
   // forward rows are 32/64-byte aligned; the reduction (d_in) is a multiple of 32
   const uint4* src = reinterpret_cast<const uint4*>(p.codes + rbase + (FMT == kFp8 ? kk : kk / 2));
+  const uint8_t* scales = static_cast<const uint8_t*>(p.scales) + G.scale_off;
   constexpr int NV = NW / 4;
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
@@ -165,17 +182,17 @@ __device__ __forceinline__ void load_raw(const Params& p, const Group& G, int tw
     }
   }
   if (FMT == kFp8) {
-    raw.sc = __float_as_uint(static_cast<const float*>(p.scales)[G.w_row0 + row]);  // fp32 channel scale
+    raw.sc = __float_as_uint(reinterpret_cast<const float*>(scales)[G.w_row0 + row]);  // fp32 channel scale
   } else {
     const int n = G.w_row0 + row;
     const bool second = valid > 32;
     if (FMT == kInt4) {
-      const uint16_t* S = static_cast<const uint16_t*>(p.scales);
+      const uint16_t* S = reinterpret_cast<const uint16_t*>(scales);
       const uint32_t s0 = S[static_cast<size_t>(kk / p.group) * p.N + n];
       const uint32_t s1 = second ? S[static_cast<size_t>((kk + 32) / p.group) * p.N + n] : 0u;
       raw.sc = s0 | (s1 << 16);
     } else {
-      const uint8_t* E = static_cast<const uint8_t*>(p.scales);
+      const uint8_t* E = scales;
       const uint32_t e0 = E[static_cast<size_t>(kk / 32) * p.N + n];
       const uint32_t e1 = second ? E[static_cast<size_t>(kk / 32 + 1) * p.N + n] : 127u;
       raw.sc = e0 | (e1 << 8);
@@ -250,7 +267,7 @@ __device__ __forceinline__ void convert(const Raw& raw, const uint8_t* sS, int s
   }
 }
 
-template <int FMT, bool BWD, bool SCHED>
+template <int FMT, bool BWD, bool SCHED, bool MOE = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_constant__ KParams<SCHED> kp) {
   const Params& p = kp.p;
   extern __shared__ uint8_t smem_raw[];
@@ -302,6 +319,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_co
       tma_prefetch_desc(&p.tmB[i]);
       tma_prefetch_desc(&p.tmY[i]);
     }
+    if (MOE) tma_prefetch_desc(&p.tmB[0]);
     if (BWD) tma_prefetch_desc(&p.tmS);
   }
   if (warp == 1) {
@@ -312,7 +330,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_co
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int total = s_meta[0], ng = s_meta[1];
+  // groups: from the launch (shared memory copy), or built on the device (MoE)
+  const Group* gsrc = MOE ? p.moe_groups : sg;
+  const int total = MOE ? p.moe_meta[0] : s_meta[0], ng = MOE ? p.moe_meta[1] : s_meta[1];
   // this CTA's units: count, and the i-th one
   int nu;
   if constexpr (SCHED) {
@@ -339,8 +359,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_co
       bool ok = true;
       for (int i = 0; i < nu && ok; ++i) {
         int g, tw, tt;
-        decode(sg, ng, unit_at(i), g, tw, tt);
-        const Group& G = sg[g];
+        decode(gsrc, ng, unit_at(i), g, tw, tt);
+        const Group& G = gsrc[g];
         const int nk = (G.kred + BK - 1) / BK;
         for (int ks = 0; ks < nk; ++ks) {
           if (!mbar_wait(&empty[stage], ph ^ 1, abort_flag, kErrWaitEmpty)) {
@@ -377,8 +397,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_co
       long long gk = 0;  // k-steps of this CTA's earlier units
       for (int i = 0; i < nu && ok; ++i) {
         int g, tw, tt;
-        decode(sg, ng, unit_at(i), g, tw, tt);
-        const int nk = (sg[g].kred + BK - 1) / BK;
+        decode(gsrc, ng, unit_at(i), g, tw, tt);
+        const int nk = (gsrc[g].kred + BK - 1) / BK;
         // Accumulator halves overlap with the epilogue at both ends of a unit: the first D
         // k-steps feed half 0 only while the epilogue still reads half 1 of the previous
         // unit, and the last D k-steps finish half 0 first, so the epilogue can drain it
@@ -473,8 +493,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_co
     uint32_t acc_ph = 0;
     for (int i = 0; i < nu; ++i) {
       int g, tw, tt;
-      decode(sg, ng, unit_at(i), g, tw, tt);
-      const Group& G = sg[g];
+      decode(gsrc, ng, unit_at(i), g, tw, tt);
+      const Group& G = gsrc[g];
       const int n0 = tw * WM + q * 32;  // first weight row of this warp's blocks
       const int m_base = tt * TP * TN;
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
@@ -483,6 +503,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_co
       auto stage_chunk = [&](const uint32_t (&r)[32], int c) {
         const int m0 = m_base + c * 32;
         if (n0 >= G.rows || m0 >= G.tokens) return;
+        if constexpr (MOE) {
+          // fp32 rows of the group's token slots: lane = weight row, so each of the 32
+          // stores of the warp writes 128 contiguous bytes; tokens past the group's end
+          // (the next expert's rows in the activation map) are not written
+          if (n0 + lane < G.rows) {
+            float* out = p.moe_out + static_cast<size_t>(G.out_row0 + m0) * p.moe_ldo + G.out_col0 + n0 + lane;
+            const int jn = min(32, G.tokens - m0);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < jn) out[static_cast<size_t>(j) * p.moe_ldo] = __uint_as_float(r[j]);
+          }
+          return;
+        }
         if (lane == 0) bulk_wait_read<SLOTS - 1>();  // the store that last read this slot is done
         __syncwarp();
         uint8_t* b = ebuf + slot * BLK;
@@ -549,8 +582,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_co
     };
     auto set_unit = [&](Cursor& c) {
       if (c.i < nu) {
-        decode(sg, ng, unit_at(c.i), c.g, c.tw, c.tt);
-        c.nk = (sg[c.g].kred + BK - 1) / BK;
+        decode(gsrc, ng, unit_at(c.i), c.g, c.tw, c.tt);
+        c.nk = (gsrc[c.g].kred + BK - 1) / BK;
       }
     };
     auto advance = [&](Cursor& c) {
@@ -570,7 +603,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_co
     auto fetch = [&](Raw& raw) {
       to_parity(ld);
       if (ld.i < nu) {
-        load_raw<FMT, BWD>(p, sg[ld.g], ld.tw, r, ld.ks, raw);
+        load_raw<FMT, BWD>(p, gsrc[ld.g], ld.tw, r, ld.ks, raw);
         advance(ld);
       }
     };

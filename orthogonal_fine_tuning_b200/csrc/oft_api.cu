@@ -23,6 +23,7 @@
 #include "rot_tc.cuh"
 #include "gemm_dq.cuh"
 #include "gemm_dq2.cuh"
+#include "moe_fused.cuh"
 
 using namespace oftk;
 
@@ -898,20 +899,28 @@ int oft_linear_bwd(const uint16_t* dY, const uint16_t* X, int M, const oft_weigh
 // ---------------------------------------------------------------------------
 namespace {
 struct MoeLayout {
-  size_t rex, xg, buf, ytk, inv, pexp, total;
+  size_t rex, xg, buf, ytk, inv, pexp, groups, meta, total;
 };
-MoeLayout moe_layout(int T, int E, int top_k, int chunk, int K, int N, int b) {
+// fused: no chunk buffers; a device-built group list instead
+MoeLayout moe_layout(int T, int E, int top_k, int chunk, int K, int N, int b, bool fused = false) {
   MoeLayout L{};
   const size_t TK = 1ull * T * top_k;
   L.rex = 0;
   L.xg = round_up(L.rex + 4ull * E * 2 * (K / b) * b * b, 256);
   L.buf = round_up(L.xg + 2ull * 2 * TK * K, 256);
-  L.ytk = round_up(L.buf + 2ull * 2 * chunk * N * K, 256);  // two chunk buffers (double-buffered)
+  L.ytk = round_up(L.buf + (fused ? 0ull : 2ull * 2 * chunk * N * K), 256);  // two chunk buffers (double-buffered)
   L.inv = round_up(L.ytk + 4ull * TK * N, 256);  // per-slot expert outputs kept in fp32
   L.pexp = round_up(L.inv + 4ull * TK, 256);
-  L.total = round_up(L.pexp + 4ull * TK, 256);
+  L.groups = round_up(L.pexp + 4ull * TK, 256);
+  L.meta = round_up(L.groups + (fused ? sizeof(gdq::Group) * 2ull * E : 0ull), 256);
+  L.total = round_up(L.meta + (fused ? 16ull : 0ull), 256);
   return L;
 }
+
+int moe_oft_fwd_impl(bool fused, const uint16_t* X, int T, const float* logits, int E, int top_k, int chunk,
+                     const oft_weight* W, int b, const uint16_t* Q, uint16_t* Y, int32_t* topk_idx, float* topk_w,
+                     int32_t* offsets, int32_t* bucket, int32_t* chunk_table, int32_t* n_active, void* ws,
+                     size_t ws_bytes, void* stream);
 }  // namespace
 
 size_t moe_chunked_oft_workspace(int T, int E, int top_k, int chunk, const oft_weight* W, int b) {
@@ -923,6 +932,30 @@ int moe_chunked_oft_fwd(const uint16_t* X, int T, const float* logits, int E, in
                         const oft_weight* W, int b, const uint16_t* Q, uint16_t* Y, int32_t* topk_idx, float* topk_w,
                         int32_t* offsets, int32_t* bucket, int32_t* chunk_table, int32_t* n_active, void* ws,
                         size_t ws_bytes, void* stream) {
+  return moe_oft_fwd_impl(false, X, T, logits, E, top_k, chunk, W, b, Q, Y, topk_idx, topk_w, offsets, bucket,
+                          chunk_table, n_active, ws, ws_bytes, stream);
+}
+
+size_t moe_fused_oft_workspace(int T, int E, int top_k, int chunk, const oft_weight* W, int b) {
+  if (W == nullptr || T <= 0 || E <= 0 || top_k <= 0 || chunk <= 0 || b <= 0) return 0;
+  return moe_layout(T, E, top_k, chunk, W->d_in, W->d_out, b, true).total;
+}
+
+int moe_fused_oft_fwd(const uint16_t* X, int T, const float* logits, int E, int top_k, int chunk,
+                      const oft_weight* W, int b, const uint16_t* Q, uint16_t* Y, int32_t* topk_idx, float* topk_w,
+                      int32_t* offsets, int32_t* bucket, int32_t* chunk_table, int32_t* n_active, void* ws,
+                      size_t ws_bytes, void* stream) {
+  return moe_oft_fwd_impl(true, X, T, logits, E, top_k, chunk, W, b, Q, Y, topk_idx, topk_w, offsets, bucket,
+                          chunk_table, n_active, ws, ws_bytes, stream);
+}
+
+}  // extern "C"
+
+namespace {
+int moe_oft_fwd_impl(bool fused, const uint16_t* X, int T, const float* logits, int E, int top_k, int chunk,
+                     const oft_weight* W, int b, const uint16_t* Q, uint16_t* Y, int32_t* topk_idx, float* topk_w,
+                     int32_t* offsets, int32_t* bucket, int32_t* chunk_table, int32_t* n_active, void* ws,
+                     size_t ws_bytes, void* stream) {
   if (int rc = check_weight(W, true)) return rc;
   if (W->fmt != OFT_W_INT4) return fail(OFT_ERR_UNSUPPORTED, "the MoE expert bank must be INT4");
   const int K = W->d_in, N = W->d_out;
@@ -939,7 +972,7 @@ int moe_chunked_oft_fwd(const uint16_t* X, int T, const float* logits, int E, in
     if (q == nullptr || !aligned16(q)) return fail(OFT_ERR_INVALID_ARG, "NULL or misaligned pointer");
   const int n_proj = N / 2, TK = T * top_k, nb = K / b;
   const int n_chunks_max = (E + chunk - 1) / chunk;
-  const MoeLayout L = moe_layout(T, E, top_k, chunk, K, N, b);
+  const MoeLayout L = moe_layout(T, E, top_k, chunk, K, N, b, fused);
   if (ws_bytes < L.total) return fail(OFT_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
   cudaStream_t st = as_stream(stream);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
@@ -989,6 +1022,47 @@ int moe_chunked_oft_fwd(const uint16_t* X, int T, const float* logits, int E, in
     }
     OFT_LAUNCHED("moe_rot_tc_kernel");
   }
+  if (fused) {
+    // 5'. one grouped fused-dequant GEMM over every (active expert, projection): the INT4
+    //     codes are decoded into the tensor-core operand; per-slot fp32 outputs to Ytk
+    gdq::Group* groups = reinterpret_cast<gdq::Group*>(wsb + L.groups);
+    int* meta = reinterpret_cast<int*>(wsb + L.meta);
+    const long long code_stride = 1ll * N * K / 2, scale_stride = 2ll * (K / W->group) * N;
+    {
+      ProfScope ps(OFT_K_ROUTE, st);
+      moe_groups_kernel<<<1, 32, 0, st>>>(chunk_table, n_active, offsets, TK, n_proj, K, code_stride, scale_stride,
+                                          groups, meta);
+      OFT_LAUNCHED("moe_groups_kernel");
+    }
+    gdq::KParams<false> kp;
+    memset(&kp, 0, sizeof(kp));
+    gdq::Params& gp = kp.p;
+    if (int rc = make_map_bf16(&gp.tmB[0], Xg, K, 2ull * TK, K, gdq::TN)) return rc;
+    gp.codes = static_cast<const uint8_t*>(W->codes);
+    gp.code_row_bytes = K / 2;
+    gp.scales = W->scales;
+    gp.N = N;
+    gp.K = K;
+    gp.group = W->group;
+    gp.num_groups = 0;
+    gp.moe_groups = groups;
+    gp.moe_meta = meta;
+    gp.moe_out = Ytk;
+    gp.moe_ldo = N;
+    {
+      static bool attr_set[64] = {false};
+      int dev = 0;
+      cudaGetDevice(&dev);
+      if (dev < 64 && !attr_set[dev]) {
+        OFT_CUDA(cudaFuncSetAttribute(gdq::gemm_dq_kernel<gdq::kInt4, false, false, true>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(gdq::kSmemBytes)));
+        attr_set[dev] = true;
+      }
+      ProfScope ps(OFT_K_GEMM, st);
+      gdq::gemm_dq_kernel<gdq::kInt4, false, false, true><<<sm_count(), gdq::NUM_THREADS, gdq::kSmemBytes, st>>>(kp);
+      OFT_LAUNCHED("gemm_dq_kernel (MoE)");
+    }
+  } else {
   // 5. chunks: transient dequant of the chunk's experts, then one grouped GEMM
   gemm::Params prm;
   memset(&prm, 0, sizeof(prm));
@@ -1035,6 +1109,7 @@ int moe_chunked_oft_fwd(const uint16_t* X, int T, const float* logits, int E, in
     if (int rc = launch_gemm(prm, 0, st)) return rc;
     OFT_CUDA(cudaEventRecord(sp->gemm_done[h], st));
   }
+  }
   // 6. weighted combine in slot order
   const long long cunits = 1ll * T * (N / 8);
   const int cgrid = static_cast<int>(std::min<long long>((cunits + 255) / 256, 148ll * 16));
@@ -1044,7 +1119,7 @@ int moe_chunked_oft_fwd(const uint16_t* X, int T, const float* logits, int E, in
   return OFT_OK;
 }
 
-}  // extern "C"
+}  // namespace
 
 // ---------------------------------------------------------------------------
 // bounded-wait self test

@@ -1,5 +1,7 @@
-"""Active-expert-chunked MoE OFT forward on the GPU through the C ABI: routing,
-buckets and chunk table bit-exact against the oracle; Y within tolerance."""
+"""Active-expert MoE OFT forward on the GPU through the C ABI, in both variants:
+chunked (experts dequantised chunk by chunk into a bf16 buffer) and fused
+(decoded inside the grouped GEMM).  Routing, buckets and chunk table bit-exact
+against the oracle; Y within tolerance."""
 
 import numpy as np
 import pytest
@@ -21,13 +23,18 @@ def oft():
     return m
 
 
-def _run(oft, case):
+def _run(oft, case, fused=False):
     spec = case["spec"]
-    dev = case["X"].device
     W = oft.Weight("int4", case["codes"], case["scales"], spec.K, 2 * spec.n_proj, spec.group, n_experts=spec.E)
-    out = oft.moe_chunked_oft_fwd(case["X"], case["logits"], W, spec.b, case["Q"], spec.top_k, spec.chunk)
+    fwd = oft.moe_fused_oft_fwd if fused else oft.moe_chunked_oft_fwd
+    out = fwd(case["X"], case["logits"], W, spec.b, case["Q"], spec.top_k, spec.chunk)
     oft.oft_check_device()
     return out
+
+
+@pytest.fixture(params=[False, True], ids=["chunked", "fused"])
+def fused(request):
+    return request.param
 
 
 def _check_routing(out, logits_np, spec):
@@ -49,11 +56,11 @@ def _to(case, dev):
 
 @pytest.mark.parametrize("T,E,top_k,chunk,b,K", [(200, 24, 4, 4, 32, 256), (77, 9, 3, 2, 16, 256), (64, 5, 1, 3, 64, 256),
                                                   (50, 7, 2, 3, 32, 160)])
-def test_small_moe(oft, T, E, top_k, chunk, b, K):
+def test_small_moe(oft, fused, T, E, top_k, chunk, b, K):
     spec = MoESpec("s", T=T, K=K, E=E, n_proj=48, top_k=top_k, chunk=chunk, group=32, b=b, q_sigma=0.05,
                    seed=T + E)
     case = make_moe_case(spec)
-    out = _run(oft, _to(case, "cuda"))
+    out = _run(oft, _to(case, "cuda"), fused)
     _check_routing(out, raw(case["logits"]), spec)
     bank = moe_ref.ExpertBank(raw(case["codes"]), raw(case["scales"]), spec.K, spec.group, spec.n_proj)
     Yref, _ = moe_ref.moe_fwd_chunked(raw(case["X"]), raw(case["logits"]), bank, raw(case["Q"]), b, top_k, chunk, E)
@@ -69,12 +76,12 @@ def test_ties_in_logits_go_to_lower_expert(oft):
     _check_routing(out, raw(case["logits"]), spec)
 
 
-def test_c3_full_routing_and_sampled_output(oft):
+def test_c3_full_routing_and_sampled_output(oft, fused):
     """Kimi-like expert layer: 4096 tokens, hidden 7168, 384 INT4-g32 experts of
     2 x 2048, top-8 over Zipf-biased logits, chunks of 16, b=32."""
     spec = MOE_CONFIGS["c3"]
     case = make_moe_case(spec, device="cuda")
-    out = _run(oft, case)
+    out = _run(oft, case, fused)
     logits = raw(case["logits"])
     _check_routing(out, logits, spec)
     rng = np.random.default_rng(0)
@@ -92,3 +99,15 @@ def test_c3_full_routing_and_sampled_output(oft):
     Yref = moe_ref.moe_fwd_direct(raw(case["X"]), logits, bank, raw(case["Q"]), spec.b, spec.top_k,
                                   tokens=toks, cols=cols)
     assert rel_err(f64(out["Y"])[toks][:, cols], Yref) < TOL
+
+
+def test_fused_matches_chunked(oft):
+    """Both variants compute the same product: identical routing, Y within tolerance
+    of each other on a ragged case (hidden size not a multiple of 64, experts with
+    a single token)."""
+    spec = MoESpec("fc", T=90, K=160, E=13, n_proj=40, top_k=3, chunk=5, group=32, b=32, q_sigma=0.05, seed=77)
+    case = _to(make_moe_case(spec), "cuda")
+    a, f = _run(oft, case, False), _run(oft, case, True)
+    for k in ("topk_idx", "offsets", "bucket", "chunk_table", "n_active"):
+        assert torch.equal(a[k], f[k]), k
+    assert rel_err(f64(f["Y"]), f64(a["Y"])) < TOL

@@ -37,7 +37,18 @@ WORKLOAD_NAMES = {
     "c2": "gated-MLP gate/up OFT linear fwd: 8192 x 4096 -> 2x12288, INT4 g128, b=64",
     "c3": "MoE active-expert-chunked OFT fwd: 4096 tok, hidden 7168, 384 experts x (2x2048), INT4 g32, top-8, chunk 16, b=32",
     "c4": "training-step OFT linear fwd+bwd: 16384 x 7168 -> 12288/3072/3072, MXFP4, b=64",
+    # decode-like checks, not among the five workloads: the same weights at 64 tokens, forward only
+    "c1-m64": "fused-QKV FP8 weights at 64 tokens, fwd: 64 x 2560 -> 4096/1024/1024, FP8 e4m3 per-channel, b=32",
+    "c4-m64": "MXFP4 weights at 64 tokens, fwd: 64 x 7168 -> 12288/3072/3072, MXFP4, b=64",
 }
+
+
+def linear_spec(name: str):
+    """The linear workload `name`: one of the five, or a 64-token forward over c1 / c4 weights."""
+    from gen import LINEAR_CONFIGS
+    if name.endswith("-m64"):
+        return LINEAR_CONFIGS[name[:-4]].with_(M=64, backward=False)
+    return LINEAR_CONFIGS[name]
 
 
 # ----------------------------------------------------------------------------
@@ -316,7 +327,7 @@ def run_ours(args, rank, world):
         outputs = dict(Y=out["Y"])
         result_keys = ("Y",)
     else:
-        spec = LINEAR_CONFIGS[name]
+        spec = linear_spec(name)
         backward = spec.backward
         case = make_linear_case(spec)
         W = oft.Weight(spec.fmt, case["codes"].to(dev), case["scales"].to(dev), spec.K, spec.N, spec.group)
@@ -413,6 +424,17 @@ def run_ours(args, rank, world):
         unit = "GB/s"
         traffic = None
         kernel = "whole step (chunk dequant + grouped GEMM), HBM"
+    elif spec.M <= 128:
+        # few tokens: the weight stream bounds the GEMM; bytes of one launch over its time
+        wbytes = weight_bytes(spec)
+        per_launch_bytes = wbytes + 2 * spec.P * spec.M * spec.K + 2 * spec.M * spec.N
+        avg_s = g_ms / g_launch / 1e3
+        bound = "hbm"
+        achieved = per_launch_bytes / avg_s / 1e9
+        peak = peaks["hbm_gbs"]
+        unit = "GB/s"
+        traffic = None
+        kernel = "gemm_dq_kernel (fused dequant, tcgen05/TMEM), weight-stream bound at this M"
     else:
         gemm_flops = flops["gemm_fwd"] + flops.get("gemm_bwd", 0.0)
         per_launch = gemm_flops / (g_launch / args.steps)
@@ -539,7 +561,7 @@ def run_reference(args, rank, world):
         value = statistics.mean(r["value"] for r in res)
         sample = res[-1]["sample"]
     else:
-        spec = LINEAR_CONFIGS[name]
+        spec = linear_spec(name)
         case = make_linear_case(spec)
         per_budget = 150.0 / (args.steps + args.warmup)
         tokens = min(spec.M, 64)

@@ -392,7 +392,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_co
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       uint32_t acc_ph = 0;
-      constexpr uint32_t idesc = idesc_bf16_f32(WM, TN);
       bool ok = true;
       long long gk = 0;  // k-steps of this CTA's earlier units
       for (int i = 0; i < nu && ok; ++i) {
@@ -407,14 +406,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_co
         const int D = nk < STAGES ? nk : STAGES;
         const int T0 = nk - D > D ? nk - D : D;  // tail [T0, nk); empty when nk <= D
         auto st_of = [&](int j) { return static_cast<int>((gk + j) % STAGES); };
+        // each token tile's MMAs are only as wide as its tokens (a multiple of 16; none
+        // for a tile past the group's end): small or ragged token counts do not pay for
+        // the full 192 columns
+        uint32_t idesc_h[TP];
+        bool live_h[TP];
+#pragma unroll
+        for (int h = 0; h < TP; ++h) {
+          const int tok = min(TN, max(0, gsrc[g].tokens - (tt * TP + h) * TN));
+          live_h[h] = tok > 0;
+          idesc_h[h] = idesc_bf16_f32(WM, live_h[h] ? (tok + 15) / 16 * 16 : TN);
+        }
         auto issue = [&](int h, int j) {
+          if (!live_h[h]) return;
           const int st = st_of(j);
           const uint32_t a0 = tmem + A_COL0 + static_cast<uint32_t>(st * 32);
           const uint32_t b0 = smem_u32(sB + st * B_BYTES + h * BT_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
-            mma_bf16_ts(tmem + static_cast<uint32_t>(h * TN), a0 + kk * 8, sdesc_sw128(b0 + kk * 32, 16, 1024), idesc,
-                        (j | kk) ? 1u : 0u);
+            mma_bf16_ts(tmem + static_cast<uint32_t>(h * TN), a0 + kk * 8, sdesc_sw128(b0 + kk * 32, 16, 1024),
+                        idesc_h[h], (j | kk) ? 1u : 0u);
         };
         auto wait_full = [&](int j) {
           const int st = st_of(j);

@@ -42,6 +42,8 @@ SMALL = [
     ("one-token", 1, 128, (8,), "int4", 128, 16),
     ("four-splits", 257, 512, (64, 136, 256, 40), "int4", 64, 64),
     ("wide-k", 130, 1024, (384,), "fp8", 0, 16),
+    ("small-m-mxfp4", 37, 2048, (264, 1032), "mxfp4", 32, 64),
+    ("small-m-fp8", 64, 1536, (256, 128, 128), "fp8", 0, 32),
 ]
 
 

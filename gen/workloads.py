@@ -231,6 +231,13 @@ def make_moe_router(spec: MoESpec, device="cpu"):
     return (noise + bias.unsqueeze(0)).to(torch.float32).contiguous().to(device)
 
 
+def make_moe_grad(spec: MoESpec, device="cpu"):
+    """Upstream gradient of the MoE layer output, bf16 [T][2 n_proj] (gate | up)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(9000 + spec.seed)
+    return torch.randn(spec.T, 2 * spec.n_proj, generator=g, device=device).to(torch.bfloat16)
+
+
 def make_moe_case(spec: MoESpec, device="cpu", experts: Optional[Sequence[int]] = None):
     """Draw one chunked-MoE OFT problem.
 

@@ -22,10 +22,26 @@ readings taken here are:
     experts are those with a non-zero count, ascending; chunk c holds
     active[c*C : (c+1)*C], the last one possibly partial.
 
-Pins (tests/test_oracle_moe.py): top-k against a brute-force Python sort;
-buckets against a dictionary build; chunked order equals the direct per-token
-sum; weights sum to one; a router that sends every token to one expert with
-k = 1 reduces to the split-projection linear of oft_ref.
+Backward (the pages train these expert layers through the adapter only; the
+frozen expert weights get no gradient).  With D_p,tk = dY_p[t] W_e,p^T (e =
+idx[t, k], p = gate / up):
+
+  dX[t]          = sum_k w_tk sum_p D_p,tk R_e,p^T            (blockwise)
+  G_e,p,blk      = sum_{(t,k): idx = e} X[t]_blk^T (w_tk D_p,tk,blk)
+  dq_e,p         = Cayley backward of G_e,p (oft_ref.cayley_grad); zero for
+                   experts no token selected
+  dw_tk          = <dY[t], Y_tk> = sum_p <D_p,tk, X[t] R_e,p>
+  dlogit[t, e_k] = w_tk (dw_tk - sum_j w_tj dw_tj)   (softmax over the selected
+                   logits); zero for logits that were not selected (top-k is
+                   piecewise constant in the logits)
+
+Pins (tests/test_oracle_moe.py, tests/test_oracle_moe_bwd.py): top-k against a
+brute-force Python sort; buckets against a dictionary build; chunked order
+equals the direct per-token sum; weights sum to one; a router that sends every
+token to one expert with k = 1 reduces to the split-projection linear of
+oft_ref (forward and backward); central finite differences of the forward for
+dX, dq and the logits; dw equals the inner product of dY with the per-slot
+expert outputs; each token's logit gradient sums to zero.
 """
 
 from __future__ import annotations
@@ -33,7 +49,7 @@ from __future__ import annotations
 import numpy as np
 
 from .codecs import bf16_bits_to_f64, dequant
-from .oft_ref import rotate, rotations
+from .oft_ref import cayley_grad, packed_len, rotate, rotate_t, rotations
 
 
 def topk(logits: np.ndarray, k: int):
@@ -84,12 +100,14 @@ class ExpertBank:
         return dequant("int4", self.codes[e], self.scales[e], self.K, self.group, rows=rows)
 
 
-def expert_outputs(X: np.ndarray, e: int, bank: ExpertBank, Qe_bits: np.ndarray, b: int, cols=None):
+def expert_outputs(X: np.ndarray, e: int, bank: ExpertBank, Qe_bits: np.ndarray, b: int, cols=None, R=None):
     """Y_tk for tokens X [m][K] routed to expert e: [m][2n] (or the given columns).
 
-    Qe_bits: packed bf16 bits [2][K/b][b(b-1)/2] for (gate, up)."""
+    Qe_bits: packed bf16 bits [2][K/b][b(b-1)/2] for (gate, up); or R, the
+    expert's rotations [2][K/b][b][b] given directly (then Qe_bits is unused)."""
     n = bank.n
-    R = rotations(Qe_bits, b)                                   # [2][K/b][b][b]
+    if R is None:
+        R = rotations(Qe_bits, b)                               # [2][K/b][b][b]
     cols = np.arange(2 * n) if cols is None else np.asarray(cols)
     out = np.empty((X.shape[0], len(cols)))
     for proj in (0, 1):
@@ -142,3 +160,38 @@ def moe_fwd_chunked(X_bits, logits, bank: ExpertBank, Q_bits, b: int, top_k: int
         Y += w[:, k:k + 1] * Ytk[pos[np.arange(T) * top_k + k]]
     routing = dict(idx=idx, w=w, counts=counts, offsets=offsets, bucket=bucket, n_active=n_active, table=table)
     return Y, routing
+
+
+def moe_bwd_direct(dY: np.ndarray, X_bits, logits, bank: ExpertBank, Q_bits, b: int, top_k: int, E: int):
+    """Backward of moe_fwd_direct, token by token in slot order.
+
+    dY float64 [T][2n] (gate | up columns).  Returns (dX [T][K],
+    dq [E][2][K/b][b(b-1)/2], dlogits [T][E], dw [T][top_k])."""
+    X = bf16_bits_to_f64(X_bits)
+    idx, w = topk(logits, top_k)
+    T, K = X.shape
+    n, nb = bank.n, K // b
+    dX = np.zeros((T, K))
+    G = np.zeros((E, 2, nb, b, b))
+    dw = np.zeros((T, top_k))
+    Rs, Ws = {}, {}
+    for t in range(T):
+        for k in range(top_k):
+            e = int(idx[t, k])
+            if e not in Rs:
+                Rs[e], Ws[e] = rotations(Q_bits[e], b), bank.weight_t(e)
+            for p in (0, 1):
+                D = dY[t, p * n:(p + 1) * n] @ Ws[e][p * n:(p + 1) * n]      # dY_p[t] W_e,p^T, [K]
+                dw[t, k] += D @ rotate(X[t:t + 1], Rs[e][p])[0]
+                dX[t] += w[t, k] * rotate_t(D[None], Rs[e][p])[0]
+                G[e, p] += w[t, k] * np.einsum("ji,jk->jik", X[t].reshape(nb, b), D.reshape(nb, b))
+    dq = np.zeros((E, 2, nb, packed_len(b)))
+    for e in Rs:
+        for p in (0, 1):
+            dq[e, p] = cayley_grad(G[e, p], Rs[e][p], b)
+    dlogits = np.zeros((T, E))
+    s = (w * dw).sum(axis=1)
+    for t in range(T):
+        for k in range(top_k):
+            dlogits[t, idx[t, k]] = w[t, k] * (dw[t, k] - s[t])
+    return dX, dq, dlogits, dw

@@ -110,6 +110,15 @@ def linear_fwd(X: np.ndarray, Wt: np.ndarray, splits, R: np.ndarray) -> np.ndarr
     return np.concatenate(outs, axis=1)
 
 
+def cayley_grad(G: np.ndarray, R: np.ndarray, b: int) -> np.ndarray:
+    """dL/dR = G per block [nb][b][b] -> dq [nb][b(b-1)/2] (Cayley backward).
+
+    dQ_full = 1/2 (I + R)^T G (I + R)^T, then dq_ij = dQ_full[i, j] - dQ_full[j, i]."""
+    T = np.swapaxes(np.eye(b) + R, -1, -2)
+    dQf = 0.5 * T @ G @ T
+    return pack_upper(dQf, b) - pack_upper(np.swapaxes(dQf, -1, -2), b)
+
+
 def linear_bwd(dY: np.ndarray, X: np.ndarray, Wt: np.ndarray, splits, R: np.ndarray, b: int,
                return_parts: bool = False):
     """Adapter backward.  Returns dX [M][K] and dq [P][K/b][b(b-1)/2]."""
@@ -117,15 +126,11 @@ def linear_bwd(dY: np.ndarray, X: np.ndarray, Wt: np.ndarray, splits, R: np.ndar
     nb = K // b
     dX = np.zeros((M, K))
     dq, parts = [], []
-    I = np.eye(b)
     for p, (n0, n1) in enumerate(split_bounds(splits)):
         dXp = dY[:, n0:n1] @ Wt[n0:n1]                       # dY_p W_p^T
         dX += rotate_t(dXp, R[p])
         G = np.einsum("mji,mjk->jik", X.reshape(M, nb, b), dXp.reshape(M, nb, b))
-        IR = I + R[p]
-        T = np.swapaxes(IR, -1, -2)
-        dQf = 0.5 * T @ G @ T
-        dq.append(pack_upper(dQf, b) - pack_upper(np.swapaxes(dQf, -1, -2), b))
+        dq.append(cayley_grad(G, R[p], b))
         parts.append(dict(dXp=dXp, G=G))
     dq = np.stack(dq)
     if return_parts:

@@ -238,12 +238,15 @@ def cpu_baseline_linear(case, backward: bool, budget_s: float = 12.0):
                       f"({cpu_model()}), {dt:.2f} s"}
 
 
-def cpu_baseline_moe(case, budget_s: float = 12.0):
+def cpu_baseline_moe(case, budget_s: float = 12.0, dY=None):
+    """Oracle tokens/s of the MoE step on the host cores (forward; with dY, forward + backward)."""
     import numpy as np
     from oracle import moe_ref
+    from oracle.codecs import bf16_bits_to_f64
     sys.path.insert(0, os.path.join(ROOT, "tests"))
     from npcase import raw
     spec = case["spec"]
+    dYf = None if dY is None else bf16_bits_to_f64(raw(dY[:8]))
     logits = raw(case["logits"])
     idx, _ = moe_ref.topk(logits, spec.top_k)
     t0 = time.perf_counter()
@@ -256,11 +259,14 @@ def cpu_baseline_moe(case, budget_s: float = 12.0):
         scales = {int(e): raw(case["scales"][int(e)]) for e in used}
         bank = moe_ref.ExpertBank(codes, scales, spec.K, spec.group, spec.n_proj)
         moe_ref.moe_fwd_direct(X[t:t + 1], logits[t:t + 1], bank, raw(case["Q"]), spec.b, spec.top_k)
+        if dYf is not None:
+            moe_ref.moe_bwd_direct(dYf[t:t + 1], X[t:t + 1], logits[t:t + 1], bank, raw(case["Q"]), spec.b,
+                                   spec.top_k, spec.E)
         done += 1
     dt = time.perf_counter() - t0
+    what = "forward + backward" if dYf is not None else "direct per-token top-%d sum" % spec.top_k
     return {"value": done / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{done} tokens of {spec.T}, direct per-token top-{spec.top_k} sum, float64 numpy "
-                      f"({cpu_model()}), {dt:.2f} s"}
+            "sample": f"{done} tokens of {spec.T}, {what}, float64 numpy ({cpu_model()}), {dt:.2f} s"}
 
 
 # ----------------------------------------------------------------------------
@@ -292,7 +298,7 @@ def gemm_kernel_hash() -> str:
 def run_ours(args, rank, world):
     import torch
     import orthogonal_fine_tuning_b200 as oft
-    from gen import LINEAR_CONFIGS, MOE_CONFIGS, make_linear_case, make_moe_case
+    from gen import LINEAR_CONFIGS, MOE_CONFIGS, make_linear_case, make_moe_case, make_moe_grad
 
     _, _, local = dist_env()
     torch.cuda.set_device(local)
@@ -313,19 +319,34 @@ def run_ours(args, rank, world):
         X, logits, Q = case["X"], case["logits"], case["Q"]
         out = moe_fwd(X, logits, W, spec.b, Q, spec.top_k, spec.chunk, workspace=ws)
         tokens = spec.T
-        backward = False
+        backward = bool(args.moe_backward)
+        if backward:
+            # adapter backward through the chunked path: dX, per-expert dQ, router-logit gradient
+            dY = make_moe_grad(spec, device=dev)
+            bws = torch.empty(oft.moe_chunked_oft_bwd_workspace(spec.T, spec.E, spec.top_k, spec.chunk, W, spec.b),
+                              dtype=torch.uint8, device=dev)
+            out.update(oft.moe_chunked_oft_bwd(dY, X, logits, W, spec.b, Q, spec.top_k, spec.chunk, workspace=bws))
 
         def new_outputs():
-            return moe_fwd(X, logits, W, spec.b, Q, spec.top_k, spec.chunk, workspace=ws)
+            o = moe_fwd(X, logits, W, spec.b, Q, spec.top_k, spec.chunk, workspace=ws)
+            if backward:
+                o.update(oft.moe_chunked_oft_bwd(dY, X, logits, W, spec.b, Q, spec.top_k, spec.chunk, workspace=bws))
+            return o
 
-        def step(Xi=X, Li=logits, Qi=Q, o=None):
+        def step(Xi=X, Li=logits, Qi=Q, o=None, dYi=None):
             o = out if o is None else o
             moe_fwd(Xi, Li, W, spec.b, Qi, spec.top_k, spec.chunk, workspace=ws, out=o)
+            if backward:
+                oft.moe_chunked_oft_bwd(dY if dYi is None else dYi, Xi, Li, W, spec.b, Qi, spec.top_k, spec.chunk,
+                                        workspace=bws, out=o)
+                allreduce_grad(o["dQ"])
             return o["Y"]
 
         inputs = dict(X=X, logits=logits, Q=Q)
-        outputs = dict(Y=out["Y"])
         result_keys = ("Y",)
+        if backward:
+            inputs["dY"] = dY
+            result_keys = ("Y", "dX", "dQ", "dlogits")
     else:
         spec = linear_spec(name)
         backward = spec.backward
@@ -397,6 +418,16 @@ def run_ours(args, rank, world):
         # the chunked variant materialises each active expert in bf16 (write + read), as the pages do
         chunk_buf_bytes = 0 if args.moe == "fused" else 2 * (2 * spec.K * 2 * spec.n_proj)
         alg_bytes = n_active * (expert_bytes + chunk_buf_bytes) + 2 * spec.T * spec.K + 2 * spec.T * 2 * spec.n_proj
+        if backward:
+            # dY W^T per routed row, its rotation back, dR, the Cayley backward; the experts stream
+            # through the chunk buffer once more; dY and the logits in, dX, dQ and dlogits out
+            flops["gemm_bwd"] = gemm_flops
+            flops["rot_bwd"] = 2 * 2.0 * TK * spec.K * spec.b * 2
+            flops["cayley_bwd"] = 4.0 * spec.b ** 3 * n_active * 2 * (spec.K // spec.b)
+            total_flops = sum(flops.values())
+            nq = spec.E * 2 * (spec.K // spec.b) * (spec.b * (spec.b - 1) // 2)
+            alg_bytes += (n_active * (expert_bytes + chunk_buf_bytes) + 2 * spec.T * 2 * spec.n_proj
+                          + 2 * spec.T * spec.K + 2 * spec.T * spec.K + 4 * spec.T * spec.E + 2 * nq + 4 * nq)
     else:
         flops = linear_flops(spec, backward)
         total_flops = sum(flops.values())
@@ -423,7 +454,7 @@ def run_ours(args, rank, world):
         peak = peaks["hbm_gbs"]
         unit = "GB/s"
         traffic = None
-        kernel = "whole step (chunk dequant + grouped GEMM), HBM"
+        kernel = "whole step (chunk dequant + grouped GEMM" + (", forward and backward" if backward else "") + "), HBM"
     elif spec.M <= 128:
         # few tokens: the weight stream bounds the GEMM; bytes of one launch over its time
         wbytes = weight_bytes(spec)
@@ -484,7 +515,7 @@ def run_ours(args, rank, world):
         comp.wait_event(ev_out[b])               # read-back of step i-2 is done with dev_out[b]
         d = dev_in[b]
         if is_moe:
-            step(d["X"], d["logits"], d["Q"], o=dev_out[b])
+            step(d["X"], d["logits"], d["Q"], o=dev_out[b], dYi=d.get("dY"))
         elif backward:
             step(d["X"], d["dY"], d["Q"], o=dev_out[b])
         else:
@@ -521,13 +552,14 @@ def run_ours(args, rank, world):
         return None
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline_moe(case) if is_moe else cpu_baseline_linear(case, backward)
+        cpu = cpu_baseline_moe(case, dY=dY if backward else None) if is_moe else cpu_baseline_linear(case, backward)
     config = {"workload": WORKLOAD_NAMES[name], "name": name, "tokens_per_gpu": tokens,
               "global_batch_tokens": tokens * world, "parallelism": f"dp{world}" if world > 1 else "single",
               "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MB write)",
               "step": "build_rotation + fwd" + (" + bwd" if backward else "") + (" + dQ all-reduce" if world > 1 and backward else "")}
     if is_moe:
         config.update(n_active_experts=n_active, moe_variant=args.moe)
+        config["step"] = "route + build_rotation + fwd" + (" + bwd (dX, dQ, dlogits)" if backward else "")
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -547,17 +579,18 @@ def run_reference(args, rank, world):
     bounded sample of the same workload per step."""
     if rank != 0:
         return None
-    from gen import LINEAR_CONFIGS, MOE_CONFIGS, make_linear_case, make_moe_case
+    from gen import LINEAR_CONFIGS, MOE_CONFIGS, make_linear_case, make_moe_case, make_moe_grad
     name = args.workload
     if name in MOE_CONFIGS:
         import torch
         spec = MOE_CONFIGS[name]
         dev = "cuda" if torch.cuda.is_available() else "cpu"
         case = make_moe_case(spec, device=dev)
+        dY = make_moe_grad(spec, device=dev) if args.moe_backward else None
         per = max(2.0, 150.0 / (args.steps + args.warmup))
         for _ in range(args.warmup):
-            cpu_baseline_moe(case, budget_s=per / 4)
-        res = [cpu_baseline_moe(case, budget_s=per) for _ in range(args.steps)]
+            cpu_baseline_moe(case, budget_s=per / 4, dY=dY)
+        res = [cpu_baseline_moe(case, budget_s=per, dY=dY) for _ in range(args.steps)]
         value = statistics.mean(r["value"] for r in res)
         sample = res[-1]["sample"]
     else:
@@ -593,6 +626,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="c1", choices=sorted(WORKLOAD_NAMES))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--moe-backward", action="store_true",
+                    help="MoE workload: time forward + adapter backward (chunked path)")
     ap.add_argument("--moe", default="chunked", choices=["chunked", "fused"],
                     help="MoE workload: the pages' chunked dequant (default) or the fused-dequant grouped GEMM")
     args = ap.parse_args(argv)

@@ -169,6 +169,31 @@ int moe_fused_oft_fwd(const uint16_t* X, int T, const float* logits, int E, int 
                       int32_t* topk_idx, float* topk_w, int32_t* offsets, int32_t* bucket, int32_t* chunk_table,
                       int32_t* n_active, void* ws, size_t ws_bytes, void* stream);
 
+/* Bytes of scratch moe_chunked_oft_bwd needs: routing tables, the active experts'
+ * rotations, dY gathered in bucket order, two transposed bf16 chunk buffers,
+ * and fp32 per-slot gradients (2 x T*top_k x K for dY W^T, T*top_k x K for the
+ * rotated-back rows). */
+size_t moe_chunked_oft_bwd_workspace(int T, int E, int top_k, int chunk, const oft_weight* W_experts, int b);
+
+/* Adapter backward of the chunked MoE layer above (the frozen experts get no
+ * gradient; the pages train the adapters only: "技术细节" of m.xxlwj.com 771001).
+ * Inputs as for moe_chunked_oft_fwd, plus dY bf16 [T][2*n_proj] (gate | up), the
+ * gradient of Y.  The routing is recomputed from `logits` (it is deterministic).
+ * With D_p = dY_p[t] W_e,p^T for every (t, k) routed to e:
+ *   dX bf16 [T][K]          = sum_k w_tk sum_p D_p R_e,p^T;
+ *   dQ fp32 [E][2][K/b][b(b-1)/2], fully overwritten: the Cayley backward of
+ *       G_e,p = sum over e's entries of blockdiag(X_t^T w_tk D_p); zero for experts
+ *       that no token selected;
+ *   dlogits fp32 [T][E], fully overwritten (NULL: not computed): through the
+ *       softmax over the selected logits, w_tk (dw_tk - sum_j w_tj dw_tj) with
+ *       dw_tk = <dY[t], Y_tk>; zero for logits that were not selected.
+ * Each expert's weight is dequantised transposed, chunk by chunk, into a bf16
+ * buffer ([chunk][gate/up][K][n_proj]) and contracted by one grouped GEMM per chunk.
+ * Same limits as the forward; the result does not depend on scheduling. */
+int moe_chunked_oft_bwd(const uint16_t* dY, const uint16_t* X, int T, const float* logits, int E, int top_k,
+                        int chunk, const oft_weight* W_experts, int b, const uint16_t* Q_experts, uint16_t* dX,
+                        float* dQ, float* dlogits, void* ws, size_t ws_bytes, void* stream);
+
 /* ---- test hooks: single steps of the path, same kernels ---- */
 
 /* Dequantise a single weight to bf16: out [N][K] (transpose = 0) or [K][N]. */

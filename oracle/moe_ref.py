@@ -162,11 +162,15 @@ def moe_fwd_chunked(X_bits, logits, bank: ExpertBank, Q_bits, b: int, top_k: int
     return Y, routing
 
 
-def moe_bwd_direct(dY: np.ndarray, X_bits, logits, bank: ExpertBank, Q_bits, b: int, top_k: int, E: int):
+def moe_bwd_direct(dY: np.ndarray, X_bits, logits, bank: ExpertBank, Q_bits, b: int, top_k: int, E: int,
+                   tokens=None):
     """Backward of moe_fwd_direct, token by token in slot order.
 
     dY float64 [T][2n] (gate | up columns).  Returns (dX [T][K],
-    dq [E][2][K/b][b(b-1)/2], dlogits [T][E], dw [T][top_k])."""
+    dq [E][2][K/b][b(b-1)/2], dlogits [T][E], dw [T][top_k]).
+    `tokens` (optional) restricts the work to those tokens, for sampled checks of
+    large problems: the rows of dX, dlogits and dw of the other tokens stay zero,
+    and dq_e is complete only for experts all of whose tokens are listed."""
     X = bf16_bits_to_f64(X_bits)
     idx, w = topk(logits, top_k)
     T, K = X.shape
@@ -175,7 +179,8 @@ def moe_bwd_direct(dY: np.ndarray, X_bits, logits, bank: ExpertBank, Q_bits, b: 
     G = np.zeros((E, 2, nb, b, b))
     dw = np.zeros((T, top_k))
     Rs, Ws = {}, {}
-    for t in range(T):
+    tokens = range(T) if tokens is None else [int(t) for t in tokens]
+    for t in tokens:
         for k in range(top_k):
             e = int(idx[t, k])
             if e not in Rs:
@@ -191,7 +196,7 @@ def moe_bwd_direct(dY: np.ndarray, X_bits, logits, bank: ExpertBank, Q_bits, b: 
             dq[e, p] = cayley_grad(G[e, p], Rs[e][p], b)
     dlogits = np.zeros((T, E))
     s = (w * dw).sum(axis=1)
-    for t in range(T):
+    for t in tokens:
         for k in range(top_k):
             dlogits[t, idx[t, k]] = w[t, k] * (dw[t, k] - s[t])
     return dX, dq, dlogits, dw

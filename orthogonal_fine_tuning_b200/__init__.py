@@ -7,6 +7,8 @@ from .binding import (  # noqa: F401
     OFTError,
     Weight,
     library_path,
+    moe_chunked_oft_bwd,
+    moe_chunked_oft_bwd_workspace,
     moe_chunked_oft_fwd,
     moe_chunked_oft_workspace,
     moe_fused_oft_fwd,

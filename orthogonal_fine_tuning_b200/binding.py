@@ -209,6 +209,34 @@ def moe_fused_oft_fwd(X: torch.Tensor, logits: torch.Tensor, W: Weight, b: int, 
     return _moe_fwd(True, X, logits, W, b, Q, top_k, chunk, workspace, out, stream)
 
 
+def moe_chunked_oft_bwd_workspace(T: int, E: int, top_k: int, chunk: int, W: Weight, b: int) -> int:
+    cw = W.c()
+    return int(_L.moe_chunked_oft_bwd_workspace(T, E, top_k, chunk, ctypes.byref(cw), b))
+
+
+def moe_chunked_oft_bwd(dY: torch.Tensor, X: torch.Tensor, logits: torch.Tensor, W: Weight, b: int, Q: torch.Tensor,
+                        top_k: int, chunk: int, want_dlogits: bool = True, workspace: Optional[torch.Tensor] = None,
+                        out: Optional[dict] = None, stream=None) -> dict:
+    """Adapter backward of the chunked MoE layer: dX bf16 [T][K], dQ fp32
+    [E][2][K/b][b(b-1)/2] and (optionally) dlogits fp32 [T][E]."""
+    T, E = logits.shape
+    dev = X.device
+    nb = W.d_in // b
+    o = out if out is not None else dict(
+        dX=torch.empty(T, W.d_in, dtype=torch.bfloat16, device=dev),
+        dQ=torch.empty(E, 2, nb, b * (b - 1) // 2, dtype=torch.float32, device=dev),
+        dlogits=torch.empty(T, E, dtype=torch.float32, device=dev) if want_dlogits else None,
+    )
+    cw = W.c()
+    nbytes = int(_L.moe_chunked_oft_bwd_workspace(T, E, top_k, chunk, ctypes.byref(cw), b))
+    ws = _ws(nbytes, dev, workspace)
+    dl = o.get("dlogits")
+    _check(_L.moe_chunked_oft_bwd(
+        _ptr(_bits(dY)), _ptr(_bits(X)), T, _ptr(logits), E, top_k, chunk, ctypes.byref(cw), b, _ptr(_bits(Q)),
+        _ptr(o["dX"]), _ptr(o["dQ"]), _ptr(dl) if dl is not None else None, _ptr(ws), ws.numel(), _stream(stream)))
+    return o
+
+
 def oft_dequant_weight(W: Weight, transpose: bool = False, out: Optional[torch.Tensor] = None,
                        stream=None) -> torch.Tensor:
     if out is None:

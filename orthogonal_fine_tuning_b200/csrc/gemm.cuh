@@ -43,10 +43,13 @@ struct Group {
 };
 
 // MoE chunk: groups are derived on the device from the routing results.
+//   forward  (bwd = 0): Y_tk[pos][p n + j] = Xg[p][pos][:] . buf[slot][p n + j][:]   (contract over K)
+//   backward (bwd = 1): D[p][pos][c]      = dYg[p][pos][:] . buft[slot][p][c][:]    (contract over n)
 struct MoESrc {
   const int* chunk_table;  // [n_chunks][chunk], -1 padded
   const int* offsets;      // [E+1]
   int chunk_idx, chunk, TK, n_proj, K;
+  int bwd;
 };
 
 struct Params {
@@ -134,14 +137,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_bf16_kernel(const __grid_
         for (int proj = 0; proj < 2; ++proj) {
           Group g{};
           g.m = cnt;
-          g.n = s.n_proj;
-          g.k = s.K;
           g.a_map = 0;
           g.b_map = 0;
           g.a_row0 = proj * s.TK + s.offsets[e];
-          g.b_row0 = (slot * 2 + proj) * s.n_proj;
-          g.c_row0 = s.offsets[e];
-          g.c_col0 = proj * s.n_proj;
+          if (s.bwd) {
+            g.n = s.K;
+            g.k = s.n_proj;
+            g.b_row0 = (slot * 2 + proj) * s.K;
+            g.c_row0 = proj * s.TK + s.offsets[e];
+            g.c_col0 = 0;
+          } else {
+            g.n = s.n_proj;
+            g.k = s.K;
+            g.b_row0 = (slot * 2 + proj) * s.n_proj;
+            g.c_row0 = s.offsets[e];
+            g.c_col0 = proj * s.n_proj;
+          }
           add(g);
         }
       }

@@ -24,6 +24,7 @@
 #include "gemm_dq.cuh"
 #include "gemm_dq2.cuh"
 #include "moe_fused.cuh"
+#include "moe_bwd.cuh"
 
 using namespace oftk;
 
@@ -1122,6 +1123,190 @@ int moe_oft_fwd_impl(bool fused, const uint16_t* X, int T, const float* logits, 
 }
 
 }  // namespace
+
+// ---------------------------------------------------------------------------
+// MoE backward
+// ---------------------------------------------------------------------------
+namespace {
+struct MoeBwdLayout {
+  size_t idx, w, offsets, bucket, table, meta, order, inv, pexp, rex, dyg, buf, d, u, dwp, total;
+};
+MoeBwdLayout moe_bwd_layout(int T, int E, int top_k, int chunk, int K, int N, int b) {
+  MoeBwdLayout L{};
+  const size_t TK = 1ull * T * top_k, n = N / 2, nb = K / b;
+  const size_t n_chunks_max = (E + chunk - 1) / chunk;
+  L.idx = 0;
+  L.w = round_up(L.idx + 4 * TK, 256);
+  L.offsets = round_up(L.w + 4 * TK, 256);
+  L.bucket = round_up(L.offsets + 4ull * (E + 1), 256);
+  L.table = round_up(L.bucket + 4 * TK, 256);
+  L.meta = round_up(L.table + 4 * n_chunks_max * chunk, 256);  // [0] n_active, [1] unit counter
+  L.order = round_up(L.meta + 16, 256);
+  L.inv = round_up(L.order + 4ull * E, 256);
+  L.pexp = round_up(L.inv + 4 * TK, 256);
+  L.rex = round_up(L.pexp + 4 * TK, 256);
+  L.dyg = round_up(L.rex + 4ull * E * 2 * nb * b * b, 256);
+  L.buf = round_up(L.dyg + 2 * 2 * TK * n, 256);
+  L.d = round_up(L.buf + 2ull * 2 * chunk * N * K, 256);  // two transposed chunk buffers
+  L.u = round_up(L.d + 4 * 2 * TK * K, 256);
+  L.dwp = round_up(L.u + 4 * TK * K, 256);
+  L.total = round_up(L.dwp + 4 * TK * nb, 256);
+  return L;
+}
+
+template <int B>
+int launch_moe_bwd_rot(const float* D, const uint16_t* X, int K, int TK, int top_k, const int* bucket,
+                       const int* offsets, const float* w, const int* order, const int* n_active, int* counter,
+                       const float* R, float* U, float* dwp, float* dQ, cudaStream_t st) {
+  constexpr size_t smem = MoeBwdCfg<B>::SMEM;
+  if (int rc = set_smem(moe_bwd_rot_kernel<B>, smem)) return rc;
+  int per_sm = 0;
+  OFT_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, moe_bwd_rot_kernel<B>, 256, smem));
+  moe_bwd_rot_kernel<B><<<sm_count() * std::max(1, per_sm), 256, smem, st>>>(D, X, K, TK, top_k, bucket, offsets, w,
+                                                                             order, n_active, counter, R, U, dwp, dQ);
+  OFT_LAUNCHED("moe_bwd_rot_kernel");
+  return OFT_OK;
+}
+}  // namespace
+
+extern "C" {
+
+size_t moe_chunked_oft_bwd_workspace(int T, int E, int top_k, int chunk, const oft_weight* W, int b) {
+  if (W == nullptr || T <= 0 || E <= 0 || top_k <= 0 || chunk <= 0 || b <= 0) return 0;
+  return moe_bwd_layout(T, E, top_k, chunk, W->d_in, W->d_out, b).total;
+}
+
+int moe_chunked_oft_bwd(const uint16_t* dY, const uint16_t* X, int T, const float* logits, int E, int top_k,
+                        int chunk, const oft_weight* W, int b, const uint16_t* Q, uint16_t* dX, float* dQ,
+                        float* dlogits, void* ws, size_t ws_bytes, void* stream) {
+  if (int rc = check_weight(W, true)) return rc;
+  if (W->fmt != OFT_W_INT4) return fail(OFT_ERR_UNSUPPORTED, "the MoE expert bank must be INT4");
+  const int K = W->d_in, N = W->d_out;
+  if (int rc = check_b(b, K)) return rc;
+  if (T <= 0) return fail(OFT_ERR_INVALID_ARG, "T must be positive");
+  if (E < 1 || E > kMaxExperts || W->n_experts != E)
+    return fail(OFT_ERR_UNSUPPORTED, "E must be 1..%d and match the bank's n_experts", kMaxExperts);
+  if (top_k < 1 || top_k > kMaxTopK || top_k > E) return fail(OFT_ERR_UNSUPPORTED, "top_k must be 1..%d", kMaxTopK);
+  if (chunk < 1 || chunk > gemm::MAX_GROUPS / 2) return fail(OFT_ERR_UNSUPPORTED, "chunk must be 1..%d", gemm::MAX_GROUPS / 2);
+  if (N % 16 != 0) return fail(OFT_ERR_UNSUPPORTED, "expert d_out (gate+up) must be a multiple of 16");
+  if (1ll * T * top_k * 2 > (1ll << 31) - 1 || 1ll * E * 2 * K > (1ll << 31) - 1)
+    return fail(OFT_ERR_UNSUPPORTED, "too many routed rows");
+  const void* ptrs[] = {dY, X, logits, Q, dX, dQ, ws};
+  for (const void* q : ptrs)
+    if (q == nullptr || !aligned16(q)) return fail(OFT_ERR_INVALID_ARG, "NULL or misaligned pointer");
+  if (dlogits != nullptr && !aligned16(dlogits)) return fail(OFT_ERR_INVALID_ARG, "misaligned dlogits");
+  const int n_proj = N / 2, TK = T * top_k, nb = K / b;
+  const int n_chunks_max = (E + chunk - 1) / chunk;
+  const MoeBwdLayout L = moe_bwd_layout(T, E, top_k, chunk, K, N, b);
+  if (ws_bytes < L.total) return fail(OFT_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
+  cudaStream_t st = as_stream(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  int* idx = reinterpret_cast<int*>(wsb + L.idx);
+  float* wts = reinterpret_cast<float*>(wsb + L.w);
+  int* offsets = reinterpret_cast<int*>(wsb + L.offsets);
+  int* bucket = reinterpret_cast<int*>(wsb + L.bucket);
+  int* table = reinterpret_cast<int*>(wsb + L.table);
+  int* n_active = reinterpret_cast<int*>(wsb + L.meta);
+  int* counter = n_active + 1;
+  int* order = reinterpret_cast<int*>(wsb + L.order);
+  int* inv = reinterpret_cast<int*>(wsb + L.inv);
+  int* pexp = reinterpret_cast<int*>(wsb + L.pexp);
+  float* Rex = reinterpret_cast<float*>(wsb + L.rex);
+  uint16_t* dYg = reinterpret_cast<uint16_t*>(wsb + L.dyg);
+  uint16_t* buf = reinterpret_cast<uint16_t*>(wsb + L.buf);
+  float* D = reinterpret_cast<float*>(wsb + L.d);
+  float* U = reinterpret_cast<float*>(wsb + L.u);
+  float* dwp = reinterpret_cast<float*>(wsb + L.dwp);
+
+  // 1. routing, as in the forward
+  {
+    ProfScope ps(OFT_K_ROUTE, st);
+    moe_topk_kernel<<<(T * 32 + 255) / 256, 256, 0, st>>>(logits, T, E, top_k, idx, wts);
+    OFT_LAUNCHED("moe_topk_kernel");
+  }
+  const size_t rsmem = sizeof(int) * (32 * E + 2 * E + 1);
+  OFT_CUDA(cudaFuncSetAttribute(moe_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(rsmem)));
+  {
+    ProfScope ps(OFT_K_ROUTE, st);
+    moe_route_kernel<<<1, 1024, rsmem, st>>>(idx, TK, E, chunk, n_chunks_max, offsets, bucket, inv, pexp, table,
+                                            n_active);
+    OFT_LAUNCHED("moe_route_kernel");
+    moe_order_kernel<<<1, 1024, 0, st>>>(offsets, table, n_active, order, counter);
+    OFT_LAUNCHED("moe_order_kernel");
+    const long long gunits = 1ll * TK * (N / 8);
+    moe_gather_dy_kernel<<<static_cast<int>(std::min<long long>((gunits + 255) / 256, 148ll * 16)), 256, 0, st>>>(
+        dY, bucket, TK, top_k, n_proj, dYg);
+    OFT_LAUNCHED("moe_gather_dy_kernel");
+  }
+  // 2. rotations of the active experts
+  if (int rc = launch_cayley(Q, E * 2 * nb, b, Rex, table, n_active, 2 * nb, st)) return rc;
+  // 3. chunks: transposed dequant of the chunk's experts (side stream, double-buffered),
+  //    then one grouped GEMM D[p][pos][:] = dYg[p][pos][:] W_e,p^T
+  gemm::Params prm;
+  memset(&prm, 0, sizeof(prm));
+  if (int rc = make_map_bf16(&prm.tmA[0], dYg, n_proj, 2ull * TK, n_proj, gemm::BM)) return rc;
+  for (int i = 1; i < gemm::MAX_MAPS; ++i) prm.tmA[i] = prm.tmA[0];
+  prm.C = D;
+  prm.c_f32 = 1;
+  prm.ldc = K;
+  prm.use_moe = 1;
+  prm.moe.chunk_table = table;
+  prm.moe.offsets = offsets;
+  prm.moe.chunk = chunk;
+  prm.moe.TK = TK;
+  prm.moe.n_proj = n_proj;
+  prm.moe.K = K;
+  prm.moe.bwd = 1;
+  const WeightView bank = view_of(W);
+  SidePipe* sp = nullptr;
+  if (int rc = side_pipe(&sp)) return rc;
+  OFT_CUDA(cudaEventRecord(sp->start, st));
+  OFT_CUDA(cudaStreamWaitEvent(sp->side, sp->start, 0));
+  const size_t buf_elems = 1ull * chunk * N * K;
+  for (int c = 0; c < n_chunks_max; ++c) {
+    const int h = c & 1;
+    uint16_t* bufc = buf + h * buf_elems;
+    if (c >= 2) OFT_CUDA(cudaStreamWaitEvent(sp->side, sp->gemm_done[h], 0));
+    {
+      ProfScope ps(OFT_K_DEQUANT, sp->side);
+      moe_chunk_dequant_t_kernel<<<dim3((K + 63) / 64, (N + 63) / 64, chunk), 256, 0, sp->side>>>(bank, table, c, chunk,
+                                                                                                  n_proj, bufc);
+      OFT_LAUNCHED("moe_chunk_dequant_t_kernel");
+    }
+    OFT_CUDA(cudaEventRecord(sp->dq_done[h], sp->side));
+    OFT_CUDA(cudaStreamWaitEvent(st, sp->dq_done[h], 0));
+    prm.moe.chunk_idx = c;
+    if (int rc = make_map_bf16(&prm.tmB[0], bufc, n_proj, 2ull * chunk * K, n_proj, gemm::BN)) return rc;
+    for (int i = 1; i < gemm::MAX_MAPS; ++i) prm.tmB[i] = prm.tmB[0];
+    if (int rc = launch_gemm(prm, 0, st)) return rc;
+    OFT_CUDA(cudaEventRecord(sp->gemm_done[h], st));
+  }
+  // 4. per (active expert, block): rows rotated back, dw partials, dR and the Cayley backward
+  OFT_CUDA(cudaMemsetAsync(dQ, 0, sizeof(float) * E * 2 * nb * (b * (b - 1) / 2), st));
+  {
+    ProfScope ps(OFT_K_GRAD, st);
+    int rc = OFT_OK;
+    if (b == 16) rc = launch_moe_bwd_rot<16>(D, X, K, TK, top_k, bucket, offsets, wts, order, n_active, counter, Rex, U, dwp, dQ, st);
+    if (b == 32) rc = launch_moe_bwd_rot<32>(D, X, K, TK, top_k, bucket, offsets, wts, order, n_active, counter, Rex, U, dwp, dQ, st);
+    if (b == 64) rc = launch_moe_bwd_rot<64>(D, X, K, TK, top_k, bucket, offsets, wts, order, n_active, counter, Rex, U, dwp, dQ, st);
+    if (rc) return rc;
+  }
+  // 5. dX[t] = sum_k w_tk U[pos(t, k)] in slot order; logit gradients
+  {
+    ProfScope ps(OFT_K_ROUTE, st);
+    const long long cunits = 1ll * T * (K / 8);
+    const int cgrid = static_cast<int>(std::min<long long>((cunits + 255) / 256, 148ll * 16));
+    moe_combine_kernel<<<cgrid, 256, 0, st>>>(U, wts, inv, T, K, top_k, dX);
+    OFT_LAUNCHED("moe_combine_kernel");
+    if (dlogits != nullptr) {
+      moe_dlogits_kernel<<<(T * 32 + 255) / 256, 256, 0, st>>>(dwp, nb, idx, wts, inv, T, E, top_k, dlogits);
+      OFT_LAUNCHED("moe_dlogits_kernel");
+    }
+  }
+  return OFT_OK;
+}
+
+}  // extern "C"
 
 // ---------------------------------------------------------------------------
 // bounded-wait self test

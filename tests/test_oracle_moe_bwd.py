@@ -110,3 +110,18 @@ def test_single_expert_reduces_to_split_linear_backward():
     assert np.abs(dq[1] - dql).max() <= 1e-12 * np.abs(dql).max()
     assert not dq[[0, 2, 3]].any()
     assert not dlog.any()
+
+
+def test_token_subset_gives_the_same_rows_and_complete_experts():
+    spec = _tiny(T=12, K=16, E=7, n_proj=4, top_k=2, b=8)
+    case, bank, dY = _setup(spec)
+    Xb, logits, Qb = raw(case["X"]), raw(case["logits"]), raw(case["Q"])
+    full = moe_ref.moe_bwd_direct(dY, Xb, logits, bank, Qb, spec.b, spec.top_k, spec.E)
+    idx, _ = moe_ref.topk(logits, spec.top_k)
+    e = int(idx[3, 0])
+    toks = sorted(set(np.nonzero((idx == e).any(axis=1))[0].tolist()) | {0, 5})
+    part = moe_ref.moe_bwd_direct(dY, Xb, logits, bank, Qb, spec.b, spec.top_k, spec.E, tokens=toks)
+    for a, b in zip(full, part):
+        if a.shape[0] == spec.T:
+            assert np.array_equal(a[toks], b[toks])
+    assert np.abs(full[1][e] - part[1][e]).max() <= 1e-13 * np.abs(full[1][e]).max()

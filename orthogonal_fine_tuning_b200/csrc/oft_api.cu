@@ -1269,7 +1269,8 @@ int moe_chunked_oft_bwd(const uint16_t* dY, const uint16_t* X, int T, const floa
     if (c >= 2) OFT_CUDA(cudaStreamWaitEvent(sp->side, sp->gemm_done[h], 0));
     {
       ProfScope ps(OFT_K_DEQUANT, sp->side);
-      moe_chunk_dequant_t_kernel<<<dim3((K + 63) / 64, (N + 63) / 64, chunk), 256, 0, sp->side>>>(bank, table, c, chunk,
+      moe_chunk_dequant_t_kernel<<<dim3((K + 64 * kDqtStrip - 1) / (64 * kDqtStrip), (N + 63) / 64, chunk), 256, 0,
+                                   sp->side>>>(bank, table, c, chunk,
                                                                                                   n_proj, bufc);
       OFT_LAUNCHED("moe_chunk_dequant_t_kernel");
     }

@@ -8,10 +8,10 @@
 // are groups of one launch (item "自定义适配器核函数"), and the backward forms only
 // the activation gradient (m.xxlwj.com 771001, section "技术细节").
 //
-// Here a cluster of two CTAs computes a 256-row weight tile against 320 tokens:
+// Here a cluster of two CTAs computes a 256-row weight tile against 384 tokens:
 // each CTA decodes its own 128 weight rows into its own TMEM, and loads only its
-// 80-token half of each 160-token activation tile.  The leader CTA issues
-// tcgen05.mma.cta_group::2 (M = 256, N = 160): the tensor cores of both SMs work
+// 96-token half of each 192-token activation tile.  The leader CTA issues
+// tcgen05.mma.cta_group::2 (M = 256, N = 192): the tensor cores of both SMs work
 // on one instruction, every activation byte a CTA loads feeds 256 weight rows, and
 // each SM's L2 -> shared-memory traffic halves against the one-CTA kernel.
 //
@@ -26,7 +26,7 @@
 //              tcgen05.commit multicast to both CTAs
 //   acc_empty[h] leader's; both CTAs' epilogue threads arrive
 //   s_full[s]  each CTA's own (backward scale tiles for its decode warps)
-// Activation stages (6) and TMEM weight slots (6) are separate rings: the slot
+// Activation stages (6) and TMEM weight slots (4) are separate rings: the slot
 // hand-off crosses both SMs, so the weight ring is as deep as TMEM allows.
 #pragma once
 

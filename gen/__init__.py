@@ -14,6 +14,7 @@ from .workloads import (  # noqa: F401
     MOE_CONFIGS,
     make_linear_case,
     make_moe_case,
+    make_moe_down,
     make_moe_grad,
     make_moe_router,
     split_offsets,

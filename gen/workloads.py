@@ -238,6 +238,27 @@ def make_moe_grad(spec: MoESpec, device="cpu"):
     return torch.randn(spec.T, 2 * spec.n_proj, generator=g, device=device).to(torch.bfloat16)
 
 
+def make_moe_down(spec: MoESpec, device="cpu", experts: Optional[Sequence[int]] = None):
+    """Down projections of a full expert layer (d_in = n_proj, d_out = K) and their
+    adapters: codes uint8 [E][K][n_proj/2], scales bf16 [E][n_proj/G][K] (INT4, group
+    G along n_proj), Q_down bf16 [E][n_proj/b][b(b-1)/2].  One generator per expert,
+    as for the gate/up bank."""
+    g = torch.Generator(device=device)
+    g.manual_seed(5000 + spec.seed)
+    qd = _draw_q(1, spec.n_proj, spec.b, spec.q_sigma, g, device, lead=(spec.E,))[:, 0].contiguous()
+    codes = torch.zeros(spec.E, spec.K, spec.n_proj // 2, dtype=torch.uint8, device=device)
+    scales = torch.ones(spec.E, spec.n_proj // spec.group, spec.K, dtype=torch.bfloat16, device=device)
+    wspec = LinearSpec("down", M=0, K=spec.n_proj, splits=(spec.K,), fmt=FMT_INT4, group=spec.group, b=spec.b,
+                       q_sigma=0.0, w_sigma=spec.w_sigma)
+    ge = torch.Generator(device=device)
+    for e in (range(spec.E) if experts is None else experts):
+        ge.manual_seed(200000 + 1000 * spec.seed + e)
+        c, s_ = _draw_weight(wspec, spec.K, ge, device)
+        codes[e].copy_(c)
+        scales[e].copy_(s_)
+    return dict(down_codes=codes, down_scales=scales, Q_down=qd)
+
+
 def make_moe_case(spec: MoESpec, device="cpu", experts: Optional[Sequence[int]] = None):
     """Draw one chunked-MoE OFT problem.
 

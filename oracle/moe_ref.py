@@ -22,6 +22,14 @@ readings taken here are:
     experts are those with a non-zero count, ascending; chunk c holds
     active[c*C : (c+1)*C], the last one possibly partial.
 
+Full expert layer (the step after the gate/up output above): each expert also has
+a down projection W_e,down (d_in = n, d_out = K) with its own OFT rotation on its
+input, and the gated activation between them is SwiGLU:
+
+  h_tk  = silu(g_tk) * u_tk,            [g_tk | u_tk] = Y_tk,  silu(x) = x sigmoid(x)
+  Z_tk  = (h_tk R_e,down) W_e,down
+  Y_t   = sum_k w_tk Z_tk
+
 Backward (the pages train these expert layers through the adapter only; the
 frozen expert weights get no gradient).  With D_p,tk = dY_p[t] W_e,p^T (e =
 idx[t, k], p = gate / up):
@@ -200,3 +208,50 @@ def moe_bwd_direct(dY: np.ndarray, X_bits, logits, bank: ExpertBank, Q_bits, b: 
         for k in range(top_k):
             dlogits[t, idx[t, k]] = w[t, k] * (dw[t, k] - s[t])
     return dX, dq, dlogits, dw
+
+
+def silu(x):
+    """x * sigmoid(x); sigmoid from exp(-|x|) on both branches, so neither overflows
+    nor cancels: 1 / (1 + e^-x) for x >= 0, e^x / (1 + e^x) for x < 0."""
+    x = np.asarray(x, dtype=np.float64)
+    z = np.exp(-np.abs(x))
+    sig = np.where(x >= 0, 1.0 / (1.0 + z), z / (1.0 + z))
+    return x * sig
+
+
+class DownBank(ExpertBank):
+    """INT4 down projections: codes uint8 [E][K][n/2], scales bf16 bits [E][n/G][K];
+    weight_t(e) is deq(W_e,down)^T [K][n] (one row per output channel)."""
+
+    def __init__(self, codes, scales_bits, n: int, group: int):
+        super().__init__(codes, scales_bits, n, group, 0)
+
+    def weight_t(self, e: int, rows=None) -> np.ndarray:
+        return dequant("int4", self.codes[e], self.scales[e], self.K, self.group, rows=rows)
+
+
+def expert_layer(X: np.ndarray, e: int, bank: ExpertBank, down: DownBank, Qe_bits, Qd_bits, b: int):
+    """Z for tokens X [m][K] through expert e: [m][K] = (silu(g) u R_e,down) W_e,down."""
+    Y = expert_outputs(X, e, bank, Qe_bits, b)
+    n = bank.n
+    h = silu(Y[:, :n]) * Y[:, n:]
+    Rd = rotations(Qd_bits, b)                                  # [n/b][b][b]
+    return rotate(h, Rd) @ down.weight_t(e).T
+
+
+def moe_layer_direct(X_bits, logits, bank: ExpertBank, down: DownBank, Q_bits, Qd_bits, b: int, top_k: int,
+                     tokens=None):
+    """Y[t] = sum_k w_tk Z_tk for the full expert layer, token by token in slot order.
+
+    Q_bits: gate/up adapters [E][2][K/b][b(b-1)/2]; Qd_bits: down adapters
+    [E][n/b][b(b-1)/2].  `tokens` optionally restricts the rows computed."""
+    X = bf16_bits_to_f64(X_bits)
+    idx, w = topk(logits, top_k)
+    T, K = X.shape
+    tokens = np.arange(T) if tokens is None else np.asarray(tokens)
+    Y = np.zeros((len(tokens), K))
+    for i, t in enumerate(tokens):
+        for k in range(top_k):
+            e = int(idx[t, k])
+            Y[i] += w[t, k] * expert_layer(X[t:t + 1], e, bank, down, Q_bits[e], Qd_bits[e], b)[0]
+    return Y

@@ -169,6 +169,25 @@ int moe_fused_oft_fwd(const uint16_t* X, int T, const float* logits, int E, int 
                       int32_t* topk_idx, float* topk_w, int32_t* offsets, int32_t* bucket, int32_t* chunk_table,
                       int32_t* n_active, void* ws, size_t ws_bytes, void* stream);
 
+/* Bytes of scratch moe_chunked_oft_layer_fwd needs: that of moe_chunked_oft_fwd plus
+ * the routing tables, the down adapters' rotations, the gated activations (bf16
+ * [T*top_k][n_proj]) and the per-slot down outputs (fp32 [T*top_k][d_in]). */
+size_t moe_chunked_oft_layer_workspace(int T, int E, int top_k, int chunk, const oft_weight* W_experts,
+                                       const oft_weight* W_down, int b);
+
+/* Full MoE expert layer, forward: the chunked gate/up projections above, SwiGLU, and
+ * a down projection with its own OFT adapter, every expert weight INT4 and
+ * dequantised chunk by chunk ("技术细节" of m.xxlwj.com 771001).  For every (t, k)
+ * routed to e, with [g | u] = [X_t R_e,g W_e,g | X_t R_e,u W_e,u]:
+ *   h = silu(g) * u (fp32),  Z_tk = (h R_e,down) W_e,down,  Y_t = sum_k w_tk Z_tk.
+ * W_down: INT4 bank with d_in = n_proj, d_out = d_in of W_experts (one row per output
+ * channel, n_experts = E); Q_down bf16 [E][n_proj/b][b(b-1)/2].  Y bf16 [T][K].
+ * h R_e,down is rounded to bf16 as the GEMM operand; everything else accumulates in
+ * fp32.  Same limits as moe_chunked_oft_fwd, and n_proj % b == 0. */
+int moe_chunked_oft_layer_fwd(const uint16_t* X, int T, const float* logits, int E, int top_k, int chunk,
+                              const oft_weight* W_experts, const oft_weight* W_down, int b, const uint16_t* Q_experts,
+                              const uint16_t* Q_down, uint16_t* Y, void* ws, size_t ws_bytes, void* stream);
+
 /* Bytes of scratch moe_chunked_oft_bwd needs: routing tables, the active experts'
  * rotations, dY gathered in bucket order, two transposed bf16 chunk buffers,
  * and fp32 per-slot gradients (2 x T*top_k x K for dY W^T, T*top_k x K for the

@@ -10,6 +10,8 @@ from .binding import (  # noqa: F401
     moe_chunked_oft_bwd,
     moe_chunked_oft_bwd_workspace,
     moe_chunked_oft_fwd,
+    moe_chunked_oft_layer_fwd,
+    moe_chunked_oft_layer_workspace,
     moe_chunked_oft_workspace,
     moe_fused_oft_fwd,
     moe_fused_oft_workspace,

@@ -26,7 +26,8 @@ EXPORTS = (
     "moe_chunked_oft_workspace", "moe_chunked_oft_fwd", "oft_dequant_weight", "oft_rotate",
     "oft_cayley_backward", "oft_debug_bounded_wait", "oft_profile_begin", "oft_profile_end",
     "oft_linear_fwd_noalloc", "oft_set_gemm_mode", "moe_fused_oft_workspace", "moe_fused_oft_fwd",
-    "moe_chunked_oft_bwd_workspace", "moe_chunked_oft_bwd",
+    "moe_chunked_oft_bwd_workspace", "moe_chunked_oft_bwd", "moe_chunked_oft_layer_workspace",
+    "moe_chunked_oft_layer_fwd",
 )
 
 
@@ -61,6 +62,8 @@ _SIGS = {
     "moe_fused_oft_fwd": (_I, [_P, _I, _P, _I, _I, _I, _WP, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _Z, _P]),
     "moe_chunked_oft_bwd_workspace": (_Z, [_I, _I, _I, _I, _WP, _I]),
     "moe_chunked_oft_bwd": (_I, [_P, _P, _I, _P, _I, _I, _I, _WP, _I, _P, _P, _P, _P, _P, _Z, _P]),
+    "moe_chunked_oft_layer_workspace": (_Z, [_I, _I, _I, _I, _WP, _WP, _I]),
+    "moe_chunked_oft_layer_fwd": (_I, [_P, _I, _P, _I, _I, _I, _WP, _WP, _I, _P, _P, _P, _P, _Z, _P]),
     "oft_dequant_weight": (_I, [_WP, _P, _I, _P]),
     "oft_rotate": (_I, [_P, _I, _I, _I, _I, _P, _P, _P]),
     "oft_cayley_backward": (_I, [_P, _P, _I, _I, _P, _P]),

@@ -237,6 +237,28 @@ def moe_chunked_oft_bwd(dY: torch.Tensor, X: torch.Tensor, logits: torch.Tensor,
     return o
 
 
+def moe_chunked_oft_layer_workspace(T: int, E: int, top_k: int, chunk: int, W: Weight, W_down: Weight, b: int) -> int:
+    cw, cd = W.c(), W_down.c()
+    return int(_L.moe_chunked_oft_layer_workspace(T, E, top_k, chunk, ctypes.byref(cw), ctypes.byref(cd), b))
+
+
+def moe_chunked_oft_layer_fwd(X: torch.Tensor, logits: torch.Tensor, W: Weight, W_down: Weight, b: int,
+                              Q: torch.Tensor, Q_down: torch.Tensor, top_k: int, chunk: int,
+                              workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                              stream=None) -> torch.Tensor:
+    """Full expert layer: Y bf16 [T][K] = sum_k w_tk ((silu(g) u) R_e,down) W_e,down, with
+    [g | u] the chunked gate/up outputs of expert e."""
+    T, E = logits.shape
+    Y = out if out is not None else torch.empty(T, W.d_in, dtype=torch.bfloat16, device=X.device)
+    cw, cd = W.c(), W_down.c()
+    nbytes = int(_L.moe_chunked_oft_layer_workspace(T, E, top_k, chunk, ctypes.byref(cw), ctypes.byref(cd), b))
+    ws = _ws(nbytes, X.device, workspace)
+    _check(_L.moe_chunked_oft_layer_fwd(
+        _ptr(_bits(X)), T, _ptr(logits), E, top_k, chunk, ctypes.byref(cw), ctypes.byref(cd), b, _ptr(_bits(Q)),
+        _ptr(_bits(Q_down)), _ptr(Y), _ptr(ws), ws.numel(), _stream(stream)))
+    return Y
+
+
 def oft_dequant_weight(W: Weight, transpose: bool = False, out: Optional[torch.Tensor] = None,
                        stream=None) -> torch.Tensor:
     if out is None:

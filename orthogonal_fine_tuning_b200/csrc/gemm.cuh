@@ -43,13 +43,15 @@ struct Group {
 };
 
 // MoE chunk: groups are derived on the device from the routing results.
-//   forward  (bwd = 0): Y_tk[pos][p n + j] = Xg[p][pos][:] . buf[slot][p n + j][:]   (contract over K)
-//   backward (bwd = 1): D[p][pos][c]      = dYg[p][pos][:] . buft[slot][p][c][:]    (contract over n)
+//   gate/up  (mode 0): Y_tk[pos][p n + j] = Xg[p][pos][:] . buf[slot][p n + j][:]   (contract over K)
+//   backward (mode 1): D[p][pos][c]      = dYg[p][pos][:] . buft[slot][p][c][:]    (contract over n)
+//   down     (mode 2): Z[pos][c]         = Hg[pos][:] . bufd[slot][c][:]           (contract over n)
+enum : int { kMoeGateUp = 0, kMoeBwd = 1, kMoeDown = 2 };
 struct MoESrc {
   const int* chunk_table;  // [n_chunks][chunk], -1 padded
   const int* offsets;      // [E+1]
   int chunk_idx, chunk, TK, n_proj, K;
-  int bwd;
+  int mode;
 };
 
 struct Params {
@@ -134,13 +136,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_bf16_kernel(const __grid_
         if (e < 0) continue;
         const int cnt = s.offsets[e + 1] - s.offsets[e];
         if (cnt <= 0) continue;
-        for (int proj = 0; proj < 2; ++proj) {
+        for (int proj = 0; proj < (s.mode == kMoeDown ? 1 : 2); ++proj) {
           Group g{};
           g.m = cnt;
           g.a_map = 0;
           g.b_map = 0;
           g.a_row0 = proj * s.TK + s.offsets[e];
-          if (s.bwd) {
+          if (s.mode == kMoeDown) {
+            g.n = s.K;
+            g.k = s.n_proj;
+            g.b_row0 = slot * s.K;
+            g.c_row0 = s.offsets[e];
+            g.c_col0 = 0;
+          } else if (s.mode == kMoeBwd) {
             g.n = s.K;
             g.k = s.n_proj;
             g.b_row0 = (slot * 2 + proj) * s.K;

@@ -25,6 +25,7 @@
 #include "gemm_dq2.cuh"
 #include "moe_fused.cuh"
 #include "moe_bwd.cuh"
+#include "moe_layer.cuh"
 
 using namespace oftk;
 
@@ -923,7 +924,7 @@ MoeLayout moe_layout(int T, int E, int top_k, int chunk, int K, int N, int b, bo
 int moe_oft_fwd_impl(bool fused, const uint16_t* X, int T, const float* logits, int E, int top_k, int chunk,
                      const oft_weight* W, int b, const uint16_t* Q, uint16_t* Y, int32_t* topk_idx, float* topk_w,
                      int32_t* offsets, int32_t* bucket, int32_t* chunk_table, int32_t* n_active, void* ws,
-                     size_t ws_bytes, void* stream);
+                     size_t ws_bytes, void* stream, bool combine = true);
 }  // namespace
 
 size_t moe_chunked_oft_workspace(int T, int E, int top_k, int chunk, const oft_weight* W, int b) {
@@ -955,10 +956,12 @@ int moe_fused_oft_fwd(const uint16_t* X, int T, const float* logits, int E, int 
 }  // extern "C"
 
 namespace {
+// combine = false stops before the weighted combine and leaves the per-slot outputs
+// Ytk (fp32, bucket order), inv_pos and pos_expert in the workspace (full expert layer).
 int moe_oft_fwd_impl(bool fused, const uint16_t* X, int T, const float* logits, int E, int top_k, int chunk,
                      const oft_weight* W, int b, const uint16_t* Q, uint16_t* Y, int32_t* topk_idx, float* topk_w,
                      int32_t* offsets, int32_t* bucket, int32_t* chunk_table, int32_t* n_active, void* ws,
-                     size_t ws_bytes, void* stream) {
+                     size_t ws_bytes, void* stream, bool combine) {
   if (int rc = check_weight(W, true)) return rc;
   if (W->fmt != OFT_W_INT4) return fail(OFT_ERR_UNSUPPORTED, "the MoE expert bank must be INT4");
   const int K = W->d_in, N = W->d_out;
@@ -970,7 +973,8 @@ int moe_oft_fwd_impl(bool fused, const uint16_t* X, int T, const float* logits, 
   if (chunk < 1 || chunk > gemm::MAX_GROUPS / 2) return fail(OFT_ERR_UNSUPPORTED, "chunk must be 1..%d", gemm::MAX_GROUPS / 2);
   if (N % 16 != 0) return fail(OFT_ERR_UNSUPPORTED, "expert d_out (gate+up) must be a multiple of 16");
   if (1ll * T * top_k * 2 > (1ll << 31) - 1) return fail(OFT_ERR_UNSUPPORTED, "too many routed rows");
-  const void* ptrs[] = {X, logits, Q, Y, topk_idx, topk_w, offsets, bucket, chunk_table, n_active, ws};
+  const void* ptrs[] = {X, logits, Q, combine ? static_cast<const void*>(Y) : ws, topk_idx, topk_w, offsets, bucket,
+                        chunk_table, n_active, ws};
   for (const void* q : ptrs)
     if (q == nullptr || !aligned16(q)) return fail(OFT_ERR_INVALID_ARG, "NULL or misaligned pointer");
   const int n_proj = N / 2, TK = T * top_k, nb = K / b;
@@ -1113,6 +1117,7 @@ int moe_oft_fwd_impl(bool fused, const uint16_t* X, int T, const float* logits, 
     OFT_CUDA(cudaEventRecord(sp->gemm_done[h], st));
   }
   }
+  if (!combine) return OFT_OK;
   // 6. weighted combine in slot order
   const long long cunits = 1ll * T * (N / 8);
   const int cgrid = static_cast<int>(std::min<long long>((cunits + 255) / 256, 148ll * 16));
@@ -1123,6 +1128,160 @@ int moe_oft_fwd_impl(bool fused, const uint16_t* X, int T, const float* logits, 
 }
 
 }  // namespace
+
+// ---------------------------------------------------------------------------
+// MoE full expert layer (gate/up, SwiGLU, down projection)
+// ---------------------------------------------------------------------------
+namespace {
+struct MoeLayerLayout {
+  MoeLayout fwd;
+  size_t idx, w, offsets, bucket, table, nact, rd, hg, z, total;
+};
+MoeLayerLayout moe_layer_layout(int T, int E, int top_k, int chunk, int K, int N, int b) {
+  MoeLayerLayout L{};
+  L.fwd = moe_layout(T, E, top_k, chunk, K, N, b);
+  const size_t TK = 1ull * T * top_k, n = N / 2, nbd = n / b;
+  const size_t n_chunks_max = (E + chunk - 1) / chunk;
+  L.idx = L.fwd.total;
+  L.w = round_up(L.idx + 4 * TK, 256);
+  L.offsets = round_up(L.w + 4 * TK, 256);
+  L.bucket = round_up(L.offsets + 4ull * (E + 1), 256);
+  L.table = round_up(L.bucket + 4 * TK, 256);
+  L.nact = round_up(L.table + 4 * n_chunks_max * chunk, 256);
+  L.rd = round_up(L.nact + 16, 256);
+  L.hg = round_up(L.rd + 4ull * E * nbd * b * b, 256);
+  L.z = round_up(L.hg + 2 * TK * n, 256);
+  L.total = round_up(L.z + 4 * TK * K, 256);
+  return L;
+}
+
+int check_down_bank(const oft_weight* Wgu, const oft_weight* Wd, int b) {
+  if (int rc = check_weight(Wd, true)) return rc;
+  if (Wd->fmt != OFT_W_INT4) return fail(OFT_ERR_UNSUPPORTED, "the down-projection bank must be INT4");
+  if (Wd->n_experts != Wgu->n_experts) return fail(OFT_ERR_INVALID_ARG, "gate/up and down banks differ in n_experts");
+  if (Wd->d_in != Wgu->d_out / 2 || Wd->d_out != Wgu->d_in)
+    return fail(OFT_ERR_INVALID_ARG, "down bank must map n_proj = %d to d_in = %d", Wgu->d_out / 2, Wgu->d_in);
+  if (int rc = check_b(b, Wd->d_in)) return rc;
+  return OFT_OK;
+}
+
+template <int B>
+int launch_swiglu_rot(const float* Ytk, const int* pexp, int TK, int n, const float* Rd, uint16_t* Hg, cudaStream_t st) {
+  const long long units = 1ll * ((TK + SwigluCfg<B>::PT - 1) / SwigluCfg<B>::PT) * (n / B);
+  const int grid = static_cast<int>(std::min<long long>(units, 148ll * 8));
+  moe_swiglu_rot_kernel<B><<<std::max(grid, 1), 256, 0, st>>>(Ytk, pexp, TK, n, Rd, Hg);
+  OFT_LAUNCHED("moe_swiglu_rot_kernel");
+  return OFT_OK;
+}
+}  // namespace
+
+extern "C" {
+
+size_t moe_chunked_oft_layer_workspace(int T, int E, int top_k, int chunk, const oft_weight* W_gu,
+                                       const oft_weight* W_down, int b) {
+  if (W_gu == nullptr || W_down == nullptr || T <= 0 || E <= 0 || top_k <= 0 || chunk <= 0 || b <= 0) return 0;
+  return moe_layer_layout(T, E, top_k, chunk, W_gu->d_in, W_gu->d_out, b).total;
+}
+
+int moe_chunked_oft_layer_fwd(const uint16_t* X, int T, const float* logits, int E, int top_k, int chunk,
+                              const oft_weight* W_gu, const oft_weight* W_down, int b, const uint16_t* Q_gu,
+                              const uint16_t* Q_down, uint16_t* Y, void* ws, size_t ws_bytes, void* stream) {
+  if (int rc = check_weight(W_gu, true)) return rc;
+  if (int rc = check_down_bank(W_gu, W_down, b)) return rc;
+  const int K = W_gu->d_in, N = W_gu->d_out, n = N / 2, nbd = n / (b > 0 ? b : 1);
+  if (T <= 0 || E <= 0 || top_k <= 0 || chunk <= 0) return fail(OFT_ERR_INVALID_ARG, "bad sizes");
+  const void* ptrs[] = {X, logits, Q_gu, Q_down, Y, ws};
+  for (const void* q : ptrs)
+    if (q == nullptr || !aligned16(q)) return fail(OFT_ERR_INVALID_ARG, "NULL or misaligned pointer");
+  const MoeLayerLayout L = moe_layer_layout(T, E, top_k, chunk, K, N, b);
+  if (ws_bytes < L.total) return fail(OFT_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
+  cudaStream_t st = as_stream(stream);
+  uint8_t* wsb = static_cast<uint8_t*>(ws);
+  int* idx = reinterpret_cast<int*>(wsb + L.idx);
+  float* wts = reinterpret_cast<float*>(wsb + L.w);
+  int* offsets = reinterpret_cast<int*>(wsb + L.offsets);
+  int* bucket = reinterpret_cast<int*>(wsb + L.bucket);
+  int* table = reinterpret_cast<int*>(wsb + L.table);
+  int* n_active = reinterpret_cast<int*>(wsb + L.nact);
+  float* Rd = reinterpret_cast<float*>(wsb + L.rd);
+  uint16_t* Hg = reinterpret_cast<uint16_t*>(wsb + L.hg);
+  float* Z = reinterpret_cast<float*>(wsb + L.z);
+  float* Ytk = reinterpret_cast<float*>(wsb + L.fwd.ytk);
+  const int* inv = reinterpret_cast<const int*>(wsb + L.fwd.inv);
+  const int* pexp = reinterpret_cast<const int*>(wsb + L.fwd.pexp);
+  uint16_t* buf = reinterpret_cast<uint16_t*>(wsb + L.fwd.buf);
+  const int TK = T * top_k, n_chunks_max = (E + chunk - 1) / chunk;
+
+  // 1. routing, gate/up rotations, rotated gather, chunked gate/up GEMMs -> Ytk (fp32, bucket order)
+  if (int rc = moe_oft_fwd_impl(false, X, T, logits, E, top_k, chunk, W_gu, b, Q_gu, nullptr, idx, wts, offsets,
+                                bucket, table, n_active, ws, L.fwd.total, stream, false))
+    return rc;
+  // 2. down adapters of the active experts
+  if (int rc = launch_cayley(Q_down, E * nbd, b, Rd, table, n_active, nbd, st)) return rc;
+  // 3. h = silu(g) * u, rotated by R_e,down, bf16 in bucket order
+  {
+    ProfScope ps(OFT_K_ROTATE, st);
+    int rc = OFT_OK;
+    if (b == 16) rc = launch_swiglu_rot<16>(Ytk, pexp, TK, n, Rd, Hg, st);
+    if (b == 32) rc = launch_swiglu_rot<32>(Ytk, pexp, TK, n, Rd, Hg, st);
+    if (b == 64) rc = launch_swiglu_rot<64>(Ytk, pexp, TK, n, Rd, Hg, st);
+    if (rc) return rc;
+  }
+  // 4. chunks of down projections: transient dequant (side stream, double-buffered, in the
+  //    gate/up chunk buffers, which every gate/up GEMM has finished reading), one grouped GEMM each
+  gemm::Params prm;
+  memset(&prm, 0, sizeof(prm));
+  if (int rc = make_map_bf16(&prm.tmA[0], Hg, n, 1ull * TK, n, gemm::BM)) return rc;
+  for (int i = 1; i < gemm::MAX_MAPS; ++i) prm.tmA[i] = prm.tmA[0];
+  prm.C = Z;
+  prm.c_f32 = 1;
+  prm.ldc = K;
+  prm.use_moe = 1;
+  prm.moe.chunk_table = table;
+  prm.moe.offsets = offsets;
+  prm.moe.chunk = chunk;
+  prm.moe.TK = TK;
+  prm.moe.n_proj = n;
+  prm.moe.K = K;
+  prm.moe.mode = gemm::kMoeDown;
+  const WeightView dbank = view_of(W_down);  // N = K rows, K = n columns per expert
+  const size_t dq_smem = sizeof(uint16_t) * kChunkRows * chunk_scale_ld(n / W_down->group);
+  if (dq_smem > 227 * 1024) return fail(OFT_ERR_UNSUPPORTED, "n_proj / group too large for the chunk dequant");
+  OFT_CUDA(cudaFuncSetAttribute(moe_chunk_dequant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(dq_smem)));
+  SidePipe* sp = nullptr;
+  if (int rc = side_pipe(&sp)) return rc;
+  OFT_CUDA(cudaEventRecord(sp->start, st));
+  OFT_CUDA(cudaStreamWaitEvent(sp->side, sp->start, 0));
+  const size_t buf_elems = 1ull * chunk * K * n;
+  for (int c = 0; c < n_chunks_max; ++c) {
+    const int h = c & 1;
+    uint16_t* bufc = buf + h * buf_elems;
+    if (c >= 2) OFT_CUDA(cudaStreamWaitEvent(sp->side, sp->gemm_done[h], 0));
+    {
+      ProfScope ps(OFT_K_DEQUANT, sp->side);
+      moe_chunk_dequant_kernel<<<dim3((K + kChunkRows - 1) / kChunkRows, chunk), 256, dq_smem, sp->side>>>(
+          dbank, table, c, chunk, bufc);
+      OFT_LAUNCHED("moe_chunk_dequant_kernel");
+    }
+    OFT_CUDA(cudaEventRecord(sp->dq_done[h], sp->side));
+    OFT_CUDA(cudaStreamWaitEvent(st, sp->dq_done[h], 0));
+    prm.moe.chunk_idx = c;
+    if (int rc = make_map_bf16(&prm.tmB[0], bufc, n, 1ull * chunk * K, n, gemm::BN)) return rc;
+    for (int i = 1; i < gemm::MAX_MAPS; ++i) prm.tmB[i] = prm.tmB[0];
+    if (int rc = launch_gemm(prm, 0, st)) return rc;
+    OFT_CUDA(cudaEventRecord(sp->gemm_done[h], st));
+  }
+  // 5. Y[t] = sum_k w_tk Z[pos(t, k)] in slot order
+  const long long cunits = 1ll * T * (K / 8);
+  const int cgrid = static_cast<int>(std::min<long long>((cunits + 255) / 256, 148ll * 16));
+  ProfScope ps(OFT_K_ROUTE, st);
+  moe_combine_kernel<<<cgrid, 256, 0, st>>>(Z, wts, inv, T, K, top_k, Y);
+  OFT_LAUNCHED("moe_combine_kernel");
+  return OFT_OK;
+}
+
+}  // extern "C"
 
 // ---------------------------------------------------------------------------
 // MoE backward
@@ -1256,7 +1415,7 @@ int moe_chunked_oft_bwd(const uint16_t* dY, const uint16_t* X, int T, const floa
   prm.moe.TK = TK;
   prm.moe.n_proj = n_proj;
   prm.moe.K = K;
-  prm.moe.bwd = 1;
+  prm.moe.mode = gemm::kMoeBwd;
   const WeightView bank = view_of(W);
   SidePipe* sp = nullptr;
   if (int rc = side_pipe(&sp)) return rc;

@@ -238,8 +238,9 @@ def cpu_baseline_linear(case, backward: bool, budget_s: float = 12.0):
                       f"({cpu_model()}), {dt:.2f} s"}
 
 
-def cpu_baseline_moe(case, budget_s: float = 12.0, dY=None):
-    """Oracle tokens/s of the MoE step on the host cores (forward; with dY, forward + backward)."""
+def cpu_baseline_moe(case, budget_s: float = 12.0, dY=None, down=None):
+    """Oracle tokens/s of the MoE step on the host cores (forward; with dY, forward +
+    backward; with the down projections, the full expert layer)."""
     import numpy as np
     from oracle import moe_ref
     from oracle.codecs import bf16_bits_to_f64
@@ -258,13 +259,21 @@ def cpu_baseline_moe(case, budget_s: float = 12.0, dY=None):
         codes = {int(e): raw(case["codes"][int(e)]) for e in used}
         scales = {int(e): raw(case["scales"][int(e)]) for e in used}
         bank = moe_ref.ExpertBank(codes, scales, spec.K, spec.group, spec.n_proj)
-        moe_ref.moe_fwd_direct(X[t:t + 1], logits[t:t + 1], bank, raw(case["Q"]), spec.b, spec.top_k)
+        if down is not None:
+            dcodes = {int(e): raw(down["down_codes"][int(e)]) for e in used}
+            dscales = {int(e): raw(down["down_scales"][int(e)]) for e in used}
+            dbank = moe_ref.DownBank(dcodes, dscales, spec.n_proj, spec.group)
+            moe_ref.moe_layer_direct(X[t:t + 1], logits[t:t + 1], bank, dbank, raw(case["Q"]), raw(down["Q_down"]),
+                                     spec.b, spec.top_k)
+        else:
+            moe_ref.moe_fwd_direct(X[t:t + 1], logits[t:t + 1], bank, raw(case["Q"]), spec.b, spec.top_k)
         if dYf is not None:
             moe_ref.moe_bwd_direct(dYf[t:t + 1], X[t:t + 1], logits[t:t + 1], bank, raw(case["Q"]), spec.b,
                                    spec.top_k, spec.E)
         done += 1
     dt = time.perf_counter() - t0
-    what = "forward + backward" if dYf is not None else "direct per-token top-%d sum" % spec.top_k
+    what = ("forward + backward" if dYf is not None else
+            "full expert layer" if down is not None else "direct per-token top-%d sum" % spec.top_k)
     return {"value": done / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
             "sample": f"{done} tokens of {spec.T}, {what}, float64 numpy ({cpu_model()}), {dt:.2f} s"}
 
@@ -298,7 +307,7 @@ def gemm_kernel_hash() -> str:
 def run_ours(args, rank, world):
     import torch
     import orthogonal_fine_tuning_b200 as oft
-    from gen import LINEAR_CONFIGS, MOE_CONFIGS, make_linear_case, make_moe_case, make_moe_grad
+    from gen import LINEAR_CONFIGS, MOE_CONFIGS, make_linear_case, make_moe_case, make_moe_down, make_moe_grad
 
     _, _, local = dist_env()
     torch.cuda.set_device(local)
@@ -347,6 +356,27 @@ def run_ours(args, rank, world):
         if backward:
             inputs["dY"] = dY
             result_keys = ("Y", "dX", "dQ", "dlogits")
+        if args.moe_layer:
+            # full expert layer: gate/up, SwiGLU, down projection with its own adapter
+            dn = make_moe_down(spec, device=dev)
+            Wd = oft.Weight("int4", dn["down_codes"], dn["down_scales"], spec.n_proj, spec.K, spec.group,
+                            n_experts=spec.E)
+            Qd = dn["Q_down"]
+            lws = torch.empty(oft.moe_chunked_oft_layer_workspace(spec.T, spec.E, spec.top_k, spec.chunk, W, Wd, spec.b),
+                              dtype=torch.uint8, device=dev)
+            lay = dict(Y=torch.empty(spec.T, spec.K, dtype=torch.bfloat16, device=dev))
+
+            def new_outputs():
+                return dict(Y=torch.empty(spec.T, spec.K, dtype=torch.bfloat16, device=dev))
+
+            def step(Xi=X, Li=logits, Qi=Q, o=None, dYi=None, Qdi=None):
+                o = lay if o is None else o
+                oft.moe_chunked_oft_layer_fwd(Xi, Li, W, Wd, spec.b, Qi, Qd if Qdi is None else Qdi, spec.top_k,
+                                              spec.chunk, workspace=lws, out=o["Y"])
+                return o["Y"]
+
+            inputs = dict(X=X, logits=logits, Q=Q, Q_down=Qd)
+            result_keys = ("Y",)
     else:
         spec = linear_spec(name)
         backward = spec.backward
@@ -418,6 +448,17 @@ def run_ours(args, rank, world):
         # the chunked variant materialises each active expert in bf16 (write + read), as the pages do
         chunk_buf_bytes = 0 if args.moe == "fused" else 2 * (2 * spec.K * 2 * spec.n_proj)
         alg_bytes = n_active * (expert_bytes + chunk_buf_bytes) + 2 * spec.T * spec.K + 2 * spec.T * 2 * spec.n_proj
+        if args.moe_layer:
+            # down projections: GEMM, rotation of h by the down adapter, its Cayley build; the down
+            # weights stream through the chunk buffer like gate/up; Y is [T][K]
+            nbd = spec.n_proj // spec.b
+            flops["gemm_down"] = 2.0 * TK * spec.n_proj * spec.K
+            flops["rot_down"] = 2.0 * TK * spec.n_proj * spec.b
+            flops["cayley_down"] = 2.0 * spec.b ** 3 * n_active * nbd
+            total_flops = sum(flops.values())
+            down_bytes = spec.K * spec.n_proj // 2 + 2 * spec.K * (spec.n_proj // spec.group)
+            down_buf = 2 * (2 * spec.K * spec.n_proj)
+            alg_bytes += n_active * (down_bytes + down_buf) - 2 * spec.T * 2 * spec.n_proj + 2 * spec.T * spec.K
         if backward:
             # dY W^T per routed row, its rotation back, dR, the Cayley backward; the experts stream
             # through the chunk buffer once more; dY and the logits in, dX, dQ and dlogits out
@@ -454,7 +495,8 @@ def run_ours(args, rank, world):
         peak = peaks["hbm_gbs"]
         unit = "GB/s"
         traffic = None
-        kernel = "whole step (chunk dequant + grouped GEMM" + (", forward and backward" if backward else "") + "), HBM"
+        kernel = ("whole step (chunk dequant + grouped GEMM" + (", forward and backward" if backward else "")
+                  + (", gate/up + SwiGLU + down" if args.moe_layer else "") + "), HBM")
     elif spec.M <= 128:
         # few tokens: the weight stream bounds the GEMM; bytes of one launch over its time
         wbytes = weight_bytes(spec)
@@ -514,7 +556,9 @@ def run_ours(args, rank, world):
         comp.wait_event(ev_in[b])
         comp.wait_event(ev_out[b])               # read-back of step i-2 is done with dev_out[b]
         d = dev_in[b]
-        if is_moe:
+        if is_moe and args.moe_layer:
+            step(d["X"], d["logits"], d["Q"], o=dev_out[b], Qdi=d["Q_down"])
+        elif is_moe:
             step(d["X"], d["logits"], d["Q"], o=dev_out[b], dYi=d.get("dY"))
         elif backward:
             step(d["X"], d["dY"], d["Q"], o=dev_out[b])
@@ -552,14 +596,18 @@ def run_ours(args, rank, world):
         return None
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline_moe(case, dY=dY if backward else None) if is_moe else cpu_baseline_linear(case, backward)
+        if is_moe:
+            cpu = cpu_baseline_moe(case, dY=dY if backward else None, down=dn if args.moe_layer else None)
+        else:
+            cpu = cpu_baseline_linear(case, backward)
     config = {"workload": WORKLOAD_NAMES[name], "name": name, "tokens_per_gpu": tokens,
               "global_batch_tokens": tokens * world, "parallelism": f"dp{world}" if world > 1 else "single",
               "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MB write)",
               "step": "build_rotation + fwd" + (" + bwd" if backward else "") + (" + dQ all-reduce" if world > 1 and backward else "")}
     if is_moe:
         config.update(n_active_experts=n_active, moe_variant=args.moe)
-        config["step"] = "route + build_rotation + fwd" + (" + bwd (dX, dQ, dlogits)" if backward else "")
+        config["step"] = ("route + build_rotation + fwd" + (" + bwd (dX, dQ, dlogits)" if backward else "")
+                          + (" (full expert layer: gate/up, SwiGLU, down)" if args.moe_layer else ""))
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -579,7 +627,7 @@ def run_reference(args, rank, world):
     bounded sample of the same workload per step."""
     if rank != 0:
         return None
-    from gen import LINEAR_CONFIGS, MOE_CONFIGS, make_linear_case, make_moe_case, make_moe_grad
+    from gen import LINEAR_CONFIGS, MOE_CONFIGS, make_linear_case, make_moe_case, make_moe_down, make_moe_grad
     name = args.workload
     if name in MOE_CONFIGS:
         import torch
@@ -587,10 +635,11 @@ def run_reference(args, rank, world):
         dev = "cuda" if torch.cuda.is_available() else "cpu"
         case = make_moe_case(spec, device=dev)
         dY = make_moe_grad(spec, device=dev) if args.moe_backward else None
+        dn = make_moe_down(spec, device=dev) if args.moe_layer else None
         per = max(2.0, 150.0 / (args.steps + args.warmup))
         for _ in range(args.warmup):
-            cpu_baseline_moe(case, budget_s=per / 4, dY=dY)
-        res = [cpu_baseline_moe(case, budget_s=per, dY=dY) for _ in range(args.steps)]
+            cpu_baseline_moe(case, budget_s=per / 4, dY=dY, down=dn)
+        res = [cpu_baseline_moe(case, budget_s=per, dY=dY, down=dn) for _ in range(args.steps)]
         value = statistics.mean(r["value"] for r in res)
         sample = res[-1]["sample"]
     else:
@@ -628,9 +677,13 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--moe-backward", action="store_true",
                     help="MoE workload: time forward + adapter backward (chunked path)")
+    ap.add_argument("--moe-layer", action="store_true",
+                    help="MoE workload: time the full expert layer (gate/up, SwiGLU, down projection)")
     ap.add_argument("--moe", default="chunked", choices=["chunked", "fused"],
                     help="MoE workload: the pages' chunked dequant (default) or the fused-dequant grouped GEMM")
     args = ap.parse_args(argv)
+    if args.moe_layer and args.moe_backward:
+        ap.error("--moe-layer times the forward of the full expert layer; --moe-backward the gate/up backward")
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":

@@ -40,7 +40,16 @@ WORKLOAD_NAMES = {
     # decode-like checks, not among the five workloads: the same weights at 64 tokens, forward only
     "c1-m64": "fused-QKV FP8 weights at 64 tokens, fwd: 64 x 2560 -> 4096/1024/1024, FP8 e4m3 per-channel, b=32",
     "c4-m64": "MXFP4 weights at 64 tokens, fwd: 64 x 7168 -> 12288/3072/3072, MXFP4, b=64",
+    # a smaller MoE case for profiler captures (the full layer holds ~12 GB): same expert shapes
+    "c3-mid": "MoE active-expert-chunked OFT: 2048 tok, hidden 7168, 128 experts x (2x2048), INT4 g32, top-8, chunk 16, b=32",
 }
+
+
+def moe_spec(name: str):
+    from gen import MOE_CONFIGS
+    if name == "c3-mid":
+        return MOE_CONFIGS["c3"].with_(name="c3-mid", T=2048, E=128)
+    return MOE_CONFIGS.get(name)
 
 
 def linear_spec(name: str):
@@ -314,11 +323,11 @@ def run_ours(args, rank, world):
     dev = torch.device("cuda", local)
     peaks, peak_src = load_peaks()
     name = args.workload
-    is_moe = name in MOE_CONFIGS
+    is_moe = moe_spec(name) is not None
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
     if is_moe:
-        spec = MOE_CONFIGS[name]
+        spec = moe_spec(name)
         case = make_moe_case(spec, device=dev)
         W = oft.Weight("int4", case["codes"], case["scales"], spec.K, 2 * spec.n_proj, spec.group, n_experts=spec.E)
         fused = args.moe == "fused"
@@ -418,22 +427,32 @@ def run_ours(args, rank, world):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    with ClockSampler(dev) as clocks, oft.profile(max_launches=max(4096, 64 * args.steps)) as prof:
+    # Two passes of the same K steps.  The first gives the step time (value): only the
+    # step's own launches, so consecutive kernels overlap their launch as they do in use.
+    # The second brackets every library kernel with CUDA events on its stream (the
+    # library's profiling hooks) for the per-kernel split and the roofline; those events
+    # sit between the kernels and add their own gaps, so its step time is reported apart.
+    def timed_pass():
+        st_, en_ = ([torch.cuda.Event(enable_timing=True) for _ in range(args.steps)] for _ in range(2))
         for i in range(args.steps):
             flush.zero_()                          # evict L2 between timed steps
-            starts[i].record()
+            st_[i].record()
             step()
-            ends[i].record()
+            en_[i].record()
         torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        return sum(s.elapsed_time(e) for s, e in zip(st_, en_)) / args.steps
+
+    with ClockSampler(dev) as clocks:
+        ms_local = timed_pass()
     oft.oft_check_device()
-    ms_steps = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    ms_local = sum(ms_steps) / len(ms_steps)
+    with oft.profile(max_launches=max(4096, 64 * args.steps)) as prof:
+        ms_prof_local = timed_pass()
+    oft.oft_check_device()
     ms_per_step = max_over_ranks(ms_local, dev)
+    ms_profiled = max_over_ranks(ms_prof_local, dev)
     value = tokens * world / (ms_per_step / 1e3)
 
     # ---- algorithmic work ----
@@ -615,6 +634,9 @@ def run_ours(args, rank, world):
         "config": config, "tflops": tflops, "algorithmic_flops_per_step": total_flops,
         "algorithmic_bytes_per_step": alg_bytes, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": int(sum(prof.launches.values())),
+        "profiled_pass": {"ms_per_step": ms_profiled,
+                          "note": "the same K steps again with CUDA events around every library kernel; "
+                                  "kernel_ms_per_step and roofline.achieved come from this pass"},
         "kernel_ms_per_step": {k: v / args.steps for k, v in prof.ms.items()},
         "kernel_launches_per_step": {k: v / args.steps for k, v in prof.launches.items()},
         "clocks": clocks.summary(),
@@ -629,9 +651,9 @@ def run_reference(args, rank, world):
         return None
     from gen import LINEAR_CONFIGS, MOE_CONFIGS, make_linear_case, make_moe_case, make_moe_down, make_moe_grad
     name = args.workload
-    if name in MOE_CONFIGS:
+    if moe_spec(name) is not None:
         import torch
-        spec = MOE_CONFIGS[name]
+        spec = moe_spec(name)
         dev = "cuda" if torch.cuda.is_available() else "cpu"
         case = make_moe_case(spec, device=dev)
         dY = make_moe_grad(spec, device=dev) if args.moe_backward else None
@@ -657,7 +679,7 @@ def run_reference(args, rank, world):
         ms = 1e3 * statistics.mean(times)
         value = tokens / (ms / 1e3)
         sample = f"first {tokens} of {spec.M} tokens per step, float64 numpy ({cpu_model()})"
-    ms_per_step = None if name in MOE_CONFIGS else ms
+    ms_per_step = None if moe_spec(name) is not None else ms
     return {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",

@@ -172,6 +172,7 @@ __global__ void __launch_bounds__(CayleyFwdCfg<B>::THREADS, CayleyFwdCfg<B>::MIN
                                                                                const int* __restrict__ n_active,
                                                                                int blocks_per_expert) {
   constexpr int BPC = CayleyFwdCfg<B>::BPC;
+  pdl_wait();
   const int total = active_list != nullptr ? min(nblocks, *n_active * blocks_per_expert) : nblocks;
   for (int base = blockIdx.x * BPC; base < total; base += gridDim.x * BPC)
     cayley_fwd_block<B, UNROLL>(Q, R, base + threadIdx.x / B, total, active_list, blocks_per_expert);
@@ -197,6 +198,7 @@ __global__ void __launch_bounds__(TPR * B) cayley_fwd_split_kernel(const uint16_
   __shared__ __align__(16) float piv[2][2 * B + 4];
   const int r = threadIdx.x / TPR, h = threadIdx.x % TPR;
   const unsigned full = 0xFFFFFFFFu;
+  pdl_wait();
   const int total = active_list != nullptr ? min(nblocks, *n_active * blocks_per_expert) : nblocks;
   for (int lin = blockIdx.x; lin < total; lin += gridDim.x) {
     int blk = lin;
@@ -279,6 +281,7 @@ __global__ void __launch_bounds__(kCayleyThreads) cayley_bwd_kernel(const float*
   float* U = csm + 2 * B * LD;  // T G
   const int tid = threadIdx.x;
   const int ti = (tid / NT) * TI, tj = (tid % NT) * TI;
+  pdl_wait();
   for (int blk = blockIdx.x; blk < nblocks; blk += gridDim.x) {
     const float* rb = R + static_cast<size_t>(blk) * B * B;
     const float* gb = G + static_cast<size_t>(blk) * nparts * B * B;

@@ -226,6 +226,13 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, const void* s
                : "memory");
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialisation may start before the previous kernel on its stream has finished;
+// pdl_wait() returns once that kernel has completed and its writes are visible.
+// Every kernel calls it before its first global-memory access (and returns at
+// once when it was launched without the attribute).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
 // wait until at most N committed bulk groups still read their shared-memory source

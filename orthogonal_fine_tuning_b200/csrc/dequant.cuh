@@ -159,6 +159,7 @@ __global__ void __launch_bounds__(256) moe_chunk_dequant_kernel(WeightView bank,
 // 2^-127, e = 255 is NaN), so the backward's producers apply a per-element scale
 // with one multiply.
 __global__ void e8m0_factor_kernel(const uint8_t* __restrict__ e, long long n, uint16_t* __restrict__ out) {
+  pdl_wait();
   const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= n) return;
   const uint32_t v = e[i];
@@ -184,6 +185,7 @@ template <bool NIB>
 __global__ void __launch_bounds__(256) pack_codes_bwd_kernel(const uint8_t* __restrict__ in, int N, int K,
                                                              PackBwdParams pp, uint8_t* __restrict__ out) {
   __shared__ uint8_t t[64][128 + 4];  // [channel][feature], one code per byte
+  pdl_wait();
   int g = 0;
   while (g + 1 < pp.num_groups && static_cast<int>(blockIdx.x) >= pp.blk0[g + 1]) ++g;
   const int local = static_cast<int>(blockIdx.x) - pp.blk0[g];

@@ -270,6 +270,7 @@ __device__ __forceinline__ void convert(const Raw& raw, const uint8_t* sS, int s
 template <int FMT, bool BWD, bool SCHED, bool MOE = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_constant__ KParams<SCHED> kp) {
   const Params& p = kp.p;
+  if constexpr (MOE) pdl_wait();  // the prologue reads the device-built group list
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sB = smem;
@@ -329,6 +330,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_dq_kernel(const __grid_co
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();
   const uint32_t tmem = *tmem_slot;
   // groups: from the launch (shared memory copy), or built on the device (MoE)
   const Group* gsrc = MOE ? p.moe_groups : sg;

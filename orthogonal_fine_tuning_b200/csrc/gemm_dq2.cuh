@@ -140,6 +140,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
   tc_fence_before();
   cluster_sync_all();  // barriers initialised and TMEM allocated in both CTAs
   tc_fence_after();
+  pdl_wait();
   const uint32_t tmem = *tmem_slot;
   const int total = s_meta[0], ng = s_meta[1];
   const int cid = static_cast<int>(cluster_id_x()), ncl = static_cast<int>(cluster_count_x());

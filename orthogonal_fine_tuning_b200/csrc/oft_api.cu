@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdarg>
+#include <cstdlib>
 #include <cstdio>
 #include <cstring>
 #include <algorithm>
@@ -12,6 +13,7 @@
 #include <queue>
 #include <vector>
 #include <string>
+#include <utility>
 
 #include "oft.h"
 
@@ -56,6 +58,33 @@ int fail(int code, const char* fmt, ...) {
   } while (0)
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Launches with programmatic stream serialisation (the kernel may be scheduled while
+// the previous kernel on the stream drains; it calls pdl_wait() before touching
+// global memory).  OFT_PDL=0 in the environment turns it off.
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = getenv("OFT_PDL");
+    return v == nullptr || v[0] != '0';
+  }();
+  return on;
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -296,15 +325,15 @@ int launch_cayley(const uint16_t* Q, int nblocks, int b, float* R, const int* ac
   const int grid = std::max(1, std::min((nblocks + bpc - 1) / bpc, sm_count() * 32 / warps));
   const int* al = active_list;
   if (nblocks >= kCayleyUnrollBlocks) {
-    if (b == 16) cayley_fwd_kernel<16, true><<<grid, 32, 0, st>>>(Q, nblocks, R, al, n_active, blocks_per_expert);
-    if (b == 32) cayley_fwd_kernel<32, true><<<grid, 32, 0, st>>>(Q, nblocks, R, al, n_active, blocks_per_expert);
-    if (b == 64) cayley_fwd_kernel<64, true><<<grid, 64, 0, st>>>(Q, nblocks, R, al, n_active, blocks_per_expert);
+    if (b == 16) OFT_CUDA(launch_pdl(cayley_fwd_kernel<16, true>, grid, 32, 0, st, Q, nblocks, R, al, n_active, blocks_per_expert));
+    if (b == 32) OFT_CUDA(launch_pdl(cayley_fwd_kernel<32, true>, grid, 32, 0, st, Q, nblocks, R, al, n_active, blocks_per_expert));
+    if (b == 64) OFT_CUDA(launch_pdl(cayley_fwd_kernel<64, true>, grid, 64, 0, st, Q, nblocks, R, al, n_active, blocks_per_expert));
   } else {
-    if (b == 16) cayley_fwd_kernel<16, false><<<grid, 32, 0, st>>>(Q, nblocks, R, al, n_active, blocks_per_expert);
+    if (b == 16) OFT_CUDA(launch_pdl(cayley_fwd_kernel<16, false>, grid, 32, 0, st, Q, nblocks, R, al, n_active, blocks_per_expert));
     // few blocks: the per-block pivot chain is the time, so two threads share each row
     const int sgrid = std::max(1, std::min(nblocks, sm_count() * 16));
-    if (b == 32) cayley_fwd_split_kernel<32, 2><<<sgrid, 64, 0, st>>>(Q, nblocks, R, al, n_active, blocks_per_expert);
-    if (b == 64) cayley_fwd_split_kernel<64, 2><<<sgrid, 128, 0, st>>>(Q, nblocks, R, al, n_active, blocks_per_expert);
+    if (b == 32) OFT_CUDA(launch_pdl(cayley_fwd_split_kernel<32, 2>, sgrid, 64, 0, st, Q, nblocks, R, al, n_active, blocks_per_expert));
+    if (b == 64) OFT_CUDA(launch_pdl(cayley_fwd_split_kernel<64, 2>, sgrid, 128, 0, st, Q, nblocks, R, al, n_active, blocks_per_expert));
   }
   OFT_LAUNCHED("cayley_fwd_kernel");
   return OFT_OK;
@@ -317,9 +346,9 @@ int launch_cayley_bwd(const float* R, const float* G, int nparts, int nblocks, i
   if (b == 32) OFT_CUDA(cudaFuncSetAttribute(cayley_bwd_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   if (b == 64) OFT_CUDA(cudaFuncSetAttribute(cayley_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   ProfScope ps(OFT_K_CAYLEY, st);
-  if (b == 16) cayley_bwd_kernel<16><<<grid, kCayleyThreads, smem, st>>>(R, G, nparts, nblocks, dQ);
-  if (b == 32) cayley_bwd_kernel<32><<<grid, kCayleyThreads, smem, st>>>(R, G, nparts, nblocks, dQ);
-  if (b == 64) cayley_bwd_kernel<64><<<grid, kCayleyThreads, smem, st>>>(R, G, nparts, nblocks, dQ);
+  if (b == 16) OFT_CUDA(launch_pdl(cayley_bwd_kernel<16>, grid, kCayleyThreads, smem, st, R, G, nparts, nblocks, dQ));
+  if (b == 32) OFT_CUDA(launch_pdl(cayley_bwd_kernel<32>, grid, kCayleyThreads, smem, st, R, G, nparts, nblocks, dQ));
+  if (b == 64) OFT_CUDA(launch_pdl(cayley_bwd_kernel<64>, grid, kCayleyThreads, smem, st, R, G, nparts, nblocks, dQ));
   OFT_LAUNCHED("cayley_bwd_kernel");
   return OFT_OK;
 }
@@ -348,7 +377,7 @@ int launch_rotate_fwd(const uint16_t* X, int M, int K, int P, int b, const float
   if (int rc = set_smem(rtc::rot_fwd_tc_kernel, rtc::kFwdSmem)) return rc;
   const int grid = std::min(sm_count(), prm.groups * prm.tiles_m);
   ProfScope ps(OFT_K_ROTATE, st);
-  rtc::rot_fwd_tc_kernel<<<grid, rtc::NUM_THREADS, rtc::kFwdSmem, st>>>(prm);
+  OFT_CUDA(launch_pdl(rtc::rot_fwd_tc_kernel, grid, rtc::NUM_THREADS, rtc::kFwdSmem, st, prm));
   OFT_LAUNCHED("rot_fwd_tc_kernel");
   return OFT_OK;
 }
@@ -370,7 +399,7 @@ int launch_rotate_bwd(const float* dXr, int M, int K, int P, int b, const float*
   if (int rc = set_smem(rtc::rot_bwd_tc_kernel, rtc::kBwdSmem)) return rc;
   const int grid = std::min(sm_count(), prm.groups * prm.tiles_m);
   ProfScope ps(OFT_K_ROTATE, st);
-  rtc::rot_bwd_tc_kernel<<<grid, rtc::NUM_THREADS, rtc::kBwdSmem, st>>>(prm);
+  OFT_CUDA(launch_pdl(rtc::rot_bwd_tc_kernel, grid, rtc::NUM_THREADS, rtc::kBwdSmem, st, prm));
   OFT_LAUNCHED("rot_bwd_tc_kernel");
   return OFT_OK;
 }
@@ -407,7 +436,7 @@ int launch_grad(const uint16_t* X, const float* dXr, int M, int K, int P, int b,
   if (int rc = set_smem(rtc::grad_tc_kernel, rtc::kGradSmem)) return rc;
   const int grid = std::min(sm_count(), prm.groups * prm.chunks);
   ProfScope ps(OFT_K_GRAD, st);
-  rtc::grad_tc_kernel<<<grid, rtc::NUM_THREADS, rtc::kGradSmem, st>>>(prm);
+  OFT_CUDA(launch_pdl(rtc::grad_tc_kernel, grid, rtc::NUM_THREADS, rtc::kGradSmem, st, prm));
   OFT_LAUNCHED("grad_tc_kernel");
   return OFT_OK;
 }
@@ -450,7 +479,7 @@ int launch_gemm_dq_k(const gdq::KParams<SCHED>& kp, int grid, cudaStream_t st) {
     attr_set[dev] = true;
   }
   ProfScope ps(OFT_K_GEMM, st);
-  gdq::gemm_dq_kernel<FMT, BWD, SCHED><<<grid, gdq::NUM_THREADS, gdq::kSmemBytes, st>>>(kp);
+  OFT_CUDA(launch_pdl(gdq::gemm_dq_kernel<FMT, BWD, SCHED>, grid, gdq::NUM_THREADS, gdq::kSmemBytes, st, kp));
   OFT_LAUNCHED("gemm_dq_kernel");
   return OFT_OK;
 }
@@ -541,7 +570,7 @@ int launch_gemm_dq2_k(const gdq::KParams<SCHED>& kp, int clusters, cudaStream_t 
     attr_set[dev] = true;
   }
   ProfScope ps(OFT_K_GEMM, st);
-  gdq2::gemm_dq2_kernel<FMT, BWD, SCHED><<<2 * clusters, gdq2::NUM_THREADS, gdq2::kSmemBytes, st>>>(kp);
+  OFT_CUDA(launch_pdl(gdq2::gemm_dq2_kernel<FMT, BWD, SCHED>, 2 * clusters, gdq2::NUM_THREADS, gdq2::kSmemBytes, st, kp));
   OFT_LAUNCHED("gemm_dq2_kernel");
   return OFT_OK;
 }
@@ -828,9 +857,9 @@ int oft_linear_bwd(const uint16_t* dY, const uint16_t* X, int M, const oft_weigh
     pp.blk0[P] = blk;
     ProfScope ps(OFT_K_DEQUANT, st);
     if (W->fmt == OFT_W_FP8)
-      pack_codes_bwd_kernel<false><<<blk, 256, 0, st>>>(static_cast<const uint8_t*>(W->codes), N, K, pp, codes_t);
+      OFT_CUDA(launch_pdl(pack_codes_bwd_kernel<false>, blk, 256, 0, st, static_cast<const uint8_t*>(W->codes), N, K, pp, codes_t));
     else
-      pack_codes_bwd_kernel<true><<<blk, 256, 0, st>>>(static_cast<const uint8_t*>(W->codes), N, K, pp, codes_t);
+      OFT_CUDA(launch_pdl(pack_codes_bwd_kernel<true>, blk, 256, 0, st, static_cast<const uint8_t*>(W->codes), N, K, pp, codes_t));
     OFT_LAUNCHED("pack_codes_bwd_kernel");
   }
 
@@ -847,8 +876,8 @@ int oft_linear_bwd(const uint16_t* dY, const uint16_t* X, int M, const oft_weigh
     const long long n = 1ll * (K / 32) * N;
     {
       ProfScope ps(OFT_K_DEQUANT, st);
-      e8m0_factor_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
-          static_cast<const uint8_t*>(W->scales), n, fac);
+      OFT_CUDA(launch_pdl(e8m0_factor_kernel, static_cast<unsigned>((n + 255) / 256), 256, 0, st,
+                          static_cast<const uint8_t*>(W->scales), n, fac));
       OFT_LAUNCHED("e8m0_factor_kernel");
     }
     if (int rc = make_map_plain_2d(&prm.tmS, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, fac, N, K / 32, 2ull * N, 64,

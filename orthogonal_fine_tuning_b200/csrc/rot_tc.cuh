@@ -168,6 +168,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) rot_fwd_tc_kernel(const __grid
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();
   const uint32_t tmem = *tmem_slot;
   int ubeg, uend;
   unit_range(p.groups * p.tiles_m, ubeg, uend);
@@ -375,6 +376,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) rot_bwd_tc_kernel(const __grid
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();
   const uint32_t tmem = *tmem_slot;
   int ubeg, uend;
   unit_range(p.groups * p.tiles_m, ubeg, uend);
@@ -562,6 +564,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grad_tc_kernel(const __grid_co
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();
   const uint32_t tmem = *tmem_slot;
   int ubeg, uend;
   unit_range(p.groups * p.chunks, ubeg, uend);

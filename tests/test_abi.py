@@ -119,3 +119,41 @@ def test_rotation_and_debug_checks(lib):
     assert lib.oft_build_rotation(0, 4, 32, 0x2000, None) == L.OFT_ERR_INVALID_ARG
     assert lib.oft_build_rotation(0x1000, 0, 32, 0x2000, None) == L.OFT_OK
     assert lib.oft_debug_bounded_wait(0, None) == L.OFT_ERR_INVALID_ARG
+
+
+def test_moe_backward_and_layer_argument_checks(lib):
+    """Each call below fails a host-side check before any launch."""
+    from orthogonal_fine_tuning_b200 import _lib as L
+    w = _w(lib, d_in=256, d_out=64, group=32, n=16)
+    p = [0x10000 * (i + 1) for i in range(12)]
+
+    def bwd(E=16, top_k=4, chunk=4, b=32, w=w, dY=p[0], ws_bytes=1 << 40, dlogits=p[6]):
+        return lib.moe_chunked_oft_bwd(dY, p[1], 32, p[2], E, top_k, chunk, ctypes.byref(w), b, p[3], p[4], p[5],
+                                       dlogits, p[7], ws_bytes, None)
+
+    assert bwd(E=600, w=_w(lib, d_in=256, d_out=64, n=600)) == L.OFT_ERR_UNSUPPORTED
+    assert bwd(top_k=9) == L.OFT_ERR_UNSUPPORTED
+    assert bwd(chunk=17) == L.OFT_ERR_UNSUPPORTED
+    assert bwd(E=8) == L.OFT_ERR_UNSUPPORTED                        # bank size mismatch
+    assert bwd(w=_w(lib, fmt=2, d_in=256, d_out=64, n=16)) == L.OFT_ERR_UNSUPPORTED
+    assert bwd(b=24) == L.OFT_ERR_UNSUPPORTED
+    assert bwd(dY=0) == L.OFT_ERR_INVALID_ARG
+    assert bwd(dlogits=p[6] + 4) == L.OFT_ERR_INVALID_ARG           # misaligned
+    assert bwd(ws_bytes=1024) == L.OFT_ERR_WORKSPACE
+    need = lib.moe_chunked_oft_bwd_workspace(32, 16, 4, 4, ctypes.byref(w), 32)
+    assert need > 2 * 4 * 32 * 4 * 256                              # D = dY W^T alone is 2 x T*k x K fp32
+
+    wd = _w(lib, d_in=32, d_out=256, group=32, n=16)                # n_proj = 32 -> K = 256
+
+    def layer(w=w, wd=wd, b=32, X=p[0], ws_bytes=1 << 40):
+        return lib.moe_chunked_oft_layer_fwd(X, 32, p[1], 16, 4, 4, ctypes.byref(w), ctypes.byref(wd), b, p[2],
+                                             p[3], p[4], p[5], ws_bytes, None)
+
+    assert layer(wd=_w(lib, d_in=64, d_out=256, group=32, n=16)) == L.OFT_ERR_INVALID_ARG   # d_in != n_proj
+    assert layer(wd=_w(lib, d_in=32, d_out=128, group=32, n=16)) == L.OFT_ERR_INVALID_ARG   # d_out != K
+    assert layer(wd=_w(lib, d_in=32, d_out=256, group=32, n=8)) == L.OFT_ERR_INVALID_ARG    # experts differ
+    assert layer(wd=_w(lib, fmt=2, d_in=32, d_out=256, group=0, n=16)) == L.OFT_ERR_UNSUPPORTED
+    assert layer(X=0) == L.OFT_ERR_INVALID_ARG
+    assert layer(ws_bytes=1024) == L.OFT_ERR_WORKSPACE
+    lneed = lib.moe_chunked_oft_layer_workspace(32, 16, 4, 4, ctypes.byref(w), ctypes.byref(wd), 32)
+    assert lneed > lib.moe_chunked_oft_workspace(32, 16, 4, 4, ctypes.byref(w), 32)

@@ -406,10 +406,18 @@ def run_ours(args, rank, world):
         def new_outputs():
             return dict(Y=torch.empty_like(Y), dX=torch.empty_like(dX), dQ=torch.empty_like(dQ))
 
+        fwd = oft.oft_linear_fwd
+        if args.weight_side:
+            # the rotation moved onto the weight: Y_p = X (R_p deq(W_p)), one plain bf16 GEMM
+            wsw = torch.empty(oft.oft_linear_fwd_weight_side_workspace(W), dtype=torch.uint8, device=dev)
+
+            def fwd(Xi, Wi, splits, b, Ri, Y=None, workspace=None):
+                return oft.oft_linear_fwd_weight_side(Xi, Wi, splits, b, Ri, Y=Y, workspace=wsw)
+
         def step(Xi=X, dYi=dY, Qi=Q, o=None):
             o = dict(Y=Y, dX=dX, dQ=dQ) if o is None else o
             oft.oft_build_rotation(Qi, spec.b, R=R)
-            oft.oft_linear_fwd(Xi, W, spec.splits, spec.b, R, Y=o["Y"], workspace=ws)
+            fwd(Xi, W, spec.splits, spec.b, R, Y=o["Y"], workspace=ws)
             if backward:
                 oft.oft_linear_bwd(dYi, Xi, W, spec.splits, spec.b, R, dX=o["dX"], dQ=o["dQ"], workspace=ws)
                 allreduce_grad(o["dQ"])
@@ -490,6 +498,9 @@ def run_ours(args, rank, world):
                           + 2 * spec.T * spec.K + 2 * spec.T * spec.K + 4 * spec.T * spec.E + 2 * nq + 4 * nq)
     else:
         flops = linear_flops(spec, backward)
+        if args.weight_side:
+            # the forward rotation on the weight (2 N K b) instead of on the activations (2 M K b P)
+            flops["rot_fwd"] = 2.0 * spec.N * spec.K * spec.b
         total_flops = sum(flops.values())
         alg_bytes = weight_bytes(spec) + 2 * spec.M * spec.K + 2 * spec.M * spec.N
         if backward:
@@ -540,6 +551,9 @@ def run_ours(args, rank, world):
         tiles1 = sum(-(-n // 128) for n in spec.splits) * (-(-(-(-spec.M // 192)) // 2))
         kernel = ("gemm_dq2_kernel (fused dequant, 2-SM pair, tcgen05 cta_group::2)" if tiles1 >= 2 * 148
                   else "gemm_dq_kernel (fused dequant, tcgen05/TMEM)")
+        if args.weight_side and not backward:
+            traffic = None
+            kernel = "gemm_bf16_kernel (plain bf16 x bf16, tcgen05/TMEM; weight-side rotation)"
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
                 "traffic": traffic, "kernel": kernel,
                 "peak_source": f"{peak_src} ({'sustained' if bound == 'tensor' else 'copy'})"}
@@ -623,6 +637,8 @@ def run_ours(args, rank, world):
               "global_batch_tokens": tokens * world, "parallelism": f"dp{world}" if world > 1 else "single",
               "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MB write)",
               "step": "build_rotation + fwd" + (" + bwd" if backward else "") + (" + dQ all-reduce" if world > 1 and backward else "")}
+    if args.weight_side and not is_moe:
+        config["variant"] = "weight-side rotation: Y_p = X (R_p deq(W_p))"
     if is_moe:
         config.update(n_active_experts=n_active, moe_variant=args.moe)
         config["step"] = ("route + build_rotation + fwd" + (" + bwd (dX, dQ, dlogits)" if backward else "")
@@ -699,6 +715,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--moe-backward", action="store_true",
                     help="MoE workload: time forward + adapter backward (chunked path)")
+    ap.add_argument("--weight-side", action="store_true",
+                    help="dense workloads: the weight-side rotation variant of the forward")
     ap.add_argument("--moe-layer", action="store_true",
                     help="MoE workload: time the full expert layer (gate/up, SwiGLU, down projection)")
     ap.add_argument("--moe", default="chunked", choices=["chunked", "fused"],

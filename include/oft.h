@@ -120,6 +120,19 @@ size_t oft_linear_fwd_workspace(int M, const oft_weight* W, const oft_split* S, 
 int oft_linear_fwd(const uint16_t* X, int M, const oft_weight* W, const oft_split* S, int b, const float* R,
                    uint16_t* Y, void* ws, size_t ws_bytes, void* stream);
 
+/* Bytes of scratch oft_linear_fwd_weight_side needs: two bf16 copies of the weight. */
+size_t oft_linear_fwd_weight_side_workspace(const oft_weight* W);
+
+/* Weight-side variant of oft_linear_fwd: the same product, with the rotation moved
+ * onto the weight, Y_p = X (R_p deq(W_p)).  deq(W) is written to bf16, the rows of
+ * each sub-projection are rotated (V_p^T = deq(W_p)^T R_p^T, bf16, on the tensor
+ * cores), and one plain bf16 GEMM gives Y = X V over all N columns.  It does
+ * 2 N K b rotation FLOP instead of 2 M K b P, so it is the cheaper rotation when
+ * N < M P, and it keeps no X' copy.  Same arguments and limits as oft_linear_fwd;
+ * here V is rounded to bf16 instead of X'. */
+int oft_linear_fwd_weight_side(const uint16_t* X, int M, const oft_weight* W, const oft_split* S, int b,
+                               const float* R, uint16_t* Y, void* ws, size_t ws_bytes, void* stream);
+
 /* Bytes of scratch oft_linear_bwd needs for this shape. */
 size_t oft_linear_bwd_workspace(int M, const oft_weight* W, const oft_split* S, int b);
 
@@ -227,10 +240,12 @@ int oft_cayley_backward(const float* R, const float* G, int n_blocks, int b, flo
 
 /* Selects the kernel of the fused-dequant GEMM inside oft_linear_fwd / oft_linear_bwd
  * (test and benchmarking hook; process-wide, not thread-safe against concurrent
- * calls): 0 = by problem size (default: the 2-SM pair kernel for launches of at
- * least two waves of one-CTA tiles), 1 = always the one-CTA kernel, 2 = always the
- * 2-SM pair kernel.  Both compute the same product.  Returns OFT_ERR_INVALID_ARG
- * for any other value. */
+ * calls): 0 = by problem size (default: from 2048 tokens, deq(W) to a bf16
+ * workspace and a plain tcgen05 GEMM; below that the fused-decode kernels, the 2-SM
+ * pair kernel for launches of at least two waves of one-CTA tiles), 1 = always the
+ * one-CTA fused kernel, 2 = always the 2-SM pair fused kernel, 3 = always the bf16
+ * copy and the plain GEMM.  All compute the same product.  Query the *_workspace
+ * sizes after setting the mode.  Returns OFT_ERR_INVALID_ARG for any other value. */
 int oft_set_gemm_mode(int mode);
 
 /* Launches a kernel that waits on a barrier nothing will complete, bounded by

@@ -24,6 +24,8 @@ from .binding import (  # noqa: F401
     oft_linear_bwd_workspace,
     oft_linear_fwd,
     oft_linear_fwd_noalloc,
+    oft_linear_fwd_weight_side,
+    oft_linear_fwd_weight_side_workspace,
     oft_linear_fwd_workspace,
     oft_rotate,
     oft_set_gemm_mode,

@@ -27,7 +27,7 @@ EXPORTS = (
     "oft_cayley_backward", "oft_debug_bounded_wait", "oft_profile_begin", "oft_profile_end",
     "oft_linear_fwd_noalloc", "oft_set_gemm_mode", "moe_fused_oft_workspace", "moe_fused_oft_fwd",
     "moe_chunked_oft_bwd_workspace", "moe_chunked_oft_bwd", "moe_chunked_oft_layer_workspace",
-    "moe_chunked_oft_layer_fwd",
+    "moe_chunked_oft_layer_fwd", "oft_linear_fwd_weight_side_workspace", "oft_linear_fwd_weight_side",
 )
 
 
@@ -54,6 +54,8 @@ _SIGS = {
     "oft_build_rotation": (_I, [_P, _I, _I, _P, _P]),
     "oft_linear_fwd_workspace": (_Z, [_I, _WP, _SP, _I]),
     "oft_linear_fwd": (_I, [_P, _I, _WP, _SP, _I, _P, _P, _P, _Z, _P]),
+    "oft_linear_fwd_weight_side_workspace": (_Z, [_WP]),
+    "oft_linear_fwd_weight_side": (_I, [_P, _I, _WP, _SP, _I, _P, _P, _P, _Z, _P]),
     "oft_linear_bwd_workspace": (_Z, [_I, _WP, _SP, _I]),
     "oft_linear_bwd": (_I, [_P, _P, _I, _WP, _SP, _I, _P, _P, _P, _P, _Z, _P]),
     "moe_chunked_oft_workspace": (_Z, [_I, _I, _I, _I, _WP, _I]),

@@ -142,6 +142,27 @@ def oft_linear_fwd(X: torch.Tensor, W: Weight, splits: Sequence[int], b: int, R:
     return Y
 
 
+def oft_linear_fwd_weight_side_workspace(W: Weight) -> int:
+    cw = W.c()
+    return int(_L.oft_linear_fwd_weight_side_workspace(ctypes.byref(cw)))
+
+
+def oft_linear_fwd_weight_side(X: torch.Tensor, W: Weight, splits: Sequence[int], b: int, R: torch.Tensor,
+                               Y: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                               stream=None) -> torch.Tensor:
+    """The same product as oft_linear_fwd with the rotation applied to the weight:
+    Y_p = X (R_p deq(W_p))."""
+    M = X.shape[0]
+    if Y is None:
+        Y = torch.empty(M, W.d_out, dtype=torch.bfloat16, device=X.device)
+    cw, cs = W.c(), _split(splits)
+    nbytes = int(_L.oft_linear_fwd_weight_side_workspace(ctypes.byref(cw)))
+    ws = _ws(nbytes, X.device, workspace)
+    _check(_L.oft_linear_fwd_weight_side(_ptr(_bits(X)), M, ctypes.byref(cw), ctypes.byref(cs), b, _ptr(R), _ptr(Y),
+                                         _ptr(ws), ws.numel(), _stream(stream)))
+    return Y
+
+
 def oft_linear_bwd(dY: torch.Tensor, X: torch.Tensor, W: Weight, splits: Sequence[int], b: int, R: torch.Tensor,
                    dX: Optional[torch.Tensor] = None, dQ: Optional[torch.Tensor] = None,
                    workspace: Optional[torch.Tensor] = None, stream=None):

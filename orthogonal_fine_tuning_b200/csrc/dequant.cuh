@@ -54,6 +54,7 @@ __device__ __forceinline__ void dequant8(const WeightView& w, const uint8_t* cod
 
 // out[n][k] = deq(W)[n][k] for all n < N, k < K.  One thread per 8 elements.
 __global__ void __launch_bounds__(256) dequant_rows_kernel(WeightView w, uint16_t* __restrict__ out) {
+  pdl_wait();
   const long long units = static_cast<long long>(w.N) * (w.K / 8);
   for (long long u = blockIdx.x * 256ll + threadIdx.x; u < units; u += static_cast<long long>(gridDim.x) * 256) {
     const int n = static_cast<int>(u / (w.K / 8));
@@ -64,33 +65,36 @@ __global__ void __launch_bounds__(256) dequant_rows_kernel(WeightView w, uint16_
   }
 }
 
-// out[k][n] = deq(W)[n][k]: 64 x 64 tiles transposed through shared memory.
+// out[k][n] = deq(W)[n][k]: 64 x 64 tiles transposed through shared memory as
+// 32-bit words (two k per word, rows padded to 33 words), so neither the decode
+// side nor the transposed side has bank conflicts; each warp stores 64-byte runs of
+// 8 k-rows.  grid = (ceil(K / 64), ceil(N / 64)).
 __global__ void __launch_bounds__(256) dequant_transposed_kernel(WeightView w, uint16_t* __restrict__ out) {
-  __shared__ uint16_t tile[64][64 + 8];
+  __shared__ uint32_t tile[64][33];  // [row n][k pair]
+  pdl_wait();
   const int n0 = blockIdx.y * 64;
   const int k0 = blockIdx.x * 64;
-  // load: 64 rows (n) x 8 chunks of 8 k
   for (int it = threadIdx.x; it < 512; it += 256) {
-    const int r = it >> 3, c = it & 7;
+    const int r = it >> 3, c = it & 7;  // row n0 + r, k = k0 + 8c .. +7
     const int n = n0 + r, k = k0 + c * 8;
     uint32_t v[4] = {0, 0, 0, 0};
     if (n < w.N && k < w.K) dequant8(w, w.codes, w.scales, n, k, v);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      tile[r][c * 8 + 2 * i] = static_cast<uint16_t>(v[i] & 0xFFFFu);
-      tile[r][c * 8 + 2 * i + 1] = static_cast<uint16_t>(v[i] >> 16);
-    }
+    for (int i = 0; i < 4; ++i) tile[r][c * 4 + i] = v[i];
   }
   __syncthreads();
-  // store: 64 rows (k) x 8 chunks of 8 n
+  const int lane = threadIdx.x & 31;
   for (int it = threadIdx.x; it < 512; it += 256) {
-    const int r = it >> 3, c = it & 7;
+    const int q = it >> 5;
+    const int r = (lane & 7) + 8 * (q & 7);    // k row
+    const int c = (lane >> 3) + 4 * (q >> 3);  // 8 consecutive n
     const int k = k0 + r, n = n0 + c * 8;
     if (k >= w.K || n >= w.N) continue;
+    const int sh = (r & 1) * 16;
     uint32_t v[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      v[i] = static_cast<uint32_t>(tile[c * 8 + 2 * i][r]) | (static_cast<uint32_t>(tile[c * 8 + 2 * i + 1][r]) << 16);
+      v[i] = ((tile[c * 8 + 2 * i][r >> 1] >> sh) & 0xFFFFu) | (((tile[c * 8 + 2 * i + 1][r >> 1] >> sh) & 0xFFFFu) << 16);
     if (n + 8 <= w.N) {
       *reinterpret_cast<uint4*>(out + static_cast<size_t>(k) * w.N + n) = make_uint4(v[0], v[1], v[2], v[3]);
     } else {

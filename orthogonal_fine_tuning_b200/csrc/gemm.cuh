@@ -68,7 +68,9 @@ struct Params {
 
 constexpr size_t kBarrierBytes = 256;
 constexpr size_t kGroupBytes = sizeof(Group) * MAX_GROUPS;
-constexpr size_t kSmemBytes = 1024 + STAGES * (A_TILE_BYTES + B_TILE_BYTES) + kBarrierBytes + kGroupBytes;
+constexpr int EPI_LD = 33;                                   // fp32 staging row: 32 columns + 1 (no bank conflicts)
+constexpr size_t kEpiBytes = 4 * 32 * EPI_LD * sizeof(float);  // one 32 x 32 fp32 block per epilogue warp
+constexpr size_t kSmemBytes = 1024 + STAGES * (A_TILE_BYTES + B_TILE_BYTES) + kBarrierBytes + kGroupBytes + kEpiBytes;
 
 __device__ __forceinline__ void decode_tile(const Group* sg, int ng, int t, int& g, int& mt, int& nt) {
   g = 0;
@@ -101,8 +103,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_bf16_kernel(const __grid_
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* s_meta = reinterpret_cast<int*>(tmem_slot + 2);  // [0] total tiles, [1] groups
   Group* sg = reinterpret_cast<Group*>(reinterpret_cast<uint8_t*>(bars) + kBarrierBytes);
+  float* s_epi = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(sg) + kGroupBytes);  // [4 warps][32][EPI_LD]
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (p.use_moe) pdl_wait();  // the prologue reads the device-built routing tables
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -181,6 +185,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_bf16_kernel(const __grid_
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();
   const uint32_t tmem_base = *tmem_slot;
   const int total = s_meta[0];
   const int ng = s_meta[1];
@@ -282,17 +287,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_bf16_kernel(const __grid_
         tmem_ld_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN + c), r);
         tmem_ld_wait();
         const int col = nt * BN + c;
-        if (row_ok && col < G.n) {
-          if (p.c_f32) {
-            float* crow = static_cast<float*>(p.C) + crow_off;
-            if (col + 32 <= G.n) {
-              uint4* dst = reinterpret_cast<uint4*>(crow + col);
+        if (p.c_f32) {
+          // transpose the warp's 32 x 32 block through shared memory, then store it as
+          // four full 128-byte row segments per instruction
+          float* stg = s_epi + q * 32 * EPI_LD;
 #pragma unroll
-              for (int v = 0; v < 8; ++v) dst[v] = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
-            } else {
-              for (int i = 0; i < 32 && col + i < G.n; ++i) crow[col + i] = __uint_as_float(r[i]);
+          for (int j = 0; j < 32; ++j) stg[lane * EPI_LD + j] = __uint_as_float(r[j]);
+          __syncwarp();
+          const int c4 = (lane & 7) * 4;
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int rr = it * 4 + (lane >> 3);
+            const int grow = mt * BM + q * 32 + rr;
+            const int gcol = col + c4;
+            if (grow < G.m && gcol < G.n) {
+              const float* sv = stg + rr * EPI_LD + c4;
+              float* dst = static_cast<float*>(p.C) + static_cast<long long>(G.c_row0 + grow) * p.ldc + G.c_col0 + gcol;
+              if (gcol + 4 <= G.n) {
+                *reinterpret_cast<float4*>(dst) = make_float4(sv[0], sv[1], sv[2], sv[3]);
+              } else {
+                for (int e = 0; e < 4 && gcol + e < G.n; ++e) dst[e] = sv[e];
+              }
             }
-          } else {
+          }
+          __syncwarp();
+        } else if (row_ok && col < G.n) {
+          {
             uint16_t* crow = static_cast<uint16_t*>(p.C) + crow_off;
             if (col + 32 <= G.n) {
               uint4* dst = reinterpret_cast<uint4*>(crow + col);

@@ -304,12 +304,12 @@ int launch_dequant(const WeightView& v, uint16_t* out, bool transpose, cudaStrea
     const long long units = 1ll * v.N * (v.K / 8);
     const int grid = static_cast<int>(std::min<long long>((units + 255) / 256, 148ll * 16));
     ProfScope ps(OFT_K_DEQUANT, st);
-    dequant_rows_kernel<<<grid, 256, 0, st>>>(v, out);
+    OFT_CUDA(launch_pdl(dequant_rows_kernel, grid, 256, 0, st, v, out));
     OFT_LAUNCHED("dequant_rows_kernel");
   } else {
     dim3 grid((v.K + 63) / 64, (v.N + 63) / 64);
     ProfScope ps(OFT_K_DEQUANT, st);
-    dequant_transposed_kernel<<<grid, 256, 0, st>>>(v, out);
+    OFT_CUDA(launch_pdl(dequant_transposed_kernel, grid, 256, 0, st, v, out));
     OFT_LAUNCHED("dequant_transposed_kernel");
   }
   return OFT_OK;
@@ -360,9 +360,11 @@ int set_smem(KernelT kernel, size_t bytes) {
 }
 
 // X'_p = X R_p on the tensor cores (all P sub-projections in one pass).
-int launch_rotate_fwd(const uint16_t* X, int M, int K, int P, int b, const float* R, uint16_t* Xr, cudaStream_t st) {
+int launch_rotate_fwd(const uint16_t* X, int M, int K, int P, int b, const float* R, uint16_t* Xr, cudaStream_t st,
+                      bool transpose = false) {
   rtc::FwdParams prm;
   memset(&prm, 0, sizeof(prm));
+  prm.transpose = transpose ? 1 : 0;
   if (int rc = make_map_bf16(&prm.tmX, X, K, M, K, rtc::TM)) return rc;
   if (int rc = make_map_bf16_3d_store(&prm.tmY, Xr, K, M, P)) return rc;
   prm.R = R;
@@ -453,7 +455,7 @@ int launch_gemm(const gemm::Params& prm, int total_tiles_hint, cudaStream_t st) 
   int grid = sm_count();
   if (total_tiles_hint > 0 && total_tiles_hint < grid) grid = total_tiles_hint;
   ProfScope ps(OFT_K_GEMM, st);
-  gemm::gemm_bf16_kernel<<<grid, gemm::NUM_THREADS, gemm::kSmemBytes, st>>>(prm);
+  OFT_CUDA(launch_pdl(gemm::gemm_bf16_kernel, grid, gemm::NUM_THREADS, gemm::kSmemBytes, st, prm));
   OFT_LAUNCHED("gemm_bf16_kernel");
   return OFT_OK;
 }
@@ -643,14 +645,25 @@ int launch_gemm_dq(int fmt, bool bwd, const gdq::Params& prm, int tiles, cudaStr
 
 
 
+// Large token counts take the weight through a bf16 copy and a plain tcgen05 GEMM
+// (gemm.cuh); the dequant pass is cheap next to the product there, and the plain
+// kernel runs closer to the tensor peak than the fused-decode kernels, which stay
+// for small token counts where streaming the low-precision codes matters.
+constexpr int kPlainMinTokens = 2048;
+bool use_plain(int M) {
+  if (g_gemm_mode == 3) return true;
+  if (g_gemm_mode == 1 || g_gemm_mode == 2) return false;
+  return M >= kPlainMinTokens;
+}
+
 struct FwdLayout {
-  size_t xr, total;
+  size_t xr, wdq, total;
 };
-FwdLayout fwd_layout(int M, int K, int N, int P) {
-  (void)N;
+FwdLayout fwd_layout(int M, int K, int N, int P, bool plain) {
   FwdLayout L{};
   L.xr = 0;
-  L.total = round_up(L.xr + 2ull * P * M * K, 256);
+  L.wdq = round_up(L.xr + 2ull * P * M * K, 256);
+  L.total = round_up(L.wdq + (plain ? 2ull * N * K : 0ull), 256);
   return L;
 }
 
@@ -667,13 +680,14 @@ size_t packed_bwd_code_bytes(int fmt, int K, const oft_split* S) {
   return blocks * (fmt == OFT_W_FP8 ? 8192ull : 4096ull);
 }
 
-BwdLayout bwd_layout(int M, int K, int N, const oft_split* S, int b, int fmt) {
+BwdLayout bwd_layout(int M, int K, int N, const oft_split* S, int b, int fmt, bool plain) {
   BwdLayout L{};
   const int P = S->n;
   L.nparts = grad_chunks(M, K).chunks;
   L.dxr = 0;
   L.codes_t = round_up(L.dxr + 4ull * P * M * K, 256);  // dX' kept in fp32
-  L.gpart = round_up(L.codes_t + packed_bwd_code_bytes(fmt, K, S), 256);
+  // packed code blocks for the fused-decode kernels, or deq(W) as bf16 [K][N] for the plain GEMM
+  L.gpart = round_up(L.codes_t + (plain ? 2ull * K * N : packed_bwd_code_bytes(fmt, K, S)), 256);
   L.factors = round_up(L.gpart + 4ull * P * (K / b) * L.nparts * b * b, 256);
   // MXFP4: one bf16 factor per e8m0 scale
   const size_t sbytes = fmt == OFT_W_MXFP4 ? 2ull * (K / 32) * N : 0ull;
@@ -690,7 +704,7 @@ const char* oft_version(void) { return "oft-b200 0.1 (sm_100a, tcgen05)"; }
 const char* oft_last_error(void) { return g_last_error.c_str(); }
 
 int oft_set_gemm_mode(int mode) {
-  if (mode < 0 || mode > 2) return fail(OFT_ERR_INVALID_ARG, "gemm mode must be 0, 1 or 2");
+  if (mode < 0 || mode > 3) return fail(OFT_ERR_INVALID_ARG, "gemm mode must be 0..3");
   g_gemm_mode = mode;
   return OFT_OK;
 }
@@ -741,10 +755,58 @@ int oft_rotate(const uint16_t* X, int M, int K, int P, int b, const float* R, ui
   return launch_rotate_fwd(X, M, K, P, b, R, Xr, as_stream(stream));
 }
 
+size_t oft_linear_fwd_weight_side_workspace(const oft_weight* W) {
+  if (W == nullptr || W->d_in <= 0 || W->d_out <= 0) return 0;
+  return round_up(2ull * W->d_out * W->d_in, 256) + round_up(2ull * W->d_out * W->d_in, 256);
+}
+
+// Weight-side forward: V_p^T = deq(W_p)^T R_p^T (rows of split p), then Y = X V in one
+// plain tcgen05 GEMM over all N columns.
+int oft_linear_fwd_weight_side(const uint16_t* X, int M, const oft_weight* W, const oft_split* S, int b,
+                               const float* R, uint16_t* Y, void* ws, size_t ws_bytes, void* stream) {
+  if (int rc = check_weight(W, false)) return rc;
+  if (int rc = check_split(S, W->d_out)) return rc;
+  const int K = W->d_in, N = W->d_out, P = S->n, nb = K / (b > 0 ? b : 1);
+  if (int rc = check_b(b, K)) return rc;
+  if (K % 32 != 0) return fail(OFT_ERR_UNSUPPORTED, "K must be a multiple of 32");
+  if (M < 0) return fail(OFT_ERR_INVALID_ARG, "M < 0");
+  if (M == 0) return OFT_OK;
+  if (!X || !R || !Y || !ws) return fail(OFT_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(X) || !aligned16(R) || !aligned16(Y) || !aligned16(ws))
+    return fail(OFT_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  const size_t need = oft_linear_fwd_weight_side_workspace(W);
+  if (ws_bytes < need) return fail(OFT_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, need);
+  cudaStream_t st = as_stream(stream);
+  uint16_t* Wd = static_cast<uint16_t*>(ws);
+  uint16_t* V = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + round_up(2ull * N * K, 256));
+  if (int rc = launch_dequant(view_of(W), Wd, false, st)) return rc;
+  int off = 0;
+  for (int p = 0; p < P; ++p) {
+    if (int rc = launch_rotate_fwd(Wd + 1ull * off * K, S->sizes[p], K, 1, b, R + 1ull * p * nb * b * b,
+                                   V + 1ull * off * K, st, true))
+      return rc;
+    off += S->sizes[p];
+  }
+  gemm::Params prm;
+  memset(&prm, 0, sizeof(prm));
+  if (int rc = make_map_bf16(&prm.tmA[0], X, K, M, K, gemm::BM)) return rc;
+  if (int rc = make_map_bf16(&prm.tmB[0], V, K, N, K, gemm::BN)) return rc;
+  prm.C = Y;
+  prm.ldc = N;
+  prm.c_f32 = 0;
+  prm.num_groups = 1;
+  gemm::Group& g = prm.groups[0];
+  g.m = M;
+  g.n = N;
+  g.k = K;
+  const int tiles = ((M + gemm::BM - 1) / gemm::BM) * ((N + gemm::BN - 1) / gemm::BN);
+  return launch_gemm(prm, tiles, st);
+}
+
 size_t oft_linear_fwd_workspace(int M, const oft_weight* W, const oft_split* S, int b) {
   if (W == nullptr || S == nullptr || M <= 0) return 0;
   (void)b;
-  return fwd_layout(M, W->d_in, W->d_out, S->n).total;
+  return fwd_layout(M, W->d_in, W->d_out, S->n, use_plain(M)).total;
 }
 
 int oft_linear_fwd(const uint16_t* X, int M, const oft_weight* W, const oft_split* S, int b, const float* R,
@@ -758,13 +820,42 @@ int oft_linear_fwd(const uint16_t* X, int M, const oft_weight* W, const oft_spli
   if (!X || !R || !Y || !ws) return fail(OFT_ERR_INVALID_ARG, "NULL pointer");
   if (!aligned16(X) || !aligned16(R) || !aligned16(Y) || !aligned16(ws))
     return fail(OFT_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
-  const FwdLayout L = fwd_layout(M, K, N, P);
+  // the plain path when the token count calls for it and the workspace holds the bf16 weight
+  const bool plain = use_plain(M) && ws_bytes >= fwd_layout(M, K, N, P, true).total;
+  const FwdLayout L = fwd_layout(M, K, N, P, plain);
   if (ws_bytes < L.total) return fail(OFT_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
   cudaStream_t st = as_stream(stream);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   uint16_t* Xr = reinterpret_cast<uint16_t*>(wsb + L.xr);
 
   if (int rc = launch_rotate_fwd(X, M, K, P, b, R, Xr, st)) return rc;
+
+  if (plain) {
+    // Y[:, cols of p] = X'_p deq(W_p)^T-rows: one plain grouped GEMM over bf16 deq(W) [N][K]
+    uint16_t* Wdq = reinterpret_cast<uint16_t*>(wsb + L.wdq);
+    if (int rc = launch_dequant(view_of(W), Wdq, false, st)) return rc;
+    gemm::Params prm;
+    memset(&prm, 0, sizeof(prm));
+    if (int rc = make_map_bf16(&prm.tmA[0], Xr, K, 1ull * P * M, K, gemm::BM)) return rc;
+    if (int rc = make_map_bf16(&prm.tmB[0], Wdq, K, N, K, gemm::BN)) return rc;
+    prm.C = Y;
+    prm.ldc = N;
+    prm.c_f32 = 0;
+    prm.num_groups = P;
+    int off = 0, tiles = 0;
+    for (int p = 0; p < P; ++p) {
+      gemm::Group& g = prm.groups[p];
+      g.m = M;
+      g.n = S->sizes[p];
+      g.k = K;
+      g.a_row0 = p * M;
+      g.b_row0 = off;
+      g.c_col0 = off;
+      tiles += ((M + gemm::BM - 1) / gemm::BM) * ((g.n + gemm::BN - 1) / gemm::BN);
+      off += S->sizes[p];
+    }
+    return launch_gemm(prm, tiles, st);
+  }
 
   // Y[:, cols of p] = X'_p deq(W_p): dequant fused into the GEMM's weight operand
   int tiles1 = 0, units2 = 0;
@@ -806,7 +897,7 @@ int oft_linear_fwd(const uint16_t* X, int M, const oft_weight* W, const oft_spli
 
 size_t oft_linear_bwd_workspace(int M, const oft_weight* W, const oft_split* S, int b) {
   if (W == nullptr || S == nullptr || M <= 0 || b <= 0) return 0;
-  return bwd_layout(M, W->d_in, W->d_out, S, b, W->fmt).total;
+  return bwd_layout(M, W->d_in, W->d_out, S, b, W->fmt, use_plain(M)).total;
 }
 
 int oft_linear_bwd(const uint16_t* dY, const uint16_t* X, int M, const oft_weight* W, const oft_split* S, int b,
@@ -825,12 +916,45 @@ int oft_linear_bwd(const uint16_t* dY, const uint16_t* X, int M, const oft_weigh
   if (!dY || !X || !dX || !ws) return fail(OFT_ERR_INVALID_ARG, "NULL pointer");
   if (!aligned16(dY) || !aligned16(X) || !aligned16(R) || !aligned16(dX) || !aligned16(dQ) || !aligned16(ws))
     return fail(OFT_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
-  const BwdLayout L = bwd_layout(M, K, N, S, b, W->fmt);
+  const bool plain = use_plain(M) && ws_bytes >= bwd_layout(M, K, N, S, b, W->fmt, true).total;
+  const BwdLayout L = bwd_layout(M, K, N, S, b, W->fmt, plain);
   if (ws_bytes < L.total) return fail(OFT_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   float* dXr = reinterpret_cast<float*>(wsb + L.dxr);
   uint8_t* codes_t = wsb + L.codes_t;
   float* Gp = reinterpret_cast<float*>(wsb + L.gpart);
+
+  if (plain) {
+    // dX'_p = dY_p deq(W_p): one plain grouped GEMM against bf16 deq(W) laid out [K][N]
+    uint16_t* WdqT = reinterpret_cast<uint16_t*>(codes_t);
+    if (int rc = launch_dequant(view_of(W), WdqT, true, st)) return rc;
+    gemm::Params prm;
+    memset(&prm, 0, sizeof(prm));
+    int off = 0, tiles = 0;
+    for (int p = 0; p < P; ++p) {
+      const int Np = S->sizes[p];
+      if (int rc = make_map_bf16(&prm.tmA[p], dY + off, Np, M, N, gemm::BM)) return rc;
+      if (int rc = make_map_bf16(&prm.tmB[p], WdqT + off, Np, K, N, gemm::BN)) return rc;
+      gemm::Group& g = prm.groups[p];
+      g.m = M;
+      g.n = K;
+      g.k = Np;
+      g.a_map = p;
+      g.b_map = p;
+      g.c_row0 = p * M;
+      tiles += ((M + gemm::BM - 1) / gemm::BM) * ((K + gemm::BN - 1) / gemm::BN);
+      off += Np;
+    }
+    prm.C = dXr;
+    prm.ldc = K;
+    prm.c_f32 = 1;
+    prm.num_groups = P;
+    if (int rc = launch_gemm(prm, tiles, st)) return rc;
+    if (int rc = launch_rotate_bwd(dXr, M, K, P, b, R, dX, st)) return rc;
+    if (int rc = launch_grad(X, dXr, M, K, P, b, Gp, st)) return rc;
+    if (int rc = launch_cayley_bwd(R, Gp, L.nparts, P * nb, b, dQ, st)) return rc;
+    return OFT_OK;
+  }
 
   // codes re-laid out per (sub-projection, 128 input features, 64 channels) block for
   // the dequant producers: one row per input feature, coalesced across a warp

@@ -66,6 +66,7 @@ struct FwdParams {
   const float* R;   // [P][nb][b][b]
   uint16_t* Xr;     // [P][M][K]
   int M, K, P, b, nb, groups, tiles_m;
+  int transpose;    // 1: X'_p = X R_p^T (weight-side rotation of deq(W)^T rows)
 };
 
 constexpr int FWD_A_BYTES = TM * 64 * 2;           // 16 KB
@@ -78,7 +79,7 @@ constexpr size_t kFwdSmem = 1024 + A_STAGES * FWD_A_BYTES + 2 * MAX_P * FWD_BP_B
 __device__ __forceinline__ void builders_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 // B[r = p*64 + c][i] = R_p[i][c] restricted to group g (block-diagonal), split
-// hi/lo.  Zero the tiles, then stream each diagonal R block in with coalesced
+// hi/lo (with p.transpose: B[r = p*64 + i][c] = R_p[i][c], i.e. R_p^T).  Zero the tiles, then stream each diagonal R block in with coalesced
 // float4 loads (eight in flight per thread) and scatter it transposed.
 __device__ void build_fwd_b(const FwdParams& p, int g, uint8_t* sBhi, uint8_t* sBlo, int tid) {
   const int b = p.b;
@@ -115,8 +116,9 @@ __device__ void build_fwd_b(const FwdParams& p, int g, uint8_t* sBhi, uint8_t* s
       const float e[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
-        const int r = sp * 64 + c0 + t;
-        const uint32_t off = swz(r, k >> 3) + (k & 7) * 2;
+        const int r = sp * 64 + (p.transpose ? k : c0 + t);
+        const int kk = p.transpose ? c0 + t : k;
+        const uint32_t off = swz(r, kk >> 3) + (kk & 7) * 2;
         const uint16_t h = bf16_rn(e[t]);
         *reinterpret_cast<uint16_t*>(sBhi + off) = h;
         *reinterpret_cast<uint16_t*>(sBlo + off) = bf16_rn(e[t] - bf16_bits_to_f32(h));

@@ -88,11 +88,16 @@ def test_argument_checks(lib):
 def test_workspace_sizes(lib):
     w, s = _w(lib, d_in=2560, d_out=6144, group=0, fmt=2), _s([4096, 1024, 1024])
     fwd = lib.oft_linear_fwd_workspace(4096, ctypes.byref(w), ctypes.byref(s), 32)
-    # rotated activations for 3 sub-projections; the dequant is fused, so no bf16 weight copy
-    assert 2 * 3 * 4096 * 2560 <= fwd < 2 * 3 * 4096 * 2560 + 2 * 6144 * 2560
+    # 4096 tokens: rotated activations for 3 sub-projections + the bf16 weight copy of the plain GEMM
+    assert 2 * 3 * 4096 * 2560 + 2 * 6144 * 2560 <= fwd < 2 * 3 * 4096 * 2560 + 2 * 6144 * 2560 + 4096
     bwd = lib.oft_linear_bwd_workspace(4096, ctypes.byref(w), ctypes.byref(s), 32)
-    # fp32 dX' for 3 sub-projections + transposed FP8 codes + dR partials
-    assert bwd >= 4 * 3 * 4096 * 2560 + 6144 * 2560
+    # fp32 dX' for 3 sub-projections + the transposed bf16 weight copy + dR partials
+    assert bwd >= 4 * 3 * 4096 * 2560 + 2 * 6144 * 2560
+    # 1024 tokens: the fused-decode kernels, so no bf16 weight copy; packed FP8 codes in the backward
+    fwd1 = lib.oft_linear_fwd_workspace(1024, ctypes.byref(w), ctypes.byref(s), 32)
+    assert 2 * 3 * 1024 * 2560 <= fwd1 < 2 * 3 * 1024 * 2560 + 4096
+    bwd1 = lib.oft_linear_bwd_workspace(1024, ctypes.byref(w), ctypes.byref(s), 32)
+    assert 4 * 3 * 1024 * 2560 + 6144 * 2560 <= bwd1 < 4 * 3 * 1024 * 2560 + 2 * 6144 * 2560
     assert lib.oft_linear_fwd_workspace(0, ctypes.byref(w), ctypes.byref(s), 32) == 0
 
 

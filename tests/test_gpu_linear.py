@@ -47,9 +47,10 @@ SMALL = [
 ]
 
 
-@pytest.fixture(params=[1, 2], ids=["one-cta", "pair"])
+@pytest.fixture(params=[1, 2, 3], ids=["one-cta", "pair", "plain"])
 def gemm_mode(oft, request):
-    """Both fused-dequant GEMM kernels: the one-CTA kernel and the 2-SM pair."""
+    """Every GEMM path: the fused-dequant one-CTA kernel, the 2-SM pair, and the bf16
+    weight copy with the plain tcgen05 GEMM."""
     oft.oft_set_gemm_mode(request.param)
     yield request.param
     oft.oft_set_gemm_mode(0)
@@ -125,3 +126,28 @@ def test_c4_sampled_fwd_bwd(oft):
     dQ = f64(got["dQ"])
     for p, j in [(0, 0), (0, 111), (1, 57), (2, 3)]:
         assert rel_err(dQ[p, j], ref.dq_block(p, j)) < TOL
+
+
+@pytest.mark.parametrize("name,M,K,splits,fmt,group,b", SMALL, ids=[s[0] for s in SMALL])
+def test_weight_side_forward(oft, name, M, K, splits, fmt, group, b):
+    """The weight-side variant, Y_p = X (R_p deq(W_p)), against the same oracle."""
+    spec = LinearSpec(name, M=M, K=K, splits=splits, fmt=fmt, group=group, b=b, q_sigma=0.05,
+                      w_mode="codes" if name == "c0" else "normal", seed=len(name) + M + 1)
+    case = make_linear_case(spec)
+    W = device_weight(case, "cuda")
+    R = oft.oft_build_rotation(case["Q"].cuda(), b)
+    Y = oft.oft_linear_fwd_weight_side(case["X"].cuda(), W, splits, b, R)
+    oft.oft_check_device()
+    assert rel_err(f64(Y), OracleLinear(case).fwd()) < TOL
+
+
+def test_weight_side_c2_sampled(oft):
+    """Gate/up INT4-g128 workload through the weight-side variant, sampled outputs."""
+    case = make_linear_case(LINEAR_CONFIGS["c2"])
+    spec = case["spec"]
+    W = device_weight(case, "cuda")
+    R = oft.oft_build_rotation(case["Q"].cuda(), spec.b)
+    Y = oft.oft_linear_fwd_weight_side(case["X"].cuda(), W, spec.splits, spec.b, R)
+    oft.oft_check_device()
+    rows, cols = _sample(8192, 64, 11), _sample(24576, 512, 12)
+    assert rel_err(f64(Y)[rows][:, cols], OracleLinear(case).fwd(rows=rows, cols=cols)) < TOL

@@ -291,23 +291,29 @@ def cpu_baseline_moe(case, budget_s: float = 12.0, dY=None, down=None):
 # our path
 # ----------------------------------------------------------------------------
 
-def gemm_traffic(flops_per_launch_unit):
-    """Per-launch DRAM bytes of the GEMM kernel from the committed ncu summary, if
-    the kernel source is unchanged since the counters were taken."""
+# device sources each GEMM kernel is built from (its traffic entry is void once they change)
+GEMM_SOURCES = {"gemm_dq2_kernel": ("gemm_dq.cuh", "gemm_dq2.cuh", "dq_pack.cuh"),
+                "gemm_bf16_kernel": ("gemm.cuh",)}
+PLAIN_MIN_TOKENS = 2048  # the library's switch to the bf16 weight copy + plain GEMM
+
+
+def gemm_traffic(kernel: str, workload: str):
+    """Per-launch DRAM bytes of a GEMM kernel from the committed ncu summary, if the
+    kernel's sources are unchanged since the counters were taken."""
     path = os.path.join(ROOT, "profiles", "gemm_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
-        d = json.load(f)
-    if d.get("kernel_sha256_16") != gemm_kernel_hash():
+        d = json.load(f).get(kernel, {})
+    if d.get("kernel_sha256_16") != gemm_kernel_hash(kernel):
         return None
-    return d.get("bytes_per_launch_by_workload", {}).get(flops_per_launch_unit)
+    return d.get("bytes_per_launch_by_workload", {}).get(workload)
 
 
-def gemm_kernel_hash() -> str:
-    """Hash of the fused-dequant GEMMs' device sources (both kernels and their decoders)."""
+def gemm_kernel_hash(kernel: str = "gemm_dq2_kernel") -> str:
+    """Hash of a GEMM kernel's device sources."""
     h = hashlib.sha256()
-    for f in ("gemm_dq.cuh", "gemm_dq2.cuh", "dq_pack.cuh"):
+    for f in GEMM_SOURCES[kernel]:
         with open(os.path.join(ROOT, "orthogonal_fine_tuning_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -321,6 +327,7 @@ def run_ours(args, rank, world):
     _, _, local = dist_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    oft.oft_set_gemm_mode(args.gemm_mode)
     peaks, peak_src = load_peaks()
     name = args.workload
     is_moe = moe_spec(name) is not None
@@ -546,11 +553,18 @@ def run_ours(args, rank, world):
         achieved = per_launch / avg_s / 1e12
         peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
         unit = "TFLOP/s"
-        traffic = gemm_traffic(name)
-        # the library picks the 2-SM pair kernel for launches of two or more one-CTA waves
+        # the library's choice: from PLAIN_MIN_TOKENS tokens the bf16 weight copy and the plain
+        # GEMM; below, the 2-SM pair kernel for launches of two or more one-CTA waves
         tiles1 = sum(-(-n // 128) for n in spec.splits) * (-(-(-(-spec.M // 192)) // 2))
-        kernel = ("gemm_dq2_kernel (fused dequant, 2-SM pair, tcgen05 cta_group::2)" if tiles1 >= 2 * 148
-                  else "gemm_dq_kernel (fused dequant, tcgen05/TMEM)")
+        if args.gemm_mode == 3 or (args.gemm_mode == 0 and spec.M >= PLAIN_MIN_TOKENS):
+            kernel = "gemm_bf16_kernel (plain bf16 GEMM, tcgen05/TMEM; the weight dequantised to bf16 first)"
+            traffic = gemm_traffic("gemm_bf16_kernel", name)
+        elif args.gemm_mode == 2 or (args.gemm_mode == 0 and tiles1 >= 2 * 148):
+            kernel = "gemm_dq2_kernel (fused dequant, 2-SM pair, tcgen05 cta_group::2)"
+            traffic = gemm_traffic("gemm_dq2_kernel", name)
+        else:
+            kernel = "gemm_dq_kernel (fused dequant, tcgen05/TMEM)"
+            traffic = None
         if args.weight_side and not backward:
             traffic = None
             kernel = "gemm_bf16_kernel (plain bf16 x bf16, tcgen05/TMEM; weight-side rotation)"
@@ -715,6 +729,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--moe-backward", action="store_true",
                     help="MoE workload: time forward + adapter backward (chunked path)")
+    ap.add_argument("--gemm-mode", type=int, default=0, choices=[0, 1, 2, 3],
+                    help="GEMM path of the dense workloads (oft_set_gemm_mode): 0 by size, 1 one-CTA fused, "
+                         "2 2-SM pair fused, 3 bf16 copy + plain GEMM")
     ap.add_argument("--weight-side", action="store_true",
                     help="dense workloads: the weight-side rotation variant of the forward")
     ap.add_argument("--moe-layer", action="store_true",

@@ -52,16 +52,27 @@ __device__ __forceinline__ void dequant8(const WeightView& w, const uint8_t* cod
   dq::mxfp4x8(word, eb, out);
 }
 
-// out[n][k] = deq(W)[n][k] for all n < N, k < K.  One thread per 8 elements.
+// out[n][k] = deq(W)[n][k] for all n < N, k < K.  A unit is 8 consecutive elements
+// of a row; each thread takes four units a stride apart per pass, so four code
+// loads are in flight before the first decode.  N * K / 8 < 2^31 (checked on the host).
 __global__ void __launch_bounds__(256) dequant_rows_kernel(WeightView w, uint16_t* __restrict__ out) {
   pdl_wait();
-  const long long units = static_cast<long long>(w.N) * (w.K / 8);
-  for (long long u = blockIdx.x * 256ll + threadIdx.x; u < units; u += static_cast<long long>(gridDim.x) * 256) {
-    const int n = static_cast<int>(u / (w.K / 8));
-    const int k0 = static_cast<int>(u % (w.K / 8)) * 8;
-    uint32_t v[4];
-    dequant8(w, w.codes, w.scales, n, k0, v);
-    *reinterpret_cast<uint4*>(out + static_cast<size_t>(n) * w.K + k0) = make_uint4(v[0], v[1], v[2], v[3]);
+  const int per_row = w.K / 8;
+  const int units = w.N * per_row;
+  const int stride = gridDim.x * 256;
+  for (int u0 = blockIdx.x * 256 + threadIdx.x; u0 < units; u0 += 4 * stride) {
+    uint32_t v[4][4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int u = u0 + j * stride;
+      if (u < units) dequant8(w, w.codes, w.scales, u / per_row, (u % per_row) * 8, v[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int u = u0 + j * stride;
+      if (u < units)
+        *reinterpret_cast<uint4*>(out + static_cast<size_t>(u) * 8) = make_uint4(v[j][0], v[j][1], v[j][2], v[j][3]);
+    }
   }
 }
 

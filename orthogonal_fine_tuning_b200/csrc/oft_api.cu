@@ -300,9 +300,10 @@ WeightView view_of(const oft_weight* W) {
 }
 
 int launch_dequant(const WeightView& v, uint16_t* out, bool transpose, cudaStream_t st) {
+  if (1ll * v.N * v.K / 8 >= (1ll << 31)) return fail(OFT_ERR_UNSUPPORTED, "weight too large for one dequant launch");
   if (!transpose) {
     const long long units = 1ll * v.N * (v.K / 8);
-    const int grid = static_cast<int>(std::min<long long>((units + 255) / 256, 148ll * 16));
+    const int grid = static_cast<int>(std::min<long long>((units + 1023) / 1024, 148ll * 8));
     ProfScope ps(OFT_K_DEQUANT, st);
     OFT_CUDA(launch_pdl(dequant_rows_kernel, grid, 256, 0, st, v, out));
     OFT_LAUNCHED("dequant_rows_kernel");

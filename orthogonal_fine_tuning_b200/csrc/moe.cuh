@@ -147,82 +147,6 @@ __global__ void __launch_bounds__(1024) moe_route_kernel(const int* __restrict__
   }
 }
 
-// Xg[proj][pos][:] = X[bucket[pos] / k] R_{e(pos), proj}  for both projections, in
-// bucket order.  grid = (ceil(K/64) column groups, ceil(TK/128) position tiles).
-// The tile's 128 gathered rows (64 columns each) are staged once in shared memory
-// as fp32 and rotated for gate and up.  Each thread owns one output column c and
-// 32 consecutive positions: it keeps column c of its expert's b x b block in
-// registers and reloads it only where the expert changes (positions are sorted
-// by expert), while the warp shares each activation row by broadcast.
-constexpr int kGatherRows = 128;
-constexpr int kGatherThreads = 256;
-
-template <int B>
-__global__ void __launch_bounds__(kGatherThreads) moe_gather_rotate_kernel(
-    const uint16_t* __restrict__ X, int K, int TK, int top_k, const int* __restrict__ bucket,
-    const int* __restrict__ pos_expert, const float* __restrict__ Rex, uint16_t* __restrict__ Xg) {
-  constexpr int LD = 64 + 4;  // padded fp32 row
-  __shared__ __align__(16) float xs[kGatherRows * LD];
-  __shared__ int s_exp[kGatherRows];
-  const int g = blockIdx.x, p0 = blockIdx.y * kGatherRows, nb = K / B;
-  for (int it = threadIdx.x; it < kGatherRows * 8; it += kGatherThreads) {
-    const int r = it >> 3, ch = it & 7;
-    const int pos = p0 + r, col = g * 64 + ch * 8;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (pos < TK && col < K) {
-      const int t = bucket[pos] / top_k;
-      v = *reinterpret_cast<const uint4*>(X + static_cast<size_t>(t) * K + col);
-    }
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    float* d = xs + r * LD + ch * 8;
-    *reinterpret_cast<float4*>(d) = make_float4(__uint_as_float(w[0] << 16), __uint_as_float(w[0] & 0xFFFF0000u),
-                                                __uint_as_float(w[1] << 16), __uint_as_float(w[1] & 0xFFFF0000u));
-    *reinterpret_cast<float4*>(d + 4) = make_float4(__uint_as_float(w[2] << 16), __uint_as_float(w[2] & 0xFFFF0000u),
-                                                    __uint_as_float(w[3] << 16), __uint_as_float(w[3] & 0xFFFF0000u));
-  }
-  for (int r = threadIdx.x; r < kGatherRows; r += kGatherThreads)
-    s_exp[r] = (p0 + r < TK) ? pos_expert[p0 + r] : -1;
-  __syncthreads();
-  const int c = threadIdx.x & 63, lanegrp = threadIdx.x >> 6;
-  const int col = g * 64 + c;
-  if (col >= K) return;
-  const int jb = col / B, cb = col % B;  // rotation block and column within it
-  const float* xrow0 = xs + (c / B) * B;  // the block's first column in the staged rows
-#pragma unroll 1
-  for (int proj = 0; proj < 2; ++proj) {
-    int cur_e = -1;
-    float rc[B];
-#pragma unroll 1
-    for (int i = 0; i < kGatherRows / 4; ++i) {
-      const int r = lanegrp * (kGatherRows / 4) + i;
-      const int e = s_exp[r];
-      if (e < 0) break;
-      if (e != cur_e) {
-        const float* Rb = Rex + ((static_cast<size_t>(e) * 2 + proj) * nb + jb) * B * B + cb;
-#pragma unroll
-        for (int l = 0; l < B; ++l) rc[l] = Rb[l * B];
-        cur_e = e;
-      }
-      const float* xr = xrow0 + r * LD;
-      float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-      for (int l = 0; l < B; l += 8) {
-        const float4 u = *reinterpret_cast<const float4*>(xr + l);
-        const float4 v = *reinterpret_cast<const float4*>(xr + l + 4);
-        a0 = fmaf(u.x, rc[l + 0], a0);
-        a1 = fmaf(u.y, rc[l + 1], a1);
-        a0 = fmaf(u.z, rc[l + 2], a0);
-        a1 = fmaf(u.w, rc[l + 3], a1);
-        a0 = fmaf(v.x, rc[l + 4], a0);
-        a1 = fmaf(v.y, rc[l + 5], a1);
-        a0 = fmaf(v.z, rc[l + 6], a0);
-        a1 = fmaf(v.w, rc[l + 7], a1);
-      }
-      Xg[(static_cast<size_t>(proj) * TK + p0 + r) * K + col] = f32_to_bf16_bits(a0 + a1);
-    }
-  }
-}
-
 // Rotated gather on the tensor cores: Xg[proj][pos][:] = X[bucket[pos] / k] R_{e,proj}.
 // Units are (active expert, 64-column group, 128-position tile of that expert's
 // bucket rows), in that order with the tile fastest, so a tile never mixes experts

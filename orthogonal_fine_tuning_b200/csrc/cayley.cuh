@@ -38,6 +38,17 @@ __host__ __device__ __forceinline__ int tri_index(int i, int j, int b) {  // i <
 // list (MoE), only the blocks of the first *n_active experts of `active` are
 // built: linear block i is block i % blocks_per_expert of expert
 // active[i / blocks_per_expert].
+// Stage one block's packed Q (B(B-1)/2 bf16 = B(B-1)/16 16-byte vectors; blocks
+// are 16-byte aligned for B = 16, 32, 64) in shared memory with coalesced vector
+// loads by the block's `nthr` threads, so each thread then gathers its row's
+// entries from shared memory instead of with scattered 2-byte global loads.
+template <int B>
+__device__ __forceinline__ void stage_q(const uint16_t* __restrict__ q, uint16_t* qs, int t, int nthr) {
+  constexpr int NV = B * (B - 1) / 16;
+  for (int v = t; v < NV; v += nthr)
+    reinterpret_cast<uint4*>(qs)[v] = reinterpret_cast<const uint4*>(q)[v];
+}
+
 template <int B>
 struct CayleyFwdCfg {
   static constexpr int THREADS = B < 32 ? 32 : B;
@@ -51,6 +62,7 @@ __device__ __forceinline__ void cayley_fwd_block(const uint16_t* __restrict__ Q,
                                                  int blocks_per_expert) {
   constexpr int BPC = CayleyFwdCfg<B>::BPC;
   __shared__ __align__(16) float piv[2][BPC][2 * B + 4];  // pivot row, right-hand side, 1 / pivot
+  __shared__ __align__(16) uint16_t qsh[BPC][B * (B - 1) / 2];
   const int sub = threadIdx.x / B, r = threadIdx.x % B;
   const bool active = lin < total;  // B = 16: the CTA's second block may run past the end
   int blk = lin;
@@ -65,7 +77,10 @@ __device__ __forceinline__ void cayley_fwd_block(const uint16_t* __restrict__ Q,
   };
 
   float a[B], rhs[B];
-  const uint16_t* q = Q + static_cast<size_t>(active ? blk : 0) * (B * (B - 1) / 2);
+  const uint16_t* q = qsh[sub];
+  block_sync();  // the previous block of this CTA is done with qsh and piv
+  if (active) stage_q<B>(Q + static_cast<size_t>(blk) * (B * (B - 1) / 2), qsh[sub], r, B);
+  block_sync();
 #pragma unroll
   for (int j = 0; j < B; ++j) {
     float v = 0.f;
@@ -90,7 +105,7 @@ __device__ __forceinline__ void cayley_fwd_block(const uint16_t* __restrict__ Q,
       float* pr = piv[c & 1][sub];
       const int k0 = c & ~3;  // first float4 holding a column >= c
       if (r == c) {
-        my_inv = 1.0f / a[c];  // >= 1 in exact arithmetic, so never a zero pivot
+        my_inv = __frcp_rn(a[c]);  // >= 1 in exact arithmetic, so never a zero pivot; correctly rounded
         pr[2 * B] = my_inv;
 #pragma unroll
         for (int k = k0; k < B; k += 4)
@@ -126,7 +141,7 @@ __device__ __forceinline__ void cayley_fwd_block(const uint16_t* __restrict__ Q,
     for (int c = 0; c < B; ++c) {
       float* pr = piv[c & 1][sub];
       if (r == c) {
-        my_inv = 1.0f / a[0];
+        my_inv = __frcp_rn(a[0]);
         pr[2 * B] = my_inv;
 #pragma unroll
         for (int k = 0; k < B; k += 4) {
@@ -196,6 +211,7 @@ __global__ void __launch_bounds__(TPR * B) cayley_fwd_split_kernel(const uint16_
   constexpr int H = B / TPR;  // columns per thread
   static_assert(H % 4 == 0 && (TPR & (TPR - 1)) == 0, "slices of whole float4s");
   __shared__ __align__(16) float piv[2][2 * B + 4];
+  __shared__ __align__(16) uint16_t qsh[B * (B - 1) / 2];
   const int r = threadIdx.x / TPR, h = threadIdx.x % TPR;
   const unsigned full = 0xFFFFFFFFu;
   pdl_wait();
@@ -203,7 +219,10 @@ __global__ void __launch_bounds__(TPR * B) cayley_fwd_split_kernel(const uint16_
   for (int lin = blockIdx.x; lin < total; lin += gridDim.x) {
     int blk = lin;
     if (active_list != nullptr) blk = active_list[lin / blocks_per_expert] * blocks_per_expert + lin % blocks_per_expert;
-    const uint16_t* q = Q + static_cast<size_t>(blk) * (B * (B - 1) / 2);
+    __syncthreads();  // the previous block is done with qsh and piv
+    stage_q<B>(Q + static_cast<size_t>(blk) * (B * (B - 1) / 2), qsh, threadIdx.x, TPR * B);
+    __syncthreads();
+    const uint16_t* q = qsh;
     float a[H], rhs[H];
 #pragma unroll
     for (int k = 0; k < H; ++k) {
@@ -224,7 +243,7 @@ __global__ void __launch_bounds__(TPR * B) cayley_fwd_split_kernel(const uint16_
       // the row's pivot-column element A[r][c] is the first thread's a[0]
       const float arc = __shfl_sync(full, a[0], threadIdx.x & ~(TPR - 1));
       if (r == c) {
-        if (h == 0) pr[2 * B] = 1.0f / a[0];  // >= 1 in exact arithmetic
+        if (h == 0) pr[2 * B] = __frcp_rn(a[0]);  // >= 1 in exact arithmetic; correctly rounded
 #pragma unroll
         for (int k = 0; k < H; k += 4) {
           *reinterpret_cast<float4*>(pr + h * H + k) = make_float4(a[k], a[k + 1], a[k + 2], a[k + 3]);

@@ -165,7 +165,7 @@ constexpr int kMoeRotThreads = 128;
 constexpr size_t kMoeRotSmem = 1024 + 3 * 16384 + 64;
 
 template <int B>
-__global__ void __launch_bounds__(kMoeRotThreads) moe_rot_tc_kernel(
+__global__ void __launch_bounds__(kMoeRotThreads, 4) moe_rot_tc_kernel(
     const uint16_t* __restrict__ X, int K, int top_k, const int* __restrict__ bucket,
     const int* __restrict__ offsets, const int* __restrict__ active, const int* __restrict__ n_active_p,
     const float* __restrict__ Rex, int TK, uint16_t* __restrict__ Xg) {
@@ -220,16 +220,53 @@ __global__ void __launch_bounds__(kMoeRotThreads) moe_rot_tc_kernel(
   const int ubeg = static_cast<int>(blockIdx.x) * per + min(static_cast<int>(blockIdx.x), rem);
   const int uend = ubeg + per + (static_cast<int>(blockIdx.x) < rem ? 1 : 0);
   constexpr uint32_t idesc = idesc_bf16_f32(128, 128);
-  int cur_e = -1, cur_g = -1, a = 0;
-  uint32_t phase = 0;
-  for (int u = ubeg; u < uend; ++u) {
-    while (a + 1 < na && s_pref[a + 1] <= u) ++a;  // units are visited in increasing order
-    const int e = active[a];
+  constexpr int NIT = 128 * 8 / kMoeRotThreads;  // 16-byte activation loads per thread and unit
+  struct Unit {
+    int e, g, pos0, nrows;
+  };
+  // units are visited in increasing order; each cursor keeps its own active-expert index
+  auto unit_at = [&](int u, int& acur) -> Unit {
+    while (acur + 1 < na && s_pref[acur + 1] <= u) ++acur;
+    const int e = active[acur];
     const int pos_beg = offsets[e], n_e = offsets[e + 1] - pos_beg;
     const int tiles = (n_e + 127) / 128;
-    const int local = u - s_pref[a];
+    const int local = u - s_pref[acur];
     const int g = local / tiles, rt = local % tiles;
-    const int pos0 = pos_beg + rt * 128, nrows = min(128, n_e - rt * 128);
+    return Unit{e, g, pos_beg + rt * 128, min(128, n_e - rt * 128)};
+  };
+  // Software pipeline: unit u's activation rows are loaded while unit u-1 is multiplied
+  // and stored, and the bucket entries that give their token ids one unit earlier still,
+  // so no load waits on another load.
+  auto load_tokens = [&](const Unit& U, bool valid, int (&tok)[NIT]) {
+#pragma unroll
+    for (int q = 0; q < NIT; ++q) {
+      const int r = (tid + q * kMoeRotThreads) >> 3;
+      tok[q] = (valid && r < U.nrows) ? bucket[U.pos0 + r] : -1;
+    }
+  };
+  auto load_rows = [&](const Unit& U, const int (&tok)[NIT], uint4 (&xv)[NIT]) {
+#pragma unroll
+    for (int q = 0; q < NIT; ++q) {
+      const int col = U.g * 64 + ((tid + q * kMoeRotThreads) & 7) * 8;
+      xv[q] = make_uint4(0, 0, 0, 0);
+      if (tok[q] >= 0 && col < K) xv[q] = *reinterpret_cast<const uint4*>(X + static_cast<size_t>(tok[q] / top_k) * K + col);
+    }
+  };
+  int cur_e = -1, cur_g = -1, a = 0, a1 = 0, a2 = 0;
+  uint32_t phase = 0;
+  uint4 xv[NIT];
+  int tok1[NIT], tok2[NIT];
+  if (ubeg < uend) {
+    const Unit u0 = unit_at(ubeg, a1);
+    load_tokens(u0, true, tok1);
+    load_rows(u0, tok1, xv);
+    const bool v1 = ubeg + 1 < uend;
+    load_tokens(v1 ? unit_at(ubeg + 1, a2) : u0, v1, tok1);
+  }
+  a1 = a2;
+  for (int u = ubeg; u < uend; ++u) {
+    const Unit U = unit_at(u, a);
+    const int e = U.e, g = U.g, pos0 = U.pos0, nrows = U.nrows;
     // 1. rotation tiles of (e, g), when they change (the previous unit's MMAs have completed)
     if (e != cur_e || g != cur_g) {
       for (int v = tid; v < 16384 / 16; v += kMoeRotThreads) {  // each tile is 16 KB
@@ -238,10 +275,10 @@ __global__ void __launch_bounds__(kMoeRotThreads) moe_rot_tc_kernel(
       }
       __syncthreads();
       constexpr int PER = 16 * B;  // float4s of one projection's diagonal blocks in the group
-      constexpr int NIT = 2 * PER / kMoeRotThreads;  // b / 4 per thread: all loads in flight first
-      float4 rv[NIT];
+      constexpr int NRT = 2 * PER / kMoeRotThreads;  // b / 4 per thread: all loads in flight first
+      float4 rv[NRT];
 #pragma unroll
-      for (int q = 0; q < NIT; ++q) {
+      for (int q = 0; q < NRT; ++q) {
         const int f = tid + q * kMoeRotThreads;
         const int pr = f / PER, rem4 = f % PER;
         const int jb = rem4 / (B * B / 4), w = rem4 % (B * B / 4);
@@ -252,7 +289,7 @@ __global__ void __launch_bounds__(kMoeRotThreads) moe_rot_tc_kernel(
                                  : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
-      for (int q = 0; q < NIT; ++q) {
+      for (int q = 0; q < NRT; ++q) {
         const int f = tid + q * kMoeRotThreads;
         const int pr = f / PER, rem4 = f % PER;
         const int jb = rem4 / (B * B / 4), w = rem4 % (B * B / 4);
@@ -271,23 +308,11 @@ __global__ void __launch_bounds__(kMoeRotThreads) moe_rot_tc_kernel(
       cur_e = e;
       cur_g = g;
     }
-    // 2. gather the tile's activation rows: the 8 loads of each thread are all in flight
-    //    before any of them is stored
-    {
-      constexpr int NIT = 128 * 8 / kMoeRotThreads;
-      uint4 xv[NIT];
+    // 2. this unit's activation rows (loaded one unit ago) into the swizzled A tile
 #pragma unroll
-      for (int q = 0; q < NIT; ++q) {
-        const int it = tid + q * kMoeRotThreads, r = it >> 3, col = g * 64 + (it & 7) * 8;
-        xv[q] = make_uint4(0, 0, 0, 0);
-        if (r < nrows && col < K)
-          xv[q] = *reinterpret_cast<const uint4*>(X + static_cast<size_t>(bucket[pos0 + r] / top_k) * K + col);
-      }
-#pragma unroll
-      for (int q = 0; q < NIT; ++q) {
-        const int it = tid + q * kMoeRotThreads;
-        *reinterpret_cast<uint4*>(sA + sw128_offset(static_cast<uint32_t>(it >> 3), static_cast<uint32_t>(it & 7))) = xv[q];
-      }
+    for (int q = 0; q < NIT; ++q) {
+      const int it = tid + q * kMoeRotThreads;
+      *reinterpret_cast<uint4*>(sA + sw128_offset(static_cast<uint32_t>(it >> 3), static_cast<uint32_t>(it & 7))) = xv[q];
     }
     fence_proxy_async_smem();
     __syncthreads();
@@ -302,6 +327,14 @@ __global__ void __launch_bounds__(kMoeRotThreads) moe_rot_tc_kernel(
         mma_bf16_ss(tmem, ad, sdesc_sw128(bl + kk * 32, 16, 1024), idesc, 1u);
       }
       mma_commit(bar);
+    }
+    // prefetch: unit u+1's rows (their token ids are already in tok1), unit u+2's token ids
+    if (u + 1 < uend) {
+      load_rows(unit_at(u + 1, a1), tok1, xv);
+      const bool v2 = u + 2 < uend;
+      load_tokens(v2 ? unit_at(u + 2, a2) : U, v2, tok2);
+#pragma unroll
+      for (int q = 0; q < NIT; ++q) tok1[q] = tok2[q];
     }
     if (!warp_wait_bounded(bar, phase, abort_flag, kErrWaitAccFull)) break;
     phase ^= 1;

@@ -53,7 +53,7 @@ template <int B>
 struct CayleyFwdCfg {
   static constexpr int THREADS = B < 32 ? 32 : B;
   static constexpr int BPC = THREADS / B;  // blocks per CTA
-  static constexpr int MIN_CTAS = B == 64 ? 4 : 16;  // resident CTAs per SM the register budget allows
+  static constexpr int MIN_CTAS = B == 64 ? 8 : 24;  // resident CTAs per SM the register budget allows
 };
 
 template <int B, bool UNROLL>
@@ -180,6 +180,77 @@ __device__ __forceinline__ void cayley_fwd_block(const uint16_t* __restrict__ Q,
   }
 }
 
+// Many-block form (UNROLL = true): in-place Gauss-Jordan inversion of A = I - Q with
+// one thread per row, then R = 2 A^-1 - I, since I + R = 2 (I - Q)^-1.  Each pivot
+// publishes one row of B values and every other row updates B entries, against 2B
+// of each for elimination on [A | I + Q]; with half the row state in registers more
+// blocks stay resident per SM.  The pivot loop is fully unrolled, so every register
+// index is static.  No pivoting: every pivot is >= 1 in exact arithmetic.
+template <int B>
+__device__ __forceinline__ void cayley_fwd_block_inv(const uint16_t* __restrict__ Q, float* __restrict__ R, int lin,
+                                                     int total, const int* __restrict__ active_list,
+                                                     int blocks_per_expert) {
+  constexpr int BPC = CayleyFwdCfg<B>::BPC;
+  __shared__ __align__(16) float piv[2][BPC][B];
+  __shared__ __align__(16) uint16_t qsh[BPC][B * (B - 1) / 2];
+  const int sub = threadIdx.x / B, r = threadIdx.x % B;
+  const bool active = lin < total;  // B = 16: the CTA's second block may run past the end
+  int blk = lin;
+  if (active && active_list != nullptr)
+    blk = active_list[lin / blocks_per_expert] * blocks_per_expert + lin % blocks_per_expert;
+  auto block_sync = [&]() {
+    if constexpr (B <= 32) {
+      __syncwarp();
+    } else {
+      __syncthreads();
+    }
+  };
+  block_sync();  // the previous block of this CTA is done with qsh and piv
+  if (active) stage_q<B>(Q + static_cast<size_t>(blk) * (B * (B - 1) / 2), qsh[sub], r, B);
+  block_sync();
+  const uint16_t* q = qsh[sub];
+  float a[B];
+#pragma unroll
+  for (int j = 0; j < B; ++j) {
+    float v = 0.f;
+    if (active && j != r) {
+      const float t = bf16_bits_to_f32(q[j > r ? tri_index(r, j, B) : tri_index(j, r, B)]);
+      v = j > r ? t : -t;  // Q[r][j]
+    }
+    a[j] = ((j == r) ? 1.f : 0.f) - v;
+  }
+#pragma unroll
+  for (int c = 0; c < B; ++c) {
+    float* pr = piv[c & 1][sub];
+    if (r == c) {
+      const float p = __frcp_rn(a[c]);  // correctly rounded
+#pragma unroll
+      for (int j = 0; j < B; ++j) a[j] = (j == c) ? p : a[j] * p;
+#pragma unroll
+      for (int j = 0; j < B; j += 4) *reinterpret_cast<float4*>(pr + j) = make_float4(a[j], a[j + 1], a[j + 2], a[j + 3]);
+    }
+    block_sync();
+    if (r != c) {
+      const float f = a[c];
+#pragma unroll
+      for (int j = 0; j < B; j += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(pr + j);
+        const float w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) a[j + t] = (j + t == c) ? -f * w[t] : fmaf(-f, w[t], a[j + t]);
+      }
+    }
+  }
+  if (active) {
+    float* out = R + (static_cast<size_t>(blk) * B + r) * B;
+#pragma unroll
+    for (int j = 0; j < B; j += 4)
+      *reinterpret_cast<float4*>(out + j) =
+          make_float4(2.f * a[j] - (j == r ? 1.f : 0.f), 2.f * a[j + 1] - (j + 1 == r ? 1.f : 0.f),
+                      2.f * a[j + 2] - (j + 2 == r ? 1.f : 0.f), 2.f * a[j + 3] - (j + 3 == r ? 1.f : 0.f));
+  }
+}
+
 template <int B, bool UNROLL>
 __global__ void __launch_bounds__(CayleyFwdCfg<B>::THREADS, CayleyFwdCfg<B>::MIN_CTAS) cayley_fwd_kernel(const uint16_t* __restrict__ Q,
                                                                                int nblocks, float* __restrict__ R,
@@ -189,8 +260,13 @@ __global__ void __launch_bounds__(CayleyFwdCfg<B>::THREADS, CayleyFwdCfg<B>::MIN
   constexpr int BPC = CayleyFwdCfg<B>::BPC;
   pdl_wait();
   const int total = active_list != nullptr ? min(nblocks, *n_active * blocks_per_expert) : nblocks;
-  for (int base = blockIdx.x * BPC; base < total; base += gridDim.x * BPC)
-    cayley_fwd_block<B, UNROLL>(Q, R, base + threadIdx.x / B, total, active_list, blocks_per_expert);
+  for (int base = blockIdx.x * BPC; base < total; base += gridDim.x * BPC) {
+    if constexpr (UNROLL) {
+      cayley_fwd_block_inv<B>(Q, R, base + threadIdx.x / B, total, active_list, blocks_per_expert);
+    } else {
+      cayley_fwd_block<B, UNROLL>(Q, R, base + threadIdx.x / B, total, active_list, blocks_per_expert);
+    }
+  }
 }
 
 // Forward for launches of a few hundred blocks (b = 32, 64), where each block's

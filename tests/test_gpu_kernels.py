@@ -72,10 +72,12 @@ def test_cayley_forward_many_blocks(oft, b):
     assert np.abs(np.swapaxes(got, -1, -2) @ got - I).max() < 1e-4
 
 
-def test_cayley_zero_is_identity(oft):
-    Q = torch.zeros(5, 32 * 31 // 2, dtype=torch.bfloat16, device="cuda")
+@pytest.mark.parametrize("nblocks", [5, 4100])
+def test_cayley_zero_is_identity(oft, nblocks):
+    """Q = 0 gives R = I exactly, for the small-launch and the many-block forms."""
+    Q = torch.zeros(nblocks, 32 * 31 // 2, dtype=torch.bfloat16, device="cuda")
     R = oft.oft_build_rotation(Q, 32)
-    assert torch.equal(R.cpu(), torch.eye(32).expand(5, 32, 32))
+    assert torch.equal(R.cpu(), torch.eye(32).expand(nblocks, 32, 32))
 
 
 @pytest.mark.parametrize("b", [16, 32, 64])

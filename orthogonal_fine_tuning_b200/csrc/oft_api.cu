@@ -829,12 +829,23 @@ int oft_linear_fwd(const uint16_t* X, int M, const oft_weight* W, const oft_spli
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   uint16_t* Xr = reinterpret_cast<uint16_t*>(wsb + L.xr);
 
+  SidePipe* sp = nullptr;
+  if (plain) {
+    // deq(W) -> bf16 [N][K] on the side stream, alongside the rotation on this one: the two
+    // read only inputs and write disjoint workspace regions, and the small dequant CTAs fit
+    // next to the rotation's on the same SMs
+    if (int rc = side_pipe(&sp)) return rc;
+    OFT_CUDA(cudaEventRecord(sp->start, st));
+    OFT_CUDA(cudaStreamWaitEvent(sp->side, sp->start, 0));
+    if (int rc = launch_dequant(view_of(W), reinterpret_cast<uint16_t*>(wsb + L.wdq), false, sp->side)) return rc;
+    OFT_CUDA(cudaEventRecord(sp->dq_done[0], sp->side));
+  }
   if (int rc = launch_rotate_fwd(X, M, K, P, b, R, Xr, st)) return rc;
 
   if (plain) {
     // Y[:, cols of p] = X'_p deq(W_p)^T-rows: one plain grouped GEMM over bf16 deq(W) [N][K]
     uint16_t* Wdq = reinterpret_cast<uint16_t*>(wsb + L.wdq);
-    if (int rc = launch_dequant(view_of(W), Wdq, false, st)) return rc;
+    OFT_CUDA(cudaStreamWaitEvent(st, sp->dq_done[0], 0));
     gemm::Params prm;
     memset(&prm, 0, sizeof(prm));
     if (int rc = make_map_bf16(&prm.tmA[0], Xr, K, 1ull * P * M, K, gemm::BM)) return rc;

@@ -32,3 +32,4 @@ from .binding import (  # noqa: F401
     profile,
     version,
 )
+from .slots import AdapterSlots  # noqa: F401,E402

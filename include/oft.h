@@ -38,6 +38,13 @@
  *   - Device-side waits are bounded.  A wait that runs out sets a device error
  *     word and the kernel returns; oft_check_device() reports it as
  *     OFT_ERR_TIMEOUT.
+ *   - Some calls (the MoE entry points, and oft_linear_fwd from 2048 tokens) run
+ *     part of their work on a library-owned side stream of the device, forked from
+ *     and joined back to `stream` with events, so they stay ordered with everything
+ *     else on `stream`.  The side stream is created on the first such call on a
+ *     device; make that call before capturing `stream` into a CUDA graph.  Calls
+ *     from several host threads share it, which orders their side work but never
+ *     breaks the ordering on each caller's stream.
  *
  * Weight storage (stored transposed, one row per output channel: W^T [N][K]):
  *   OFT_W_INT4   codes uint8 [N][K/2]  (element k in byte k/2, low nibble for

@@ -107,7 +107,7 @@ __device__ __forceinline__ bool gemm_drain_wait(uint64_t* bar, uint32_t parity) 
   return true;
 }
 
-// Warp-uniform bounded wait: lane 0 waits, the verdict is broadcast so the whole
+// Warp-uniform bounded wait: lane 0 waits, the outcome is broadcast so the whole
 // warp stays converged for the .sync.aligned instructions that follow.
 __device__ __forceinline__ bool warp_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort, unsigned err) {
   bool ok = false;

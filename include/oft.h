@@ -255,6 +255,20 @@ int oft_cayley_backward(const float* R, const float* G, int n_blocks, int b, flo
  * sizes after setting the mode.  Returns OFT_ERR_INVALID_ARG for any other value. */
 int oft_set_gemm_mode(int mode);
 
+/* The static tile schedule of the plain GEMM (host only, launches nothing).  Groups
+ * g < n_groups are m[g] x n[g] outputs contracted over k[g], cut into 128 x 256
+ * tiles numbered group by group, row band by row band, as the kernel numbers them.
+ * When the groups differ in depth (the dX' product of sub-projections of different
+ * widths), tiles in decreasing depth go to the CTA with the least work so far (ties
+ * to the lowest index).  For `grid` CTAs, sets *used = 1 and writes off[0..grid] and
+ * tiles[0..off[grid]): CTA c runs tiles[off[c] .. off[c+1]) in that order.  Sets
+ * *used = 0 and writes nothing else when the kernel runs round-robin instead: equal
+ * depths, more than 2048 tiles or more than 160 CTAs.  `tiles` holds at least the
+ * total tile count.  OFT_ERR_INVALID_ARG: a NULL pointer, n_groups outside 1..32,
+ * grid < 1. */
+int oft_gemm_schedule(int n_groups, const int* m, const int* n, const int* k, int grid, int* used, int* off,
+                      int* tiles);
+
 /* Launches a kernel that waits on a barrier nothing will complete, bounded by
  * timeout_us microseconds; it must return on its own and set the device error
  * word.  Exercises the timeout path without faulting or hanging the GPU. */

@@ -28,6 +28,7 @@ EXPORTS = (
     "oft_linear_fwd_noalloc", "oft_set_gemm_mode", "moe_fused_oft_workspace", "moe_fused_oft_fwd",
     "moe_chunked_oft_bwd_workspace", "moe_chunked_oft_bwd", "moe_chunked_oft_layer_workspace",
     "moe_chunked_oft_layer_fwd", "oft_linear_fwd_weight_side_workspace", "oft_linear_fwd_weight_side",
+    "oft_gemm_schedule",
 )
 
 
@@ -71,6 +72,7 @@ _SIGS = {
     "oft_cayley_backward": (_I, [_P, _P, _I, _I, _P, _P]),
     "oft_debug_bounded_wait": (_I, [_I, _P]),
     "oft_set_gemm_mode": (_I, [_I]),
+    "oft_gemm_schedule": (_I, [_I, _P, _P, _P, _I, _P, _P, _P]),
     "oft_linear_fwd_noalloc": (_I, [_P, _I, _WP, _SP, _I, _P, _P, _P]),
     "oft_profile_begin": (_I, [_I]),
     "oft_profile_end": (_I, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int), _I,

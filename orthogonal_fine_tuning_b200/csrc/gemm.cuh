@@ -33,6 +33,8 @@ constexpr int MAX_GROUPS = 32;
 constexpr int MAX_MAPS = 4;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr int GM = 16;  // m-tiles per raster band (L2 reuse of the B tiles)
+constexpr int MAX_SCHED_CTAS = 160;
+constexpr int MAX_SCHED_TILES = 2048;
 
 struct Group {
   int m, n, k;
@@ -64,6 +66,25 @@ struct Params {
   int use_moe;
   Group groups[MAX_GROUPS];
   MoESrc moe;
+  // Optional static schedule for groups of unequal depth (sub-projections of different
+  // widths contracted in the backward): CTA c runs tiles sched[sched_off[c] .. sched_off[c+1])
+  // in that order.  sched_ctas == 0 means round-robin over the tiles.
+  int sched_ctas;
+  uint16_t sched_off[MAX_SCHED_CTAS + 1];
+  uint16_t sched[MAX_SCHED_TILES];
+};
+
+// This CTA's tiles: a slice of the static schedule, or every gridDim.x-th tile.
+struct TileIter {
+  int i, end, step;
+  bool tab;
+  __device__ __forceinline__ TileIter(const Params& p, int total) {
+    tab = p.sched_ctas == static_cast<int>(gridDim.x);
+    i = tab ? p.sched_off[blockIdx.x] : static_cast<int>(blockIdx.x);
+    end = tab ? p.sched_off[blockIdx.x + 1] : total;
+    step = tab ? 1 : static_cast<int>(gridDim.x);
+  }
+  __device__ __forceinline__ int tile(const Params& p) const { return tab ? p.sched[i] : i; }
 };
 
 constexpr size_t kBarrierBytes = 256;
@@ -195,7 +216,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_bf16_kernel(const __grid_
       int stage = 0;
       uint32_t ph = 0;
       long long issued = 0;
-      for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      for (TileIter it(p, total); it.i < it.end; it.i += it.step) {
+        const int t = it.tile(p);
+        if (t >= total) continue;
         int g, mt, nt;
         decode_tile(sg, ng, t, g, mt, nt);
         const Group& G = sg[g];
@@ -229,7 +252,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_bf16_kernel(const __grid_
       int acc = 0;
       uint32_t acc_ph = 0;
       constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
-      for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      for (TileIter it(p, total); it.i < it.end; it.i += it.step) {
+        const int t = it.tile(p);
+        if (t >= total) continue;
         int g, mt, nt;
         decode_tile(sg, ng, t, g, mt, nt);
         const int nk = (sg[g].k + BK - 1) / BK;
@@ -268,7 +293,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_bf16_kernel(const __grid_
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     int acc = 0;
     uint32_t acc_ph = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+    for (TileIter it(p, total); it.i < it.end; it.i += it.step) {
+      const int t = it.tile(p);
+      if (t >= total) continue;
       int g, mt, nt;
       decode_tile(sg, ng, t, g, mt, nt);
       const Group& G = sg[g];

@@ -444,7 +444,59 @@ int launch_grad(const uint16_t* X, const float* dXr, int M, int K, int P, int b,
   return OFT_OK;
 }
 
-int launch_gemm(const gemm::Params& prm, int total_tiles_hint, cudaStream_t st) {
+// Longest-first static schedule for a plain grouped GEMM whose groups differ in depth (the
+// dX' product of sub-projections of different widths): tiles in decreasing depth go to
+// the CTA with the least work so far (ties to the lowest index), and each CTA runs its
+// tiles in that order.  Round-robin would leave the CTAs that draw an extra deep tile
+// with up to a quarter more work than the mean.  The last schedule built on this thread
+// is kept, since a training loop repeats the same shapes.
+bool build_gemm_schedule(gemm::Params& prm, int grid) {
+  if (prm.use_moe || grid <= 0 || grid > gemm::MAX_SCHED_CTAS) return false;
+  std::vector<int> key{grid};
+  std::vector<int> depth;  // k-steps per tile, in the order the kernel numbers the tiles
+  int kmin = 1 << 30, kmax = 0;
+  for (int gi = 0; gi < prm.num_groups; ++gi) {
+    const gemm::Group& g = prm.groups[gi];
+    if (g.m <= 0 || g.n <= 0) continue;
+    const int tiles = ((g.m + gemm::BM - 1) / gemm::BM) * ((g.n + gemm::BN - 1) / gemm::BN);
+    const int nk = (g.k + gemm::BK - 1) / gemm::BK;
+    kmin = std::min(kmin, nk);
+    kmax = std::max(kmax, nk);
+    depth.insert(depth.end(), tiles, nk);
+    key.insert(key.end(), {g.m, g.n, g.k});
+  }
+  if (depth.empty() || kmin == kmax || depth.size() > static_cast<size_t>(gemm::MAX_SCHED_TILES)) return false;
+  static thread_local std::vector<int> last_key;
+  static thread_local std::vector<uint16_t> last_off, last_tab;
+  if (key != last_key) {
+    std::vector<int> order(depth.size());
+    for (size_t i = 0; i < order.size(); ++i) order[i] = static_cast<int>(i);
+    std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return depth[a] > depth[b]; });
+    using Slot = std::pair<long long, int>;  // (work so far, CTA)
+    std::priority_queue<Slot, std::vector<Slot>, std::greater<Slot>> heap;
+    for (int c = 0; c < grid; ++c) heap.push({0, c});
+    std::vector<std::vector<uint16_t>> per(grid);
+    for (int t : order) {
+      Slot s = heap.top();
+      heap.pop();
+      per[s.second].push_back(static_cast<uint16_t>(t));
+      heap.push({s.first + depth[t], s.second});
+    }
+    last_off.assign(grid + 1, 0);
+    last_tab.clear();
+    for (int c = 0; c < grid; ++c) {
+      last_tab.insert(last_tab.end(), per[c].begin(), per[c].end());
+      last_off[c + 1] = static_cast<uint16_t>(last_tab.size());
+    }
+    last_key = key;
+  }
+  std::copy(last_off.begin(), last_off.end(), prm.sched_off);
+  std::copy(last_tab.begin(), last_tab.end(), prm.sched);
+  prm.sched_ctas = grid;
+  return true;
+}
+
+int launch_gemm(gemm::Params prm, int total_tiles_hint, cudaStream_t st) {
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -455,6 +507,8 @@ int launch_gemm(const gemm::Params& prm, int total_tiles_hint, cudaStream_t st) 
   }
   int grid = sm_count();
   if (total_tiles_hint > 0 && total_tiles_hint < grid) grid = total_tiles_hint;
+  prm.sched_ctas = 0;
+  build_gemm_schedule(prm, grid);
   ProfScope ps(OFT_K_GEMM, st);
   OFT_CUDA(launch_pdl(gemm::gemm_bf16_kernel, grid, gemm::NUM_THREADS, gemm::kSmemBytes, st, prm));
   OFT_LAUNCHED("gemm_bf16_kernel");
@@ -707,6 +761,28 @@ const char* oft_last_error(void) { return g_last_error.c_str(); }
 int oft_set_gemm_mode(int mode) {
   if (mode < 0 || mode > 3) return fail(OFT_ERR_INVALID_ARG, "gemm mode must be 0..3");
   g_gemm_mode = mode;
+  return OFT_OK;
+}
+
+int oft_gemm_schedule(int n_groups, const int* m, const int* n, const int* k, int grid, int* used, int* off,
+                      int* tiles) {
+  if (!m || !n || !k || !used || !off || !tiles) return fail(OFT_ERR_INVALID_ARG, "NULL pointer");
+  if (n_groups < 1 || n_groups > gemm::MAX_GROUPS) return fail(OFT_ERR_INVALID_ARG, "n_groups must be 1..32");
+  if (grid < 1) return fail(OFT_ERR_INVALID_ARG, "grid < 1");
+  gemm::Params* prm = new gemm::Params;
+  memset(prm, 0, sizeof(*prm));
+  prm->num_groups = n_groups;
+  for (int g = 0; g < n_groups; ++g) {
+    prm->groups[g].m = m[g];
+    prm->groups[g].n = n[g];
+    prm->groups[g].k = k[g];
+  }
+  *used = build_gemm_schedule(*prm, grid) ? 1 : 0;
+  if (*used) {
+    for (int c = 0; c <= grid; ++c) off[c] = prm->sched_off[c];
+    for (int i = 0; i < off[grid]; ++i) tiles[i] = prm->sched[i];
+  }
+  delete prm;
   return OFT_OK;
 }
 

@@ -162,3 +162,52 @@ def test_moe_backward_and_layer_argument_checks(lib):
     assert layer(ws_bytes=1024) == L.OFT_ERR_WORKSPACE
     lneed = lib.moe_chunked_oft_layer_workspace(32, 16, 4, 4, ctypes.byref(w), ctypes.byref(wd), 32)
     assert lneed > lib.moe_chunked_oft_workspace(32, 16, 4, 4, ctypes.byref(w), 32)
+
+
+def _schedule(lib, groups, grid):
+    ng = len(groups)
+    arr = ctypes.c_int * ng
+    m, n, k = (arr(*[g[i] for g in groups]) for i in range(3))
+    total = sum(-(-g[0] // 128) * -(-g[1] // 256) for g in groups)
+    used = ctypes.c_int(-1)
+    off = (ctypes.c_int * (grid + 1))()
+    tiles = (ctypes.c_int * max(total, 1))()
+    rc = lib.oft_gemm_schedule(ng, m, n, k, grid, ctypes.byref(used), off, tiles)
+    depth = []
+    for g in groups:
+        depth += [-(-g[2] // 64)] * (-(-g[0] // 128) * -(-g[1] // 256))
+    return rc, used.value, list(off), list(tiles)[:off[grid]] if used.value == 1 else [], depth
+
+
+def test_gemm_schedule_balances_unequal_depths(lib):
+    # dX' of the fused-QKV workload: 320 tiles 64 k-steps deep (Q), 2 x 320 tiles 16 deep
+    rc, used, off, tiles, depth = _schedule(lib, [(4096, 2560, 4096), (4096, 2560, 1024), (4096, 2560, 1024)], 148)
+    assert rc == 0 and used == 1
+    assert sorted(tiles) == list(range(960))
+    assert off[0] == 0 and all(a <= b for a, b in zip(off, off[1:]))
+    loads = [sum(depth[t] for t in tiles[off[c]:off[c + 1]]) for c in range(148)]
+    round_robin = max(sum(depth[t] for t in range(c, 960, 148)) for c in range(148))
+    # two deep tiles per CTA, 24 CTAs take a third; shallow ones fill the rest up to 208
+    assert max(loads) == 208 and round_robin == 256
+    for c in range(148):  # deepest first within a CTA
+        d = [depth[t] for t in tiles[off[c]:off[c + 1]]]
+        assert d == sorted(d, reverse=True)
+
+
+def test_gemm_schedule_ragged_groups(lib):
+    groups = [(300, 352, 264), (300, 352, 8), (300, 352, 136)]  # 6 tiles each, depths 5, 1, 3
+    rc, used, off, tiles, depth = _schedule(lib, groups, 18)
+    assert rc == 0 and used == 1 and sorted(tiles) == list(range(18))
+    loads = [sum(depth[t] for t in tiles[off[c]:off[c + 1]]) for c in range(18)]
+    assert max(loads) == 5  # one tile per CTA
+
+
+def test_gemm_schedule_falls_back_to_round_robin(lib):
+    assert _schedule(lib, [(4096, 4096, 2560), (4096, 1024, 2560)], 148)[:2] == (0, 0)  # equal depths
+    assert _schedule(lib, [(16384, 7168, 9216), (16384, 7168, 4096)], 148)[:2] == (0, 0)  # 7168 tiles
+    assert _schedule(lib, [(4096, 2560, 4096), (4096, 2560, 1024)], 161)[:2] == (0, 0)  # too many CTAs
+    used = ctypes.c_int()
+    one = (ctypes.c_int * 1)(1)
+    assert lib.oft_gemm_schedule(0, one, one, one, 4, ctypes.byref(used), one, one) == 1
+    assert lib.oft_gemm_schedule(1, one, one, one, 0, ctypes.byref(used), one, one) == 1
+    assert lib.oft_gemm_schedule(1, None, one, one, 4, ctypes.byref(used), one, one) == 1

@@ -293,7 +293,7 @@ def cpu_baseline_moe(case, budget_s: float = 12.0, dY=None, down=None):
 
 # device sources each GEMM kernel is built from (its traffic entry is void once they change)
 GEMM_SOURCES = {"gemm_dq2_kernel": ("gemm_dq.cuh", "gemm_dq2.cuh", "dq_pack.cuh"),
-                "gemm_bf16_kernel": ("gemm.cuh",)}
+                "gemm_bf16_kernel": ("gemm.cuh",), "gemm_bf16_pair_kernel": ("gemm.cuh",)}
 PLAIN_MIN_TOKENS = 2048  # the library's switch to the bf16 weight copy + plain GEMM
 
 
@@ -556,9 +556,13 @@ def run_ours(args, rank, world):
         # the library's choice: from PLAIN_MIN_TOKENS tokens the bf16 weight copy and the plain
         # GEMM; below, the 2-SM pair kernel for launches of two or more one-CTA waves
         tiles1 = sum(-(-n // 128) for n in spec.splits) * (-(-(-(-spec.M // 192)) // 2))
-        if args.gemm_mode == 3 or (args.gemm_mode == 0 and spec.M >= PLAIN_MIN_TOKENS):
-            kernel = "gemm_bf16_kernel (plain bf16 GEMM, tcgen05/TMEM; the weight dequantised to bf16 first)"
+        if args.gemm_mode == 4:
+            kernel = "gemm_bf16_kernel (plain bf16 GEMM, one CTA per tile, tcgen05/TMEM; the weight dequantised first)"
             traffic = gemm_traffic("gemm_bf16_kernel", name)
+        elif args.gemm_mode == 3 or (args.gemm_mode == 0 and spec.M >= PLAIN_MIN_TOKENS):
+            kernel = ("gemm_bf16_pair_kernel (plain bf16 GEMM on 2-SM pairs, tcgen05 cta_group::2; "
+                      "the weight dequantised to bf16 first)")
+            traffic = gemm_traffic("gemm_bf16_pair_kernel", name)
         elif args.gemm_mode == 2 or (args.gemm_mode == 0 and tiles1 >= 2 * 148):
             kernel = "gemm_dq2_kernel (fused dequant, 2-SM pair, tcgen05 cta_group::2)"
             traffic = gemm_traffic("gemm_dq2_kernel", name)
@@ -567,7 +571,8 @@ def run_ours(args, rank, world):
             traffic = None
         if args.weight_side and not backward:
             traffic = None
-            kernel = "gemm_bf16_kernel (plain bf16 x bf16, tcgen05/TMEM; weight-side rotation)"
+            kernel = ("gemm_bf16_kernel (plain bf16 x bf16, one CTA per tile; weight-side rotation)" if args.gemm_mode == 4
+                      else "gemm_bf16_pair_kernel (plain bf16 x bf16 on 2-SM pairs; weight-side rotation)")
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
                 "traffic": traffic, "kernel": kernel,
                 "peak_source": f"{peak_src} ({'sustained' if bound == 'tensor' else 'copy'})"}
@@ -729,9 +734,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--moe-backward", action="store_true",
                     help="MoE workload: time forward + adapter backward (chunked path)")
-    ap.add_argument("--gemm-mode", type=int, default=0, choices=[0, 1, 2, 3],
+    ap.add_argument("--gemm-mode", type=int, default=0, choices=[0, 1, 2, 3, 4],
                     help="GEMM path of the dense workloads (oft_set_gemm_mode): 0 by size, 1 one-CTA fused, "
-                         "2 2-SM pair fused, 3 bf16 copy + plain GEMM")
+                         "2 2-SM pair fused, 3 bf16 copy + plain pair GEMM, 4 bf16 copy + plain one-CTA GEMM")
     ap.add_argument("--weight-side", action="store_true",
                     help="dense workloads: the weight-side rotation variant of the forward")
     ap.add_argument("--moe-layer", action="store_true",

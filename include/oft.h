@@ -245,29 +245,33 @@ int oft_rotate(const uint16_t* X, int M, int K, int P, int b, const float* R, ui
  * R, G fp32 [n_blocks][b][b]; dQ fp32 [n_blocks][b(b-1)/2]. */
 int oft_cayley_backward(const float* R, const float* G, int n_blocks, int b, float* dQ, void* stream);
 
-/* Selects the kernel of the fused-dequant GEMM inside oft_linear_fwd / oft_linear_bwd
- * (test and benchmarking hook; process-wide, not thread-safe against concurrent
- * calls): 0 = by problem size (default: from 2048 tokens, deq(W) to a bf16
- * workspace and a plain tcgen05 GEMM; below that the fused-decode kernels, the 2-SM
- * pair kernel for launches of at least two waves of one-CTA tiles), 1 = always the
- * one-CTA fused kernel, 2 = always the 2-SM pair fused kernel, 3 = always the bf16
- * copy and the plain GEMM.  All compute the same product.  Query the *_workspace
+/* Selects the GEMM inside oft_linear_fwd / oft_linear_bwd and
+ * oft_linear_fwd_weight_side (test and benchmarking hook; process-wide, not
+ * thread-safe against concurrent calls): 0 = by problem size (default: from 2048
+ * tokens, deq(W) to a bf16 workspace and the plain tcgen05 GEMM on 2-SM pairs; below
+ * that the fused-decode kernels, the 2-SM pair kernel for launches of at least two
+ * waves of one-CTA tiles), 1 = always the one-CTA fused kernel, 2 = always the 2-SM
+ * pair fused kernel, 3 = always the bf16 copy and the plain pair GEMM, 4 = always the
+ * bf16 copy and the plain one-CTA GEMM.  The weight-side forward always takes the
+ * plain GEMM: the pair kernel unless the mode is 4.  All compute the same product.  Query the *_workspace
  * sizes after setting the mode.  Returns OFT_ERR_INVALID_ARG for any other value. */
 int oft_set_gemm_mode(int mode);
 
 /* The static tile schedule of the plain GEMM (host only, launches nothing).  Groups
- * g < n_groups are m[g] x n[g] outputs contracted over k[g], cut into 128 x 256
+ * g < n_groups are m[g] x n[g] outputs contracted over k[g], cut into tile_rows x 256
  * tiles numbered group by group, row band by row band, as the kernel numbers them.
- * When the groups differ in depth (the dX' product of sub-projections of different
- * widths), tiles in decreasing depth go to the CTA with the least work so far (ties
- * to the lowest index).  For `grid` CTAs, sets *used = 1 and writes off[0..grid] and
- * tiles[0..off[grid]): CTA c runs tiles[off[c] .. off[c+1]) in that order.  Sets
+ * A worker is a CTA of the one-CTA kernel (tile_rows = 128) or a CTA pair of the 2-SM
+ * kernel (tile_rows = 256).  When the groups differ in depth (the dX' product of
+ * sub-projections of different widths), tiles in decreasing depth go to the worker
+ * with the least work so far (ties to the lowest index).  For `grid` workers, sets
+ * *used = 1 and writes off[0..grid] and tiles[0..off[grid]): worker c runs
+ * tiles[off[c] .. off[c+1]) in that order.  Sets
  * *used = 0 and writes nothing else when the kernel runs round-robin instead: equal
- * depths, more than 2048 tiles or more than 160 CTAs.  `tiles` holds at least the
+ * depths, more than 2048 tiles or more than 160 workers.  `tiles` holds at least the
  * total tile count.  OFT_ERR_INVALID_ARG: a NULL pointer, n_groups outside 1..32,
- * grid < 1. */
-int oft_gemm_schedule(int n_groups, const int* m, const int* n, const int* k, int grid, int* used, int* off,
-                      int* tiles);
+ * tile_rows not 128 or 256, grid < 1. */
+int oft_gemm_schedule(int n_groups, const int* m, const int* n, const int* k, int tile_rows, int grid, int* used,
+                      int* off, int* tiles);
 
 /* Launches a kernel that waits on a barrier nothing will complete, bounded by
  * timeout_us microseconds; it must return on its own and set the device error

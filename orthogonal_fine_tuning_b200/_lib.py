@@ -72,7 +72,7 @@ _SIGS = {
     "oft_cayley_backward": (_I, [_P, _P, _I, _I, _P, _P]),
     "oft_debug_bounded_wait": (_I, [_I, _P]),
     "oft_set_gemm_mode": (_I, [_I]),
-    "oft_gemm_schedule": (_I, [_I, _P, _P, _P, _I, _P, _P, _P]),
+    "oft_gemm_schedule": (_I, [_I, _P, _P, _P, _I, _I, _P, _P, _P]),
     "oft_linear_fwd_noalloc": (_I, [_P, _I, _WP, _SP, _I, _P, _P, _P]),
     "oft_profile_begin": (_I, [_I]),
     "oft_profile_end": (_I, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int), _I,

@@ -311,8 +311,9 @@ def oft_cayley_backward(R: torch.Tensor, G: torch.Tensor, b: int, out: Optional[
 
 
 def oft_set_gemm_mode(mode: int) -> None:
-    """Fused-dequant GEMM kernel inside the linear calls: 0 by size (default),
-    1 the one-CTA kernel, 2 the 2-SM pair kernel (same product)."""
+    """GEMM inside the linear calls: 0 by size (default), 1 the one-CTA fused-dequant
+    kernel, 2 the 2-SM pair fused-dequant kernel, 3 the bf16 weight copy and the plain
+    GEMM on 2-SM pairs, 4 the same on one CTA per tile (same product)."""
     _check(_L.oft_set_gemm_mode(int(mode)))
 
 

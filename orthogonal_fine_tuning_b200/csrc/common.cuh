@@ -283,6 +283,18 @@ __device__ __forceinline__ void mma_bf16_ts_pair(uint32_t d_tmem, uint32_t a_tme
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// D (+)= A * B^T over the pair with both operands in shared memory: A rows 0..127 from
+// the leader's, 128..255 from the peer's; B columns split in halves the same way (same
+// descriptor offsets in both CTAs); each CTA's TMEM receives its own 128 rows of D.
+__device__ __forceinline__ void mma_bf16_ss_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // Arrive once on the mbarrier at the same offset in both CTAs of the pair when all
 // tcgen05 ops issued so far by this thread complete.
 __device__ __forceinline__ void mma_commit_pair_both(uint64_t* bar) {

@@ -450,15 +450,15 @@ int launch_grad(const uint16_t* X, const float* dXr, int M, int K, int P, int b,
 // tiles in that order.  Round-robin would leave the CTAs that draw an extra deep tile
 // with up to a quarter more work than the mean.  The last schedule built on this thread
 // is kept, since a training loop repeats the same shapes.
-bool build_gemm_schedule(gemm::Params& prm, int grid) {
+bool build_gemm_schedule(gemm::Params& prm, int grid, int tile_rows) {
   if (prm.use_moe || grid <= 0 || grid > gemm::MAX_SCHED_CTAS) return false;
-  std::vector<int> key{grid};
+  std::vector<int> key{grid, tile_rows};
   std::vector<int> depth;  // k-steps per tile, in the order the kernel numbers the tiles
   int kmin = 1 << 30, kmax = 0;
   for (int gi = 0; gi < prm.num_groups; ++gi) {
     const gemm::Group& g = prm.groups[gi];
     if (g.m <= 0 || g.n <= 0) continue;
-    const int tiles = ((g.m + gemm::BM - 1) / gemm::BM) * ((g.n + gemm::BN - 1) / gemm::BN);
+    const int tiles = ((g.m + tile_rows - 1) / tile_rows) * ((g.n + gemm::BN - 1) / gemm::BN);
     const int nk = (g.k + gemm::BK - 1) / gemm::BK;
     kmin = std::min(kmin, nk);
     kmax = std::max(kmax, nk);
@@ -508,7 +508,7 @@ int launch_gemm(gemm::Params prm, int total_tiles_hint, cudaStream_t st) {
   int grid = sm_count();
   if (total_tiles_hint > 0 && total_tiles_hint < grid) grid = total_tiles_hint;
   prm.sched_ctas = 0;
-  build_gemm_schedule(prm, grid);
+  build_gemm_schedule(prm, grid, gemm::BM);
   ProfScope ps(OFT_K_GEMM, st);
   OFT_CUDA(launch_pdl(gemm::gemm_bf16_kernel, grid, gemm::NUM_THREADS, gemm::kSmemBytes, st, prm));
   OFT_LAUNCHED("gemm_bf16_kernel");
@@ -675,6 +675,40 @@ int launch_gemm_dq2_t(const gdq::Params& prm, int units, cudaStream_t st) {
   return launch_gemm_dq2_k<FMT, BWD, false>(kp, clusters, st);
 }
 
+// The plain GEMM on 2-SM pairs: one persistent cluster per resident pair (the same
+// one-CTA-per-SM footprint as the fused pair kernel), schedule in units of pair tiles.
+int launch_gemm_pair(gemm::Params prm, int pair_tiles, cudaStream_t st) {
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    OFT_CUDA(cudaFuncSetAttribute(gemm::gemm_bf16_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(gemm::kPairSmemBytes)));
+    attr_set[dev] = true;
+  }
+  const int clusters = std::max(1, std::min(pair_clusters_resident(), pair_tiles));
+  prm.sched_ctas = 0;
+  build_gemm_schedule(prm, clusters, gemm::PM);
+  ProfScope ps(OFT_K_GEMM, st);
+  OFT_CUDA(launch_pdl(gemm::gemm_bf16_pair_kernel, 2 * clusters, gemm::NUM_THREADS, gemm::kPairSmemBytes, st, prm));
+  OFT_LAUNCHED("gemm_bf16_pair_kernel");
+  return OFT_OK;
+}
+
+// The dense path's plain GEMM: the pair kernel, or the one-CTA kernel in gemm mode 4.
+// B tensor maps must have boxes of plain_b_rows() rows.
+bool plain_pair() { return g_gemm_mode != 4; }
+uint32_t plain_b_rows() { return plain_pair() ? 128u : static_cast<uint32_t>(gemm::BN); }
+int launch_plain_gemm(const gemm::Params& prm, cudaStream_t st) {
+  const int bm = plain_pair() ? gemm::PM : gemm::BM;
+  int tiles = 0;
+  for (int g = 0; g < prm.num_groups; ++g) {
+    const gemm::Group& G = prm.groups[g];
+    if (G.m > 0 && G.n > 0) tiles += ((G.m + bm - 1) / bm) * ((G.n + gemm::BN - 1) / gemm::BN);
+  }
+  return plain_pair() ? launch_gemm_pair(prm, tiles, st) : launch_gemm(prm, tiles, st);
+}
+
 // Pair kernel for launches of at least two one-CTA waves (unless forced).
 bool use_pair(int tiles_one_cta) {
   if (g_gemm_mode == 1) return false;
@@ -706,7 +740,7 @@ int launch_gemm_dq(int fmt, bool bwd, const gdq::Params& prm, int tiles, cudaStr
 // for small token counts where streaming the low-precision codes matters.
 constexpr int kPlainMinTokens = 2048;
 bool use_plain(int M) {
-  if (g_gemm_mode == 3) return true;
+  if (g_gemm_mode == 3 || g_gemm_mode == 4) return true;
   if (g_gemm_mode == 1 || g_gemm_mode == 2) return false;
   return M >= kPlainMinTokens;
 }
@@ -759,15 +793,16 @@ const char* oft_version(void) { return "oft-b200 0.1 (sm_100a, tcgen05)"; }
 const char* oft_last_error(void) { return g_last_error.c_str(); }
 
 int oft_set_gemm_mode(int mode) {
-  if (mode < 0 || mode > 3) return fail(OFT_ERR_INVALID_ARG, "gemm mode must be 0..3");
+  if (mode < 0 || mode > 4) return fail(OFT_ERR_INVALID_ARG, "gemm mode must be 0..4");
   g_gemm_mode = mode;
   return OFT_OK;
 }
 
-int oft_gemm_schedule(int n_groups, const int* m, const int* n, const int* k, int grid, int* used, int* off,
-                      int* tiles) {
+int oft_gemm_schedule(int n_groups, const int* m, const int* n, const int* k, int tile_rows, int grid, int* used,
+                      int* off, int* tiles) {
   if (!m || !n || !k || !used || !off || !tiles) return fail(OFT_ERR_INVALID_ARG, "NULL pointer");
   if (n_groups < 1 || n_groups > gemm::MAX_GROUPS) return fail(OFT_ERR_INVALID_ARG, "n_groups must be 1..32");
+  if (tile_rows != gemm::BM && tile_rows != gemm::PM) return fail(OFT_ERR_INVALID_ARG, "tile_rows must be 128 or 256");
   if (grid < 1) return fail(OFT_ERR_INVALID_ARG, "grid < 1");
   gemm::Params* prm = new gemm::Params;
   memset(prm, 0, sizeof(*prm));
@@ -777,7 +812,7 @@ int oft_gemm_schedule(int n_groups, const int* m, const int* n, const int* k, in
     prm->groups[g].n = n[g];
     prm->groups[g].k = k[g];
   }
-  *used = build_gemm_schedule(*prm, grid) ? 1 : 0;
+  *used = build_gemm_schedule(*prm, grid, tile_rows) ? 1 : 0;
   if (*used) {
     for (int c = 0; c <= grid; ++c) off[c] = prm->sched_off[c];
     for (int i = 0; i < off[grid]; ++i) tiles[i] = prm->sched[i];
@@ -867,7 +902,7 @@ int oft_linear_fwd_weight_side(const uint16_t* X, int M, const oft_weight* W, co
   gemm::Params prm;
   memset(&prm, 0, sizeof(prm));
   if (int rc = make_map_bf16(&prm.tmA[0], X, K, M, K, gemm::BM)) return rc;
-  if (int rc = make_map_bf16(&prm.tmB[0], V, K, N, K, gemm::BN)) return rc;
+  if (int rc = make_map_bf16(&prm.tmB[0], V, K, N, K, plain_b_rows())) return rc;
   prm.C = Y;
   prm.ldc = N;
   prm.c_f32 = 0;
@@ -876,8 +911,7 @@ int oft_linear_fwd_weight_side(const uint16_t* X, int M, const oft_weight* W, co
   g.m = M;
   g.n = N;
   g.k = K;
-  const int tiles = ((M + gemm::BM - 1) / gemm::BM) * ((N + gemm::BN - 1) / gemm::BN);
-  return launch_gemm(prm, tiles, st);
+  return launch_plain_gemm(prm, st);
 }
 
 size_t oft_linear_fwd_workspace(int M, const oft_weight* W, const oft_split* S, int b) {
@@ -925,12 +959,12 @@ int oft_linear_fwd(const uint16_t* X, int M, const oft_weight* W, const oft_spli
     gemm::Params prm;
     memset(&prm, 0, sizeof(prm));
     if (int rc = make_map_bf16(&prm.tmA[0], Xr, K, 1ull * P * M, K, gemm::BM)) return rc;
-    if (int rc = make_map_bf16(&prm.tmB[0], Wdq, K, N, K, gemm::BN)) return rc;
+    if (int rc = make_map_bf16(&prm.tmB[0], Wdq, K, N, K, plain_b_rows())) return rc;
     prm.C = Y;
     prm.ldc = N;
     prm.c_f32 = 0;
     prm.num_groups = P;
-    int off = 0, tiles = 0;
+    int off = 0;
     for (int p = 0; p < P; ++p) {
       gemm::Group& g = prm.groups[p];
       g.m = M;
@@ -939,10 +973,9 @@ int oft_linear_fwd(const uint16_t* X, int M, const oft_weight* W, const oft_spli
       g.a_row0 = p * M;
       g.b_row0 = off;
       g.c_col0 = off;
-      tiles += ((M + gemm::BM - 1) / gemm::BM) * ((g.n + gemm::BN - 1) / gemm::BN);
       off += S->sizes[p];
     }
-    return launch_gemm(prm, tiles, st);
+    return launch_plain_gemm(prm, st);
   }
 
   // Y[:, cols of p] = X'_p deq(W_p): dequant fused into the GEMM's weight operand
@@ -1018,11 +1051,11 @@ int oft_linear_bwd(const uint16_t* dY, const uint16_t* X, int M, const oft_weigh
     if (int rc = launch_dequant(view_of(W), WdqT, true, st)) return rc;
     gemm::Params prm;
     memset(&prm, 0, sizeof(prm));
-    int off = 0, tiles = 0;
+    int off = 0;
     for (int p = 0; p < P; ++p) {
       const int Np = S->sizes[p];
       if (int rc = make_map_bf16(&prm.tmA[p], dY + off, Np, M, N, gemm::BM)) return rc;
-      if (int rc = make_map_bf16(&prm.tmB[p], WdqT + off, Np, K, N, gemm::BN)) return rc;
+      if (int rc = make_map_bf16(&prm.tmB[p], WdqT + off, Np, K, N, plain_b_rows())) return rc;
       gemm::Group& g = prm.groups[p];
       g.m = M;
       g.n = K;
@@ -1030,14 +1063,13 @@ int oft_linear_bwd(const uint16_t* dY, const uint16_t* X, int M, const oft_weigh
       g.a_map = p;
       g.b_map = p;
       g.c_row0 = p * M;
-      tiles += ((M + gemm::BM - 1) / gemm::BM) * ((K + gemm::BN - 1) / gemm::BN);
       off += Np;
     }
     prm.C = dXr;
     prm.ldc = K;
     prm.c_f32 = 1;
     prm.num_groups = P;
-    if (int rc = launch_gemm(prm, tiles, st)) return rc;
+    if (int rc = launch_plain_gemm(prm, st)) return rc;
     if (int rc = launch_rotate_bwd(dXr, M, K, P, b, R, dX, st)) return rc;
     if (int rc = launch_grad(X, dXr, M, K, P, b, Gp, st)) return rc;
     if (int rc = launch_cayley_bwd(R, Gp, L.nparts, P * nb, b, dQ, st)) return rc;

@@ -164,18 +164,18 @@ def test_moe_backward_and_layer_argument_checks(lib):
     assert lneed > lib.moe_chunked_oft_workspace(32, 16, 4, 4, ctypes.byref(w), 32)
 
 
-def _schedule(lib, groups, grid):
+def _schedule(lib, groups, grid, rows=128):
     ng = len(groups)
     arr = ctypes.c_int * ng
     m, n, k = (arr(*[g[i] for g in groups]) for i in range(3))
-    total = sum(-(-g[0] // 128) * -(-g[1] // 256) for g in groups)
+    total = sum(-(-g[0] // rows) * -(-g[1] // 256) for g in groups)
     used = ctypes.c_int(-1)
     off = (ctypes.c_int * (grid + 1))()
     tiles = (ctypes.c_int * max(total, 1))()
-    rc = lib.oft_gemm_schedule(ng, m, n, k, grid, ctypes.byref(used), off, tiles)
+    rc = lib.oft_gemm_schedule(ng, m, n, k, rows, grid, ctypes.byref(used), off, tiles)
     depth = []
     for g in groups:
-        depth += [-(-g[2] // 64)] * (-(-g[0] // 128) * -(-g[1] // 256))
+        depth += [-(-g[2] // 64)] * (-(-g[0] // rows) * -(-g[1] // 256))
     return rc, used.value, list(off), list(tiles)[:off[grid]] if used.value == 1 else [], depth
 
 
@@ -194,6 +194,15 @@ def test_gemm_schedule_balances_unequal_depths(lib):
         assert d == sorted(d, reverse=True)
 
 
+def test_gemm_schedule_pairs(lib):
+    # the same dX' on 74 CTA pairs with 256 x 256 tiles: 160 tiles 64 deep, 320 tiles 16 deep
+    rc, used, off, tiles, depth = _schedule(lib, [(4096, 2560, 4096), (4096, 2560, 1024), (4096, 2560, 1024)], 74,
+                                            rows=256)
+    assert rc == 0 and used == 1 and sorted(tiles) == list(range(480))
+    loads = [sum(depth[t] for t in tiles[off[c]:off[c + 1]]) for c in range(74)]
+    assert max(loads) == 208 and sum(loads) == 160 * 64 + 320 * 16
+
+
 def test_gemm_schedule_ragged_groups(lib):
     groups = [(300, 352, 264), (300, 352, 8), (300, 352, 136)]  # 6 tiles each, depths 5, 1, 3
     rc, used, off, tiles, depth = _schedule(lib, groups, 18)
@@ -208,6 +217,14 @@ def test_gemm_schedule_falls_back_to_round_robin(lib):
     assert _schedule(lib, [(4096, 2560, 4096), (4096, 2560, 1024)], 161)[:2] == (0, 0)  # too many CTAs
     used = ctypes.c_int()
     one = (ctypes.c_int * 1)(1)
-    assert lib.oft_gemm_schedule(0, one, one, one, 4, ctypes.byref(used), one, one) == 1
-    assert lib.oft_gemm_schedule(1, one, one, one, 0, ctypes.byref(used), one, one) == 1
-    assert lib.oft_gemm_schedule(1, None, one, one, 4, ctypes.byref(used), one, one) == 1
+    assert lib.oft_gemm_schedule(0, one, one, one, 128, 4, ctypes.byref(used), one, one) == 1
+    assert lib.oft_gemm_schedule(1, one, one, one, 128, 0, ctypes.byref(used), one, one) == 1
+    assert lib.oft_gemm_schedule(1, one, one, one, 64, 4, ctypes.byref(used), one, one) == 1
+    assert lib.oft_gemm_schedule(1, None, one, one, 256, 4, ctypes.byref(used), one, one) == 1
+
+
+def test_gemm_mode_range(lib):
+    for mode in range(5):
+        assert lib.oft_set_gemm_mode(mode) == 0
+    assert lib.oft_set_gemm_mode(5) == 1 and lib.oft_set_gemm_mode(-1) == 1
+    assert lib.oft_set_gemm_mode(0) == 0

@@ -47,10 +47,10 @@ SMALL = [
 ]
 
 
-@pytest.fixture(params=[1, 2, 3], ids=["one-cta", "pair", "plain"])
+@pytest.fixture(params=[1, 2, 3, 4], ids=["one-cta", "pair", "plain-pair", "plain"])
 def gemm_mode(oft, request):
     """Every GEMM path: the fused-dequant one-CTA kernel, the 2-SM pair, and the bf16
-    weight copy with the plain tcgen05 GEMM."""
+    weight copy with the plain tcgen05 GEMM on 2-SM pairs or on one CTA per tile."""
     oft.oft_set_gemm_mode(request.param)
     yield request.param
     oft.oft_set_gemm_mode(0)

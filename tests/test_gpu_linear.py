@@ -44,6 +44,9 @@ SMALL = [
     ("wide-k", 130, 1024, (384,), "fp8", 0, 16),
     ("small-m-mxfp4", 37, 2048, (264, 1032), "mxfp4", 32, 64),
     ("small-m-fp8", 64, 1536, (256, 128, 128), "fp8", 0, 32),
+    # 80 tiles of 256 x 256 on 74 CTA pairs (a second, partial wave), ragged in both
+    # tokens and columns
+    ("wave-tail", 1000, 256, (2560, 2440), "int4", 32, 32),
 ]
 
 

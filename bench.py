@@ -443,11 +443,23 @@ def run_ours(args, rank, world):
                 allreduce_grad(o["dQ"])
             return o["Y"]
 
+        def bwd_part():
+            oft.oft_linear_bwd(dY, X, W, spec.splits, spec.b, R, dX=dX, dQ=dQ, workspace=ws)
+            allreduce_grad(dQ)
+
+        # the same step as its API calls, each timed on its own in a third pass
+        step_parts = [("build_rotation", lambda: oft.oft_build_rotation(Q, spec.b, R=R)),
+                      ("fwd", lambda: fwd(X, W, spec.splits, spec.b, R, Y=Y, workspace=ws))]
+        if backward:
+            step_parts.append(("bwd", bwd_part))
+
         inputs = dict(X=X, Q=Q) if not backward else dict(X=X, dY=dY, Q=Q)
         outputs = dict(Y=Y) if not backward else dict(Y=Y, dX=dX, dQ=dQ)
         result_keys = tuple(outputs)
 
     # ---- device-resident timing ----
+    if is_moe:
+        step_parts = None
     for _ in range(args.warmup):
         step()
     oft.oft_check_device()
@@ -479,6 +491,27 @@ def run_ours(args, rank, world):
     with oft.profile(max_launches=max(4096, 64 * args.steps)) as prof:
         ms_prof_local = timed_pass()
     oft.oft_check_device()
+    # Third pass (dense workloads): CUDA events around each API call of the step, L2
+    # flushed before each step.  Supplementary: a failure here is reported in the line.
+    part_ms = None
+    if step_parts is not None:
+        try:
+            ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in step_parts]
+                  for _ in range(args.steps)]
+            for i in range(args.steps):
+                flush.zero_()
+                for (e0, e1), (_pname, call) in zip(ev[i], step_parts):
+                    e0.record()
+                    call()
+                    e1.record()
+            torch.cuda.synchronize()
+            part_ms = {}
+            for j, (pname, _call) in enumerate(step_parts):
+                ms_j = sum(ev[k][j][0].elapsed_time(ev[k][j][1]) for k in range(args.steps)) / args.steps
+                part_ms[pname] = max_over_ranks(ms_j, dev)
+        except Exception as exc:  # never fatal to the measurement above
+            part_ms = {"error": repr(exc)[:200]}
+        oft.oft_check_device()
     ms_per_step = max_over_ranks(ms_local, dev)
     ms_profiled = max_over_ranks(ms_prof_local, dev)
     value = tokens * world / (ms_per_step / 1e3)
@@ -689,6 +722,7 @@ def run_ours(args, rank, world):
                                   "kernel_ms_per_step and roofline.achieved come from this pass"},
         "kernel_ms_per_step": {k: v / args.steps for k, v in prof.ms.items()},
         "kernel_launches_per_step": {k: v / args.steps for k, v in prof.launches.items()},
+        **({"part_ms_per_step": part_ms} if part_ms is not None else {}),
         "clocks": clk,
     }
     return line

@@ -5,12 +5,16 @@ A step is one pass of the whole path over one batch: Cayley build of every
 rotation block, the split-projection forward (rotate, dequant, tcgen05 GEMM),
 and for the training workloads the adapter backward (dX' GEMM, dX rotation,
 dR reduction, Cayley backward), plus the dQ all-reduce when several ranks run
-data-parallel replicas.  Default workload: the dense fused-QKV FP8 forward +
-backward (4096 tokens x 2560 -> 4096/1024/1024, b = 32).
+data-parallel replicas.  The headline workload (default) is the largest one that
+fits one GPU: the MXFP4 training step, forward + backward (16384 tokens x 7168 ->
+12288/3072/3072, b = 64).  On one GPU the other four workloads are timed after it
+(--also) and reported in the same line under "workloads".
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c1] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c4] [--also c0,c1,c2,c3]
+                    [--impl ours|reference]
 
-Prints one JSON line (rank 0).
+With --gpus N > 1 and no WORLD_SIZE in the environment, the script starts N ranks
+itself (torch.distributed.run, one process per GPU).  Prints one JSON line (rank 0).
 """
 
 from __future__ import annotations
@@ -95,6 +99,38 @@ def allreduce_grad(dQ):
     if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
         dist.all_reduce(dQ)
     return dQ
+
+
+def token_shard(M: int, rank: int, world: int):
+    """Contiguous token range [t0, t1) of `rank` when one batch of M tokens is split
+    over `world` data-parallel replicas (the first M % world ranks take one more)."""
+    base, extra = divmod(M, world)
+    t0 = rank * base + min(rank, extra)
+    return t0, t0 + base + (1 if rank < extra else 0)
+
+
+def launch_cmd(argv, nproc: int, port: int, limit_s: int = 3600):
+    """The command that runs this script as `nproc` ranks on one node (one process
+    per GPU), bounded by `timeout`."""
+    return ["timeout", "-k", "60", str(limit_s), sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={nproc}", "--master-addr", "127.0.0.1", f"--master-port={port}",
+            os.path.abspath(__file__), *argv]
+
+
+def workload_config(name: str, tokens: int, world: int, backward: bool, args, n_active=None):
+    """The `config` object of a line: the same for our arm and the reference arm."""
+    config = {"workload": WORKLOAD_NAMES[name], "name": name, "tokens_per_gpu": tokens,
+              "global_batch_tokens": tokens * world, "parallelism": f"dp{world}" if world > 1 else "single",
+              "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MB write)",
+              "step": "build_rotation + fwd" + (" + bwd" if backward else "")
+                      + (" + dQ all-reduce" if world > 1 and backward else "")}
+    if moe_spec(name) is not None:
+        config.update(n_active_experts=n_active, moe_variant=args.moe)
+        config["step"] = ("route + build_rotation + fwd" + (" + bwd (dX, dQ, dlogits)" if backward else "")
+                          + (" (full expert layer: gate/up, SwiGLU, down)" if args.moe_layer else ""))
+    elif args.weight_side:
+        config["variant"] = "weight-side rotation: Y_p = X (R_p deq(W_p))"
+    return config
 
 
 def load_peaks():
@@ -332,7 +368,7 @@ def gemm_kernel_hash(kernel: str = "gemm_dq2_kernel") -> str:
     return h.hexdigest()[:16]
 
 
-def run_ours(args, rank, world):
+def run_ours(args, rank, world, name):
     import torch
     import orthogonal_fine_tuning_b200 as oft
     from gen import LINEAR_CONFIGS, MOE_CONFIGS, make_linear_case, make_moe_case, make_moe_down, make_moe_grad
@@ -342,7 +378,6 @@ def run_ours(args, rank, world):
     dev = torch.device("cuda", local)
     oft.oft_set_gemm_mode(args.gemm_mode)
     peaks, peak_src = load_peaks()
-    name = args.workload
     is_moe = moe_spec(name) is not None
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
 
@@ -413,6 +448,15 @@ def run_ours(args, rank, world):
         W = oft.Weight(spec.fmt, case["codes"].to(dev), case["scales"].to(dev), spec.K, spec.N, spec.group)
         X, Q = case["X"].to(dev), case["Q"].to(dev)
         dY = case["dY"].to(dev) if backward else None
+        if rank > 0:
+            # data-parallel replicas: the same frozen weight and adapter; rank r holds tokens
+            # [t0, t1) of a global batch of world x M (weak scaling), drawn from their own seed
+            t0, _t1 = token_shard(spec.M * world, rank, world)
+            g = torch.Generator(device=dev)
+            g.manual_seed(10007 * t0 + spec.seed)
+            X = torch.randn(spec.M, spec.K, generator=g, device=dev).to(torch.bfloat16)
+            if backward:
+                dY = torch.randn(spec.M, spec.N, generator=g, device=dev).to(torch.bfloat16)
         nbytes = oft.oft_linear_fwd_workspace(spec.M, W, spec.splits, spec.b)
         if backward:
             nbytes = max(nbytes, oft.oft_linear_bwd_workspace(spec.M, W, spec.splits, spec.b))
@@ -443,9 +487,8 @@ def run_ours(args, rank, world):
                 allreduce_grad(o["dQ"])
             return o["Y"]
 
-        def bwd_part():
+        def bwd_part():  # rank-local: the all-reduce is not one of the library calls timed here
             oft.oft_linear_bwd(dY, X, W, spec.splits, spec.b, R, dX=dX, dQ=dQ, workspace=ws)
-            allreduce_grad(dQ)
 
         # the same step as its API calls, each timed on its own in a third pass
         step_parts = [("build_rotation", lambda: oft.oft_build_rotation(Q, spec.b, R=R)),
@@ -485,16 +528,21 @@ def run_ours(args, rank, world):
         torch.cuda.synchronize()
         return sum(s.elapsed_time(e) for s, e in zip(st_, en_)) / args.steps
 
-    with ClockSampler(dev) as clocks:
-        ms_local = timed_pass()
+    # The clock sampler runs over every timed pass (the step, the profiled step, the
+    # per-call pass and the end-to-end leg) so that short steps still get samples.
+    clocks = ClockSampler(dev).__enter__()
+    ms_local = timed_pass()
     oft.oft_check_device()
     with oft.profile(max_launches=max(4096, 64 * args.steps)) as prof:
         ms_prof_local = timed_pass()
     oft.oft_check_device()
     # Third pass (dense workloads): CUDA events around each API call of the step, L2
-    # flushed before each step.  Supplementary: a failure here is reported in the line.
+    # flushed before each step.  Rank-local (no collective inside); supplementary: a
+    # failure here is reported in the line, and every rank then takes the same
+    # max-over-ranks reductions below (a failed part reports -1).
     part_ms = None
     if step_parts is not None:
+        part_local, part_err = [-1.0] * len(step_parts), None
         try:
             ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in step_parts]
                   for _ in range(args.steps)]
@@ -505,12 +553,13 @@ def run_ours(args, rank, world):
                     call()
                     e1.record()
             torch.cuda.synchronize()
-            part_ms = {}
-            for j, (pname, _call) in enumerate(step_parts):
-                ms_j = sum(ev[k][j][0].elapsed_time(ev[k][j][1]) for k in range(args.steps)) / args.steps
-                part_ms[pname] = max_over_ranks(ms_j, dev)
+            for j in range(len(step_parts)):
+                part_local[j] = sum(ev[k][j][0].elapsed_time(ev[k][j][1]) for k in range(args.steps)) / args.steps
         except Exception as exc:  # never fatal to the measurement above
-            part_ms = {"error": repr(exc)[:200]}
+            part_err = repr(exc)[:200]
+        part_ms = {pname: max_over_ranks(part_local[j], dev) for j, (pname, _c) in enumerate(step_parts)}
+        if part_err is not None:
+            part_ms["error"] = part_err
         oft.oft_check_device()
     ms_per_step = max_over_ranks(ms_local, dev)
     ms_profiled = max_over_ranks(ms_prof_local, dev)
@@ -560,8 +609,76 @@ def run_ours(args, rank, world):
             alg_bytes += 2 * spec.M * spec.N + 2 * spec.M * spec.K + 4 * dQ.numel() + 2 * dQ.numel()
     tflops = total_flops / (ms_per_step / 1e3) / 1e12
 
-    # ---- dominant kernel roofline ----
+    # ---- end to end through the public API with host buffers ----
+    # Every step copies its own inputs from pinned host memory and reads all of its
+    # outputs back into pinned host memory.  Copies in, compute and copies out run on
+    # three streams, double-buffered, so step i's read-back and step i+1's upload
+    # overlap step i+1's / step i's compute (one step in flight on each engine).
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    host_in = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in inputs.items()}
+    for k, v in inputs.items():
+        host_in[k].copy_(v)
+    dev_in = [{k: torch.empty_like(v) for k, v in inputs.items()} for _ in range(2)]
+    dev_out = [new_outputs() for _ in range(2)]
+    host_out = [{k: torch.empty(dev_out[b][k].shape, dtype=dev_out[b][k].dtype, pin_memory=True)
+                 for k in result_keys} for b in range(2)]
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    for b in range(2):  # all buffers free at the start
+        ev_comp[b].record(comp)
+        ev_out[b].record(comp)
+
+    def e2e_step(i):
+        b = i % 2
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(ev_comp[b])          # compute of step i-2 is done with dev_in[b]
+            for k in dev_in[b]:
+                dev_in[b][k].copy_(host_in[k], non_blocking=True)
+            ev_in[b].record(s_in)
+        comp.wait_event(ev_in[b])
+        comp.wait_event(ev_out[b])               # read-back of step i-2 is done with dev_out[b]
+        d = dev_in[b]
+        if is_moe and args.moe_layer:
+            step(d["X"], d["logits"], d["Q"], o=dev_out[b], Qdi=d["Q_down"])
+        elif is_moe:
+            step(d["X"], d["logits"], d["Q"], o=dev_out[b], dYi=d.get("dY"))
+        elif backward:
+            step(d["X"], d["dY"], d["Q"], o=dev_out[b])
+        else:
+            step(d["X"], None, d["Q"], o=dev_out[b])
+        ev_comp[b].record(comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_comp[b])
+            for k in result_keys:
+                host_out[b][k].copy_(dev_out[b][k], non_blocking=True)
+            ev_out[b].record(s_out)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    es.record(comp)
+    s_in.wait_event(es)
+    for i in range(args.steps):
+        e2e_step(i)
+    for b in range(2):
+        comp.wait_event(ev_out[b])
+    ee.record(comp)
+    torch.cuda.synchronize()
+    clocks.__exit__(None, None, None)
     clk = clocks.summary()
+    e2e_ms = max_over_ranks(es.elapsed_time(ee) / args.steps, dev)
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+    d2h = sum(v.numel() * v.element_size() for v in host_out[0].values())
+    e2e = {"value": tokens * world / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+           "pipelining": "double-buffered: upload, compute and read-back on three streams"}
+
+    # ---- dominant kernel roofline ----
     peak_kind = "copy"
     g_launch = prof.launches["gemm"]
     g_ms = prof.ms["gemm"]
@@ -625,73 +742,6 @@ def run_ours(args, rank, world):
                 "traffic": traffic, "kernel": kernel,
                 "peak_source": f"{peak_src} ({peak_kind})"}
 
-    # ---- end to end through the public API with host buffers ----
-    # Every step copies its own inputs from pinned host memory and reads all of its
-    # outputs back into pinned host memory.  Copies in, compute and copies out run on
-    # three streams, double-buffered, so step i's read-back and step i+1's upload
-    # overlap step i+1's / step i's compute (one step in flight on each engine).
-    comp = torch.cuda.current_stream()
-    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
-    host_in = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in inputs.items()}
-    for k, v in inputs.items():
-        host_in[k].copy_(v)
-    dev_in = [{k: torch.empty_like(v) for k, v in inputs.items()} for _ in range(2)]
-    dev_out = [new_outputs() for _ in range(2)]
-    host_out = [{k: torch.empty(dev_out[b][k].shape, dtype=dev_out[b][k].dtype, pin_memory=True)
-                 for k in result_keys} for b in range(2)]
-    ev_in = [torch.cuda.Event() for _ in range(2)]
-    ev_comp = [torch.cuda.Event() for _ in range(2)]
-    ev_out = [torch.cuda.Event() for _ in range(2)]
-    for b in range(2):  # all buffers free at the start
-        ev_comp[b].record(comp)
-        ev_out[b].record(comp)
-
-    def e2e_step(i):
-        b = i % 2
-        with torch.cuda.stream(s_in):
-            s_in.wait_event(ev_comp[b])          # compute of step i-2 is done with dev_in[b]
-            for k in dev_in[b]:
-                dev_in[b][k].copy_(host_in[k], non_blocking=True)
-            ev_in[b].record(s_in)
-        comp.wait_event(ev_in[b])
-        comp.wait_event(ev_out[b])               # read-back of step i-2 is done with dev_out[b]
-        d = dev_in[b]
-        if is_moe and args.moe_layer:
-            step(d["X"], d["logits"], d["Q"], o=dev_out[b], Qdi=d["Q_down"])
-        elif is_moe:
-            step(d["X"], d["logits"], d["Q"], o=dev_out[b], dYi=d.get("dY"))
-        elif backward:
-            step(d["X"], d["dY"], d["Q"], o=dev_out[b])
-        else:
-            step(d["X"], None, d["Q"], o=dev_out[b])
-        ev_comp[b].record(comp)
-        with torch.cuda.stream(s_out):
-            s_out.wait_event(ev_comp[b])
-            for k in result_keys:
-                host_out[b][k].copy_(dev_out[b][k], non_blocking=True)
-            ev_out[b].record(s_out)
-
-    for i in range(args.warmup):
-        e2e_step(i)
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    es.record(comp)
-    s_in.wait_event(es)
-    for i in range(args.steps):
-        e2e_step(i)
-    for b in range(2):
-        comp.wait_event(ev_out[b])
-    ee.record(comp)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(es.elapsed_time(ee) / args.steps, dev)
-    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
-    d2h = sum(v.numel() * v.element_size() for v in host_out[0].values())
-    e2e = {"value": tokens * world / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-           "pipelining": "double-buffered: upload, compute and read-back on three streams"}
-
     if rank != 0:
         return None
     cpu = None
@@ -700,16 +750,7 @@ def run_ours(args, rank, world):
             cpu = cpu_baseline_moe(case, dY=dY if backward else None, down=dn if args.moe_layer else None)
         else:
             cpu = cpu_baseline_linear(case, backward)
-    config = {"workload": WORKLOAD_NAMES[name], "name": name, "tokens_per_gpu": tokens,
-              "global_batch_tokens": tokens * world, "parallelism": f"dp{world}" if world > 1 else "single",
-              "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MB write)",
-              "step": "build_rotation + fwd" + (" + bwd" if backward else "") + (" + dQ all-reduce" if world > 1 and backward else "")}
-    if args.weight_side and not is_moe:
-        config["variant"] = "weight-side rotation: Y_p = X (R_p deq(W_p))"
-    if is_moe:
-        config.update(n_active_experts=n_active, moe_variant=args.moe)
-        config["step"] = ("route + build_rotation + fwd" + (" + bwd (dX, dQ, dlogits)" if backward else "")
-                          + (" (full expert layer: gate/up, SwiGLU, down)" if args.moe_layer else ""))
+    config = workload_config(name, tokens, world, backward, args, n_active if is_moe else None)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -728,6 +769,12 @@ def run_ours(args, rank, world):
     return line
 
 
+# keys of a workload's own line kept in the headline line's "workloads" object
+WORKLOAD_KEYS = ("value", "unit", "ms_per_step", "tflops", "config", "algorithmic_flops_per_step",
+                 "algorithmic_bytes_per_step", "roofline", "cpu_baseline", "e2e", "gpu_launches", "profiled_pass",
+                 "kernel_ms_per_step", "kernel_launches_per_step", "part_ms_per_step", "clocks")
+
+
 def run_reference(args, rank, world):
     """The oracle (float64 numpy, as it stands) timed on the host cores, on a
     bounded sample of the same workload per step."""
@@ -735,13 +782,22 @@ def run_reference(args, rank, world):
         return None
     from gen import LINEAR_CONFIGS, MOE_CONFIGS, make_linear_case, make_moe_case, make_moe_down, make_moe_grad
     name = args.workload
+    n_active = None
     if moe_spec(name) is not None:
+        import numpy as np
         import torch
+        from oracle import moe_ref
+        sys.path.insert(0, os.path.join(ROOT, "tests"))
+        from npcase import raw
         spec = moe_spec(name)
         dev = "cuda" if torch.cuda.is_available() else "cpu"
         case = make_moe_case(spec, device=dev)
         dY = make_moe_grad(spec, device=dev) if args.moe_backward else None
         dn = make_moe_down(spec, device=dev) if args.moe_layer else None
+        idx, _ = moe_ref.topk(raw(case["logits"]), spec.top_k)
+        n_active = int(np.unique(idx).size)
+        backward = args.moe_backward
+        tokens = spec.T
         per = max(2.0, 150.0 / (args.steps + args.warmup))
         for _ in range(args.warmup):
             cpu_baseline_moe(case, budget_s=per / 4, dY=dY, down=dn)
@@ -750,6 +806,8 @@ def run_reference(args, rank, world):
         sample = res[-1]["sample"]
     else:
         spec = linear_spec(name)
+        backward = spec.backward
+        tokens = spec.M
         case = make_linear_case(spec)
         per_budget = 150.0 / (args.steps + args.warmup)
         tokens = min(spec.M, 64)
@@ -767,7 +825,7 @@ def run_reference(args, rank, world):
     return {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": WORKLOAD_NAMES[name], "name": name},
+            "config": workload_config(name, tokens, world, backward, args, n_active),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -778,7 +836,11 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="c1", choices=sorted(WORKLOAD_NAMES))
+    ap.add_argument("--workload", default="c4", choices=sorted(WORKLOAD_NAMES),
+                    help="the headline workload (default: the MXFP4 training step, the largest that fits one GPU)")
+    ap.add_argument("--also", default="c0,c1,c2,c3",
+                    help="comma-separated workloads timed after the headline one on a single GPU and reported "
+                         "under 'workloads' in the same line ('' for none)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--moe-backward", action="store_true",
@@ -797,6 +859,15 @@ def main(argv=None):
         ap.error("--moe-layer times the forward of the full expert layer; --moe-backward the gate/up backward")
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # one process per GPU: start the ranks and hand back their exit status
+        import subprocess
+        import socket
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        argv = sys.argv[1:] if argv is None else list(argv)
+        sys.exit(subprocess.call(launch_cmd(argv, args.gpus, port)))
     if args.impl == "reference":
         rank, world, _ = dist_env()
         line = run_reference(args, rank, world)
@@ -804,7 +875,21 @@ def main(argv=None):
         rank, world = init_dist("nccl")
         if world != args.gpus:
             print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
-        line = run_ours(args, rank, world)
+        line = run_ours(args, rank, world, args.workload)
+        # the other workloads, on a single GPU only (no collective runs in this loop)
+        extras = [w for w in args.also.split(",") if w and w != args.workload] if world == 1 else []
+        if extras and line is not None:
+            line["workloads"] = {}
+            for name in extras:
+                import gc
+                import torch
+                gc.collect()
+                torch.cuda.empty_cache()
+                try:
+                    sub = run_ours(args, rank, world, name)
+                    line["workloads"][name] = {k: sub[k] for k in WORKLOAD_KEYS if k in sub}
+                except Exception as exc:  # reported, never fatal to the headline line
+                    line["workloads"][name] = {"error": repr(exc)[:300]}
         import torch.distributed as dist
         if dist.is_initialized():
             dist.barrier()

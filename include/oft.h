@@ -121,7 +121,9 @@ int oft_build_rotation(const uint16_t* Q, int n_blocks, int b, float* R, void* s
 /* Bytes of scratch oft_linear_fwd needs for this shape. */
 size_t oft_linear_fwd_workspace(int M, const oft_weight* W, const oft_split* S, int b);
 
-/* Split-projection OFT linear forward:  Y[:, cols of p] = (X R_p) deq(W_p).
+/* Split-projection OFT linear forward (chooseai.io news 4086, item "分投影适配器支持";
+ * the frozen base dequantised on the fly, section "技术原理：低精度基座 + BF16 适配器 + OFT"):
+ *   Y[:, cols of p] = (X R_p) deq(W_p).
  * X bf16 [M][K]; R fp32 [P][K/b][b][b] (from oft_build_rotation); Y bf16 [M][N].
  * fp32 accumulation, bf16 output (round to nearest even).  K % 32 == 0. */
 int oft_linear_fwd(const uint16_t* X, int M, const oft_weight* W, const oft_split* S, int b, const float* R,
@@ -143,7 +145,9 @@ int oft_linear_fwd_weight_side(const uint16_t* X, int M, const oft_weight* W, co
 /* Bytes of scratch oft_linear_bwd needs for this shape. */
 size_t oft_linear_bwd_workspace(int M, const oft_weight* W, const oft_split* S, int b);
 
-/* Adapter backward (no gradient for the frozen weight).
+/* Adapter backward (no gradient for the frozen weight: m.xxlwj.com 771001, section
+ * "技术细节", DeepSeek V4 paragraph; the adapter alone carries the gradient,
+ * chooseai.io news 4086, section "技术原理：低精度基座 + BF16 适配器 + OFT").
  * dY bf16 [M][N], X bf16 [M][K], R as in the forward.
  * Outputs: dX bf16 [M][K] = sum_p (dY_p W_p^T) R_p^T;
  *          dQ fp32 [P][K/b][b(b-1)/2], fully overwritten (not accumulated):
@@ -245,6 +249,21 @@ int oft_rotate(const uint16_t* X, int M, int K, int P, int b, const float* R, ui
  * R, G fp32 [n_blocks][b][b]; dQ fp32 [n_blocks][b(b-1)/2]. */
 int oft_cayley_backward(const float* R, const float* G, int n_blocks, int b, float* dQ, void* stream);
 
+/* One chunk of the MoE transient dequant (the pages' "Active-expert-chunked
+ * dequantization", section "技术细节" of m.xxlwj.com 771001), with the kernels and
+ * launch shapes the MoE calls use.  bank: an INT4 expert bank (n_experts = E,
+ * d_out = N per expert); chunk_table: device int32, slot s of chunk c is entry
+ * c * chunk + s, an expert id or -1 (empty).  For every non-empty slot s of chunk
+ * chunk_idx, with e its expert:
+ *   transpose = 0: out[s][r][k]    = deq(W_e)[r][k],       out bf16 [chunk][N][K]
+ *                  (the forward's chunk buffer; the full layer's down projections
+ *                  use it with the down bank);
+ *   transpose = 1: out[s][p][k][j] = deq(W_e)[p*N/2 + j][k], out bf16 [chunk][2][K][N/2]
+ *                  (the backward's transposed buffer; N % 16 == 0).
+ * Slots of -1 are left untouched.  Bit-exact: w = bf16_rne(q * s). */
+int oft_moe_chunk_dequant(const oft_weight* bank, const int32_t* chunk_table, int chunk_idx, int chunk, int transpose,
+                          uint16_t* out, void* stream);
+
 /* Selects the GEMM inside oft_linear_fwd / oft_linear_bwd and
  * oft_linear_fwd_weight_side (test and benchmarking hook; process-wide, not
  * thread-safe against concurrent calls): 0 = by problem size (default: from 2048
@@ -285,13 +304,17 @@ int oft_debug_bounded_wait(int timeout_us, void* stream);
  * the card for its KV cache, where cudaMalloc would fail), or a plugin
  * interface whose signature carries only inputs and outputs.
  *
- * Same result as oft_linear_fwd (same kernels, same launch sequence), but the
- * scratch (rotated activations and the bf16 copy of the weight) lives in a
+ * Same result as oft_linear_fwd given a workspace of OFT_NOALLOC_SCRATCH_BYTES
+ * (same kernels, same launch sequence), but the scratch (rotated activations and,
+ * from 2048 tokens when it fits too, the bf16 copy of the weight) lives in a
  * fixed file-scope device array of OFT_NOALLOC_SCRATCH_BYTES (32 MiB) that every
  * GPU loading this library holds until the process exits.  Allocates nothing:
  * no cudaMalloc/cudaFree and no allocating library call.
- *   - Shapes whose oft_linear_fwd_workspace() exceeds OFT_NOALLOC_SCRATCH_BYTES
- *     are rejected with OFT_ERR_WORKSPACE and a message giving both sizes.
+ *   - From 2048 tokens the bf16-weight path runs when X' (2 P M K bytes) and the
+ *     weight copy (2 N K bytes) both fit in the array, else the fused-decode path,
+ *     which needs X' only.
+ *   - Shapes whose X' alone exceeds OFT_NOALLOC_SCRATCH_BYTES are rejected with
+ *     OFT_ERR_WORKSPACE and a message giving both sizes.
  *   - The first call on a device (with that device current) looks up the
  *     array's device address; make that first call before any stream capture.
  *   - All calls share the one array and it keeps the last call's contents.

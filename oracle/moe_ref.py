@@ -13,6 +13,11 @@ readings taken here are:
   * top-k by logit, descending; ties go to the lower expert index; the slot
     order k is the rank;
   * gating weights are a softmax over the k selected logits (they sum to 1);
+  * non-finite logits (a diverging router): NaN ranks as -inf; where selected
+    values are infinite the weights are the softmax's limit -- if the largest
+    selected logit is +inf, the selected +inf entries share the weight equally
+    and the others get 0; if it is -inf (all k selected are -inf or NaN), each
+    gets 1/k;
   * each expert e has gate and up projections with independent OFT rotations
     (split-projection applied to the expert's fused gate/up tensor):
         Y_tk = [ (X_t R_e,gate) W_e,gate  |  (X_t R_e,up) W_e,up ]
@@ -61,12 +66,24 @@ from .oft_ref import cayley_grad, packed_len, rotate, rotate_t, rotations
 
 
 def topk(logits: np.ndarray, k: int):
-    """logits fp32 [T][E] -> (idx int32 [T][k], w float64 [T][k])."""
+    """logits fp32 [T][E] -> (idx int32 [T][k], w float64 [T][k]).
+
+    NaN ranks as -inf; the weights follow the limits stated in the module
+    docstring when a selected logit is infinite."""
     logits = np.asarray(logits, dtype=np.float32)
-    order = np.argsort(-logits, axis=1, kind="stable")[:, :k]
-    sel = np.take_along_axis(logits, order, axis=1).astype(np.float64)
-    z = np.exp(sel - sel.max(axis=1, keepdims=True))
-    return order.astype(np.int32), z / z.sum(axis=1, keepdims=True)
+    v = np.where(np.isnan(logits), np.float32(-np.inf), logits)
+    order = np.argsort(-v, axis=1, kind="stable")[:, :k]
+    sel = np.take_along_axis(v, order, axis=1).astype(np.float64)
+    mx = sel.max(axis=1)
+    w = np.empty_like(sel)
+    fin = np.isfinite(mx)
+    z = np.exp(sel[fin] - mx[fin, None])
+    w[fin] = z / z.sum(axis=1, keepdims=True)
+    top = mx == np.inf
+    hit = (sel[top] == np.inf).astype(np.float64)
+    w[top] = hit / hit.sum(axis=1, keepdims=True)
+    w[mx == -np.inf] = 1.0 / k
+    return order.astype(np.int32), w
 
 
 def buckets(idx: np.ndarray, E: int):

@@ -27,6 +27,7 @@ from .binding import (  # noqa: F401
     oft_linear_fwd_weight_side,
     oft_linear_fwd_weight_side_workspace,
     oft_linear_fwd_workspace,
+    oft_moe_chunk_dequant,
     oft_rotate,
     oft_set_gemm_mode,
     profile,

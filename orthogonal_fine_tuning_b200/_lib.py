@@ -28,7 +28,7 @@ EXPORTS = (
     "oft_linear_fwd_noalloc", "oft_set_gemm_mode", "moe_fused_oft_workspace", "moe_fused_oft_fwd",
     "moe_chunked_oft_bwd_workspace", "moe_chunked_oft_bwd", "moe_chunked_oft_layer_workspace",
     "moe_chunked_oft_layer_fwd", "oft_linear_fwd_weight_side_workspace", "oft_linear_fwd_weight_side",
-    "oft_gemm_schedule",
+    "oft_gemm_schedule", "oft_moe_chunk_dequant",
 )
 
 
@@ -68,6 +68,7 @@ _SIGS = {
     "moe_chunked_oft_layer_workspace": (_Z, [_I, _I, _I, _I, _WP, _WP, _I]),
     "moe_chunked_oft_layer_fwd": (_I, [_P, _I, _P, _I, _I, _I, _WP, _WP, _I, _P, _P, _P, _P, _Z, _P]),
     "oft_dequant_weight": (_I, [_WP, _P, _I, _P]),
+    "oft_moe_chunk_dequant": (_I, [_WP, _P, _I, _I, _I, _P, _P]),
     "oft_rotate": (_I, [_P, _I, _I, _I, _I, _P, _P, _P]),
     "oft_cayley_backward": (_I, [_P, _P, _I, _I, _P, _P]),
     "oft_debug_bounded_wait": (_I, [_I, _P]),
@@ -85,7 +86,7 @@ KERNEL_CLASSES = ("gemm", "rotate", "dequant", "cayley", "grad", "route")
 def load(path: str = LIB_PATH) -> ctypes.CDLL:
     if not os.path.exists(path):
         raise ImportError(
-            f"{path} is missing: build it with `python -m orthogonal_fine_tuning_b200.build` "
+            f"{path} is missing: build it with `python orthogonal_fine_tuning_b200/build.py` "
             "(the OFT path has no CPU fallback)")
     lib = ctypes.CDLL(path)
     for name, (res, args) in _SIGS.items():

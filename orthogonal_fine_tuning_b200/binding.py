@@ -290,6 +290,20 @@ def oft_dequant_weight(W: Weight, transpose: bool = False, out: Optional[torch.T
     return out
 
 
+def oft_moe_chunk_dequant(W: Weight, chunk_table: torch.Tensor, chunk_idx: int, chunk: int,
+                          transpose: bool = False, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """One chunk of the MoE transient dequant: bf16 [chunk][N][K], or with transpose
+    [chunk][2][K][N/2].  Slots whose table entry is -1 are left as they were."""
+    N, K = W.d_out, W.d_in
+    if out is None:
+        shape = (chunk, 2, K, N // 2) if transpose else (chunk, N, K)
+        out = torch.zeros(*shape, dtype=torch.bfloat16, device=W.codes.device)
+    cw = W.c()
+    _check(_L.oft_moe_chunk_dequant(ctypes.byref(cw), _ptr(chunk_table), int(chunk_idx), int(chunk),
+                                    int(bool(transpose)), _ptr(out), _stream(stream)))
+    return out
+
+
 def oft_rotate(X: torch.Tensor, R: torch.Tensor, b: int, out: Optional[torch.Tensor] = None,
                stream=None) -> torch.Tensor:
     """X bf16 [M][K], R fp32 [P][K/b][b][b] -> X R_p, bf16 [P][M][K]."""

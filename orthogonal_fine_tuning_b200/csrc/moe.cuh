@@ -20,6 +20,13 @@ constexpr int kMaxTopK = 8;
 
 // One warp per token: top_k by (logit desc, expert id asc), then softmax over
 // the selected logits (fp32).
+//
+// Non-finite logits (a diverging router): NaN ranks as -inf.  Only lanes holding a
+// real expert (e < E) are ever candidates and k <= E, so every emitted index is in
+// [0, E) whatever the logits hold.  The weights are the softmax's limit where the
+// selected values are infinite: if the largest is +inf, the +inf entries share the
+// weight equally and the rest get 0; if it is -inf (every selected logit is -inf or
+// NaN), each of the k gets 1/k.
 __global__ void __launch_bounds__(256) moe_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
                                                        int* __restrict__ idx_out, float* __restrict__ w_out) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) / 32;
@@ -32,7 +39,8 @@ __global__ void __launch_bounds__(256) moe_topk_kernel(const float* __restrict__
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     const int e = lane + 32 * i;
-    v[i] = e < E ? row[e] : -INFINITY;
+    const float x = e < E ? row[e] : -INFINITY;
+    v[i] = isnan(x) ? -INFINITY : x;
     if (e >= E) taken |= 1u << i;
   }
   float sel_v[kMaxTopK];
@@ -57,6 +65,8 @@ __global__ void __launch_bounds__(256) moe_topk_kernel(const float* __restrict__
         be = oe;
       }
     }
+    // some lane with e < E is still free (k <= E), and it beats the (-inf, INT_MAX)
+    // placeholder of lanes without a candidate, so be < E here
     if ((be & 31) == lane) taken |= 1u << (be >> 5);
     sel_v[s] = bv;
     sel_e[s] = be;
@@ -66,7 +76,12 @@ __global__ void __launch_bounds__(256) moe_topk_kernel(const float* __restrict__
     float ex[kMaxTopK];
     float sum = 0.f;
     for (int s = 0; s < k; ++s) {
-      ex[s] = expf(sel_v[s] - mx);
+      if (mx == INFINITY)
+        ex[s] = sel_v[s] == INFINITY ? 1.f : 0.f;
+      else if (mx == -INFINITY)
+        ex[s] = 1.f;
+      else
+        ex[s] = expf(sel_v[s] - mx);
       sum += ex[s];
     }
     for (int s = 0; s < k; ++s) {

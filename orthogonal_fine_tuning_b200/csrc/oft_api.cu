@@ -93,18 +93,25 @@ inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // Per-device side stream and events for the MoE chunk pipeline (dequant of chunk
 // c + 1 overlaps the grouped GEMM of chunk c).  Created on first use, kept until
 // exit; they hold no device memory.
+// The events are shared by every call on the device, so a call holds the pipe's lock
+// from its first record to its last wait (host-side enqueue only): two host threads
+// then never interleave their records and waits on the same event.
 struct SidePipe {
   bool ready = false;
   cudaStream_t side = nullptr;
   cudaEvent_t start = nullptr, dq_done[2] = {nullptr, nullptr}, gemm_done[2] = {nullptr, nullptr};
+  std::mutex mu;
 };
 SidePipe g_side[64];
+std::mutex g_side_create_mu;
 
-int side_pipe(SidePipe** out) {
+// On success *out is the device's pipe and *lock holds its mutex.
+int side_pipe(SidePipe** out, std::unique_lock<std::mutex>* lock) {
   int dev = 0;
   OFT_CUDA(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64) return fail(OFT_ERR_UNSUPPORTED, "device index %d out of range", dev);
   SidePipe& sp = g_side[dev];
+  std::lock_guard<std::mutex> create(g_side_create_mu);
   if (!sp.ready) {
     OFT_CUDA(cudaStreamCreateWithFlags(&sp.side, cudaStreamNonBlocking));
     OFT_CUDA(cudaEventCreateWithFlags(&sp.start, cudaEventDisableTiming));
@@ -114,6 +121,7 @@ int side_pipe(SidePipe** out) {
     }
     sp.ready = true;
   }
+  *lock = std::unique_lock<std::mutex>(sp.mu);
   *out = &sp;
   return OFT_OK;
 }
@@ -940,11 +948,12 @@ int oft_linear_fwd(const uint16_t* X, int M, const oft_weight* W, const oft_spli
   uint16_t* Xr = reinterpret_cast<uint16_t*>(wsb + L.xr);
 
   SidePipe* sp = nullptr;
+  std::unique_lock<std::mutex> sp_lock;
   if (plain) {
     // deq(W) -> bf16 [N][K] on the side stream, alongside the rotation on this one: the two
     // read only inputs and write disjoint workspace regions, and the small dequant CTAs fit
     // next to the rotation's on the same SMs
-    if (int rc = side_pipe(&sp)) return rc;
+    if (int rc = side_pipe(&sp, &sp_lock)) return rc;
     OFT_CUDA(cudaEventRecord(sp->start, st));
     OFT_CUDA(cudaStreamWaitEvent(sp->side, sp->start, 0));
     if (int rc = launch_dequant(view_of(W), reinterpret_cast<uint16_t*>(wsb + L.wdq), false, sp->side)) return rc;
@@ -1367,7 +1376,8 @@ int moe_oft_fwd_impl(bool fused, const uint16_t* X, int T, const float* logits, 
   // GEMM of chunk c - 1 runs on the caller's stream; the dequant of chunk c waits
   // for the GEMM of chunk c - 2 (the last reader of its buffer).
   SidePipe* sp = nullptr;
-  if (int rc = side_pipe(&sp)) return rc;
+  std::unique_lock<std::mutex> sp_lock;
+  if (int rc = side_pipe(&sp, &sp_lock)) return rc;
   OFT_CUDA(cudaEventRecord(sp->start, st));
   OFT_CUDA(cudaStreamWaitEvent(sp->side, sp->start, 0));
   const size_t buf_elems = 1ull * chunk * N * K;
@@ -1523,7 +1533,8 @@ int moe_chunked_oft_layer_fwd(const uint16_t* X, int T, const float* logits, int
   OFT_CUDA(cudaFuncSetAttribute(moe_chunk_dequant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 static_cast<int>(dq_smem)));
   SidePipe* sp = nullptr;
-  if (int rc = side_pipe(&sp)) return rc;
+  std::unique_lock<std::mutex> sp_lock;
+  if (int rc = side_pipe(&sp, &sp_lock)) return rc;
   OFT_CUDA(cudaEventRecord(sp->start, st));
   OFT_CUDA(cudaStreamWaitEvent(sp->side, sp->start, 0));
   const size_t buf_elems = 1ull * chunk * K * n;
@@ -1691,7 +1702,8 @@ int moe_chunked_oft_bwd(const uint16_t* dY, const uint16_t* X, int T, const floa
   prm.moe.mode = gemm::kMoeBwd;
   const WeightView bank = view_of(W);
   SidePipe* sp = nullptr;
-  if (int rc = side_pipe(&sp)) return rc;
+  std::unique_lock<std::mutex> sp_lock;
+  if (int rc = side_pipe(&sp, &sp_lock)) return rc;
   OFT_CUDA(cudaEventRecord(sp->start, st));
   OFT_CUDA(cudaStreamWaitEvent(sp->side, sp->start, 0));
   const size_t buf_elems = 1ull * chunk * N * K;
@@ -1740,6 +1752,38 @@ int moe_chunked_oft_bwd(const uint16_t* dY, const uint16_t* X, int T, const floa
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// test hook: one chunk of the MoE transient dequant, as the MoE calls run it
+// ---------------------------------------------------------------------------
+extern "C" int oft_moe_chunk_dequant(const oft_weight* bank, const int32_t* chunk_table, int chunk_idx, int chunk,
+                                     int transpose, uint16_t* out, void* stream) {
+  if (int rc = check_weight(bank, true)) return rc;
+  if (bank->fmt != OFT_W_INT4) return fail(OFT_ERR_UNSUPPORTED, "the MoE expert bank must be INT4");
+  if (chunk < 1 || chunk > gemm::MAX_GROUPS / 2) return fail(OFT_ERR_UNSUPPORTED, "chunk must be 1..%d", gemm::MAX_GROUPS / 2);
+  if (chunk_idx < 0) return fail(OFT_ERR_INVALID_ARG, "chunk_idx < 0");
+  if (!chunk_table || !out || !aligned16(chunk_table) || !aligned16(out))
+    return fail(OFT_ERR_INVALID_ARG, "NULL or misaligned pointer");
+  const int K = bank->d_in, N = bank->d_out;
+  const WeightView v = view_of(bank);
+  cudaStream_t st = as_stream(stream);
+  ProfScope ps(OFT_K_DEQUANT, st);
+  if (!transpose) {
+    const size_t dq_smem = sizeof(uint16_t) * kChunkRows * chunk_scale_ld(K / bank->group);
+    if (dq_smem > 227 * 1024) return fail(OFT_ERR_UNSUPPORTED, "d_in / group too large for the chunk dequant");
+    OFT_CUDA(cudaFuncSetAttribute(moe_chunk_dequant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(dq_smem)));
+    moe_chunk_dequant_kernel<<<dim3((N + kChunkRows - 1) / kChunkRows, chunk), 256, dq_smem, st>>>(v, chunk_table,
+                                                                                                  chunk_idx, chunk, out);
+    OFT_LAUNCHED("moe_chunk_dequant_kernel");
+  } else {
+    if (N % 16 != 0) return fail(OFT_ERR_UNSUPPORTED, "the transposed chunk needs d_out (gate+up) % 16 == 0");
+    moe_chunk_dequant_t_kernel<<<dim3((K + 64 * kDqtStrip - 1) / (64 * kDqtStrip), (N + 63) / 64, chunk), 256, 0, st>>>(
+        v, chunk_table, chunk_idx, chunk, N / 2, out);
+    OFT_LAUNCHED("moe_chunk_dequant_t_kernel");
+  }
+  return OFT_OK;
+}
 
 // ---------------------------------------------------------------------------
 // bounded-wait self test
@@ -1839,7 +1883,10 @@ extern "C" int oft_linear_fwd_noalloc(const uint16_t* X, int M, const oft_weight
   if (int rc = check_b(b, W->d_in)) return rc;
   if (M < 0) return fail(OFT_ERR_INVALID_ARG, "M < 0");
   if (M == 0) return OFT_OK;
-  const size_t need = oft_linear_fwd_workspace(M, W, S, b);
+  // oft_linear_fwd takes the bf16-weight path only when its workspace also holds the
+  // weight copy, and the fused-decode path otherwise; the smaller (fused) layout is
+  // what must fit
+  const size_t need = fwd_layout(M, W->d_in, W->d_out, S->n, false).total;
   if (need > OFT_NOALLOC_SCRATCH_BYTES)
     return fail(OFT_ERR_WORKSPACE,
                 "oft_linear_fwd_noalloc: this shape needs %zu bytes of scratch, more than the fixed %u-byte "

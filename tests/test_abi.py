@@ -118,6 +118,20 @@ def test_moe_argument_checks(lib):
     assert call(w=_w(lib, fmt=2, d_in=256, d_out=64, n=16)) == L.OFT_ERR_UNSUPPORTED
 
 
+def test_chunk_dequant_hook_checks(lib):
+    """oft_moe_chunk_dequant rejects bad arguments on the host, before any launch."""
+    from orthogonal_fine_tuning_b200 import _lib as L
+    w = _w(lib, d_in=256, d_out=64, group=32, n=16)
+    assert lib.oft_moe_chunk_dequant(ctypes.byref(w), 0, 0, 4, 0, 0x20000, None) == L.OFT_ERR_INVALID_ARG
+    assert lib.oft_moe_chunk_dequant(ctypes.byref(w), 0x10000, 0, 4, 0, 0x20008, None) == L.OFT_ERR_INVALID_ARG
+    assert lib.oft_moe_chunk_dequant(ctypes.byref(w), 0x10000, -1, 4, 0, 0x20000, None) == L.OFT_ERR_INVALID_ARG
+    assert lib.oft_moe_chunk_dequant(ctypes.byref(w), 0x10000, 0, 17, 0, 0x20000, None) == L.OFT_ERR_UNSUPPORTED
+    fp8 = _w(lib, fmt=2, d_in=256, d_out=64, n=16)
+    assert lib.oft_moe_chunk_dequant(ctypes.byref(fp8), 0x10000, 0, 4, 0, 0x20000, None) == L.OFT_ERR_UNSUPPORTED
+    odd = _w(lib, d_in=256, d_out=40, group=32, n=16)
+    assert lib.oft_moe_chunk_dequant(ctypes.byref(odd), 0x10000, 0, 4, 1, 0x20000, None) == L.OFT_ERR_UNSUPPORTED
+
+
 def test_rotation_and_debug_checks(lib):
     from orthogonal_fine_tuning_b200 import _lib as L
     assert lib.oft_build_rotation(0x1000, 4, 24, 0x2000, None) == L.OFT_ERR_UNSUPPORTED

@@ -76,6 +76,36 @@ def test_ties_in_logits_go_to_lower_expert(oft):
     _check_routing(out, raw(case["logits"]), spec)
 
 
+def test_non_finite_logits(oft, fused):
+    """A diverging router: rows of NaN, -inf and +inf logits.  NaN ranks as -inf, so
+    every index stays a real expert; routing is bit-exact with the oracle, the weights
+    follow the softmax's limits, and Y stays within tolerance."""
+    spec = MoESpec("nf", T=96, K=128, E=12, n_proj=32, top_k=4, chunk=3, group=32, b=32, q_sigma=0.05, seed=11)
+    case = make_moe_case(spec)
+    g = torch.Generator().manual_seed(5)
+    lg = torch.randn(spec.T, spec.E, generator=g)
+    u = torch.rand(spec.T, spec.E, generator=g)
+    lg[u < 0.25] = float("nan")
+    lg[(u >= 0.25) & (u < 0.35)] = float("-inf")
+    lg[(u >= 0.35) & (u < 0.40)] = float("inf")
+    lg[0] = float("nan")
+    lg[1] = float("-inf")
+    lg[2, :] = float("nan")
+    lg[2, 7] = 0.5
+    case["logits"] = lg
+    out = _run(oft, _to(case, "cuda"), fused)
+    idx = _check_routing(out, raw(case["logits"]), spec)
+    assert idx.min() >= 0 and idx.max() < spec.E
+    _, w = moe_ref.topk(raw(case["logits"]), spec.top_k)
+    assert np.array_equal(out["topk_w"].cpu().numpy()[:2], w[:2].astype(np.float32))
+    bank = moe_ref.ExpertBank(raw(case["codes"]), raw(case["scales"]), spec.K, spec.group, spec.n_proj)
+    Yref, _ = moe_ref.moe_fwd_chunked(raw(case["X"]), raw(case["logits"]), bank, raw(case["Q"]), spec.b, spec.top_k,
+                                      spec.chunk, spec.E)
+    Y = f64(out["Y"])
+    assert np.all(np.isfinite(Y))
+    assert rel_err(Y, Yref) < TOL
+
+
 def test_c3_full_routing_and_sampled_output(oft, fused):
     """Kimi-like expert layer: 4096 tokens, hidden 7168, 384 INT4-g32 experts of
     2 x 2048, top-8 over Zipf-biased logits, chunks of 16, b=32."""

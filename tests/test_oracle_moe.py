@@ -26,6 +26,47 @@ def test_topk_matches_brute_force_with_ties():
     np.testing.assert_allclose(w.sum(axis=1), 1.0, rtol=1e-15)
 
 
+def test_topk_non_finite_logits():
+    """A diverging router: NaN ranks as -inf (ties to the lower id), every index is a
+    real expert, and the weights are the softmax's limits: +inf entries share the
+    weight, an all -inf / NaN selection is uniform."""
+    nan, inf = np.float32(np.nan), np.float32(np.inf)
+    rng = np.random.default_rng(4)
+    E, k = 9, 4
+    rows = [
+        [nan] * E,                                             # all NaN
+        [-inf] * E,                                            # all -inf
+        [nan, -inf, 0.5, nan, -inf, nan, nan, nan, nan],       # one finite value
+        [nan, 1.0, inf, 2.0, inf, nan, -inf, 0.0, 3.0],        # two +inf
+        [-1.0, nan, -2.0, -3.0, -inf, nan, -0.5, nan, -inf],   # finite values mixed with NaN and -inf
+        [nan, nan, 2.0, 2.0, nan, 2.0, -inf, 2.0, 2.0],        # ties among finite values
+    ]
+    rows += [list(np.where(rng.random(E) < 0.3, nan, rng.integers(-2, 3, E)).astype(np.float32))
+             for _ in range(40)]
+    logits = np.array(rows, dtype=np.float32)
+    idx, w = moe_ref.topk(logits, k)
+    for t in range(len(rows)):
+        key = [(-np.inf if np.isnan(x) else float(x)) for x in logits[t]]
+        ref = sorted(range(E), key=lambda e: (-key[e], e))[:k]
+        assert list(idx[t]) == ref
+        assert np.all((idx[t] >= 0) & (idx[t] < E))
+        sel = np.array([key[e] for e in ref])
+        if sel.max() == np.inf:
+            want = (sel == np.inf) / np.sum(sel == np.inf)
+        elif sel.max() == -np.inf:
+            want = np.full(k, 1.0 / k)
+        else:
+            z = np.exp(sel - sel.max())
+            want = z / z.sum()
+        np.testing.assert_allclose(w[t], want, rtol=1e-15, atol=0)
+        assert abs(w[t].sum() - 1.0) < 1e-15 and np.all(np.isfinite(w[t]))
+    # closed forms of the special rows
+    assert list(idx[0]) == [0, 1, 2, 3] and np.all(w[0] == 0.25)
+    assert list(idx[1]) == [0, 1, 2, 3] and np.all(w[1] == 0.25)
+    assert list(idx[2]) == [2, 0, 1, 3] and list(w[2]) == [1.0, 0.0, 0.0, 0.0]
+    assert list(idx[3]) == [2, 4, 8, 3] and list(w[3]) == [0.5, 0.5, 0.0, 0.0]
+
+
 def test_buckets_match_dictionary_build():
     rng = np.random.default_rng(1)
     T, k, E = 300, 4, 17

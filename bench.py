@@ -709,7 +709,9 @@ def run_ours(args, rank, world, name):
         peak = peaks["hbm_gbs"]
         unit = "GB/s"
         traffic = None
-        kernel = "gemm_dq_kernel (fused dequant, tcgen05/TMEM), weight-stream bound at this M"
+        kernel = ("gemm_sm_kernel (small-M split-K fused dequant: TMA-staged codes, 16 decode warps into a "
+                  "TMEM operand ring, tcgen05), weight-stream bound at this M" if args.gemm_mode in (0, 5) else
+                  "gemm_dq_kernel (fused dequant, tcgen05/TMEM), weight-stream bound at this M")
     else:
         gemm_flops = flops["gemm_fwd"] + flops.get("gemm_bwd", 0.0)
         per_launch = gemm_flops / (g_launch / args.steps)
@@ -838,7 +840,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="c4", choices=sorted(WORKLOAD_NAMES),
                     help="the headline workload (default: the MXFP4 training step, the largest that fits one GPU)")
-    ap.add_argument("--also", default="c0,c1,c2,c3",
+    ap.add_argument("--also", default="c0,c1,c2,c3,c1-m64,c4-m64",
                     help="comma-separated workloads timed after the headline one on a single GPU and reported "
                          "under 'workloads' in the same line ('' for none)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -846,8 +848,9 @@ def main(argv=None):
     ap.add_argument("--moe-backward", action="store_true",
                     help="MoE workload: time forward + adapter backward (chunked path)")
     ap.add_argument("--gemm-mode", type=int, default=0, choices=[0, 1, 2, 3, 4],
-                    help="GEMM path of the dense workloads (oft_set_gemm_mode): 0 by size, 1 one-CTA fused, "
-                         "2 2-SM pair fused, 3 bf16 copy + plain pair GEMM, 4 bf16 copy + plain one-CTA GEMM")
+                    help="GEMM path of the dense workloads (oft_set_gemm_mode): 0 by size (the small-M split-K "
+                         "kernel up to 128 tokens), 1 one-CTA fused, 2 2-SM pair fused, 3 bf16 copy + plain pair "
+                         "GEMM, 4 bf16 copy + plain one-CTA GEMM")
     ap.add_argument("--weight-side", action="store_true",
                     help="dense workloads: the weight-side rotation variant of the forward")
     ap.add_argument("--moe-layer", action="store_true",

@@ -269,9 +269,10 @@ int oft_moe_chunk_dequant(const oft_weight* bank, const int32_t* chunk_table, in
  * thread-safe against concurrent calls): 0 = by problem size (default: from 2048
  * tokens, deq(W) to a bf16 workspace and the plain tcgen05 GEMM on 2-SM pairs; below
  * that the fused-decode kernels, the 2-SM pair kernel for launches of at least two
- * waves of one-CTA tiles), 1 = always the one-CTA fused kernel, 2 = always the 2-SM
- * pair fused kernel, 3 = always the bf16 copy and the plain pair GEMM, 4 = always the
- * bf16 copy and the plain one-CTA GEMM.  The weight-side forward always takes the
+ * waves of one-CTA tiles, and for forwards of 1 to 128 tokens the small-M split-K
+ * kernel), 1 = always the one-CTA fused kernel, 2 = always the 2-SM pair fused
+ * kernel, 3 = always the bf16 copy and the plain pair GEMM, 4 = always the bf16 copy
+ * and the plain one-CTA GEMM.  The weight-side forward always takes the
  * plain GEMM: the pair kernel unless the mode is 4.  All compute the same product.  Query the *_workspace
  * sizes after setting the mode.  Returns OFT_ERR_INVALID_ARG for any other value. */
 int oft_set_gemm_mode(int mode);

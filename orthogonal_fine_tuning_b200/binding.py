@@ -327,7 +327,8 @@ def oft_cayley_backward(R: torch.Tensor, G: torch.Tensor, b: int, out: Optional[
 def oft_set_gemm_mode(mode: int) -> None:
     """GEMM inside the linear calls: 0 by size (default), 1 the one-CTA fused-dequant
     kernel, 2 the 2-SM pair fused-dequant kernel, 3 the bf16 weight copy and the plain
-    GEMM on 2-SM pairs, 4 the same on one CTA per tile (same product)."""
+    GEMM on 2-SM pairs, 4 the same on one CTA per tile (same product).  Mode 0 runs
+    forwards of up to 128 tokens on the small-M split-K kernel."""
     _check(_L.oft_set_gemm_mode(int(mode)))
 
 

@@ -93,6 +93,37 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// mbar_wait for waits that may last long (a producer ahead of its consumer, decode warps
+// ahead of their code tiles): each retry suspends the thread in try_wait for up to
+// `hint_ns` or until the phase completes, so waiting warps do not take issue slots from
+// the warps that are working.  Same bound and abort behaviour as mbar_wait.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint32_t addr, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(addr), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, volatile int* abort, unsigned err_bit,
+                                                uint32_t hint_ns = 20000u) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait(a, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait_hint(a, parity, hint_ns)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+      *abort = 1;
+      atomicOr(&g_dev_err, err_bit);
+      return false;
+    }
+  }
+}
+
 // Waits for a phase ignoring the abort flag (teardown drain of in-flight copies
 // and MMAs); bounded by 200 ms, after which it records kErrWaitDrain.
 __device__ __forceinline__ bool gemm_drain_wait(uint64_t* bar, uint32_t parity) {

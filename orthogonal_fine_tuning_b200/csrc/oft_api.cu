@@ -9,6 +9,7 @@
 #include <cstdio>
 #include <cstring>
 #include <algorithm>
+#include <memory>
 #include <mutex>
 #include <queue>
 #include <vector>
@@ -25,6 +26,7 @@
 #include "rot_tc.cuh"
 #include "gemm_dq.cuh"
 #include "gemm_dq2.cuh"
+#include "gemm_sm.cuh"
 #include "moe_fused.cuh"
 #include "moe_bwd.cuh"
 #include "moe_layer.cuh"
@@ -370,10 +372,12 @@ int set_smem(KernelT kernel, size_t bytes) {
 
 // X'_p = X R_p on the tensor cores (all P sub-projections in one pass).
 int launch_rotate_fwd(const uint16_t* X, int M, int K, int P, int b, const float* R, uint16_t* Xr, cudaStream_t st,
-                      bool transpose = false) {
+                      bool transpose = false, int* zero_ptr = nullptr, int zero_n = 0) {
   rtc::FwdParams prm;
   memset(&prm, 0, sizeof(prm));
   prm.transpose = transpose ? 1 : 0;
+  prm.zero_ptr = zero_ptr;
+  prm.zero_n = zero_ptr != nullptr ? zero_n : 0;
   if (int rc = make_map_bf16(&prm.tmX, X, K, M, K, rtc::TM)) return rc;
   if (int rc = make_map_bf16_3d_store(&prm.tmY, Xr, K, M, P)) return rc;
   prm.R = R;
@@ -753,15 +757,63 @@ bool use_plain(int M) {
   return M >= kPlainMinTokens;
 }
 
-struct FwdLayout {
-  size_t xr, wdq, total;
+// The small-M path (few tokens against the whole weight, gsm::gemm_sm_kernel): forwards
+// of 1 to 128 tokens in gemm mode 0.  Its e8m0 scale rows must be 16-byte strided.
+constexpr int kSmallMaxTokens = gsm::MAX_TOKENS;
+bool use_small(int M, int fmt, int N) {
+  if (g_gemm_mode != 0) return false;
+  if (M < 1 || M > kSmallMaxTokens) return false;
+  return fmt != OFT_W_MXFP4 || N % 16 == 0;
+}
+
+// Split-K plan of the small-M kernel: 128-row weight tiles x `splits` reduction ranges,
+// with the split count that minimises waves / splits over the SMs (ties to fewer splits).
+struct SmallPlan {
+  int tiles, splits, nkb, MN;
+  size_t part_bytes, cnt_bytes;
 };
-FwdLayout fwd_layout(int M, int K, int N, int P, bool plain) {
+SmallPlan small_plan(int M, int K, int fmt, const oft_split* S) {
+  SmallPlan pl{};
+  pl.MN = (M + 15) / 16 * 16;
+  const int kbe = fmt == OFT_W_FP8 ? 128 : 256;
+  pl.nkb = (K + kbe - 1) / kbe;
+  for (int p = 0; p < S->n; ++p) pl.tiles += (S->sizes[p] + gsm::WM - 1) / gsm::WM;
+  const int sms = sm_count();
+  double best = 1e30;
+  pl.splits = 1;
+  for (int sp = 1; sp <= std::min(gsm::MAX_SPLITS, pl.nkb); ++sp) {
+    const double waves = static_cast<double>((1ll * pl.tiles * sp + sms - 1) / sms) / sp;
+    if (waves < best - 1e-9) {
+      best = waves;
+      pl.splits = sp;
+    }
+  }
+  pl.cnt_bytes = pl.splits > 1 ? round_up(4ull * pl.tiles, 256) : 0;
+  pl.part_bytes = pl.splits > 1 ? 4ull * pl.tiles * pl.splits * pl.MN * gsm::WM : 0;
+  return pl;
+}
+
+struct FwdLayout {
+  size_t xr, wdq, cnt, part, total;
+};
+// plain: the bf16 weight copy follows X'; small_extra: the small-M kernel's split-K
+// counters and partial tiles follow X' instead
+FwdLayout fwd_layout(int M, int K, int N, int P, bool plain, size_t cnt_bytes = 0, size_t part_bytes = 0) {
   FwdLayout L{};
   L.xr = 0;
   L.wdq = round_up(L.xr + 2ull * P * M * K, 256);
-  L.total = round_up(L.wdq + (plain ? 2ull * N * K : 0ull), 256);
+  L.cnt = L.wdq;
+  L.part = round_up(L.cnt + cnt_bytes, 256);
+  L.total = plain ? round_up(L.wdq + 2ull * N * K, 256) : round_up(L.part + part_bytes, 256);
   return L;
+}
+// The layout oft_linear_fwd uses when the plain (bf16 weight copy) path is not taken.
+FwdLayout fwd_layout_fused(int M, const oft_weight* W, const oft_split* S) {
+  if (use_small(M, W->fmt, W->d_out)) {
+    const SmallPlan pl = small_plan(M, W->d_in, W->fmt, S);
+    return fwd_layout(M, W->d_in, W->d_out, S->n, false, pl.cnt_bytes, pl.part_bytes);
+  }
+  return fwd_layout(M, W->d_in, W->d_out, S->n, false);
 }
 
 
@@ -790,6 +842,88 @@ BwdLayout bwd_layout(int M, int K, int N, const oft_split* S, int b, int fmt, bo
   const size_t sbytes = fmt == OFT_W_MXFP4 ? 2ull * (K / 32) * N : 0ull;
   L.total = round_up(L.factors + sbytes, 256);
   return L;
+}
+
+// Tensor maps and launch of the small-M kernel (one CTA per SM, persistent over the
+// tiles x splits units).
+template <int FMT>
+int launch_gemm_small_t(const gsm::Params& prm, int grid, size_t smem, cudaStream_t st) {
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    OFT_CUDA(cudaFuncSetAttribute(gsm::gemm_sm_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(227 * 1024)));
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
+  ProfScope ps(OFT_K_GEMM, st);
+  OFT_CUDA(launch_pdl(gsm::gemm_sm_kernel<FMT>, grid, gsm::NUM_THREADS, smem, st, prm));
+  OFT_LAUNCHED("gemm_sm_kernel");
+  return OFT_OK;
+}
+
+int launch_gemm_small(const oft_weight* W, const oft_split* S, int M, const uint16_t* Xr, uint16_t* Y,
+                      const SmallPlan& pl, int* counters, float* part, cudaStream_t st) {
+  const int K = W->d_in, N = W->d_out, P = S->n;
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return fail(OFT_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  gsm::Params* prm = new gsm::Params;  // large (three tensor maps + groups): off the stack
+  std::unique_ptr<gsm::Params> own(prm);
+  memset(prm, 0, sizeof(*prm));
+  {
+    // codes: [N][row bytes] uint8, 128 x 128-byte boxes with the 128-byte swizzle
+    const uint64_t row_bytes = W->fmt == OFT_W_FP8 ? 1ull * K : 1ull * K / 2;
+    cuuint64_t dims[2] = {row_bytes, static_cast<cuuint64_t>(N)};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {128, gsm::WM};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(&prm->tmC, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(W->codes), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(OFT_ERR_CUDA, "cuTensorMapEncodeTiled (codes) failed (%d)", int(r));
+  }
+  if (W->fmt == OFT_W_INT4) {
+    if (int rc = make_map_plain_2d(&prm->tmS, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W->scales, N, K / W->group, 2ull * N,
+                                   gsm::WM, 256 / W->group))
+      return rc;
+  } else if (W->fmt == OFT_W_MXFP4) {
+    // e8m0 rows: the box starts at the 16-byte boundary at or below the tile's first column
+    if (int rc = make_map_plain_2d(&prm->tmS, CU_TENSOR_MAP_DATA_TYPE_UINT8, W->scales, N, K / 32, 1ull * N, 144, 8))
+      return rc;
+  }
+  if (int rc = make_map_bf16(&prm->tmX, Xr, K, 1ull * P * M, K, pl.MN)) return rc;
+  prm->fp8_scales = W->fmt == OFT_W_FP8 ? static_cast<const float*>(W->scales) : nullptr;
+  prm->Y = Y;
+  prm->part = part;
+  prm->counters = counters;
+  prm->M = M;
+  prm->MN = pl.MN;
+  prm->K = K;
+  prm->N = N;
+  prm->group = W->fmt == OFT_W_INT4 ? W->group : 32;
+  prm->splits = pl.splits;
+  prm->nkb = pl.nkb;
+  prm->total_tiles = pl.tiles;
+  prm->units = pl.tiles * pl.splits;
+  const size_t base = gsm::smem_bytes(pl.MN, 0);
+  prm->sx = static_cast<int>(std::min<size_t>(gsm::MAX_SX, (227ull * 1024 - base) / (pl.MN * 128ull)));
+  prm->num_groups = P;
+  int off = 0, tile0 = 0;
+  for (int p = 0; p < P; ++p) {
+    gsm::Group& g = prm->groups[p];
+    g.rows = S->sizes[p];
+    g.w_row0 = off;
+    g.b_row0 = p * M;
+    g.tiles = (S->sizes[p] + gsm::WM - 1) / gsm::WM;
+    g.tile0 = tile0;
+    tile0 += g.tiles;
+    off += S->sizes[p];
+  }
+  const size_t smem = gsm::smem_bytes(pl.MN, prm->sx);
+  const int grid = std::min(prm->units, sm_count());
+  if (W->fmt == OFT_W_INT4) return launch_gemm_small_t<gsm::kInt4>(*prm, grid, smem, st);
+  if (W->fmt == OFT_W_FP8) return launch_gemm_small_t<gsm::kFp8>(*prm, grid, smem, st);
+  return launch_gemm_small_t<gsm::kMxfp4>(*prm, grid, smem, st);
 }
 
 }  // namespace
@@ -923,9 +1057,9 @@ int oft_linear_fwd_weight_side(const uint16_t* X, int M, const oft_weight* W, co
 }
 
 size_t oft_linear_fwd_workspace(int M, const oft_weight* W, const oft_split* S, int b) {
-  if (W == nullptr || S == nullptr || M <= 0) return 0;
+  if (W == nullptr || S == nullptr || M <= 0 || S->n < 1 || S->n > 4) return 0;
   (void)b;
-  return fwd_layout(M, W->d_in, W->d_out, S->n, use_plain(M)).total;
+  return use_plain(M) ? fwd_layout(M, W->d_in, W->d_out, S->n, true).total : fwd_layout_fused(M, W, S).total;
 }
 
 int oft_linear_fwd(const uint16_t* X, int M, const oft_weight* W, const oft_split* S, int b, const float* R,
@@ -941,11 +1075,22 @@ int oft_linear_fwd(const uint16_t* X, int M, const oft_weight* W, const oft_spli
     return fail(OFT_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
   // the plain path when the token count calls for it and the workspace holds the bf16 weight
   const bool plain = use_plain(M) && ws_bytes >= fwd_layout(M, K, N, P, true).total;
-  const FwdLayout L = fwd_layout(M, K, N, P, plain);
+  const bool small = !plain && use_small(M, W->fmt, N);
+  const FwdLayout L = plain ? fwd_layout(M, K, N, P, true) : fwd_layout_fused(M, W, S);
   if (ws_bytes < L.total) return fail(OFT_ERR_WORKSPACE, "workspace %zu < %zu bytes", ws_bytes, L.total);
   cudaStream_t st = as_stream(stream);
   uint8_t* wsb = static_cast<uint8_t*>(ws);
   uint16_t* Xr = reinterpret_cast<uint16_t*>(wsb + L.xr);
+
+  if (small) {
+    // few tokens: the weight stream bounds the product (gsm::gemm_sm_kernel); the
+    // rotation kernel also clears the split-K counters of the tiles
+    const SmallPlan pl = small_plan(M, K, W->fmt, S);
+    int* counters = reinterpret_cast<int*>(wsb + L.cnt);
+    if (int rc = launch_rotate_fwd(X, M, K, P, b, R, Xr, st, false, pl.splits > 1 ? counters : nullptr, pl.tiles))
+      return rc;
+    return launch_gemm_small(W, S, M, Xr, Y, pl, counters, reinterpret_cast<float*>(wsb + L.part), st);
+  }
 
   SidePipe* sp = nullptr;
   std::unique_lock<std::mutex> sp_lock;
@@ -1886,7 +2031,7 @@ extern "C" int oft_linear_fwd_noalloc(const uint16_t* X, int M, const oft_weight
   // oft_linear_fwd takes the bf16-weight path only when its workspace also holds the
   // weight copy, and the fused-decode path otherwise; the smaller (fused) layout is
   // what must fit
-  const size_t need = fwd_layout(M, W->d_in, W->d_out, S->n, false).total;
+  const size_t need = fwd_layout_fused(M, W, S).total;
   if (need > OFT_NOALLOC_SCRATCH_BYTES)
     return fail(OFT_ERR_WORKSPACE,
                 "oft_linear_fwd_noalloc: this shape needs %zu bytes of scratch, more than the fixed %u-byte "

@@ -67,6 +67,8 @@ struct FwdParams {
   uint16_t* Xr;     // [P][M][K]
   int M, K, P, b, nb, groups, tiles_m;
   int transpose;    // 1: X'_p = X R_p^T (weight-side rotation of deq(W)^T rows)
+  int* zero_ptr;    // optional: zero_n ints CTA 0 clears for the kernel that follows (its split-K counters)
+  int zero_n;
 };
 
 constexpr int FWD_A_BYTES = TM * 64 * 2;           // 16 KB
@@ -171,6 +173,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) rot_fwd_tc_kernel(const __grid
   __syncthreads();
   tc_fence_after();
   pdl_wait();
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < p.zero_n; i += blockDim.x) p.zero_ptr[i] = 0;
   const uint32_t tmem = *tmem_slot;
   int ubeg, uend;
   unit_range(p.groups * p.tiles_m, ubeg, uend);

@@ -54,7 +54,8 @@ equals the direct per-token sum; weights sum to one; a router that sends every
 token to one expert with k = 1 reduces to the split-projection linear of
 oft_ref (forward and backward); central finite differences of the forward for
 dX, dq and the logits; dw equals the inner product of dY with the per-slot
-expert outputs; each token's logit gradient sums to zero.
+expert outputs; each token's logit gradient sums to zero; one expert's dq from
+its own entries (expert_dq) equals the full backward's.
 """
 
 from __future__ import annotations
@@ -225,6 +226,28 @@ def moe_bwd_direct(dY: np.ndarray, X_bits, logits, bank: ExpertBank, Q_bits, b: 
         for k in range(top_k):
             dlogits[t, idx[t, k]] = w[t, k] * (dw[t, k] - s[t])
     return dX, dq, dlogits, dw
+
+
+def expert_dq(e: int, dY: np.ndarray, X_bits, logits, bank: ExpertBank, Q_bits, b: int, top_k: int):
+    """dq_e [2][K/b][b(b-1)/2] of one expert, from the (t, k) entries routed to it
+    only: the same sums as moe_bwd_direct's G_e,p (slot order within each token,
+    tokens ascending), batched over the expert's tokens, then the Cayley backward.
+    For checks of a heavily loaded expert at full size, where moe_bwd_direct would
+    also work through every other expert of those tokens."""
+    X = bf16_bits_to_f64(X_bits)
+    idx, w = topk(logits, top_k)
+    T, K = X.shape
+    n, nb = bank.n, K // b
+    ts, ks = np.nonzero(idx == e)                  # entries in (t, k) order
+    R = rotations(Q_bits[e], b)
+    Wt = bank.weight_t(e)
+    dq = np.zeros((2, nb, packed_len(b)))
+    for p in (0, 1):
+        D = dY[ts, p * n:(p + 1) * n] @ Wt[p * n:(p + 1) * n]           # [entries][K]
+        wD = w[ts, ks][:, None] * D
+        G = np.einsum("mji,mjk->jik", X[ts].reshape(-1, nb, b), wD.reshape(-1, nb, b))
+        dq[p] = cayley_grad(G, R[p], b)
+    return dq
 
 
 def silu(x):

@@ -129,9 +129,14 @@ int side_pipe(SidePipe** out, std::unique_lock<std::mutex>* lock) {
 }
 
 int sm_count() {
+  static int cached[64] = {0};
   int dev = 0, n = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n > 0 ? n : 148;
+  if (cudaGetDevice(&dev) != cudaSuccess) return n;
+  if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  n = n > 0 ? n : 148;
+  if (dev >= 0 && dev < 64) cached[dev] = n;
+  return n;
 }
 
 // ---- launch profiler: CUDA event pairs around launches, per kernel class ----
@@ -389,7 +394,15 @@ int launch_rotate_fwd(const uint16_t* X, int M, int K, int P, int b, const float
   prm.nb = K / b;
   prm.groups = (K + 63) / 64;
   prm.tiles_m = (M + rtc::TM - 1) / rtc::TM;
-  if (int rc = set_smem(rtc::rot_fwd_tc_kernel, rtc::kFwdSmem)) return rc;
+  {
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+      if (int rc = set_smem(rtc::rot_fwd_tc_kernel, rtc::kFwdSmem)) return rc;
+      if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
+  }
   const int grid = std::min(sm_count(), prm.groups * prm.tiles_m);
   ProfScope ps(OFT_K_ROTATE, st);
   OFT_CUDA(launch_pdl(rtc::rot_fwd_tc_kernel, grid, rtc::NUM_THREADS, rtc::kFwdSmem, st, prm));
@@ -862,13 +875,59 @@ int launch_gemm_small_t(const gsm::Params& prm, int grid, size_t smem, cudaStrea
   return OFT_OK;
 }
 
+// The launch parameters of the last few small-M calls on this host thread, keyed by
+// everything they are built from: a decode loop calls the same layers again and again,
+// and encoding three tensor maps per call would dominate these short kernels' launch.
+struct SmallKey {
+  const void *codes, *scales, *xr, *y, *part, *counters;
+  int dev, M, K, N, fmt, group, splits, sizes[4], n;
+  bool operator==(const SmallKey& o) const { return memcmp(this, &o, sizeof(*this)) == 0; }
+};
+struct SmallEntry {
+  SmallKey key;
+  gsm::Params prm;
+  int grid;
+  size_t smem;
+  bool valid = false;
+};
+
 int launch_gemm_small(const oft_weight* W, const oft_split* S, int M, const uint16_t* Xr, uint16_t* Y,
                       const SmallPlan& pl, int* counters, float* part, cudaStream_t st) {
   const int K = W->d_in, N = W->d_out, P = S->n;
+  SmallKey key;
+  memset(&key, 0, sizeof(key));
+  key.codes = W->codes;
+  key.scales = W->scales;
+  key.xr = Xr;
+  key.y = Y;
+  key.part = part;
+  key.counters = counters;
+  cudaGetDevice(&key.dev);
+  key.M = M;
+  key.K = K;
+  key.N = N;
+  key.fmt = W->fmt;
+  key.group = W->group;
+  key.splits = pl.splits;
+  key.n = P;
+  for (int i = 0; i < P; ++i) key.sizes[i] = S->sizes[i];
+  constexpr int kCache = 8;
+  static thread_local std::unique_ptr<SmallEntry[]> cache(new SmallEntry[kCache]);
+  static thread_local int next_slot = 0;
+  for (int i = 0; i < kCache; ++i) {
+    const SmallEntry& e = cache[i];
+    if (e.valid && e.key == key) {
+      if (W->fmt == OFT_W_INT4) return launch_gemm_small_t<gsm::kInt4>(e.prm, e.grid, e.smem, st);
+      if (W->fmt == OFT_W_FP8) return launch_gemm_small_t<gsm::kFp8>(e.prm, e.grid, e.smem, st);
+      return launch_gemm_small_t<gsm::kMxfp4>(e.prm, e.grid, e.smem, st);
+    }
+  }
+  SmallEntry& ent = cache[next_slot];
+  next_slot = (next_slot + 1) % kCache;
+  ent.valid = false;
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return fail(OFT_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
-  gsm::Params* prm = new gsm::Params;  // large (three tensor maps + groups): off the stack
-  std::unique_ptr<gsm::Params> own(prm);
+  gsm::Params* prm = &ent.prm;
   memset(prm, 0, sizeof(*prm));
   {
     // codes: [N][row bytes] uint8, 128 x 128-byte boxes with the 128-byte swizzle
@@ -921,6 +980,10 @@ int launch_gemm_small(const oft_weight* W, const oft_split* S, int M, const uint
   }
   const size_t smem = gsm::smem_bytes(pl.MN, prm->sx);
   const int grid = std::min(prm->units, sm_count());
+  ent.key = key;
+  ent.grid = grid;
+  ent.smem = smem;
+  ent.valid = true;
   if (W->fmt == OFT_W_INT4) return launch_gemm_small_t<gsm::kInt4>(*prm, grid, smem, st);
   if (W->fmt == OFT_W_FP8) return launch_gemm_small_t<gsm::kFp8>(*prm, grid, smem, st);
   return launch_gemm_small_t<gsm::kMxfp4>(*prm, grid, smem, st);

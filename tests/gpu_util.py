@@ -72,6 +72,16 @@ class OracleLinear:
             out += oft_ref.rotate_t(dY[:, n0:n1] @ self.Wt[n0:n1], self.R[p])
         return out
 
+    def dq_split(self, p):
+        """dq of every rotation block of sub-projection p (needs every token): the
+        oracle backward of that sub-projection alone."""
+        b = self.spec.b
+        n0, n1 = oft_ref.split_bounds(self.spec.splits)[p]
+        dY = bf16_bits_to_f64(self.c["dY"][:, n0:n1])
+        Wt = oft_ref.weight_t(self.c, rows=np.arange(n0, n1))                  # [N_p][K]
+        _, dq = oft_ref.linear_bwd(dY, self.X, Wt, (n1 - n0,), self.R[p:p + 1], b)
+        return dq[0]
+
     def dq_block(self, p, j):
         """dq of rotation block j of sub-projection p (needs every token)."""
         b = self.spec.b

@@ -93,7 +93,9 @@ class _Rows:
 def test_c3_backward_sampled(oft):
     """Kimi-like expert layer (4096 tokens, hidden 7168, 384 INT4-g32 experts of
     2 x 2048, top-8, chunks of 16, b = 32): dX and dlogits on sampled tokens, dq
-    of two lightly loaded experts (computed from all of their tokens)."""
+    of two lightly loaded experts (computed from all of their tokens), and the full
+    dq of a heavily loaded expert (the eighth most loaded, over a thousand routed
+    tokens, several 128-row tiles of its grouped GEMM)."""
     spec = MOE_CONFIGS["c3"]
     case = make_moe_case(spec, device="cuda")
     dY = make_moe_grad(spec, device="cuda")
@@ -117,3 +119,8 @@ def test_c3_backward_sampled(oft):
         assert rel_err(got_dq[e], dq[e]) < TOL
     idle = counts == 0
     assert not got_dq[idle].any()
+    heavy = int(np.argsort(-counts, kind="stable")[7])
+    assert counts[heavy] > 1000
+    dq_h = moe_ref.expert_dq(heavy, bf16_bits_to_f64(raw(dY)), raw(case["X"]), logits, bank, raw(case["Q"]), spec.b,
+                             spec.top_k)
+    assert rel_err(got_dq[heavy], dq_h) < TOL

@@ -125,3 +125,23 @@ def test_token_subset_gives_the_same_rows_and_complete_experts():
         if a.shape[0] == spec.T:
             assert np.array_equal(a[toks], b[toks])
     assert np.abs(full[1][e] - part[1][e]).max() <= 1e-13 * np.abs(full[1][e]).max()
+
+
+def test_expert_dq_equals_the_full_backward():
+    """expert_dq, which works from one expert's routed entries only, gives the same dq
+    as the token-by-token full backward, for heavily and lightly loaded experts."""
+    spec = MoESpec("edq", T=60, K=64, E=7, n_proj=16, top_k=3, chunk=3, group=32, b=16, q_sigma=0.1, seed=12)
+    case = make_moe_case(spec)
+    bank = moe_ref.ExpertBank(raw(case["codes"]), raw(case["scales"]), spec.K, spec.group, spec.n_proj)
+    rng = np.random.default_rng(3)
+    dY = rng.standard_normal((spec.T, 2 * spec.n_proj))
+    logits = raw(case["logits"])
+    _, dq, _, _ = moe_ref.moe_bwd_direct(dY, raw(case["X"]), logits, bank, raw(case["Q"]), spec.b, spec.top_k,
+                                         spec.E)
+    idx, _ = moe_ref.topk(logits, spec.top_k)
+    counts = np.bincount(idx.reshape(-1), minlength=spec.E)
+    for e in range(spec.E):
+        got = moe_ref.expert_dq(e, dY, raw(case["X"]), logits, bank, raw(case["Q"]), spec.b, spec.top_k)
+        scale = max(np.abs(dq[e]).max(), 1e-300)
+        assert np.abs(got - dq[e]).max() <= 1e-12 * scale, e
+        assert (counts[e] == 0) == (not got.any())

@@ -49,6 +49,18 @@ __device__ __forceinline__ void stage_q(const uint16_t* __restrict__ q, uint16_t
     reinterpret_cast<uint4*>(qs)[v] = reinterpret_cast<const uint4*>(q)[v];
 }
 
+// Second output form of the forward (lo_off > 0): R^T of each block as bf16 hi and lo
+// parts, hi = bf16_rne(R[r][c]) at element [c][r] of the block's B x B slice of
+// (uint16_t*)R, and lo = bf16_rne(R[r][c] - hi) lo_off elements further.  This is the
+// operand the MoE rotated gather feeds to its bf16 MMAs (R = hi + lo to about 2^-16),
+// laid out so that 8 consecutive reduction indices are one 16-byte load.
+__device__ __forceinline__ void store_r_hl_t(float* R, long long lo_off, int blk, int B, int r, int c, float v) {
+  uint16_t* hi = reinterpret_cast<uint16_t*>(R) + (static_cast<long long>(blk) * B + c) * B + r;
+  const uint16_t h = f32_to_bf16_bits(v);
+  hi[0] = h;
+  hi[lo_off] = f32_to_bf16_bits(v - bf16_bits_to_f32(h));
+}
+
 template <int B>
 struct CayleyFwdCfg {
   static constexpr int THREADS = B < 32 ? 32 : B;
@@ -59,7 +71,7 @@ struct CayleyFwdCfg {
 template <int B, bool UNROLL>
 __device__ __forceinline__ void cayley_fwd_block(const uint16_t* __restrict__ Q, float* __restrict__ R, int lin,
                                                  int total, const int* __restrict__ active_list,
-                                                 int blocks_per_expert) {
+                                                 int blocks_per_expert, long long lo_off) {
   constexpr int BPC = CayleyFwdCfg<B>::BPC;
   __shared__ __align__(16) float piv[2][BPC][2 * B + 4];  // pivot row, right-hand side, 1 / pivot
   __shared__ __align__(16) uint16_t qsh[BPC][B * (B - 1) / 2];
@@ -172,7 +184,10 @@ __device__ __forceinline__ void cayley_fwd_block(const uint16_t* __restrict__ Q,
   }
 #pragma unroll
   for (int k = 0; k < B; ++k) rhs[k] *= my_inv;
-  if (active) {
+  if (active && lo_off > 0) {
+#pragma unroll
+    for (int j = 0; j < B; ++j) store_r_hl_t(R, lo_off, blk, B, r, j, rhs[j]);
+  } else if (active) {
     float* out = R + (static_cast<size_t>(blk) * B + r) * B;
 #pragma unroll
     for (int j = 0; j < B; j += 4)
@@ -189,7 +204,7 @@ __device__ __forceinline__ void cayley_fwd_block(const uint16_t* __restrict__ Q,
 template <int B>
 __device__ __forceinline__ void cayley_fwd_block_inv(const uint16_t* __restrict__ Q, float* __restrict__ R, int lin,
                                                      int total, const int* __restrict__ active_list,
-                                                     int blocks_per_expert) {
+                                                     int blocks_per_expert, long long lo_off) {
   constexpr int BPC = CayleyFwdCfg<B>::BPC;
   __shared__ __align__(16) float piv[2][BPC][B];
   __shared__ __align__(16) uint16_t qsh[BPC][B * (B - 1) / 2];
@@ -241,7 +256,10 @@ __device__ __forceinline__ void cayley_fwd_block_inv(const uint16_t* __restrict_
       }
     }
   }
-  if (active) {
+  if (active && lo_off > 0) {
+#pragma unroll
+    for (int j = 0; j < B; ++j) store_r_hl_t(R, lo_off, blk, B, r, j, 2.f * a[j] - (j == r ? 1.f : 0.f));
+  } else if (active) {
     float* out = R + (static_cast<size_t>(blk) * B + r) * B;
 #pragma unroll
     for (int j = 0; j < B; j += 4)
@@ -256,15 +274,15 @@ __global__ void __launch_bounds__(CayleyFwdCfg<B>::THREADS, CayleyFwdCfg<B>::MIN
                                                                                int nblocks, float* __restrict__ R,
                                                                                const int* __restrict__ active_list,
                                                                                const int* __restrict__ n_active,
-                                                                               int blocks_per_expert) {
+                                                                               int blocks_per_expert, long long lo_off) {
   constexpr int BPC = CayleyFwdCfg<B>::BPC;
   pdl_wait();
   const int total = active_list != nullptr ? min(nblocks, *n_active * blocks_per_expert) : nblocks;
   for (int base = blockIdx.x * BPC; base < total; base += gridDim.x * BPC) {
     if constexpr (UNROLL) {
-      cayley_fwd_block_inv<B>(Q, R, base + threadIdx.x / B, total, active_list, blocks_per_expert);
+      cayley_fwd_block_inv<B>(Q, R, base + threadIdx.x / B, total, active_list, blocks_per_expert, lo_off);
     } else {
-      cayley_fwd_block<B, UNROLL>(Q, R, base + threadIdx.x / B, total, active_list, blocks_per_expert);
+      cayley_fwd_block<B, UNROLL>(Q, R, base + threadIdx.x / B, total, active_list, blocks_per_expert, lo_off);
     }
   }
 }
@@ -283,7 +301,7 @@ __global__ void __launch_bounds__(TPR * B) cayley_fwd_split_kernel(const uint16_
                                                                  float* __restrict__ R,
                                                                  const int* __restrict__ active_list,
                                                                  const int* __restrict__ n_active,
-                                                                 int blocks_per_expert) {
+                                                                 int blocks_per_expert, long long lo_off) {
   constexpr int H = B / TPR;  // columns per thread
   static_assert(H % 4 == 0 && (TPR & (TPR - 1)) == 0, "slices of whole float4s");
   __shared__ __align__(16) float piv[2][2 * B + 4];
@@ -349,11 +367,16 @@ __global__ void __launch_bounds__(TPR * B) cayley_fwd_split_kernel(const uint16_
       for (int k = 0; k < H - 1; ++k) a[k] = a[k + 1];
       a[H - 1] = h < TPR - 1 ? nxt : 0.f;
     }
-    float* out = R + (static_cast<size_t>(blk) * B + r) * B + h * H;
+    if (lo_off > 0) {
 #pragma unroll
-    for (int k = 0; k < H; k += 4)
-      *reinterpret_cast<float4*>(out + k) =
-          make_float4(rhs[k] * my_inv, rhs[k + 1] * my_inv, rhs[k + 2] * my_inv, rhs[k + 3] * my_inv);
+      for (int k = 0; k < H; ++k) store_r_hl_t(R, lo_off, blk, B, r, h * H + k, rhs[k] * my_inv);
+    } else {
+      float* out = R + (static_cast<size_t>(blk) * B + r) * B + h * H;
+#pragma unroll
+      for (int k = 0; k < H; k += 4)
+        *reinterpret_cast<float4*>(out + k) =
+            make_float4(rhs[k] * my_inv, rhs[k + 1] * my_inv, rhs[k + 2] * my_inv, rhs[k + 3] * my_inv);
+    }
   }
 }
 

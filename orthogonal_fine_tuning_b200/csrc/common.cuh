@@ -257,6 +257,15 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, const void* s
                : "memory");
 }
 
+// 16-byte asynchronous copies global -> shared (cp.async, completion by wait_all).  Their
+// shared-memory writes are generic-proxy writes: a tcgen05.mma that reads them needs
+// fence.proxy.async after the wait.
+__device__ __forceinline__ void cp_async_16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // Programmatic dependent launch: a kernel launched with programmatic stream
 // serialisation may start before the previous kernel on its stream has finished;
 // pdl_wait() returns once that kernel has completed and its writes are visible.

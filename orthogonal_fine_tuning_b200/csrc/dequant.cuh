@@ -26,30 +26,54 @@ struct WeightView {
   long long scales_expert_stride;  // bytes between experts (bank only)
 };
 
-// Dequantise 8 consecutive elements k0..k0+7 (k0 % 8 == 0) of stored row n into
-// four packed bf16x2 words (element k0 in the low half of out[0]), with the same
-// packed decoders the fused GEMM's producer warps use (dq_pack.cuh).
-__device__ __forceinline__ void dequant8(const WeightView& w, const uint8_t* codes, const void* scales, int n, int k0,
-                                         uint32_t out[4]) {
+// The codes and scale of 8 consecutive elements k0..k0+7 (k0 % 8 == 0) of stored row
+// n, loaded ahead of their decode.
+struct Raw8 {
+  uint32_t c0, c1;  // FP8: 8 codes; INT4 / MXFP4: c0 holds 8 nibbles
+  uint32_t s;       // FP8: fp32 bits; INT4: bf16 bits; MXFP4: e8m0
+};
+
+__device__ __forceinline__ Raw8 load8(const WeightView& w, const uint8_t* codes, const void* scales, int n, int k0) {
+  Raw8 r;
   if (w.fmt == kFmtFp8) {
     const uint2 c = *reinterpret_cast<const uint2*>(codes + static_cast<size_t>(n) * w.K + k0);
-    const float s = static_cast<const float*>(scales)[n];
+    r.c0 = c.x;
+    r.c1 = c.y;
+    r.s = __float_as_uint(static_cast<const float*>(scales)[n]);
+    return r;
+  }
+  r.c0 = *reinterpret_cast<const uint32_t*>(codes + static_cast<size_t>(n) * (w.K / 2) + k0 / 2);
+  r.c1 = 0;
+  r.s = w.fmt == kFmtInt4 ? static_cast<const uint16_t*>(scales)[static_cast<size_t>(k0 / w.group) * w.N + n]
+                          : static_cast<const uint8_t*>(scales)[static_cast<size_t>(k0 / 32) * w.N + n];
+  return r;
+}
+
+// The 8 elements as four packed bf16x2 words (element k0 in the low half of out[0]),
+// with the same packed decoders the fused GEMM's producer warps use (dq_pack.cuh).
+__device__ __forceinline__ void decode8(int fmt, const Raw8& r, uint32_t out[4]) {
+  if (fmt == kFmtFp8) {
+    const float s = __uint_as_float(r.s);
     uint32_t v[4];
-    dq::e4m3x4(c.x, v);      // exact bf16 codes
-    dq::e4m3x4(c.y, v + 2);
+    dq::e4m3x4(r.c0, v);      // exact bf16 codes
+    dq::e4m3x4(r.c1, v + 2);
 #pragma unroll
     for (int i = 0; i < 4; ++i)  // canonical chain: fp32 product, then bf16
       out[i] = pack_bf16x2(__fmul_rn(__uint_as_float(v[i] << 16), s), __fmul_rn(__uint_as_float(v[i] & 0xFFFF0000u), s));
     return;
   }
-  const uint32_t word = *reinterpret_cast<const uint32_t*>(codes + static_cast<size_t>(n) * (w.K / 2) + k0 / 2);
-  if (w.fmt == kFmtInt4) {
-    const uint16_t sb = static_cast<const uint16_t*>(scales)[static_cast<size_t>(k0 / w.group) * w.N + n];
-    dq::int4x8(word, dq::bf2_splat(sb), out);
+  if (fmt == kFmtInt4) {
+    dq::int4x8(r.c0, dq::bf2_splat(static_cast<uint16_t>(r.s)), out);
     return;
   }
-  const uint8_t eb = static_cast<const uint8_t*>(scales)[static_cast<size_t>(k0 / 32) * w.N + n];
-  dq::mxfp4x8(word, eb, out);
+  dq::mxfp4x8(r.c0, r.s, out);
+}
+
+// Dequantise 8 consecutive elements k0..k0+7 (k0 % 8 == 0) of stored row n into
+// four packed bf16x2 words.
+__device__ __forceinline__ void dequant8(const WeightView& w, const uint8_t* codes, const void* scales, int n, int k0,
+                                         uint32_t out[4]) {
+  decode8(w.fmt, load8(w, codes, scales, n, k0), out);
 }
 
 // out[n][k] = deq(W)[n][k] for all n < N, k < K.  A unit is 8 consecutive elements
@@ -79,39 +103,59 @@ __global__ void __launch_bounds__(256) dequant_rows_kernel(WeightView w, uint16_
 // out[k][n] = deq(W)[n][k]: 64 x 64 tiles transposed through shared memory as
 // 32-bit words (two k per word, rows padded to 33 words), so neither the decode
 // side nor the transposed side has bank conflicts; each warp stores 64-byte runs of
-// 8 k-rows.  grid = (ceil(K / 64), ceil(N / 64)).
+// 8 k-rows.  A CTA walks a strip of kDeqTStrip tiles along K with every code and
+// scale load of the strip issued before the first decode.
+// grid = (ceil(K / (64 * kDeqTStrip)), ceil(N / 64)).
+constexpr int kDeqTStrip = 4;
+
 __global__ void __launch_bounds__(256) dequant_transposed_kernel(WeightView w, uint16_t* __restrict__ out) {
   __shared__ uint32_t tile[64][33];  // [row n][k pair]
   pdl_wait();
   const int n0 = blockIdx.y * 64;
-  const int k0 = blockIdx.x * 64;
-  for (int it = threadIdx.x; it < 512; it += 256) {
-    const int r = it >> 3, c = it & 7;  // row n0 + r, k = k0 + 8c .. +7
-    const int n = n0 + r, k = k0 + c * 8;
-    uint32_t v[4] = {0, 0, 0, 0};
-    if (n < w.N && k < w.K) dequant8(w, w.codes, w.scales, n, k, v);
+  const int kb = blockIdx.x * 64 * kDeqTStrip;
+  Raw8 raw[kDeqTStrip][2];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) tile[r][c * 4 + i] = v[i];
-  }
-  __syncthreads();
-  const int lane = threadIdx.x & 31;
-  for (int it = threadIdx.x; it < 512; it += 256) {
-    const int q = it >> 5;
-    const int r = (lane & 7) + 8 * (q & 7);    // k row
-    const int c = (lane >> 3) + 4 * (q >> 3);  // 8 consecutive n
-    const int k = k0 + r, n = n0 + c * 8;
-    if (k >= w.K || n >= w.N) continue;
-    const int sh = (r & 1) * 16;
-    uint32_t v[4];
+  for (int t = 0; t < kDeqTStrip; ++t)
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      v[i] = ((tile[c * 8 + 2 * i][r >> 1] >> sh) & 0xFFFFu) | (((tile[c * 8 + 2 * i + 1][r >> 1] >> sh) & 0xFFFFu) << 16);
-    if (n + 8 <= w.N) {
-      *reinterpret_cast<uint4*>(out + static_cast<size_t>(k) * w.N + n) = make_uint4(v[0], v[1], v[2], v[3]);
-    } else {
-      for (int i = 0; i < 8 && n + i < w.N; ++i)
-        out[static_cast<size_t>(k) * w.N + n + i] = static_cast<uint16_t>((v[i / 2] >> (16 * (i & 1))) & 0xFFFFu);
+    for (int h = 0; h < 2; ++h) {
+      const int it = threadIdx.x + 256 * h;
+      const int n = n0 + (it >> 3), k = kb + t * 64 + (it & 7) * 8;
+      raw[t][h] = (n < w.N && k < w.K) ? load8(w, w.codes, w.scales, n, k) : Raw8{0u, 0u, 0u};
     }
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int t = 0; t < kDeqTStrip; ++t) {
+    const int k0 = kb + t * 64;
+    if (k0 >= w.K) break;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int it = threadIdx.x + 256 * h;
+      const int r = it >> 3, c = it & 7;  // row n0 + r, k = k0 + 8c .. +7
+      uint32_t v[4] = {0, 0, 0, 0};
+      if (n0 + r < w.N && k0 + c * 8 < w.K) decode8(w.fmt, raw[t][h], v);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) tile[r][c * 4 + i] = v[i];
+    }
+    __syncthreads();
+    for (int it = threadIdx.x; it < 512; it += 256) {
+      const int q = it >> 5;
+      const int r = (lane & 7) + 8 * (q & 7);    // k row
+      const int c = (lane >> 3) + 4 * (q >> 3);  // 8 consecutive n
+      const int k = k0 + r, n = n0 + c * 8;
+      if (k >= w.K || n >= w.N) continue;
+      const int sh = (r & 1) * 16;
+      uint32_t v[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        v[i] = ((tile[c * 8 + 2 * i][r >> 1] >> sh) & 0xFFFFu) | (((tile[c * 8 + 2 * i + 1][r >> 1] >> sh) & 0xFFFFu) << 16);
+      if (n + 8 <= w.N) {
+        *reinterpret_cast<uint4*>(out + static_cast<size_t>(k) * w.N + n) = make_uint4(v[0], v[1], v[2], v[3]);
+      } else {
+        for (int i = 0; i < 8 && n + i < w.N; ++i)
+          out[static_cast<size_t>(k) * w.N + n + i] = static_cast<uint16_t>((v[i / 2] >> (16 * (i & 1))) & 0xFFFFu);
+      }
+    }
+    __syncthreads();  // the tile is free for the next
   }
 }
 

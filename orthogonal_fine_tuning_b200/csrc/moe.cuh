@@ -168,10 +168,14 @@ __global__ void __launch_bounds__(1024) moe_route_kernel(const int* __restrict__
 // and consecutive units of a CTA share the expert's rotation tiles.  A CTA (128
 // threads, four resident per SM) walks a contiguous range of units:
 //   gather the tile's 128 activation rows (64 bf16 columns) into a 128B-swizzled
-//   K-major tile; on an (expert, group) change rebuild B[p*64 + c][i] =
-//   R_{e,p}[i][c] over the group's diagonal blocks for p = gate, up, split into
-//   bf16 hi + lo; one thread issues 8 tcgen05.mma (M = 128, N = 128, K = 64 as
-//   4 x 16, hi and lo) into TMEM; the epilogue writes the tile's valid rows.
+//   K-major tile; on an (expert, group) change the B tiles B[p*64 + c][i] =
+//   R_{e,p}[i][c] over the group's diagonal blocks for p = gate, up hold bf16 hi + lo
+//   parts; one thread issues 8 tcgen05.mma (M = 128, N = 128, K = 64 as 4 x 16, hi
+//   and lo) into TMEM; the epilogue writes the tile's valid rows.
+// The rotations come from the Cayley build already split into hi / lo and
+// transposed (Rhi / Rlo [e][p][block][c][i]), so each 8 reduction indices of a B row
+// are one 16-byte cp.async; the tiles' off-diagonal zeros are written once, and the
+// next unit's diagonal blocks are fetched while the current unit's epilogue runs.
 // The rotation of activations in front of the frozen weight is the OFT adapter
 // ("Orbit", chooseai.io news 4086, section "技术原理：低精度基座 + BF16 适配器 + OFT");
 // the per-expert split into gate and up is its split-projection form (item
@@ -183,7 +187,7 @@ template <int B>
 __global__ void __launch_bounds__(kMoeRotThreads, 4) moe_rot_tc_kernel(
     const uint16_t* __restrict__ X, int K, int top_k, const int* __restrict__ bucket,
     const int* __restrict__ offsets, const int* __restrict__ active, const int* __restrict__ n_active_p,
-    const float* __restrict__ Rex, int TK, uint16_t* __restrict__ Xg) {
+    const uint16_t* __restrict__ Rhi, const uint16_t* __restrict__ Rlo, int TK, uint16_t* __restrict__ Xg) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;                 // 128 positions x 64 columns, bf16, 128B swizzle
@@ -226,6 +230,11 @@ __global__ void __launch_bounds__(kMoeRotThreads, 4) moe_rot_tc_kernel(
     tmem_alloc(tmem_slot, 128);
     tmem_relinquish();
   }
+  // the B tiles' off-diagonal blocks stay zero for the whole launch
+  for (int v = tid; v < 16384 / 16; v += kMoeRotThreads) {
+    reinterpret_cast<uint4*>(sBhi)[v] = make_uint4(0, 0, 0, 0);
+    reinterpret_cast<uint4*>(sBlo)[v] = make_uint4(0, 0, 0, 0);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -267,7 +276,32 @@ __global__ void __launch_bounds__(kMoeRotThreads, 4) moe_rot_tc_kernel(
       if (tok[q] >= 0 && col < K) xv[q] = *reinterpret_cast<const uint4*>(X + static_cast<size_t>(tok[q] / top_k) * K + col);
     }
   };
-  int cur_e = -1, cur_g = -1, a = 0, a1 = 0, a2 = 0;
+  // the diagonal blocks of (e, g) into the B tiles: 16-byte cp.async per 8 reduction
+  // indices of one output column, hi and lo (zeros for a block past K)
+  auto issue_b = [&](int e, int g) {
+    constexpr int NBG = 64 / B, CH = B / 8;
+    constexpr int NCOPY = 2 * NBG * B * CH;
+    for (int v = tid; v < NCOPY; v += kMoeRotThreads) {
+      const int pr = v / (NBG * B * CH);
+      int rem = v % (NBG * B * CH);
+      const int jb = rem / (B * CH);
+      rem %= B * CH;
+      const int c = rem / CH, i8 = rem % CH;
+      const int j = (g * 64) / B + jb;
+      const uint32_t off = sw128_offset(static_cast<uint32_t>(pr * 64 + jb * B + c),
+                                        static_cast<uint32_t>((jb * B + i8 * 8) >> 3));
+      if ((j + 1) * B <= K) {
+        const size_t src = (((static_cast<size_t>(e) * 2 + pr) * nb + j) * B + c) * B + i8 * 8;
+        cp_async_16(sBhi + off, Rhi + src);
+        cp_async_16(sBlo + off, Rlo + src);
+      } else {
+        *reinterpret_cast<uint4*>(sBhi + off) = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(sBlo + off) = make_uint4(0, 0, 0, 0);
+      }
+    }
+    cp_async_commit();
+  };
+  int cur_e = -1, cur_g = -1, pf_e = -1, pf_g = -1, a = 0, a1 = 0, a2 = 0, ab = 0;
   uint32_t phase = 0;
   uint4 xv[NIT];
   int tok1[NIT], tok2[NIT];
@@ -282,46 +316,14 @@ __global__ void __launch_bounds__(kMoeRotThreads, 4) moe_rot_tc_kernel(
   for (int u = ubeg; u < uend; ++u) {
     const Unit U = unit_at(u, a);
     const int e = U.e, g = U.g, pos0 = U.pos0, nrows = U.nrows;
-    // 1. rotation tiles of (e, g), when they change (the previous unit's MMAs have completed)
+    // 1. rotation tiles of (e, g), when they change (fetched during the previous unit's
+    //    epilogue, after its MMAs had completed; the first unit's here)
     if (e != cur_e || g != cur_g) {
-      for (int v = tid; v < 16384 / 16; v += kMoeRotThreads) {  // each tile is 16 KB
-        reinterpret_cast<uint4*>(sBhi)[v] = make_uint4(0, 0, 0, 0);
-        reinterpret_cast<uint4*>(sBlo)[v] = make_uint4(0, 0, 0, 0);
-      }
-      __syncthreads();
-      constexpr int PER = 16 * B;  // float4s of one projection's diagonal blocks in the group
-      constexpr int NRT = 2 * PER / kMoeRotThreads;  // b / 4 per thread: all loads in flight first
-      float4 rv[NRT];
-#pragma unroll
-      for (int q = 0; q < NRT; ++q) {
-        const int f = tid + q * kMoeRotThreads;
-        const int pr = f / PER, rem4 = f % PER;
-        const int jb = rem4 / (B * B / 4), w = rem4 % (B * B / 4);
-        const int i = w / (B / 4), c4 = (w % (B / 4)) * 4;
-        const int j = (g * 64) / B + jb;
-        rv[q] = (j + 1) * B <= K ? *reinterpret_cast<const float4*>(
-                                       Rex + (((static_cast<size_t>(e) * 2 + pr) * nb + j) * B + i) * B + c4)
-                                 : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-      for (int q = 0; q < NRT; ++q) {
-        const int f = tid + q * kMoeRotThreads;
-        const int pr = f / PER, rem4 = f % PER;
-        const int jb = rem4 / (B * B / 4), w = rem4 % (B * B / 4);
-        const int i = w / (B / 4), c4 = (w % (B / 4)) * 4;
-        const float ev[4] = {rv[q].x, rv[q].y, rv[q].z, rv[q].w};
-        const int k = jb * B + i;  // reduction index within the group
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const int r = pr * 64 + jb * B + c4 + t;  // output column (gate 0..63, up 64..127)
-          const uint32_t off = sw128_offset(static_cast<uint32_t>(r), static_cast<uint32_t>(k >> 3)) + (k & 7) * 2;
-          const uint16_t h = f32_to_bf16_bits(ev[t]);
-          *reinterpret_cast<uint16_t*>(sBhi + off) = h;
-          *reinterpret_cast<uint16_t*>(sBlo + off) = f32_to_bf16_bits(ev[t] - bf16_bits_to_f32(h));
-        }
-      }
+      if (e != pf_e || g != pf_g) issue_b(e, g);
+      cp_async_wait_all();
       cur_e = e;
       cur_g = g;
+      pf_e = pf_g = -1;
     }
     // 2. this unit's activation rows (loaded one unit ago) into the swizzled A tile
 #pragma unroll
@@ -354,6 +356,15 @@ __global__ void __launch_bounds__(kMoeRotThreads, 4) moe_rot_tc_kernel(
     if (!warp_wait_bounded(bar, phase, abort_flag, kErrWaitAccFull)) break;
     phase ^= 1;
     tc_fence_after();
+    // the product has read the B tiles: start the next unit's, if they differ
+    if (u + 1 < uend) {
+      const Unit Un = unit_at(u + 1, ab);
+      if (Un.e != cur_e || Un.g != cur_g) {
+        issue_b(Un.e, Un.g);
+        pf_e = Un.e;
+        pf_g = Un.g;
+      }
+    }
     // 4. epilogue: TMEM lane = position row, 64 columns per projection
     const int r = warp * 32 + lane;
 #pragma unroll 1

@@ -323,7 +323,7 @@ int launch_dequant(const WeightView& v, uint16_t* out, bool transpose, cudaStrea
     OFT_CUDA(launch_pdl(dequant_rows_kernel, grid, 256, 0, st, v, out));
     OFT_LAUNCHED("dequant_rows_kernel");
   } else {
-    dim3 grid((v.K + 63) / 64, (v.N + 63) / 64);
+    dim3 grid((v.K + 64 * kDeqTStrip - 1) / (64 * kDeqTStrip), (v.N + 63) / 64);
     ProfScope ps(OFT_K_DEQUANT, st);
     OFT_CUDA(launch_pdl(dequant_transposed_kernel, grid, 256, 0, st, v, out));
     OFT_LAUNCHED("dequant_transposed_kernel");
@@ -332,8 +332,10 @@ int launch_dequant(const WeightView& v, uint16_t* out, bool transpose, cudaStrea
 }
 
 // active_list / n_active (device): build only the blocks of the active experts.
+// lo_off > 0: R is written as the bf16 hi / lo parts of each block's transpose, hi at
+// (uint16_t*)R and lo lo_off elements further (the MoE rotated gather's operand).
 int launch_cayley(const uint16_t* Q, int nblocks, int b, float* R, const int* active_list, const int* n_active,
-                  int blocks_per_expert, cudaStream_t st) {
+                  int blocks_per_expert, cudaStream_t st, long long lo_off = 0) {
   ProfScope ps(OFT_K_CAYLEY, st);
   // unrolled pivots pay off once many blocks run from a warm instruction cache;
   // persistent grid of about 32 resident warps per SM
@@ -341,15 +343,15 @@ int launch_cayley(const uint16_t* Q, int nblocks, int b, float* R, const int* ac
   const int grid = std::max(1, std::min((nblocks + bpc - 1) / bpc, sm_count() * 32 / warps));
   const int* al = active_list;
   if (nblocks >= kCayleyUnrollBlocks) {
-    if (b == 16) OFT_CUDA(launch_pdl(cayley_fwd_kernel<16, true>, grid, 32, 0, st, Q, nblocks, R, al, n_active, blocks_per_expert));
-    if (b == 32) OFT_CUDA(launch_pdl(cayley_fwd_kernel<32, true>, grid, 32, 0, st, Q, nblocks, R, al, n_active, blocks_per_expert));
-    if (b == 64) OFT_CUDA(launch_pdl(cayley_fwd_kernel<64, true>, grid, 64, 0, st, Q, nblocks, R, al, n_active, blocks_per_expert));
+    if (b == 16) OFT_CUDA(launch_pdl(cayley_fwd_kernel<16, true>, grid, 32, 0, st, Q, nblocks, R, al, n_active, blocks_per_expert, lo_off));
+    if (b == 32) OFT_CUDA(launch_pdl(cayley_fwd_kernel<32, true>, grid, 32, 0, st, Q, nblocks, R, al, n_active, blocks_per_expert, lo_off));
+    if (b == 64) OFT_CUDA(launch_pdl(cayley_fwd_kernel<64, true>, grid, 64, 0, st, Q, nblocks, R, al, n_active, blocks_per_expert, lo_off));
   } else {
-    if (b == 16) OFT_CUDA(launch_pdl(cayley_fwd_kernel<16, false>, grid, 32, 0, st, Q, nblocks, R, al, n_active, blocks_per_expert));
+    if (b == 16) OFT_CUDA(launch_pdl(cayley_fwd_kernel<16, false>, grid, 32, 0, st, Q, nblocks, R, al, n_active, blocks_per_expert, lo_off));
     // few blocks: the per-block pivot chain is the time, so two threads share each row
     const int sgrid = std::max(1, std::min(nblocks, sm_count() * 16));
-    if (b == 32) OFT_CUDA(launch_pdl(cayley_fwd_split_kernel<32, 2>, sgrid, 64, 0, st, Q, nblocks, R, al, n_active, blocks_per_expert));
-    if (b == 64) OFT_CUDA(launch_pdl(cayley_fwd_split_kernel<64, 2>, sgrid, 128, 0, st, Q, nblocks, R, al, n_active, blocks_per_expert));
+    if (b == 32) OFT_CUDA(launch_pdl(cayley_fwd_split_kernel<32, 2>, sgrid, 64, 0, st, Q, nblocks, R, al, n_active, blocks_per_expert, lo_off));
+    if (b == 64) OFT_CUDA(launch_pdl(cayley_fwd_split_kernel<64, 2>, sgrid, 128, 0, st, Q, nblocks, R, al, n_active, blocks_per_expert, lo_off));
   }
   OFT_LAUNCHED("cayley_fwd_kernel");
   return OFT_OK;
@@ -432,16 +434,32 @@ int launch_rotate_bwd(const float* dXr, int M, int K, int P, int b, const float*
   return OFT_OK;
 }
 
-// Token chunking of the dR reduction (deterministic in the shape): about one
-// (128-column group, chunk) unit per SM of a 148-SM part.
+// Token chunking of the dR reduction (deterministic in the shape, fixed for a 148-SM
+// part so the workspace size does not depend on the device): units are (128-column
+// group, chunk of token tiles), spread over 148 CTAs in contiguous ranges.  The chunk
+// length minimises the busiest CTA's work, ceil(units / 148) x (tiles per chunk + 1),
+// the one counting a unit's accumulator drain and partial-sum writes; ties go to
+// longer chunks (fewer partial sums).  The MXFP4 training step (56 groups, 128 token
+// tiles) takes 5 chunks of 26 tiles: 52 tiles on the busiest CTA, against 64 with one
+// chunk per SM's worth of groups.
 struct GradChunks {
   int chunks, tiles_per_chunk;
 };
 GradChunks grad_chunks(int M, int K) {
   const int groups = (K + 127) / 128, tiles_m = (M + 127) / 128;
-  const int want = std::max(1, std::min(tiles_m, 148 / groups));
-  const int tpc = (tiles_m + want - 1) / want;
-  return GradChunks{(tiles_m + tpc - 1) / tpc, tpc};
+  int best_tpc = tiles_m;
+  long long best = 1ll << 60;
+  for (int tpc = tiles_m; tpc >= 1; --tpc) {
+    const int chunks = (tiles_m + tpc - 1) / tpc;
+    if ((chunks - 1) * tpc >= tiles_m) continue;  // the same chunking as a longer tpc
+    const long long units = 1ll * groups * chunks;
+    const long long cost = (units + 147) / 148 * (tpc + 1);
+    if (cost < best) {
+      best = cost;
+      best_tpc = tpc;
+    }
+  }
+  return GradChunks{(tiles_m + best_tpc - 1) / best_tpc, best_tpc};
 }
 
 int launch_grad(const uint16_t* X, const float* dXr, int M, int K, int P, int b, float* Gp, cudaStream_t st) {
@@ -1496,7 +1514,11 @@ int moe_oft_fwd_impl(bool fused, const uint16_t* X, int T, const float* logits, 
     OFT_LAUNCHED("moe_route_kernel");
   }
   // 3. rotations of the active experts (gate and up)
-  if (int rc = launch_cayley(Q, E * 2 * nb, b, Rex, chunk_table, n_active, 2 * nb, st)) return rc;
+  // (as bf16 hi / lo parts of each block's transpose: the gather's MMA operand)
+  const long long r_elems = 1ll * E * 2 * nb * b * b;
+  if (int rc = launch_cayley(Q, E * 2 * nb, b, Rex, chunk_table, n_active, 2 * nb, st, r_elems)) return rc;
+  const uint16_t* Rhi = reinterpret_cast<const uint16_t*>(Rex);
+  const uint16_t* Rlo = Rhi + r_elems;
   // 4. rotated gather in bucket order: Xg[proj][pos] = X[t] R_{e,proj}
   //    on the tensor cores, units (active expert, 64-column group, 128-position tile)
   {
@@ -1505,17 +1527,17 @@ int moe_oft_fwd_impl(bool fused, const uint16_t* X, int T, const float* logits, 
     if (b == 16) {
       if (int rc = set_smem(moe_rot_tc_kernel<16>, kMoeRotSmem)) return rc;
       moe_rot_tc_kernel<16><<<rgrid, kMoeRotThreads, kMoeRotSmem, st>>>(X, K, top_k, bucket, offsets, chunk_table,
-                                                                         n_active, Rex, TK, Xg);
+                                                                         n_active, Rhi, Rlo, TK, Xg);
     }
     if (b == 32) {
       if (int rc = set_smem(moe_rot_tc_kernel<32>, kMoeRotSmem)) return rc;
       moe_rot_tc_kernel<32><<<rgrid, kMoeRotThreads, kMoeRotSmem, st>>>(X, K, top_k, bucket, offsets, chunk_table,
-                                                                         n_active, Rex, TK, Xg);
+                                                                         n_active, Rhi, Rlo, TK, Xg);
     }
     if (b == 64) {
       if (int rc = set_smem(moe_rot_tc_kernel<64>, kMoeRotSmem)) return rc;
       moe_rot_tc_kernel<64><<<rgrid, kMoeRotThreads, kMoeRotSmem, st>>>(X, K, top_k, bucket, offsets, chunk_table,
-                                                                         n_active, Rex, TK, Xg);
+                                                                         n_active, Rhi, Rlo, TK, Xg);
     }
     OFT_LAUNCHED("moe_rot_tc_kernel");
   }

@@ -156,5 +156,32 @@ __device__ __forceinline__ void mxfp4x8_mul(uint32_t w, uint32_t e, uint32_t out
   out[3] = e2m1x2_lanes_mul(prmt(hi, 0u, 0x4342u), f2, g2, two_step);
 }
 
+// mxfp4x8_mul for four words sharing one e8m0 scale (a 32-element group), with the
+// choice between the one-step factor (e <= 128, every realistic weight) and the
+// two-step one taken once for the group rather than per pair.
+__device__ __forceinline__ void mxfp4x32_mul(const uint32_t (&w)[4], uint32_t e, uint32_t (&out)[16]) {
+  if (e <= 128u) {
+    const uint32_t f2 = ((e + 126u) << 7) * 0x10001u;  // 2^(e-1)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t x0 = w[i] & 0x0F0F0F0Fu;
+      const uint32_t x1 = (w[i] >> 4) & 0x0F0F0F0Fu;
+      const uint32_t lo = prmt(x0, x1, 0x5140u);
+      const uint32_t hi = prmt(x0, x1, 0x7362u);
+      out[4 * i] = bf2_mul((prmt(lo, 0u, 0x4140u) * 0x1040u) & 0x81C081C0u, f2);
+      out[4 * i + 1] = bf2_mul((prmt(lo, 0u, 0x4342u) * 0x1040u) & 0x81C081C0u, f2);
+      out[4 * i + 2] = bf2_mul((prmt(hi, 0u, 0x4140u) * 0x1040u) & 0x81C081C0u, f2);
+      out[4 * i + 3] = bf2_mul((prmt(hi, 0u, 0x4342u) * 0x1040u) & 0x81C081C0u, f2);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t t[4];
+      mxfp4x8_mul(w[i], e, t);
+      out[4 * i] = t[0], out[4 * i + 1] = t[1], out[4 * i + 2] = t[2], out[4 * i + 3] = t[3];
+    }
+  }
+}
+
 }  // namespace dq
 }  // namespace oftk

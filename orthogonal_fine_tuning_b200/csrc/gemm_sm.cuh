@@ -7,11 +7,11 @@
 //   * TMA brings 128-row x 128-byte code tiles (256 INT4 / MXFP4 codes, or 128 FP8
 //     codes, per row) into a 6-stage shared-memory ring with the 128-byte swizzle,
 //     together with their scale tiles; about 100 KB per SM are in flight.
-//   * 16 decode warps (four per TMEM lane quarter) each take every fourth 64-wide
-//     k-chunk: one weight row per thread, its 32 or 64 code bytes read from the
+//   * 16 decode warps (four per TMEM lane quarter) each take every fourth 128-wide
+//     k-chunk: one weight row per thread, its 64 or 128 code bytes read from the
 //     swizzled tile without bank conflicts, decoded to bf16 in registers and
-//     written with tcgen05.st into a ring of 32-column A slots in tensor memory
-//     (12 to 15 slots, all of TMEM the accumulator does not use).
+//     written with tcgen05.st into a ring of 64-column A slots in tensor memory
+//     (4 to 7 slots, all of TMEM the accumulators do not use).
 //   * Two threads issue tcgen05.mma (kind::f16, A = 128 weight rows from TMEM,
 //     B = the M tokens of X' from a shared-memory TMA ring, N = M rounded up to 16),
 //     the even chunks into one accumulator and the odd ones into another, and
@@ -36,7 +36,7 @@
 //   warp 0        TMA producer of code + scale tiles
 //   warps 1, 19   MMA issuers (even / odd chunks into accumulators 0 / 1); warp 1 also
 //                 allocates TMEM
-//   warps 2..17   decode (chunk j goes to the warps with (j mod 4) == (warp - 2) / 4),
+//   warps 2..17   decode (128-wide chunk j goes to the warps with (j mod 4) == (warp - 2) / 4),
 //                 then the epilogue of the unit
 //   warp 18       TMA producer of X' tiles (apart from the codes, so the code ring runs
 //                 as far ahead as its stages allow)
@@ -57,7 +57,7 @@ constexpr int MAX_TOKENS = 128;         // MMA N = tokens rounded up to 16
 constexpr int SC = 6;                   // code stages
 constexpr int CODE_BYTES = WM * 128;    // one code tile: 128 rows x 128 bytes, 128B swizzle
 constexpr int SCALE_STAGE = 2304;       // INT4: <= 8 x 128 bf16; MXFP4: 8 x 144 e8m0
-constexpr int MAX_SX = 12;              // X' stages (64 k each)
+constexpr int MAX_SX = 12;              // X' stages (128 k each)
 constexpr int NUM_THREADS = 640;
 constexpr int X_WARP = 18;              // the X' producer
 constexpr int MMA_WARP2 = 19;           // the second MMA issuer
@@ -91,16 +91,22 @@ struct Params {
   Group groups[MAX_GROUPS];
 };
 
-// k elements per code tile row (128 bytes) and 64-wide chunks per tile
+// k elements per code tile row (128 bytes); a chunk (one A slot, one X' stage, one
+// MMA hand-off) is KC = 128 of them: the fixed cost of each hand-off (barriers,
+// tensor-memory stores, commits) is paid once per 128 x 128 weight elements
+constexpr int KC = 128;
 template <int FMT>
 __host__ __device__ constexpr int kb_elems() { return FMT == kFp8 ? 128 : 256; }
 template <int FMT>
-__host__ __device__ constexpr int chunks_per_kb() { return kb_elems<FMT>() / 64; }
+__host__ __device__ constexpr int chunks_per_kb() { return kb_elems<FMT>() / KC; }
+
+// one X' stage: two 64-column boxes of MN rows
+__host__ __device__ inline size_t x_stage_bytes(int MN) { return static_cast<size_t>(MN) * 128 * 2; }
 
 // dynamic shared memory: alignment slack, code + scale stages (padded to 1 KB), X' stages, barriers
 __host__ __device__ inline size_t smem_bytes(int MN, int sx) {
   const size_t cs = (static_cast<size_t>(SC) * (CODE_BYTES + SCALE_STAGE) + 1023) / 1024 * 1024;
-  return 1024 + cs + static_cast<size_t>(sx) * MN * 128 + 1024;
+  return 1024 + cs + static_cast<size_t>(sx) * x_stage_bytes(MN) + 1024;
 }
 
 __device__ __forceinline__ void unit_of(const Params& p, int u, int& g, int& tile, int& s) {
@@ -117,12 +123,12 @@ __device__ __forceinline__ void split_range(const Params& p, int s, int& kb0, in
   kb1 = static_cast<int>((static_cast<long long>(s + 1) * p.nkb) / p.splits);
 }
 
-// 64-wide chunks of k-blocks [kb0, kb1): the last block may be partial along K
+// KC-wide chunks of k-blocks [kb0, kb1): the last block may be partial along K
 template <int FMT>
 __device__ __forceinline__ int chunks_in(const Params& p, int kb0, int kb1) {
   const int k0 = kb0 * kb_elems<FMT>();
   const int k1 = min(p.K, kb1 * kb_elems<FMT>());
-  return k1 > k0 ? (k1 - k0 + 63) / 64 : 0;
+  return k1 > k0 ? (k1 - k0 + KC - 1) / KC : 0;
 }
 
 // One 64-wide chunk of one weight row -> 32 bf16x2 words (element 2i in the low half of word i).
@@ -160,12 +166,10 @@ __device__ __forceinline__ void decode_chunk(const uint8_t* crow, int r, int c, 
         }
       } else {
         const uint32_t e = srow_base[(2 * c + h) * 144 + srem + r];  // [32-group][144] e8m0
+        uint32_t t[16];
+        dq::mxfp4x32_mul(ws, e, t);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          uint32_t t[4];
-          dq::mxfp4x8_mul(ws[i], e, t);
-          o[16 * h + 4 * i] = t[0], o[16 * h + 4 * i + 1] = t[1], o[16 * h + 4 * i + 2] = t[2], o[16 * h + 4 * i + 3] = t[3];
-        }
+        for (int i = 0; i < 16; ++i) o[16 * h + i] = t[i];
       }
     }
   }
@@ -197,15 +201,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_sm_kernel(const __grid_co
   uint8_t* sC = smem;
   uint8_t* sS = sC + SC * CODE_BYTES;
   uint8_t* sX = smem + (static_cast<size_t>(SC) * (CODE_BYTES + SCALE_STAGE) + 1023) / 1024 * 1024;
-  const int XB = p.MN * 128;           // one X' stage
+  const int XB = static_cast<int>(x_stage_bytes(p.MN));  // one X' stage (two boxes)
+  const int XH = XB / 2;                                  // one box
   uint64_t* bars = reinterpret_cast<uint64_t*>(sX + p.sx * XB);
   uint64_t* c_full = bars;
   uint64_t* c_empty = c_full + SC;
   uint64_t* x_full = c_empty + SC;
-  uint64_t* x_empty = x_full + MAX_SX;
-  uint64_t* a_full = x_empty + MAX_SX;  // up to 15 A slots
-  uint64_t* a_empty = a_full + 16;
-  uint64_t* acc_full = a_empty + 16;     // one per accumulator
+  uint64_t* chunk_empty = x_full + MAX_SX;
+  uint64_t* a_full = chunk_empty + MAX_SX;  // up to 12 slots
+  uint64_t* acc_full = a_full + MAX_SX;  // one per accumulator
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* drain = acc_empty + 1;       // one per issuer
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
@@ -214,7 +218,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_sm_kernel(const __grid_co
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
   const int AC = (p.MN + 31) / 32 * 32;          // columns of each of the two accumulators
-  const int NS = min(15, (512 - 2 * AC) / 32);   // A slots after them
+  // One ring of chunk slots: slot s is A slot s in TMEM (64 columns after the
+  // accumulators, KC bf16 each) and X' stage s in shared memory, released together by
+  // one tcgen05.commit on chunk_empty[s] after the chunk's MMAs.
+  const int NS = min(p.sx, min(15, (512 - 2 * AC) / 64));
   const uint32_t A_COL0 = static_cast<uint32_t>(2 * AC);
 
   if (threadIdx.x == 0) {
@@ -224,11 +231,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_sm_kernel(const __grid_co
     }
     for (int s = 0; s < MAX_SX; ++s) {
       mbar_init(&x_full[s], 1);
-      mbar_init(&x_empty[s], 1);
-    }
-    for (int s = 0; s < 16; ++s) {
+      mbar_init(&chunk_empty[s], 1);
       mbar_init(&a_full[s], 4);
-      mbar_init(&a_empty[s], 1);
     }
     mbar_init(&acc_full[0], 1);
     mbar_init(&acc_full[1], 1);
@@ -312,19 +316,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_sm_kernel(const __grid_co
         const int nch = chunks_in<FMT>(p, kb0, kb1);
         const int k0 = kb0 * kb_elems<FMT>();
         for (int j = 0; j < nch; ++j) {
-          if (!mbar_wait_sleep(&x_empty[xs], ph ^ 1u, abort_flag, kErrWaitEmpty)) {
+          if (!mbar_wait_sleep(&chunk_empty[xs], ph ^ 1u, abort_flag, kErrWaitEmpty)) {
             ok = false;
             break;
           }
           mbar_arrive_expect_tx(&x_full[xs], static_cast<uint32_t>(XB));
-          tma_load_2d(sX + xs * XB, &p.tmX, &x_full[xs], k0 + j * 64, p.groups[g].b_row0);
+          tma_load_2d(sX + xs * XB, &p.tmX, &x_full[xs], k0 + j * KC, p.groups[g].b_row0);
+          tma_load_2d(sX + xs * XB + XH, &p.tmX, &x_full[xs], k0 + j * KC + 64, p.groups[g].b_row0);
           ++issued;
-          ring_next(xs, ph, p.sx);
+          ring_next(xs, ph, NS);
         }
       }
       if (*abort_flag)
-        for (int i = (issued > p.sx ? issued - p.sx : 0); i < issued; ++i)
-          gemm_drain_wait(&x_full[i % p.sx], static_cast<uint32_t>((i / p.sx) & 1));
+        for (int i = (issued > NS ? issued - NS : 0); i < issued; ++i)
+          gemm_drain_wait(&x_full[i % NS], static_cast<uint32_t>((i / NS) & 1));
     }
   } else if (warp == 1 || warp == MMA_WARP2) {
     // ---------------- MMA issuers ----------------
@@ -336,8 +341,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_sm_kernel(const __grid_co
       const int h = warp == 1 ? 0 : 1;
       const uint32_t d_acc = tmem + static_cast<uint32_t>(h * AC);
       const uint32_t idesc = idesc_bf16_f32(WM, p.MN);
-      int sl = 0, xs = 0;
-      uint32_t aph = 0, xph = 0;
+      int sl = 0;  // chunk slot: A slot and X' stage
+      uint32_t aph = 0;
       bool ok = true;
       for (int i = 0; i < nu && ok; ++i) {
         int g, tile, s, kb0, kb1;
@@ -352,21 +357,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_sm_kernel(const __grid_co
         for (int j = 0; j < nch; ++j) {
           if ((j & 1) == h) {
             if (!mbar_wait_sleep(&a_full[sl], aph, abort_flag, kErrWaitDequant, 2000u) ||
-                !mbar_wait_sleep(&x_full[xs], xph, abort_flag, kErrWaitFull, 2000u)) {
+                !mbar_wait_sleep(&x_full[sl], aph, abort_flag, kErrWaitFull, 2000u)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint32_t a0 = tmem + A_COL0 + static_cast<uint32_t>(sl * 32);
-            const uint64_t b0 = sdesc_sw128(smem_u32(sX + xs * XB), 16, 1024);
+            const uint32_t a0 = tmem + A_COL0 + static_cast<uint32_t>(sl * 64);
+            const uint64_t b0 = sdesc_sw128(smem_u32(sX + sl * XB), 16, 1024);
+            const uint64_t b1 = sdesc_sw128(smem_u32(sX + sl * XB + XH), 16, 1024);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)  // +32 bytes along K per 16 elements: +2 in the descriptor's address field
-              mma_bf16_ts(d_acc, a0 + kk * 8, b0 + static_cast<uint64_t>(2 * kk), idesc, (j >= 2 || kk) ? 1u : 0u);
-            mma_commit(&a_empty[sl]);
-            mma_commit(&x_empty[xs]);
+            for (int kk = 0; kk < 8; ++kk)  // +32 bytes along K per 16 elements: +2 in the descriptor's address field
+              mma_bf16_ts(d_acc, a0 + kk * 8, (kk < 4 ? b0 : b1) + static_cast<uint64_t>(2 * (kk & 3)), idesc,
+                          (j >= 2 || kk) ? 1u : 0u);
+            mma_commit(&chunk_empty[sl]);
           }
           ring_next(sl, aph, NS);
-          ring_next(xs, xph, p.sx);
         }
         if (!ok) break;
         // (an accumulator that took no chunk -- nch <= h -- is committed unwritten: the
@@ -413,17 +418,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_sm_kernel(const __grid_co
             }
             mbar_try_wait(smem_u32(&c_full[cst]), cph);  // every lane acquires the tile
             if (real) {
+              // two 64-wide halves: decode, store into the slot's 32-column halves
+              const uint8_t* crow = sC + cst * CODE_BYTES + r * 128;
+              const uint8_t* srow = sS + cst * SCALE_STAGE;
               uint32_t o[32];
-              decode_chunk<FMT>(sC + cst * CODE_BYTES + r * 128, r, c, sS + cst * SCALE_STAGE, srem, p.group,
-                                fp8_scale, o);
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&c_empty[cst]);
-              if (!warp_wait_bounded_sleep(&a_empty[sl], aph ^ 1u, abort_flag, kErrWaitEmpty)) {
+              decode_chunk<FMT>(crow, r, 2 * c, srow, srem, p.group, fp8_scale, o);
+              if (!warp_wait_bounded_sleep(&chunk_empty[sl], aph ^ 1u, abort_flag, kErrWaitEmpty)) {
                 ok = false;
                 break;
               }
               tc_fence_after();
-              tmem_st_32x32b_x32(tmem + trow + A_COL0 + static_cast<uint32_t>(sl * 32), o);
+              tmem_st_32x32b_x32(tmem + trow + A_COL0 + static_cast<uint32_t>(sl * 64), o);
+              decode_chunk<FMT>(crow, r, 2 * c + 1, srow, srem, p.group, fp8_scale, o);
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&c_empty[cst]);
+              tmem_st_32x32b_x32(tmem + trow + A_COL0 + static_cast<uint32_t>(sl * 64 + 32), o);
               tmem_st_wait();
               tc_fence_before();
               __syncwarp();

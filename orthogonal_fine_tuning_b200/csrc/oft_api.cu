@@ -983,7 +983,7 @@ int launch_gemm_small(const oft_weight* W, const oft_split* S, int M, const uint
   prm->total_tiles = pl.tiles;
   prm->units = pl.tiles * pl.splits;
   const size_t base = gsm::smem_bytes(pl.MN, 0);
-  prm->sx = static_cast<int>(std::min<size_t>(gsm::MAX_SX, (227ull * 1024 - base) / (pl.MN * 128ull)));
+  prm->sx = static_cast<int>(std::min<size_t>(gsm::MAX_SX, (227ull * 1024 - base) / gsm::x_stage_bytes(pl.MN)));
   prm->num_groups = P;
   int off = 0, tile0 = 0;
   for (int p = 0; p < P; ++p) {

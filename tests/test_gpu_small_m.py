@@ -71,15 +71,22 @@ def test_small_m_token_counts(oft, M, fmt, group):
     assert rel_err(f64(Y), OracleLinear(case).fwd()) < TOL
 
 
-@pytest.mark.parametrize("fmt,group,K", [("int4", 32, 352), ("int4", 128, 512), ("fp8", 0, 320), ("mxfp4", 32, 512)])
-def test_small_m_decode_exact(oft, fmt, group, K):
+@pytest.mark.parametrize("fmt,group,K,extreme", [("int4", 32, 352, False), ("int4", 128, 512, False),
+                                                 ("fp8", 0, 320, False), ("mxfp4", 32, 512, False),
+                                                 ("mxfp4", 32, 768, True)])
+def test_small_m_decode_exact(oft, fmt, group, K, extreme):
     """One-hot tokens with Q = 0 (R = I exactly): token m selects input feature k_m, so
     Y[m][n] = deq(W)[n][k_m] -- a single product 1 * w summed with exact zeros, split-K
-    partials included.  Every k of the reduction is covered by windows of 64 tokens."""
+    partials included.  Every k of the reduction is covered by windows of 64 tokens.
+    The extreme case draws e8m0 exponents over 2..252, so both the one-step and the
+    two-step scale factors of the MXFP4 decode are exercised."""
     splits = (264, 136)
     N = sum(splits)
     spec = LinearSpec("ex", M=64, K=K, splits=splits, fmt=fmt, group=group, b=32, q_sigma=0.0, seed=K + N)
     case = make_linear_case(spec, q_zero=True)
+    if extreme:
+        g = torch.Generator().manual_seed(K)
+        case["scales"] = torch.randint(2, 253, case["scales"].shape, generator=g).to(torch.uint8)
     c = linear_np(case)
     ref = codecs.dequant(fmt, c["codes"], c["scales"], K, group)     # float64 [N][K]
     W = device_weight(case, "cuda")

@@ -304,16 +304,19 @@ __global__ void __launch_bounds__(kMoeRotThreads, 4) moe_rot_tc_kernel(
   int cur_e = -1, cur_g = -1, pf_e = -1, pf_g = -1, a = 0, a1 = 0, a2 = 0, ab = 0;
   uint32_t phase = 0;
   uint4 xv[NIT];
-  int tok1[NIT], tok2[NIT];
+  // token ids of the unit after next go to one of two buffers by unit parity (the loop
+  // below is unrolled by two), so no instruction waits on loads still in flight
+  int tokE[NIT], tokO[NIT];
   if (ubeg < uend) {
     const Unit u0 = unit_at(ubeg, a1);
-    load_tokens(u0, true, tok1);
-    load_rows(u0, tok1, xv);
+    load_tokens(u0, true, tokE);
+    load_rows(u0, tokE, xv);
     const bool v1 = ubeg + 1 < uend;
-    load_tokens(v1 ? unit_at(ubeg + 1, a2) : u0, v1, tok1);
+    load_tokens(v1 ? unit_at(ubeg + 1, a2) : u0, v1, tokO);
   }
   a1 = a2;
-  for (int u = ubeg; u < uend; ++u) {
+  // one unit: tok_next holds the token ids of unit u + 1; unit u + 2's are loaded into tok_dst
+  auto run_unit = [&](int u, const int (&tok_next)[NIT], int (&tok_dst)[NIT]) -> bool {
     const Unit U = unit_at(u, a);
     const int e = U.e, g = U.g, pos0 = U.pos0, nrows = U.nrows;
     // 1. rotation tiles of (e, g), when they change (fetched during the previous unit's
@@ -345,15 +348,13 @@ __global__ void __launch_bounds__(kMoeRotThreads, 4) moe_rot_tc_kernel(
       }
       mma_commit(bar);
     }
-    // prefetch: unit u+1's rows (their token ids are already in tok1), unit u+2's token ids
+    // prefetch: unit u+1's rows (their token ids are already in tok_next), unit u+2's token ids
     if (u + 1 < uend) {
-      load_rows(unit_at(u + 1, a1), tok1, xv);
+      load_rows(unit_at(u + 1, a1), tok_next, xv);
       const bool v2 = u + 2 < uend;
-      load_tokens(v2 ? unit_at(u + 2, a2) : U, v2, tok2);
-#pragma unroll
-      for (int q = 0; q < NIT; ++q) tok1[q] = tok2[q];
+      load_tokens(v2 ? unit_at(u + 2, a2) : U, v2, tok_dst);
     }
-    if (!warp_wait_bounded(bar, phase, abort_flag, kErrWaitAccFull)) break;
+    if (!warp_wait_bounded(bar, phase, abort_flag, kErrWaitAccFull)) return false;
     phase ^= 1;
     tc_fence_after();
     // the product has read the B tiles: start the next unit's, if they differ
@@ -390,6 +391,11 @@ __global__ void __launch_bounds__(kMoeRotThreads, 4) moe_rot_tc_kernel(
     }
     tc_fence_before();
     __syncthreads();  // TMEM and the shared tiles are free for the next unit
+    return true;
+  };
+  for (int u = ubeg; u < uend; u += 2) {
+    if (!run_unit(u, tokO, tokE)) break;
+    if (u + 1 < uend && !run_unit(u + 1, tokE, tokO)) break;
   }
   __syncthreads();
   if (warp == 1) {

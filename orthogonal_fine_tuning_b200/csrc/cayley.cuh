@@ -383,12 +383,16 @@ __global__ void __launch_bounds__(TPR * B) cayley_fwd_split_kernel(const uint16_
 // dQ[blk] = pack(D - D^T), D = 1/2 (I+R)^T G (I+R)^T.
 // G is read either directly ([nblocks][b][b], nparts = 1) or as `nparts` partial
 // sums laid out [nblocks][nparts][b][b], summed in part order (deterministic).
+// With a map (the MoE's active experts), only the blocks map[i] * per + r for
+// i < *n_map and r < per are computed; the others are left as they are.
 // One CTA per block; each thread owns a TI x TI tile of the two b x b products.
 // Dynamic shared memory: 3 * B * (B + 1) floats.
 template <int B>
 __global__ void __launch_bounds__(kCayleyThreads) cayley_bwd_kernel(const float* __restrict__ R,
                                                                     const float* __restrict__ G, int nparts,
-                                                                    int nblocks, float* __restrict__ dQ) {
+                                                                    int nblocks, float* __restrict__ dQ,
+                                                                    const int* __restrict__ map,
+                                                                    const int* __restrict__ n_map, int per) {
   constexpr int TI = (B == 64) ? 4 : (B == 32 ? 2 : 1);
   constexpr int NT = B / TI;  // threads per output row of tiles
   static_assert(NT * NT == kCayleyThreads, "tile grid must cover the CTA");
@@ -400,7 +404,9 @@ __global__ void __launch_bounds__(kCayleyThreads) cayley_bwd_kernel(const float*
   const int tid = threadIdx.x;
   const int ti = (tid / NT) * TI, tj = (tid % NT) * TI;
   pdl_wait();
-  for (int blk = blockIdx.x; blk < nblocks; blk += gridDim.x) {
+  const int count = map != nullptr ? *n_map * per : nblocks;
+  for (int it = blockIdx.x; it < count; it += gridDim.x) {
+    const int blk = map != nullptr ? map[it / per] * per + it % per : it;
     const float* rb = R + static_cast<size_t>(blk) * B * B;
     const float* gb = G + static_cast<size_t>(blk) * nparts * B * B;
     constexpr int EPT = B * B / kCayleyThreads;  // elements per thread

@@ -491,4 +491,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// fp32 -> the nearest tf32 value (ties away from zero), held in an fp32 register.  A
+// kind::tf32 MMA reads only the top 19 bits of each operand (truncation, a bias of
+// half a tf32 ulp on average); operands rounded here first lose nothing more.
+__device__ __forceinline__ float tf32_rn(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+
 }  // namespace oftk

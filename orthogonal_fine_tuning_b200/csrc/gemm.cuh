@@ -173,7 +173,9 @@ __device__ __forceinline__ uint32_t pack2(uint32_t lo, uint32_t hi) {
 // Epilogue of one warp: the 32 accumulator lanes at `tacc` are rows row0 + lane of group
 // G (row0 relative to the group), columns nt * BN + [0, BN).  bf16 rows are stored
 // directly; fp32 goes through the warp's 32 x 32 staging block `stg`, so every store
-// instruction writes four full 128-byte row segments.
+// instruction writes four full 128-byte row segments.  fp32 outputs (dX', the MoE's
+// D) are only ever read as tf32 MMA operands, so they are stored rounded to the
+// nearest tf32 value.
 __device__ __forceinline__ void store_rows(const Params& p, const Group& G, int row0, int nt, uint32_t tacc, float* stg,
                                            int lane) {
   const int row = row0 + lane;
@@ -188,7 +190,7 @@ __device__ __forceinline__ void store_rows(const Params& p, const Group& G, int 
     const int col = nt * BN + c;
     if (p.c_f32) {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) stg[lane * EPI_LD + j] = __uint_as_float(r[j]);
+      for (int j = 0; j < 32; ++j) stg[lane * EPI_LD + j] = tf32_rn(__uint_as_float(r[j]));
       __syncwarp();
       const int c4 = (lane & 7) * 4;
 #pragma unroll

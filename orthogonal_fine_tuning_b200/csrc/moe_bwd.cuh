@@ -17,7 +17,8 @@
 // selected logits, dlogit[t, e_k] = w_tk (dw_tk - sum_j w_tj dw_tj).
 //
 // Everything below works in bucket order (positions sorted by expert, stable in
-// (t, k)), the order the forward's grouped GEMM uses.
+// (t, k)), the order the forward's grouped GEMM uses.  The rotations back, G and
+// the Cayley backward run on the tensor cores in moe_bwd_tc.cuh.
 #pragma once
 
 #include "cayley.cuh"
@@ -113,11 +114,11 @@ __global__ void __launch_bounds__(256) moe_chunk_dequant_t_kernel(WeightView ban
 }
 
 // Active experts ordered by bucket size, largest first (ties: lower id first),
-// so that the per-(expert, block) units below start with the longest ones; also
-// resets the units' work counter.  One CTA; n_active <= E <= kMaxExperts.
+// so that the per-(expert, column group) units of the backward's rotation kernels
+// (moe_bwd_tc.cuh) start with the longest ones.  One CTA; n_active <= E <= kMaxExperts.
 __global__ void __launch_bounds__(1024) moe_order_kernel(const int* __restrict__ offsets,
                                                          const int* __restrict__ active, const int* __restrict__ n_active,
-                                                         int* __restrict__ order, int* __restrict__ counter) {
+                                                         int* __restrict__ order) {
   __shared__ int cnt[kMaxExperts];
   const int na = *n_active;
   for (int a = threadIdx.x; a < na; a += 1024) cnt[a] = offsets[active[a] + 1] - offsets[active[a]];
@@ -126,279 +127,6 @@ __global__ void __launch_bounds__(1024) moe_order_kernel(const int* __restrict__
     int rank = 0;
     for (int b = 0; b < na; ++b) rank += (cnt[b] > cnt[a]) || (cnt[b] == cnt[a] && b < a);
     order[rank] = active[a];
-  }
-  if (threadIdx.x == 0) *counter = 0;
-}
-
-template <int B>
-struct MoeBwdCfg {
-  static constexpr int PT = 2048 / B;   // positions per tile (128 U threads x 4 positions x 4 columns)
-  static constexpr int LDT = PT + 4;    // transposed tile rows [column][position] (float4-aligned)
-  static constexpr int LDR = B + 4;     // rows of the stacked [R_gate^T; R_up^T]
-  static constexpr int GI = B / 16, GJ = B / 8;  // G thread tile: rows gi + 16 ii, columns gj + 8 jj
-  static constexpr int LDC = B + 1;     // Cayley scratch rows
-  static constexpr int TILE_FLOATS = 3 * B * LDT + PT;  // D_gate^T, D_up^T, X^T, w
-  static constexpr int SCRATCH_FLOATS = 2 * B * LDC;    // G, then T G
-  static constexpr int REGION = TILE_FLOATS > SCRATCH_FLOATS ? TILE_FLOATS : SCRATCH_FLOATS;
-  static constexpr size_t SMEM = sizeof(float) * (2 * B * LDR + REGION);
-  static constexpr int TI = (B == 64) ? 4 : (B == 32 ? 2 : 1);  // Cayley thread tile
-  static constexpr int NT = B / TI;
-  static constexpr int D_VEC = 2 * PT * (B / 4) / 256;  // float4 of D per thread and tile
-  static constexpr int X_VEC = PT * (B / 8) / 256;      // 8 x bf16 of X per thread and tile
-  static_assert(D_VEC * 256 == 2 * PT * (B / 4) && X_VEC * 256 == PT * (B / 8), "tile loads must cover the CTA");
-};
-
-// Position swizzle of the transposed tiles: element (row, pos) lives at
-// row * LDT + (pos ^ moe_swz(row)).  XOR with a multiple of 4 keeps every aligned
-// group of four positions together (float4 reads stay whole), and it spreads the
-// transposing stores over all banks; the G and U reads stay conflict-free.
-__device__ __forceinline__ int moe_swz(int row) { return ((row >> 3) & 7) << 2; }
-
-// One unit = (active expert e, rotation block blk), taken heaviest expert first
-// from a work counter.  The unit walks e's bucket range in tiles of PT positions,
-// staged transposed in shared memory (the next tile's loads are in flight, in
-// registers, while the current one is computed):
-//   warps 0-3:  U[pos][blk]   = sum_p D_p[pos][blk] R_e,p,blk^T    -> U (fp32, bucket order)
-//               dwp[pos][blk] = <U[pos][blk], X[t][blk]>            (partial of dw over blocks)
-//   warps 4-7:  G_p          += X[t][blk]^T (w D_p[pos][blk])       (registers)
-// and finally all warps run the Cayley backward of G_gate, G_up -> dq_e,p,blk.
-// D is fp32 [2][TK][K]; R fp32 [E][2][nb][B][B]; dQ fp32 [E][2][nb][B(B-1)/2].
-template <int B>
-__global__ void __launch_bounds__(256, (B == 64 ? 2 : 3)) moe_bwd_rot_kernel(const float* __restrict__ D, const uint16_t* __restrict__ X,
-                                                          int K, int TK, int top_k, const int* __restrict__ bucket,
-                                                          const int* __restrict__ offsets, const float* __restrict__ topk_w,
-                                                          const int* __restrict__ order,
-                                                          const int* __restrict__ n_active, int* __restrict__ counter,
-                                                          const float* __restrict__ R, float* __restrict__ U,
-                                                          float* __restrict__ dwp, float* __restrict__ dQ) {
-  using C = MoeBwdCfg<B>;
-  constexpr int PT = C::PT, LDT = C::LDT, LDR = C::LDR, GI = C::GI, GJ = C::GJ, LDC = C::LDC, TI = C::TI, NT = C::NT;
-  constexpr int D_VEC = C::D_VEC, X_VEC = C::X_VEC;
-  extern __shared__ float4 msm4[];
-  float* sm = reinterpret_cast<float*>(msm4);
-  float* Rc = sm;                   // [2B][LDR]: row p*B + i holds column i of R_p (R_p^T), later (I + R_p)^T
-  float* region = sm + 2 * B * LDR;
-  float* Dt = region;               // [2][B][LDT]
-  float* Xt = region + 2 * B * LDT;  // [B][LDT]
-  float* ws = region + 3 * B * LDT;  // [PT]
-  float* Gs = region;               // [B][LDC]  (after the tile loop)
-  float* Us = region + B * LDC;     // [B][LDC]
-  __shared__ int s_unit;
-  const int tid = threadIdx.x, warp = tid / 32;
-  const int nb = K / B;
-  const int total = *n_active * nb;
-  const int ti = (tid / NT) * TI, tj = (tid % NT) * TI;
-  for (;;) {
-    if (tid == 0) s_unit = atomicAdd(counter, 1);
-    __syncthreads();
-    const int u = s_unit;
-    if (u >= total) break;
-    const int e = order[u / nb], blk = u % nb;
-    const int o0 = offsets[e], o1 = offsets[e + 1];
-    for (int idx = tid; idx < 2 * B * B; idx += 256) {
-      const int p = idx / (B * B), r = (idx / B) % B, c = idx % B;  // R_p[r][c]
-      Rc[(p * B + c) * LDR + r] = R[((static_cast<size_t>(e) * 2 + p) * nb + blk) * B * B + r * B + c];
-    }
-    // tile loads into registers (zeros past the end of e's range)
-    float4 dreg[D_VEC];
-    uint4 xreg[X_VEC];
-    float wreg = 0.f;
-    auto fetch = [&](int t0) {
-      const int np = min(PT, o1 - t0);
-#pragma unroll
-      for (int v = 0; v < D_VEC; ++v) {
-        const int it = tid + 256 * v;
-        const int p = it / (PT * (B / 4)), rem = it % (PT * (B / 4));
-        const int r = rem / (B / 4), c4 = (rem % (B / 4)) * 4;
-        dreg[v] = r < np ? *reinterpret_cast<const float4*>(D + (static_cast<size_t>(p) * TK + t0 + r) * K + blk * B + c4)
-                         : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-      for (int v = 0; v < X_VEC; ++v) {
-        const int it = tid + 256 * v;
-        const int r = it / (B / 8), c8 = (it % (B / 8)) * 8;
-        xreg[v] = r < np ? *reinterpret_cast<const uint4*>(X + static_cast<size_t>(bucket[t0 + r] / top_k) * K + blk * B + c8)
-                         : make_uint4(0u, 0u, 0u, 0u);
-      }
-      if (tid < PT) wreg = tid < np ? topk_w[bucket[t0 + tid]] : 0.f;
-    };
-    auto stage = [&]() {
-#pragma unroll
-      for (int v = 0; v < D_VEC; ++v) {
-        const int it = tid + 256 * v;
-        const int p = it / (PT * (B / 4)), rem = it % (PT * (B / 4));
-        const int r = rem / (B / 4), c4 = (rem % (B / 4)) * 4;
-        const int row = p * B + c4;
-        Dt[row * LDT + (r ^ moe_swz(row))] = dreg[v].x;
-        Dt[(row + 1) * LDT + (r ^ moe_swz(row + 1))] = dreg[v].y;
-        Dt[(row + 2) * LDT + (r ^ moe_swz(row + 2))] = dreg[v].z;
-        Dt[(row + 3) * LDT + (r ^ moe_swz(row + 3))] = dreg[v].w;
-      }
-#pragma unroll
-      for (int v = 0; v < X_VEC; ++v) {
-        const int it = tid + 256 * v;
-        const int r = it / (B / 8), c8 = (it % (B / 8)) * 8;
-        const uint32_t q[4] = {xreg[v].x, xreg[v].y, xreg[v].z, xreg[v].w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int row = c8 + 2 * i;
-          Xt[row * LDT + (r ^ moe_swz(row))] = __uint_as_float(q[i] << 16);
-          Xt[(row + 1) * LDT + (r ^ moe_swz(row + 1))] = __uint_as_float(q[i] & 0xFFFF0000u);
-        }
-      }
-      if (tid < PT) ws[tid] = wreg;
-    };
-    float g[2][GI][GJ];
-#pragma unroll
-    for (int p = 0; p < 2; ++p)
-#pragma unroll
-      for (int ii = 0; ii < GI; ++ii)
-#pragma unroll
-        for (int jj = 0; jj < GJ; ++jj) g[p][ii][jj] = 0.f;
-    fetch(o0);
-    for (int t0 = o0; t0 < o1; t0 += PT) {
-      const int np = min(PT, o1 - t0);
-      __syncthreads();  // previous tile consumed (and R^T written, on the first tile)
-      stage();
-      __syncthreads();
-      if (t0 + PT < o1) fetch(t0 + PT);
-      if (warp < 4) {
-        // U: 4 positions x 4 columns per thread, and the partial dw of this block
-        const int jg = tid % (B / 4), pos0 = (tid / (B / 4)) * 4;
-        float acc[4][4];
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) acc[a][c] = 0.f;
-        float s[4] = {0.f, 0.f, 0.f, 0.f};
-        if (pos0 < np) {
-#pragma unroll 8
-          for (int i2 = 0; i2 < 2 * B; ++i2) {
-            const float4 dv = *reinterpret_cast<const float4*>(Dt + i2 * LDT + (pos0 ^ moe_swz(i2)));
-            const float4 rv = *reinterpret_cast<const float4*>(Rc + i2 * LDR + jg * 4);
-            const float d4[4] = {dv.x, dv.y, dv.z, dv.w}, r4[4] = {rv.x, rv.y, rv.z, rv.w};
-#pragma unroll
-            for (int a = 0; a < 4; ++a)
-#pragma unroll
-              for (int c = 0; c < 4; ++c) acc[a][c] = fmaf(d4[a], r4[c], acc[a][c]);
-          }
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const int row = jg * 4 + c;
-            const float4 xv = *reinterpret_cast<const float4*>(Xt + row * LDT + (pos0 ^ moe_swz(row)));
-            s[0] = fmaf(acc[0][c], xv.x, s[0]);
-            s[1] = fmaf(acc[1][c], xv.y, s[1]);
-            s[2] = fmaf(acc[2][c], xv.z, s[2]);
-            s[3] = fmaf(acc[3][c], xv.w, s[3]);
-          }
-        }
-#pragma unroll
-        for (int o = 1; o < B / 4; o <<= 1)
-#pragma unroll
-          for (int a = 0; a < 4; ++a) s[a] += __shfl_xor_sync(0xFFFFFFFFu, s[a], o);
-#pragma unroll
-        for (int a = 0; a < 4; ++a) {
-          if (pos0 + a < np) {
-            *reinterpret_cast<float4*>(U + static_cast<size_t>(t0 + pos0 + a) * K + blk * B + jg * 4) =
-                make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
-            if (jg == 0) dwp[static_cast<size_t>(t0 + pos0 + a) * nb + blk] = s[a];
-          }
-        }
-      } else {
-        // G_p += X^T (w D_p): rows gi + 16 ii, columns gj + 8 jj, four positions per step
-        const int gt = tid - 128, gj = gt % 8, gi = gt / 8;
-        for (int pos0 = 0; pos0 < np; pos0 += 4) {
-          const float4 w4 = *reinterpret_cast<const float4*>(ws + pos0);
-          float4 xv[GI];
-#pragma unroll
-          for (int ii = 0; ii < GI; ++ii) {
-            const int row = gi + 16 * ii;
-            const float4 x = *reinterpret_cast<const float4*>(Xt + row * LDT + (pos0 ^ moe_swz(row)));
-            xv[ii] = make_float4(x.x * w4.x, x.y * w4.y, x.z * w4.z, x.w * w4.w);
-          }
-#pragma unroll
-          for (int p = 0; p < 2; ++p)
-#pragma unroll
-            for (int jj = 0; jj < GJ; ++jj) {
-              const int row = p * B + gj + 8 * jj;
-              const float4 dv = *reinterpret_cast<const float4*>(Dt + row * LDT + (pos0 ^ moe_swz(row)));
-#pragma unroll
-              for (int ii = 0; ii < GI; ++ii) {
-                float a = g[p][ii][jj];
-                a = fmaf(xv[ii].x, dv.x, a);
-                a = fmaf(xv[ii].y, dv.y, a);
-                a = fmaf(xv[ii].z, dv.z, a);
-                a = fmaf(xv[ii].w, dv.w, a);
-                g[p][ii][jj] = a;
-              }
-            }
-        }
-      }
-    }
-    __syncthreads();  // tiles consumed: the region becomes Cayley scratch
-    for (int idx = tid; idx < 2 * B; idx += 256) Rc[(idx / B) * B * LDR + (idx % B) * (LDR + 1)] += 1.f;  // (I + R_p)^T
-#pragma unroll
-    for (int p = 0; p < 2; ++p) {
-      if (warp >= 4) {
-        const int gt = tid - 128, gj = gt % 8, gi = gt / 8;
-#pragma unroll
-        for (int ii = 0; ii < GI; ++ii)
-#pragma unroll
-          for (int jj = 0; jj < GJ; ++jj) Gs[(gi + 16 * ii) * LDC + gj + 8 * jj] = g[p][ii][jj];
-      }
-      __syncthreads();
-      const float* T = Rc + p * B * LDR;
-      float o[TI][TI];
-#pragma unroll
-      for (int x = 0; x < TI; ++x)
-#pragma unroll
-        for (int y = 0; y < TI; ++y) o[x][y] = 0.f;
-#pragma unroll 4
-      for (int l = 0; l < B; ++l) {  // U = T G
-        float tv[TI], gv[TI];
-#pragma unroll
-        for (int x = 0; x < TI; ++x) tv[x] = T[(ti + x) * LDR + l];
-#pragma unroll
-        for (int y = 0; y < TI; ++y) gv[y] = Gs[l * LDC + tj + y];
-#pragma unroll
-        for (int x = 0; x < TI; ++x)
-#pragma unroll
-          for (int y = 0; y < TI; ++y) o[x][y] = fmaf(tv[x], gv[y], o[x][y]);
-      }
-#pragma unroll
-      for (int x = 0; x < TI; ++x)
-#pragma unroll
-        for (int y = 0; y < TI; ++y) Us[(ti + x) * LDC + tj + y] = o[x][y];
-      __syncthreads();
-#pragma unroll
-      for (int x = 0; x < TI; ++x)
-#pragma unroll
-        for (int y = 0; y < TI; ++y) o[x][y] = 0.f;
-#pragma unroll 4
-      for (int l = 0; l < B; ++l) {  // 2 dQ_full = (T G) T
-        float uv[TI], tv[TI];
-#pragma unroll
-        for (int x = 0; x < TI; ++x) uv[x] = Us[(ti + x) * LDC + l];
-#pragma unroll
-        for (int y = 0; y < TI; ++y) tv[y] = T[l * LDR + tj + y];
-#pragma unroll
-        for (int x = 0; x < TI; ++x)
-#pragma unroll
-          for (int y = 0; y < TI; ++y) o[x][y] = fmaf(uv[x], tv[y], o[x][y]);
-      }
-      __syncthreads();  // every thread is done reading G before it is overwritten
-#pragma unroll
-      for (int x = 0; x < TI; ++x)
-#pragma unroll
-        for (int y = 0; y < TI; ++y) Gs[(ti + x) * LDC + tj + y] = o[x][y];
-      __syncthreads();
-      float* out = dQ + ((static_cast<size_t>(e) * 2 + p) * nb + blk) * (B * (B - 1) / 2);
-      for (int idx = tid; idx < B * B; idx += 256) {
-        const int i = idx / B, j = idx % B;
-        if (i < j) out[tri_index(i, j, B)] = 0.5f * (Gs[i * LDC + j] - Gs[j * LDC + i]);
-      }
-      __syncthreads();
-    }
   }
 }
 

@@ -29,6 +29,7 @@
 #include "gemm_sm.cuh"
 #include "moe_fused.cuh"
 #include "moe_bwd.cuh"
+#include "moe_bwd_tc.cuh"
 #include "moe_layer.cuh"
 
 using namespace oftk;
@@ -203,15 +204,15 @@ int make_map_bf16(CUtensorMap* m, const void* base, uint64_t inner, uint64_t out
   return OFT_OK;
 }
 
-// 3-D fp32 tensor [P][M][K] (dX'), box {32, 128, 1}; rows past M read as zero.  `swizzle` is the
+// 3-D fp32 tensor [P][M][K] (dX'), box {32, box_rows, 1}; rows past M read as zero.  `swizzle` is the
 // 128B swizzle (K-major operands) or its 32-byte-atom variant (MN-major tf32 operands).
 int make_map_f32_3d(CUtensorMap* m, const void* base, uint64_t K, uint64_t M, uint64_t P,
-                    CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
+                    CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B, uint32_t box_rows = 128) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return fail(OFT_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   cuuint64_t dims[3] = {K, M, P};
   cuuint64_t strides[2] = {K * 4, M * K * 4};
-  cuuint32_t box[3] = {32, 128, 1};
+  cuuint32_t box[3] = {32, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -357,16 +358,17 @@ int launch_cayley(const uint16_t* Q, int nblocks, int b, float* R, const int* ac
   return OFT_OK;
 }
 
-int launch_cayley_bwd(const float* R, const float* G, int nparts, int nblocks, int b, float* dQ, cudaStream_t st) {
+int launch_cayley_bwd(const float* R, const float* G, int nparts, int nblocks, int b, float* dQ, cudaStream_t st,
+                      const int* map = nullptr, const int* n_map = nullptr, int per = 1) {
   const size_t smem = 3ull * b * (b + 1) * sizeof(float);
   const int grid = std::min(nblocks, sm_count() * 8);
   if (b == 16) OFT_CUDA(cudaFuncSetAttribute(cayley_bwd_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   if (b == 32) OFT_CUDA(cudaFuncSetAttribute(cayley_bwd_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   if (b == 64) OFT_CUDA(cudaFuncSetAttribute(cayley_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   ProfScope ps(OFT_K_CAYLEY, st);
-  if (b == 16) OFT_CUDA(launch_pdl(cayley_bwd_kernel<16>, grid, kCayleyThreads, smem, st, R, G, nparts, nblocks, dQ));
-  if (b == 32) OFT_CUDA(launch_pdl(cayley_bwd_kernel<32>, grid, kCayleyThreads, smem, st, R, G, nparts, nblocks, dQ));
-  if (b == 64) OFT_CUDA(launch_pdl(cayley_bwd_kernel<64>, grid, kCayleyThreads, smem, st, R, G, nparts, nblocks, dQ));
+  if (b == 16) OFT_CUDA(launch_pdl(cayley_bwd_kernel<16>, grid, kCayleyThreads, smem, st, R, G, nparts, nblocks, dQ, map, n_map, per));
+  if (b == 32) OFT_CUDA(launch_pdl(cayley_bwd_kernel<32>, grid, kCayleyThreads, smem, st, R, G, nparts, nblocks, dQ, map, n_map, per));
+  if (b == 64) OFT_CUDA(launch_pdl(cayley_bwd_kernel<64>, grid, kCayleyThreads, smem, st, R, G, nparts, nblocks, dQ, map, n_map, per));
   OFT_LAUNCHED("cayley_bwd_kernel");
   return OFT_OK;
 }
@@ -1813,32 +1815,76 @@ MoeBwdLayout moe_bwd_layout(int T, int E, int top_k, int chunk, int K, int N, in
   L.offsets = round_up(L.w + 4 * TK, 256);
   L.bucket = round_up(L.offsets + 4ull * (E + 1), 256);
   L.table = round_up(L.bucket + 4 * TK, 256);
-  L.meta = round_up(L.table + 4 * n_chunks_max * chunk, 256);  // [0] n_active, [1] unit counter
+  L.meta = round_up(L.table + 4 * n_chunks_max * chunk, 256);  // n_active
   L.order = round_up(L.meta + 16, 256);
   L.inv = round_up(L.order + 4ull * E, 256);
   L.pexp = round_up(L.inv + 4 * TK, 256);
   L.rex = round_up(L.pexp + 4 * TK, 256);
   L.dyg = round_up(L.rex + 4ull * E * 2 * nb * b * b, 256);
   L.buf = round_up(L.dyg + 2 * 2 * TK * n, 256);
-  L.d = round_up(L.buf + 2ull * 2 * chunk * N * K, 256);  // two transposed chunk buffers
+  // two transposed chunk buffers; after the last chunk's GEMM the same bytes hold the
+  // active experts' adapter gradients G [E][2][nb][b][b]
+  L.d = round_up(L.buf + std::max(2ull * 2 * chunk * N * K, 4ull * E * 2 * nb * b * b), 256);
   L.u = round_up(L.d + 4 * 2 * TK * K, 256);
   L.dwp = round_up(L.u + 4 * TK * K, 256);
   L.total = round_up(L.dwp + 4 * TK * nb, 256);
   return L;
 }
 
-template <int B>
-int launch_moe_bwd_rot(const float* D, const uint16_t* X, int K, int TK, int top_k, const int* bucket,
-                       const int* offsets, const float* w, const int* order, const int* n_active, int* counter,
-                       const float* R, float* U, float* dwp, float* dQ, cudaStream_t st) {
-  constexpr size_t smem = MoeBwdCfg<B>::SMEM;
-  if (int rc = set_smem(moe_bwd_rot_kernel<B>, smem)) return rc;
-  int per_sm = 0;
-  OFT_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, moe_bwd_rot_kernel<B>, 256, smem));
-  moe_bwd_rot_kernel<B><<<sm_count() * std::max(1, per_sm), 256, smem, st>>>(D, X, K, TK, top_k, bucket, offsets, w,
-                                                                             order, n_active, counter, R, U, dwp, dQ);
-  OFT_LAUNCHED("moe_bwd_rot_kernel");
-  return OFT_OK;
+// Step 4 of the MoE backward on the tensor cores: U and the dw partials, each active
+// expert's adapter gradient G (into `G`, [E][2][nb][b][b]), then its Cayley backward.
+int launch_moe_bwd_tc(const float* D, const uint16_t* X, int K, int TK, int top_k, int E, int b, const int* bucket,
+                      const int* offsets, const float* w, const int* order, const int* n_active, const float* R,
+                      float* U, float* dwp, float* G, float* dQ, cudaStream_t st) {
+  const int nb = K / b;
+  {
+    rtc::MoeRotbParams prm;
+    memset(&prm, 0, sizeof(prm));
+    if (int rc = make_map_f32_3d(&prm.tmD, D, K, TK, 2)) return rc;
+    prm.R = R;
+    prm.X = X;
+    prm.bucket = bucket;
+    prm.offsets = offsets;
+    prm.order = order;
+    prm.n_active = n_active;
+    prm.U = U;
+    prm.dwp = dwp;
+    prm.K = K;
+    prm.TK = TK;
+    prm.top_k = top_k;
+    prm.b = b;
+    prm.nb = nb;
+    prm.groups = (K + 63) / 64;
+    if (int rc = set_smem(rtc::moe_rotb_tc_kernel, rtc::kMoeRotbSmem)) return rc;
+    const int grid = static_cast<int>(std::min<long long>(sm_count(), 1ll * E * prm.groups));
+    ProfScope ps(OFT_K_ROTATE, st);
+    OFT_CUDA(launch_pdl(rtc::moe_rotb_tc_kernel, grid, rtc::NUM_THREADS, rtc::kMoeRotbSmem, st, prm));
+    OFT_LAUNCHED("moe_rotb_tc_kernel");
+  }
+  {
+    rtc::MoeGradParams prm;
+    memset(&prm, 0, sizeof(prm));
+    if (int rc = make_map_f32_3d(&prm.tmD, D, K, TK, 2, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B, rtc::MG_TP)) return rc;
+    prm.X = X;
+    prm.bucket = bucket;
+    prm.w = w;
+    prm.offsets = offsets;
+    prm.order = order;
+    prm.n_active = n_active;
+    prm.G = G;
+    prm.K = K;
+    prm.TK = TK;
+    prm.top_k = top_k;
+    prm.b = b;
+    prm.nb = nb;
+    prm.groups = (K + 127) / 128;
+    if (int rc = set_smem(rtc::moe_grad_tc_kernel, rtc::kMoeGradSmem)) return rc;
+    const int grid = static_cast<int>(std::min<long long>(sm_count(), 1ll * E * prm.groups));
+    ProfScope ps(OFT_K_GRAD, st);
+    OFT_CUDA(launch_pdl(rtc::moe_grad_tc_kernel, grid, rtc::NUM_THREADS, rtc::kMoeGradSmem, st, prm));
+    OFT_LAUNCHED("moe_grad_tc_kernel");
+  }
+  return launch_cayley_bwd(R, G, 1, E * 2 * nb, b, dQ, st, order, n_active, 2 * nb);
 }
 }  // namespace
 
@@ -1880,7 +1926,6 @@ int moe_chunked_oft_bwd(const uint16_t* dY, const uint16_t* X, int T, const floa
   int* bucket = reinterpret_cast<int*>(wsb + L.bucket);
   int* table = reinterpret_cast<int*>(wsb + L.table);
   int* n_active = reinterpret_cast<int*>(wsb + L.meta);
-  int* counter = n_active + 1;
   int* order = reinterpret_cast<int*>(wsb + L.order);
   int* inv = reinterpret_cast<int*>(wsb + L.inv);
   int* pexp = reinterpret_cast<int*>(wsb + L.pexp);
@@ -1904,15 +1949,16 @@ int moe_chunked_oft_bwd(const uint16_t* dY, const uint16_t* X, int T, const floa
     moe_route_kernel<<<1, 1024, rsmem, st>>>(idx, TK, E, chunk, n_chunks_max, offsets, bucket, inv, pexp, table,
                                             n_active);
     OFT_LAUNCHED("moe_route_kernel");
-    moe_order_kernel<<<1, 1024, 0, st>>>(offsets, table, n_active, order, counter);
+    moe_order_kernel<<<1, 1024, 0, st>>>(offsets, table, n_active, order);
     OFT_LAUNCHED("moe_order_kernel");
     const long long gunits = 1ll * TK * (N / 8);
     moe_gather_dy_kernel<<<static_cast<int>(std::min<long long>((gunits + 255) / 256, 148ll * 16)), 256, 0, st>>>(
         dY, bucket, TK, top_k, n_proj, dYg);
     OFT_LAUNCHED("moe_gather_dy_kernel");
   }
-  // 2. rotations of the active experts
+  // 2. rotations of the active experts; the inactive experts' dQ is zero
   if (int rc = launch_cayley(Q, E * 2 * nb, b, Rex, table, n_active, 2 * nb, st)) return rc;
+  OFT_CUDA(cudaMemsetAsync(dQ, 0, sizeof(float) * E * 2 * nb * (b * (b - 1) / 2), st));
   // 3. chunks: transposed dequant of the chunk's experts (side stream, double-buffered),
   //    then one grouped GEMM D[p][pos][:] = dYg[p][pos][:] W_e,p^T
   gemm::Params prm;
@@ -1956,16 +2002,12 @@ int moe_chunked_oft_bwd(const uint16_t* dY, const uint16_t* X, int T, const floa
     if (int rc = launch_gemm(prm, 0, st)) return rc;
     OFT_CUDA(cudaEventRecord(sp->gemm_done[h], st));
   }
-  // 4. per (active expert, block): rows rotated back, dw partials, dR and the Cayley backward
-  OFT_CUDA(cudaMemsetAsync(dQ, 0, sizeof(float) * E * 2 * nb * (b * (b - 1) / 2), st));
-  {
-    ProfScope ps(OFT_K_GRAD, st);
-    int rc = OFT_OK;
-    if (b == 16) rc = launch_moe_bwd_rot<16>(D, X, K, TK, top_k, bucket, offsets, wts, order, n_active, counter, Rex, U, dwp, dQ, st);
-    if (b == 32) rc = launch_moe_bwd_rot<32>(D, X, K, TK, top_k, bucket, offsets, wts, order, n_active, counter, Rex, U, dwp, dQ, st);
-    if (b == 64) rc = launch_moe_bwd_rot<64>(D, X, K, TK, top_k, bucket, offsets, wts, order, n_active, counter, Rex, U, dwp, dQ, st);
-    if (rc) return rc;
-  }
+  // 4. per (active expert, column group): rows rotated back with the dw partials, the
+  //    expert's adapter gradient (into the chunk buffers, free after the last GEMM), and
+  //    the Cayley backward of the active experts' blocks
+  if (int rc = launch_moe_bwd_tc(D, X, K, TK, top_k, E, b, bucket, offsets, wts, order, n_active, Rex, U, dwp,
+                                 reinterpret_cast<float*>(buf), dQ, st))
+    return rc;
   // 5. dX[t] = sum_k w_tk U[pos(t, k)] in slot order; logit gradients
   {
     ProfScope ps(OFT_K_ROUTE, st);

@@ -308,14 +308,20 @@ constexpr int BWD_BP_BYTES = 64 * 64 * 4;          // 16 KB: one 64 x 64 fp32 ti
 constexpr size_t kBwdSmem = 1024 + A_STAGES * BWD_A_BYTES + MAX_P * BWD_BP_BYTES + 256;
 
 // B_p[i][l] = R_p[i][l] restricted to group g (block-diagonal), fp32, K-major in
-// two 32-wide chunks.  Zero the tiles, then stream the diagonal blocks in with
-// coalesced float4 loads (eight in flight per thread).
-__device__ void build_bwd_b(const BwdParams& p, int g, uint8_t* sB, int tid) {
-  const int b = p.b;
-  for (int v = tid; v < p.P * BWD_BP_BYTES / 16; v += 128) reinterpret_cast<uint4*>(sB)[v] = make_uint4(0, 0, 0, 0);
+// two 32-wide chunks, for the P rotations R[P][nb][b][b] of d_in = K.  Zero the
+// tiles, then stream the diagonal blocks in with coalesced float4 loads (eight in
+// flight per thread).  With sBlo, R is split into its nearest tf32 value (sB) and
+// the nearest tf32 value of the remainder (sBlo): two tf32 MMAs then carry R to
+// about 2^-22 of its size.
+__device__ void build_bwd_b(const float* R, int P, int nb, int b, int K, int g, uint8_t* sB, int tid,
+                            uint8_t* sBlo = nullptr) {
+  for (int v = tid; v < P * BWD_BP_BYTES / 16; v += 128) {
+    reinterpret_cast<uint4*>(sB)[v] = make_uint4(0, 0, 0, 0);
+    if (sBlo != nullptr) reinterpret_cast<uint4*>(sBlo)[v] = make_uint4(0, 0, 0, 0);
+  }
   builders_sync();
   const int per_split = 16 * b;
-  const int total = p.P * per_split;
+  const int total = P * per_split;
   for (int base = 0; base < total; base += 128 * 8) {
     float4 v[8];
     int meta[8];
@@ -329,8 +335,8 @@ __device__ void build_bwd_b(const BwdParams& p, int g, uint8_t* sB, int tid) {
         const int jb = rem / (b * b / 4), w = rem % (b * b / 4);
         const int i = w / (b / 4), l4 = (w % (b / 4)) * 4;
         const int j = (g * 64) / b + jb;
-        if ((j + 1) * b <= p.K) {
-          v[u] = *reinterpret_cast<const float4*>(p.R + ((static_cast<size_t>(sp) * p.nb + j) * b + i) * b + l4);
+        if ((j + 1) * b <= K) {
+          v[u] = *reinterpret_cast<const float4*>(R + ((static_cast<size_t>(sp) * nb + j) * b + i) * b + l4);
           meta[u] = (sp << 16) | ((jb * b + i) << 8) | (jb * b + l4);  // split, row i in group, first l in group
         }
       }
@@ -339,7 +345,15 @@ __device__ void build_bwd_b(const BwdParams& p, int g, uint8_t* sB, int tid) {
     for (int u = 0; u < 8; ++u) {
       if (meta[u] < 0) continue;
       const int sp = meta[u] >> 16, r = (meta[u] >> 8) & 255, k = meta[u] & 255;
-      *reinterpret_cast<float4*>(sB + sp * BWD_BP_BYTES + (k >> 5) * 8192 + swz(r, (k & 31) >> 2)) = v[u];
+      const uint32_t off = sp * BWD_BP_BYTES + (k >> 5) * 8192 + swz(r, (k & 31) >> 2);
+      if (sBlo == nullptr) {
+        *reinterpret_cast<float4*>(sB + off) = v[u];
+      } else {
+        const float4 hi = make_float4(tf32_rn(v[u].x), tf32_rn(v[u].y), tf32_rn(v[u].z), tf32_rn(v[u].w));
+        *reinterpret_cast<float4*>(sB + off) = hi;
+        *reinterpret_cast<float4*>(sBlo + off) = make_float4(tf32_rn(v[u].x - hi.x), tf32_rn(v[u].y - hi.y),
+                                                             tf32_rn(v[u].z - hi.z), tf32_rn(v[u].w - hi.w));
+      }
     }
   }
 }
@@ -466,7 +480,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) rot_bwd_tc_kernel(const __grid
     for (int u = ubeg; u < uend; ++u) {
       const int g = u / p.tiles_m, mt = u % p.tiles_m;
       if (g != cur_g) {
-        build_bwd_b(p, g, sB, tid);
+        build_bwd_b(p.R, p.P, p.nb, p.b, p.K, g, sB, tid);
         fence_proxy_async_smem();
         mbar_arrive(b_full);
         cur_g = g;

@@ -42,6 +42,10 @@ def _to(case, dev):
     (64, 6, 1, 3, 64, 256, 128),    # k = 1: the logit gradient vanishes
     (50, 7, 2, 3, 32, 160, 72),     # hidden and projection widths not multiples of 64
     (300, 40, 4, 16, 32, 128, 64),  # idle experts (dq must be zero), one full chunk
+    (600, 4, 2, 2, 32, 192, 64),    # experts of about 300 rows: several row tiles per unit
+    (96, 8, 2, 4, 32, 4096, 32),    # wide hidden: several (expert, column group) units per CTA
+    (96, 8, 2, 4, 64, 4096, 32),
+    (96, 8, 3, 4, 16, 2048, 32),
 ])
 def test_small_moe_backward(oft, T, E, top_k, chunk, b, K, n):
     spec = MoESpec("sb", T=T, K=K, E=E, n_proj=n, top_k=top_k, chunk=chunk, group=32, b=b, q_sigma=0.05,

@@ -11,7 +11,7 @@
 //   U         = sum_p D_p R_e,p^T                  (blockwise)
 //   dX[t]    += w_tk U
 //   G_e,p,blk += X[t]_blk^T (w_tk D_p,blk)
-//   dw_tk     = <U, X[t]>  (= sum_p <D_p, X[t] R_e,p> = <dY[t], Y_tk>)
+//   dw_tk     = <U, X[t]>  (= sum_p <D_p, X[t] R_e,p> = <dY[t], Y_tk>), with dX[t] in one pass over U
 //
 // then dq_e,p = Cayley backward of G_e,p and, through the softmax over the k
 // selected logits, dlogit[t, e_k] = w_tk (dw_tk - sum_j w_tj dw_tj).
@@ -28,19 +28,26 @@
 
 namespace oftk {
 
-// dYg[p][pos][j] = dY[bucket[pos] / k][p * n + j]   (n % 8 == 0).
+// dYg[p][pos][j] = dY[bucket[pos] / k][p * n + j]   (n % 8 == 0), and each position's
+// routed token and gating weight: row_t[pos] = bucket[pos] / k, row_w[pos] = w[bucket[pos]].
 __global__ void __launch_bounds__(256) moe_gather_dy_kernel(const uint16_t* __restrict__ dY,
-                                                            const int* __restrict__ bucket, int TK, int k, int n,
-                                                            uint16_t* __restrict__ dYg) {
+                                                            const int* __restrict__ bucket, const float* __restrict__ w,
+                                                            int TK, int k, int n, uint16_t* __restrict__ dYg,
+                                                            int* __restrict__ row_t, float* __restrict__ row_w) {
   const int per_row = (2 * n) / 8;
   const long long units = static_cast<long long>(TK) * per_row;
   for (long long u = blockIdx.x * 256ll + threadIdx.x; u < units; u += static_cast<long long>(gridDim.x) * 256) {
     const int pos = static_cast<int>(u / per_row);
     const int col = static_cast<int>(u % per_row) * 8;
     const int p = col / n, j = col - p * n;
-    const int t = bucket[pos] / k;
+    const int ent = bucket[pos];
+    const int t = ent / k;
     const uint4 v = *reinterpret_cast<const uint4*>(dY + static_cast<size_t>(t) * 2 * n + col);
     *reinterpret_cast<uint4*>(dYg + (static_cast<size_t>(p) * TK + pos) * n + j) = v;
+    if (col == 0) {
+      row_t[pos] = t;
+      row_w[pos] = w[ent];
+    }
   }
 }
 
@@ -130,32 +137,71 @@ __global__ void __launch_bounds__(1024) moe_order_kernel(const int* __restrict__
   }
 }
 
-// dlogits[t][:] = 0 except dlogits[t][idx[t,s]] = w_ts (dw_ts - sum_j w_tj dw_tj),
-// dw_ts = sum over blocks of dwp[pos(t, s)][blk] (fixed order).  One warp per token.
-__global__ void __launch_bounds__(256) moe_dlogits_kernel(const float* __restrict__ dwp, int nb,
-                                                          const int* __restrict__ idx, const float* __restrict__ w,
-                                                          const int* __restrict__ inv_pos, int T, int E, int k,
+// dX[t] = sum_s w_ts U[pos(t, s)] (fp32 in slot order, stored as bf16) and
+// dw_ts = <U[pos(t, s)], X[t]> (each lane sums its columns in order, then a fixed
+// xor-shuffle tree).  One warp per token; K % 256 == 0 is not required (K % 8 == 0).
+__global__ void __launch_bounds__(256) moe_combine_bwd_kernel(const float* __restrict__ U, const float* __restrict__ w,
+                                                              const int* __restrict__ inv_pos,
+                                                              const uint16_t* __restrict__ X, int T, int K, int k,
+                                                              uint16_t* __restrict__ dX, float* __restrict__ dw) {
+  const int lane = threadIdx.x % 32;
+  for (int t = (blockIdx.x * 256 + threadIdx.x) / 32; t < T; t += gridDim.x * 8) {
+    int pos[kMaxTopK];
+    float ws[kMaxTopK], dws[kMaxTopK];
+#pragma unroll
+    for (int s = 0; s < kMaxTopK; ++s) {
+      pos[s] = s < k ? inv_pos[static_cast<size_t>(t) * k + s] : 0;
+      ws[s] = s < k ? w[static_cast<size_t>(t) * k + s] : 0.f;
+      dws[s] = 0.f;
+    }
+    for (int c = lane * 8; c < K; c += 256) {
+      const uint4 xq = *reinterpret_cast<const uint4*>(X + static_cast<size_t>(t) * K + c);
+      const float x[8] = {__uint_as_float(xq.x << 16), __uint_as_float(xq.x & 0xFFFF0000u),
+                          __uint_as_float(xq.y << 16), __uint_as_float(xq.y & 0xFFFF0000u),
+                          __uint_as_float(xq.z << 16), __uint_as_float(xq.z & 0xFFFF0000u),
+                          __uint_as_float(xq.w << 16), __uint_as_float(xq.w & 0xFFFF0000u)};
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int s = 0; s < kMaxTopK; ++s) {
+        if (s >= k) break;
+        const float4 a = *reinterpret_cast<const float4*>(U + static_cast<size_t>(pos[s]) * K + c);
+        const float4 b = *reinterpret_cast<const float4*>(U + static_cast<size_t>(pos[s]) * K + c + 4);
+        const float u[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          acc[e] = fmaf(ws[s], u[e], acc[e]);
+          dws[s] = fmaf(u[e], x[e], dws[s]);
+        }
+      }
+      *reinterpret_cast<uint4*>(dX + static_cast<size_t>(t) * K + c) =
+          make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
+                     pack_bf16x2(acc[6], acc[7]));
+    }
+#pragma unroll
+    for (int s = 0; s < kMaxTopK; ++s) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) dws[s] += __shfl_xor_sync(0xFFFFFFFFu, dws[s], o);
+      if (lane == 0 && s < k) dw[static_cast<size_t>(t) * k + s] = dws[s];
+    }
+  }
+}
+
+// dlogits[t][:] = 0 except dlogits[t][idx[t,s]] = w_ts (dw_ts - sum_j w_tj dw_tj)
+// (the sum in slot order).  One warp per token.
+__global__ void __launch_bounds__(256) moe_dlogits_kernel(const float* __restrict__ dw, const int* __restrict__ idx,
+                                                          const float* __restrict__ w, int T, int E, int k,
                                                           float* __restrict__ dlogits) {
   const int warp = (blockIdx.x * 256 + threadIdx.x) / 32, lane = threadIdx.x % 32;
   if (warp >= T) return;
   const int t = warp;
-  float mine = 0.f, s = 0.f;
-  for (int j = 0; j < k; ++j) {
-    const float* row = dwp + static_cast<size_t>(inv_pos[static_cast<size_t>(t) * k + j]) * nb;
-    float acc = 0.f;
-    for (int b = lane; b < nb; b += 32) acc += row[b];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
-    const float wj = w[static_cast<size_t>(t) * k + j];
-    s = fmaf(wj, acc, s);
-    if (lane == j) mine = acc;
-  }
+  float s = 0.f;
+  for (int j = 0; j < k; ++j) s = fmaf(w[static_cast<size_t>(t) * k + j], dw[static_cast<size_t>(t) * k + j], s);
   float* out = dlogits + static_cast<size_t>(t) * E;
   for (int e = lane; e < E; e += 32) out[e] = 0.f;
   __syncwarp();
   if (lane < k) {
-    const float wl = w[static_cast<size_t>(t) * k + lane];
-    out[idx[static_cast<size_t>(t) * k + lane]] = wl * (mine - s);
+    const size_t tk = static_cast<size_t>(t) * k + lane;
+    out[idx[tk]] = w[tk] * (dw[tk] - s);
   }
 }
 

@@ -54,19 +54,16 @@ __device__ __forceinline__ bool moe_unit(const int* order, const int* offsets, i
 }
 
 // ===========================================================================
-// U = sum_p D_p R_e,p^T and the dw partials
+// U = sum_p D_p R_e,p^T
 // ===========================================================================
 struct MoeRotbParams {
   CUtensorMap tmD;          // D fp32 3-D {K, TK, 2}, box {32, 128, 1}, 128B swizzle
   const float* R;           // [E][2][nb][b][b]
-  const uint16_t* X;        // [T][K]
-  const int* bucket;        // [TK] routed entry t * top_k + slot, bucket order
   const int* offsets;       // [E + 1]
   const int* order;         // active experts, heaviest first
   const int* n_active;
   float* U;                 // [TK][K], bucket order
-  float* dwp;               // [TK][nb]
-  int K, TK, top_k, b, nb, groups;  // groups of 64 columns
+  int K, TK, nb, groups;    // groups of 64 columns
 };
 
 constexpr int MRB_A_BYTES = TM * 64 * 4;  // one split's 128-row x 64-column fp32 tile (two 32-column boxes)
@@ -75,11 +72,50 @@ constexpr int MRB_ACC = 4;                // 64-column accumulators in TMEM
 constexpr int MRB_B_BYTES = 2 * 2 * BWD_BP_BYTES;  // one unit's R tiles, both splits, tf32 hi then lo
 constexpr size_t kMoeRotbSmem = 1024 + MRB_STAGES * MRB_A_BYTES + 2 * MRB_B_BYTES + 256;
 
-__device__ __forceinline__ float bf16_lane(const uint4 (&v)[8], int e) {
-  const uint32_t w = (&v[e >> 3].x)[(e & 7) >> 1];
-  return __uint_as_float((e & 1) ? (w & 0xFFFF0000u) : (w << 16));
+// The diagonal R blocks of one (expert, 64-column group) unit, both splits: 2 (64/b) b^2
+// floats, 32 b / 128 float4s per builder thread, loaded one unit ahead of their store.
+template <int B>
+struct RbRegs {
+  static constexpr int N = 2 * 16 * B / 128;
+  float4 v[N];
+};
+
+template <int B>
+__device__ __forceinline__ void rb_load(const float* Re, int nb, int K, int g, int tid, RbRegs<B>& r) {
+#pragma unroll
+  for (int u = 0; u < RbRegs<B>::N; ++u) {
+    const int f = u * 128 + tid;  // float4 index over both splits' diagonal blocks
+    const int sp = f / (16 * B), rem = f % (16 * B);
+    const int jb = rem / (B * B / 4), w = rem % (B * B / 4);
+    const int i = w / (B / 4), l4 = (w % (B / 4)) * 4;
+    const int j = (g * 64) / B + jb;
+    r.v[u] = (j + 1) * B <= K ? *reinterpret_cast<const float4*>(Re + ((static_cast<size_t>(sp) * nb + j) * B + i) * B + l4)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
 }
 
+// Into one unit buffer (hi tiles of both splits, then lo tiles), K-major in two 32-wide
+// chunks as the dense dX rotation lays them out.  Positions off the diagonal blocks are
+// never written: they stay zero from the kernel's start.
+template <int B>
+__device__ __forceinline__ void rb_store(const RbRegs<B>& r, uint8_t* buf, int tid) {
+#pragma unroll
+  for (int u = 0; u < RbRegs<B>::N; ++u) {
+    const int f = u * 128 + tid;
+    const int sp = f / (16 * B), rem = f % (16 * B);
+    const int jb = rem / (B * B / 4), w = rem % (B * B / 4);
+    const int i = w / (B / 4), l4 = (w % (B / 4)) * 4;
+    const int row = jb * B + i, k = jb * B + l4;
+    const uint32_t off = sp * BWD_BP_BYTES + (k >> 5) * 8192 + swz(row, (k & 31) >> 2);
+    const float4 v = r.v[u];
+    const float4 hi = make_float4(tf32_rn(v.x), tf32_rn(v.y), tf32_rn(v.z), tf32_rn(v.w));
+    *reinterpret_cast<float4*>(buf + off) = hi;
+    *reinterpret_cast<float4*>(buf + 2 * BWD_BP_BYTES + off) =
+        make_float4(tf32_rn(v.x - hi.x), tf32_rn(v.y - hi.y), tf32_rn(v.z - hi.z), tf32_rn(v.w - hi.w));
+  }
+}
+
+template <int B>
 __global__ void __launch_bounds__(NUM_THREADS, 1) moe_rotb_tc_kernel(const __grid_constant__ MoeRotbParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -125,7 +161,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) moe_rotb_tc_kernel(const __gri
   pdl_wait();
   const uint32_t tmem = *tmem_slot;
   const int n_units = *p.n_active * p.groups;
-  const size_t r_expert = 2ull * p.nb * p.b * p.b;
+  const size_t r_expert = 2ull * p.nb * B * B;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -215,50 +251,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) moe_rotb_tc_kernel(const __gri
   } else {
     const int q = warp & 3, tid = threadIdx.x - 64;
     const int r = q * 32 + lane;  // this thread's row of every tile
+    for (int v = tid; v < 2 * MRB_B_BYTES / 16; v += 128) reinterpret_cast<uint4*>(sB)[v] = make_uint4(0, 0, 0, 0);
+    builders_sync();
     int acc = 0;
     uint32_t acc_ph = 0;
-    MoeUnit u, un;
+    RbRegs<B> rv;
+    MoeUnit u, un, un2;
     bool have = moe_unit(p.order, p.offsets, n_units, p.groups, 0, u);
     if (have) {
-      build_bwd_b(p.R + u.e * r_expert, 2, p.nb, p.b, p.K, u.g, sB, tid, sB + 2 * BWD_BP_BYTES);
+      rb_load<B>(p.R + u.e * r_expert, p.nb, p.K, u.g, tid, rv);
+      rb_store<B>(rv, sB, tid);
       fence_proxy_async_smem();
       mbar_arrive(&b_full[0]);
     }
+    bool next = have && moe_unit(p.order, p.offsets, n_units, p.groups, 1, un);
+    if (next) rb_load<B>(p.R + un.e * r_expert, p.nb, p.K, un.g, tid, rv);
     for (int k = 0; have; ++k) {
-      // the next unit's R tiles go into the other buffer while this unit's MMAs run
-      const bool next = moe_unit(p.order, p.offsets, n_units, p.groups, k + 1, un);
+      // the next unit's R tiles (loaded during this unit's predecessor) go into the other
+      // buffer, and the loads of the one after start, while this unit's MMAs run
+      bool next2 = false;
       if (next) {
         const int bb = (k + 1) & 1;
         if (k + 1 >= 2 &&
             !warp_wait(&b_empty[bb], static_cast<uint32_t>((((k + 1) >> 1) - 1) & 1), abort_flag, kErrWaitEmpty))
           break;
-        build_bwd_b(p.R + un.e * r_expert, 2, p.nb, p.b, p.K, un.g, sB + bb * MRB_B_BYTES, tid,
-                    sB + bb * MRB_B_BYTES + 2 * BWD_BP_BYTES);
+        rb_store<B>(rv, sB + bb * MRB_B_BYTES, tid);
         fence_proxy_async_smem();
         mbar_arrive(&b_full[bb]);
+        next2 = moe_unit(p.order, p.offsets, n_units, p.groups, k + 2, un2);
+        if (next2) rb_load<B>(p.R + un2.e * r_expert, p.nb, p.K, un2.g, tid, rv);
       }
       const int nt = (u.r1 - u.r0 + TM - 1) / TM;
       bool ok = true;
       for (int mt = 0; mt < nt; ++mt) {
         const int pos = u.r0 + mt * TM + r;
-        const bool valid = pos < u.r1;
-        // this row's X columns of the group, for the dw partials (loaded before the accumulator wait)
-        uint4 xv[8];
-#pragma unroll
-        for (int v = 0; v < 8; ++v) xv[v] = make_uint4(0u, 0u, 0u, 0u);
-        if (valid) {
-          const uint4* src = reinterpret_cast<const uint4*>(
-              p.X + static_cast<size_t>(p.bucket[pos] / p.top_k) * p.K + u.g * 64);
-#pragma unroll
-          for (int v = 0; v < 8; ++v)
-            if (u.g * 64 + v * 8 < p.K) xv[v] = __ldg(src + v);
-        }
         if (!warp_wait(&acc_full[acc], acc_ph, abort_flag, kErrWaitAccFull)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        float part = 0.f;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint32_t rr[32];
@@ -266,26 +297,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) moe_rotb_tc_kernel(const __gri
           tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * 64 + h * 32), rr);
           tmem_ld_wait();
           const int col = u.g * 64 + h * 32;
-          if (valid && col < p.K) {
+          if (pos < u.r1 && col < p.K) {
             float4* dst = reinterpret_cast<float4*>(p.U + static_cast<size_t>(pos) * p.K + col);
 #pragma unroll
             for (int v = 0; v < 8; ++v)
               dst[v] = make_float4(__uint_as_float(rr[4 * v]), __uint_as_float(rr[4 * v + 1]),
                                    __uint_as_float(rr[4 * v + 2]), __uint_as_float(rr[4 * v + 3]));
-            float s[2] = {0.f, 0.f};  // dot products over the half's first and second 16 columns
-#pragma unroll
-            for (int e = 0; e < 32; ++e) s[e >> 4] = fmaf(__uint_as_float(rr[e]), bf16_lane(xv, h * 32 + e), s[e >> 4]);
-            float* dw = p.dwp + static_cast<size_t>(pos) * p.nb;
-            if (p.b == 16) {
-              dw[col / 16] = s[0];
-              dw[col / 16 + 1] = s[1];
-            } else if (p.b == 32) {
-              dw[col / 32] = s[0] + s[1];
-            } else if (h == 0) {
-              part = s[0] + s[1];
-            } else {
-              dw[col / 64] = part + (s[0] + s[1]);
-            }
           }
         }
         tc_fence_before();
@@ -297,7 +314,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) moe_rotb_tc_kernel(const __gri
       }
       if (!ok) break;
       u = un;
+      un = un2;
       have = next;
+      next = next2;
     }
   }
   __syncthreads();
@@ -310,24 +329,49 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) moe_rotb_tc_kernel(const __gri
 // ===========================================================================
 // G_e,p,blk = sum over the expert's positions of (w X[t, blk])^T D_p[pos, blk]
 // ===========================================================================
-struct MoeGradParams {
-  CUtensorMap tmD;          // D fp32 3-D {K, TK, 2}, box {32, 64, 1}, 128B swizzle with 32-byte atoms
-  const uint16_t* X;        // [T][K]
-  const int* bucket;        // [TK]
-  const float* w;           // [TK] gating weights, indexed by routed entry
-  const int* offsets;
-  const int* order;
-  const int* n_active;
-  float* G;                 // [E][2][nb][b][b]
-  int K, TK, top_k, b, nb, groups;  // groups of 128 columns
-};
-
 constexpr int MG_TP = 64;                        // positions per tile (8 MMAs of K = 8)
 constexpr int MG_REGION = MG_TP * 128;           // 8 KB: 64 positions x 32 fp32 columns
 constexpr int MG_D_BYTES = 2 * 4 * MG_REGION;    // both splits, 128 columns: the N = 256 B operand
 constexpr int MG_X_BYTES = 4 * MG_REGION;        // 128 weighted X columns: the M = 128 A operand
 constexpr int MG_STAGES = 2;
 constexpr size_t kMoeGradSmem = 1024 + MG_STAGES * (MG_D_BYTES + MG_X_BYTES) + 256;
+
+struct MoeGradParams {
+  CUtensorMap tmD;          // D fp32 3-D {K, TK, 2}, box {32, 64, 1}, 128B swizzle with 32-byte atoms
+  const uint16_t* X;        // [T][K]
+  const int* row_t;         // [TK] routed token of each position
+  const float* row_w;       // [TK] gating weight of each position
+  const int* offsets;
+  const int* order;
+  const int* n_active;
+  float* G;                 // [E][2][nb][b][b]
+  int K, TK, b, nb, groups;  // groups of 128 columns
+};
+
+// Position in a CTA's sequence of (unit, 64-row tile) steps.
+struct TileCursor {
+  MoeUnit u;
+  int k, mt, nt;
+  bool valid;
+};
+
+__device__ __forceinline__ void cursor_init(TileCursor& c, const int* order, const int* offsets, int n_units,
+                                            int groups) {
+  c.k = 0;
+  c.mt = 0;
+  c.valid = moe_unit(order, offsets, n_units, groups, 0, c.u);
+  c.nt = c.valid ? (c.u.r1 - c.u.r0 + MG_TP - 1) / MG_TP : 0;
+}
+
+__device__ __forceinline__ void cursor_next(TileCursor& c, const int* order, const int* offsets, int n_units,
+                                            int groups) {
+  if (!c.valid) return;
+  if (++c.mt < c.nt) return;
+  c.mt = 0;
+  c.valid = moe_unit(order, offsets, n_units, groups, ++c.k, c.u);
+  c.nt = c.valid ? (c.u.r1 - c.u.r0 + MG_TP - 1) / MG_TP : 0;
+}
+
 
 __global__ void __launch_bounds__(NUM_THREADS, 1) moe_grad_tc_kernel(const __grid_constant__ MoeGradParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -495,31 +539,46 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) moe_grad_tc_kernel(const __gri
       mbar_arrive(&acc_empty[acc]);
       return true;
     };
-    // weighted X rows of one tile: thread chunk ci of rows (tid >> 4) + 8 it, loaded into
-    // registers one tile ahead of their conversion
-    uint4 xr[8];
-    float wr[8];
-    auto fetch = [&](const MoeUnit& v, int mt) {
-      const int col = v.g * 128 + ci * 8;
+    // Weighted X rows of one tile: thread chunk ci of rows (tid >> 4) + 8 it.  Three tiles
+    // are in flight: the X rows of tile i + 1 and the token ids / weights of tile i + 2
+    // load while tile i is converted and stored.
+    uint4 xr[8];    // X chunks of the next tile to stage
+    float xw[8];    // their weights
+    int mt_[8];     // token ids of the tile after (then of the one after that)
+    float mw[8];    // its weights
+    auto load_meta = [&](const TileCursor& c) {
 #pragma unroll
       for (int it = 0; it < 8; ++it) {
-        const int pos = v.r0 + mt * MG_TP + (tid >> 4) + 8 * it;
-        xr[it] = make_uint4(0u, 0u, 0u, 0u);
-        wr[it] = 0.f;
-        if (pos < v.r1 && col < p.K) {
-          const int ent = p.bucket[pos];
-          xr[it] = __ldg(reinterpret_cast<const uint4*>(p.X + static_cast<size_t>(ent / p.top_k) * p.K + col));
-          wr[it] = p.w[ent];
-        }
+        const int pos = c.u.r0 + c.mt * MG_TP + (tid >> 4) + 8 * it;
+        const bool ok = c.valid && pos < c.u.r1;
+        mt_[it] = ok ? p.row_t[pos] : -1;
+        mw[it] = ok ? p.row_w[pos] : 0.f;
+      }
+    };
+    auto load_x = [&](const TileCursor& c) {  // from the meta registers, which then free up
+      const int col = c.u.g * 128 + ci * 8;
+#pragma unroll
+      for (int it = 0; it < 8; ++it) {
+        xr[it] = (mt_[it] >= 0 && col < p.K)
+                     ? __ldg(reinterpret_cast<const uint4*>(p.X + static_cast<size_t>(mt_[it]) * p.K + col))
+                     : make_uint4(0u, 0u, 0u, 0u);
+        xw[it] = mw[it];
       }
     };
     int stage = 0;
     uint32_t ph = 0;
-    MoeUnit cur, prev;
-    int k = 0, mt = 0;
-    bool have = moe_unit(p.order, p.offsets, n_units, p.groups, 0, cur);
-    if (have) fetch(cur, 0);
-    while (have) {
+    TileCursor c0, c1;  // the tile being staged, the tile after the next one
+    cursor_init(c0, p.order, p.offsets, n_units, p.groups);
+    c1 = c0;
+    if (c0.valid) {
+      load_meta(c0);
+      load_x(c0);
+      cursor_next(c1, p.order, p.offsets, n_units, p.groups);
+      load_meta(c1);
+      cursor_next(c1, p.order, p.offsets, n_units, p.groups);
+    }
+    MoeUnit prev;
+    while (c0.valid) {
       if (!warp_wait(&x_empty[stage], ph ^ 1, abort_flag, kErrWaitEmpty)) break;
       uint8_t* base = sX + stage * MG_X_BYTES + (ci >> 2) * MG_REGION;
       const uint32_t c16 = (ci & 3) * 2;
@@ -527,7 +586,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) moe_grad_tc_kernel(const __gri
       for (int it = 0; it < 8; ++it) {
         const int row = (tid >> 4) + 8 * it;
         const uint4 v = xr[it];
-        const float s = wr[it];
+        const float s = xw[it];
         *reinterpret_cast<float4*>(base + swz32(row, c16)) =
             make_float4(tf32_rn(__uint_as_float(v.x << 16) * s), tf32_rn(__uint_as_float(v.x & 0xFFFF0000u) * s),
                         tf32_rn(__uint_as_float(v.y << 16) * s), tf32_rn(__uint_as_float(v.y & 0xFFFF0000u) * s));
@@ -541,21 +600,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) moe_grad_tc_kernel(const __gri
         stage = 0;
         ph ^= 1;
       }
-      // move to the next tile and start its loads, then drain the unit before this one
-      // once this unit's first tile is staged (its MMAs keep the tensor pipe busy meanwhile)
-      const MoeUnit staged = cur;
-      const int ks = k;
-      const bool first = (mt == 0);
-      if (++mt == (cur.r1 - cur.r0 + MG_TP - 1) / MG_TP) {
-        mt = 0;
-        have = moe_unit(p.order, p.offsets, n_units, p.groups, ++k, cur);
+      const TileCursor done = c0;
+      cursor_next(c0, p.order, p.offsets, n_units, p.groups);
+      if (c0.valid) load_x(c0);  // the meta registers hold c0's tile
+      load_meta(c1);
+      cursor_next(c1, p.order, p.offsets, n_units, p.groups);
+      // once a unit's first tile is staged, drain the unit before it (its MMAs keep the
+      // tensor pipe busy meanwhile); after the last tile, drain the last unit
+      if (done.mt == 0) {
+        if (done.k > 0 && !epilogue(done.k - 1, prev)) break;
+        prev = done.u;
       }
-      if (have) fetch(cur, mt);
-      if (first) {
-        if (ks > 0 && !epilogue(ks - 1, prev)) break;
-        prev = staged;
-      }
-      if (!have) epilogue(ks, staged);
+      if (!c0.valid) epilogue(done.k, done.u);
     }
   }
   __syncthreads();

@@ -1804,7 +1804,7 @@ int moe_chunked_oft_layer_fwd(const uint16_t* X, int T, const float* logits, int
 // ---------------------------------------------------------------------------
 namespace {
 struct MoeBwdLayout {
-  size_t idx, w, offsets, bucket, table, meta, order, inv, pexp, rex, dyg, buf, d, u, dwp, total;
+  size_t idx, w, offsets, bucket, table, meta, order, inv, pexp, rex, dyg, buf, d, u, dw, row_t, row_w, total;
 };
 MoeBwdLayout moe_bwd_layout(int T, int E, int top_k, int chunk, int K, int N, int b) {
   MoeBwdLayout L{};
@@ -1826,39 +1826,44 @@ MoeBwdLayout moe_bwd_layout(int T, int E, int top_k, int chunk, int K, int N, in
   // active experts' adapter gradients G [E][2][nb][b][b]
   L.d = round_up(L.buf + std::max(2ull * 2 * chunk * N * K, 4ull * E * 2 * nb * b * b), 256);
   L.u = round_up(L.d + 4 * 2 * TK * K, 256);
-  L.dwp = round_up(L.u + 4 * TK * K, 256);
-  L.total = round_up(L.dwp + 4 * TK * nb, 256);
+  L.dw = round_up(L.u + 4 * TK * K, 256);
+  L.row_t = round_up(L.dw + 4 * TK, 256);
+  L.row_w = round_up(L.row_t + 4 * TK, 256);
+  L.total = round_up(L.row_w + 4 * TK, 256);
   return L;
 }
 
-// Step 4 of the MoE backward on the tensor cores: U and the dw partials, each active
-// expert's adapter gradient G (into `G`, [E][2][nb][b][b]), then its Cayley backward.
-int launch_moe_bwd_tc(const float* D, const uint16_t* X, int K, int TK, int top_k, int E, int b, const int* bucket,
-                      const int* offsets, const float* w, const int* order, const int* n_active, const float* R,
-                      float* U, float* dwp, float* G, float* dQ, cudaStream_t st) {
+// Step 4 of the MoE backward on the tensor cores: U = sum_p D_p R^T per routed row, each
+// active expert's adapter gradient G (into `G`, [E][2][nb][b][b]), then its Cayley backward.
+int launch_moe_bwd_tc(const float* D, const uint16_t* X, int K, int TK, int E, int b, const int* row_t,
+                      const float* row_w, const int* offsets, const int* order, const int* n_active, const float* R,
+                      float* U, float* G, float* dQ, cudaStream_t st) {
   const int nb = K / b;
   {
     rtc::MoeRotbParams prm;
     memset(&prm, 0, sizeof(prm));
     if (int rc = make_map_f32_3d(&prm.tmD, D, K, TK, 2)) return rc;
     prm.R = R;
-    prm.X = X;
-    prm.bucket = bucket;
     prm.offsets = offsets;
     prm.order = order;
     prm.n_active = n_active;
     prm.U = U;
-    prm.dwp = dwp;
     prm.K = K;
     prm.TK = TK;
-    prm.top_k = top_k;
-    prm.b = b;
     prm.nb = nb;
     prm.groups = (K + 63) / 64;
-    if (int rc = set_smem(rtc::moe_rotb_tc_kernel, rtc::kMoeRotbSmem)) return rc;
     const int grid = static_cast<int>(std::min<long long>(sm_count(), 1ll * E * prm.groups));
-    ProfScope ps(OFT_K_ROTATE, st);
-    OFT_CUDA(launch_pdl(rtc::moe_rotb_tc_kernel, grid, rtc::NUM_THREADS, rtc::kMoeRotbSmem, st, prm));
+    auto go = [&](auto kernel) -> int {
+      if (int rc = set_smem(kernel, rtc::kMoeRotbSmem)) return rc;
+      ProfScope ps(OFT_K_ROTATE, st);
+      OFT_CUDA(launch_pdl(kernel, grid, rtc::NUM_THREADS, rtc::kMoeRotbSmem, st, prm));
+      return OFT_OK;
+    };
+    int rc = OFT_OK;
+    if (b == 16) rc = go(rtc::moe_rotb_tc_kernel<16>);
+    if (b == 32) rc = go(rtc::moe_rotb_tc_kernel<32>);
+    if (b == 64) rc = go(rtc::moe_rotb_tc_kernel<64>);
+    if (rc) return rc;
     OFT_LAUNCHED("moe_rotb_tc_kernel");
   }
   {
@@ -1866,15 +1871,14 @@ int launch_moe_bwd_tc(const float* D, const uint16_t* X, int K, int TK, int top_
     memset(&prm, 0, sizeof(prm));
     if (int rc = make_map_f32_3d(&prm.tmD, D, K, TK, 2, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B, rtc::MG_TP)) return rc;
     prm.X = X;
-    prm.bucket = bucket;
-    prm.w = w;
+    prm.row_t = row_t;
+    prm.row_w = row_w;
     prm.offsets = offsets;
     prm.order = order;
     prm.n_active = n_active;
     prm.G = G;
     prm.K = K;
     prm.TK = TK;
-    prm.top_k = top_k;
     prm.b = b;
     prm.nb = nb;
     prm.groups = (K + 127) / 128;
@@ -1934,7 +1938,9 @@ int moe_chunked_oft_bwd(const uint16_t* dY, const uint16_t* X, int T, const floa
   uint16_t* buf = reinterpret_cast<uint16_t*>(wsb + L.buf);
   float* D = reinterpret_cast<float*>(wsb + L.d);
   float* U = reinterpret_cast<float*>(wsb + L.u);
-  float* dwp = reinterpret_cast<float*>(wsb + L.dwp);
+  float* dw = reinterpret_cast<float*>(wsb + L.dw);
+  int* row_t = reinterpret_cast<int*>(wsb + L.row_t);
+  float* row_w = reinterpret_cast<float*>(wsb + L.row_w);
 
   // 1. routing, as in the forward
   {
@@ -1953,7 +1959,7 @@ int moe_chunked_oft_bwd(const uint16_t* dY, const uint16_t* X, int T, const floa
     OFT_LAUNCHED("moe_order_kernel");
     const long long gunits = 1ll * TK * (N / 8);
     moe_gather_dy_kernel<<<static_cast<int>(std::min<long long>((gunits + 255) / 256, 148ll * 16)), 256, 0, st>>>(
-        dY, bucket, TK, top_k, n_proj, dYg);
+        dY, bucket, wts, TK, top_k, n_proj, dYg, row_t, row_w);
     OFT_LAUNCHED("moe_gather_dy_kernel");
   }
   // 2. rotations of the active experts; the inactive experts' dQ is zero
@@ -2005,18 +2011,17 @@ int moe_chunked_oft_bwd(const uint16_t* dY, const uint16_t* X, int T, const floa
   // 4. per (active expert, column group): rows rotated back with the dw partials, the
   //    expert's adapter gradient (into the chunk buffers, free after the last GEMM), and
   //    the Cayley backward of the active experts' blocks
-  if (int rc = launch_moe_bwd_tc(D, X, K, TK, top_k, E, b, bucket, offsets, wts, order, n_active, Rex, U, dwp,
+  if (int rc = launch_moe_bwd_tc(D, X, K, TK, E, b, row_t, row_w, offsets, order, n_active, Rex, U,
                                  reinterpret_cast<float*>(buf), dQ, st))
     return rc;
-  // 5. dX[t] = sum_k w_tk U[pos(t, k)] in slot order; logit gradients
+  // 5. dX[t] = sum_k w_tk U[pos(t, k)] in slot order with dw_tk = <U[pos(t, k)], X[t]>; logit gradients
   {
     ProfScope ps(OFT_K_ROUTE, st);
-    const long long cunits = 1ll * T * (K / 8);
-    const int cgrid = static_cast<int>(std::min<long long>((cunits + 255) / 256, 148ll * 16));
-    moe_combine_kernel<<<cgrid, 256, 0, st>>>(U, wts, inv, T, K, top_k, dX);
-    OFT_LAUNCHED("moe_combine_kernel");
+    const int cgrid = static_cast<int>(std::min<long long>((T + 7) / 8, 148ll * 16));
+    moe_combine_bwd_kernel<<<cgrid, 256, 0, st>>>(U, wts, inv, X, T, K, top_k, dX, dw);
+    OFT_LAUNCHED("moe_combine_bwd_kernel");
     if (dlogits != nullptr) {
-      moe_dlogits_kernel<<<(T * 32 + 255) / 256, 256, 0, st>>>(dwp, nb, idx, wts, inv, T, E, top_k, dlogits);
+      moe_dlogits_kernel<<<(T * 32 + 255) / 256, 256, 0, st>>>(dw, idx, wts, T, E, top_k, dlogits);
       OFT_LAUNCHED("moe_dlogits_kernel");
     }
   }

@@ -206,7 +206,7 @@ __device__ __forceinline__ void cayley_fwd_block_inv(const uint16_t* __restrict_
                                                      int total, const int* __restrict__ active_list,
                                                      int blocks_per_expert, long long lo_off) {
   constexpr int BPC = CayleyFwdCfg<B>::BPC;
-  __shared__ __align__(16) float piv[2][BPC][B];
+  __shared__ __align__(16) float piv[2][BPC][B + 4];  // pivot row, then its reciprocal
   __shared__ __align__(16) uint16_t qsh[BPC][B * (B - 1) / 2];
   const int sub = threadIdx.x / B, r = threadIdx.x % B;
   const bool active = lin < total;  // B = 16: the CTA's second block may run past the end
@@ -234,27 +234,32 @@ __device__ __forceinline__ void cayley_fwd_block_inv(const uint16_t* __restrict_
     }
     a[j] = ((j == r) ? 1.f : 0.f) - v;
   }
+  // Pivot c in one uniform update for every row: with p = 1 / A[c][c] and the pivot row
+  // P = A[c][:] published as it is, each row r takes f = (A[r][c] - [r == c]) p and
+  // A[r][j] -= f P[j] for j != c, then A[r][c] = -f (r != c) or p (r = c).  For r != c
+  // this is the elimination step of the in-place inverse; for r = c it scales the row
+  // by p (A[c][j] - (A[c][c] - 1) p A[c][j] = A[c][j] p).  Only the publication (one
+  // reciprocal and B / 4 vector stores) runs on the pivot row's thread alone.
 #pragma unroll
   for (int c = 0; c < B; ++c) {
     float* pr = piv[c & 1][sub];
     if (r == c) {
-      const float p = __frcp_rn(a[c]);  // correctly rounded
-#pragma unroll
-      for (int j = 0; j < B; ++j) a[j] = (j == c) ? p : a[j] * p;
+      pr[B] = __frcp_rn(a[c]);  // correctly rounded; A[c][c] >= 1 in exact arithmetic
 #pragma unroll
       for (int j = 0; j < B; j += 4) *reinterpret_cast<float4*>(pr + j) = make_float4(a[j], a[j + 1], a[j + 2], a[j + 3]);
     }
     block_sync();
-    if (r != c) {
-      const float f = a[c];
+    const float pinv = pr[B];
+    const float f = (a[c] - (r == c ? 1.f : 0.f)) * pinv;
 #pragma unroll
-      for (int j = 0; j < B; j += 4) {
-        const float4 v = *reinterpret_cast<const float4*>(pr + j);
-        const float w[4] = {v.x, v.y, v.z, v.w};
+    for (int j = 0; j < B; j += 4) {
+      const float4 v = *reinterpret_cast<const float4*>(pr + j);
+      const float w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int t = 0; t < 4; ++t) a[j + t] = (j + t == c) ? -f * w[t] : fmaf(-f, w[t], a[j + t]);
-      }
+      for (int t = 0; t < 4; ++t)
+        if (j + t != c) a[j + t] = fmaf(-f, w[t], a[j + t]);
     }
+    a[c] = (r == c) ? pinv : -f;
   }
   if (active && lo_off > 0) {
 #pragma unroll
@@ -385,106 +390,127 @@ __global__ void __launch_bounds__(TPR * B) cayley_fwd_split_kernel(const uint16_
 // sums laid out [nblocks][nparts][b][b], summed in part order (deterministic).
 // With a map (the MoE's active experts), only the blocks map[i] * per + r for
 // i < *n_map and r < per are computed; the others are left as they are.
-// One CTA per block; each thread owns a TI x TI tile of the two b x b products.
-// Dynamic shared memory: 3 * B * (B + 1) floats.
+// Each thread owns a 4 x 4 tile of the two b x b products, so a CTA works on
+// kCayleyThreads / (b/4)^2 blocks at once (16, 4, 1 for b = 16, 32, 64).  Per block
+// the shared memory holds I + R, its transpose T, G (later 2D) and (T G)^T, rows
+// padded to b + 4 floats, so that both operands of every product step are float4
+// reads: 2 vector loads per 16 FMAs.
+template <int B>
+struct CayleyBwdCfg {
+  static constexpr int NT = (B / 4) * (B / 4);        // threads per block
+  static constexpr int BPC = kCayleyThreads / NT;     // blocks per CTA
+  static constexpr int LD = B + 4;
+  static constexpr int SZ = B * LD;                   // floats per array
+  static constexpr size_t SMEM = sizeof(float) * BPC * 4 * SZ;
+};
+
 template <int B>
 __global__ void __launch_bounds__(kCayleyThreads) cayley_bwd_kernel(const float* __restrict__ R,
                                                                     const float* __restrict__ G, int nparts,
                                                                     int nblocks, float* __restrict__ dQ,
                                                                     const int* __restrict__ map,
                                                                     const int* __restrict__ n_map, int per) {
-  constexpr int TI = (B == 64) ? 4 : (B == 32 ? 2 : 1);
-  constexpr int NT = B / TI;  // threads per output row of tiles
-  static_assert(NT * NT == kCayleyThreads, "tile grid must cover the CTA");
-  constexpr int LD = B + 1;
-  extern __shared__ float csm[];
-  float* T = csm;               // (I + R)^T
-  float* Gs = csm + B * LD;     // G, then D * 2
-  float* U = csm + 2 * B * LD;  // T G
-  const int tid = threadIdx.x;
-  const int ti = (tid / NT) * TI, tj = (tid % NT) * TI;
+  using C = CayleyBwdCfg<B>;
+  constexpr int NT = C::NT, BPC = C::BPC, LD = C::LD, SZ = C::SZ;
+  constexpr int V = B * B / 4 / NT;  // float4s of a block per thread (4)
+  extern __shared__ float4 cbw_smem[];
+  const int sub = threadIdx.x / NT, t = threadIdx.x % NT;
+  float* Tt = reinterpret_cast<float*>(cbw_smem) + sub * 4 * SZ;  // I + R: Tt[l][i] = T[i][l]
+  float* T = Tt + SZ;                                              // T = (I + R)^T
+  float* Gs = T + SZ;                                              // G, then 2D
+  float* Mt = Gs + SZ;                                             // (T G)^T
+  const int ti = (t / (B / 4)) * 4, tj = (t % (B / 4)) * 4;
   pdl_wait();
   const int count = map != nullptr ? *n_map * per : nblocks;
-  for (int it = blockIdx.x; it < count; it += gridDim.x) {
-    const int blk = map != nullptr ? map[it / per] * per + it % per : it;
-    const float* rb = R + static_cast<size_t>(blk) * B * B;
-    const float* gb = G + static_cast<size_t>(blk) * nparts * B * B;
-    constexpr int EPT = B * B / kCayleyThreads;  // elements per thread
-    float acc[EPT], rv[EPT];
+  for (int base = blockIdx.x * BPC; base < count; base += gridDim.x * BPC) {
+    const int it = base + sub;
+    const bool act = it < count;
+    const int blk = !act ? 0 : (map != nullptr ? map[it / per] * per + it % per : it);
+    __syncthreads();  // the previous blocks are done with shared memory
+    if (act) {
+      const float4* rb = reinterpret_cast<const float4*>(R + static_cast<size_t>(blk) * B * B);
+      const float4* gb = reinterpret_cast<const float4*>(G + static_cast<size_t>(blk) * nparts * B * B);
+      float4 rv[V], acc[V];
 #pragma unroll
-    for (int k = 0; k < EPT; ++k) {
-      rv[k] = rb[tid + k * kCayleyThreads];
-      acc[k] = 0.f;
-    }
-    for (int p = 0; p < nparts; p += 4) {  // 4 * EPT independent loads in flight, summed in part order
-      float t[4][EPT];
+      for (int v = 0; v < V; ++v) {
+        rv[v] = rb[t + v * NT];
+        acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      for (int q = 0; q < nparts; q += 2) {  // two parts' loads in flight, summed in part order
+        float4 g0[V], g1[V];
 #pragma unroll
-      for (int pp = 0; pp < 4; ++pp)
+        for (int v = 0; v < V; ++v) {
+          g0[v] = gb[static_cast<size_t>(q) * (B * B / 4) + t + v * NT];
+          g1[v] = q + 1 < nparts ? gb[static_cast<size_t>(q + 1) * (B * B / 4) + t + v * NT]
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
 #pragma unroll
-        for (int k = 0; k < EPT; ++k)
-          t[pp][k] = (p + pp < nparts) ? gb[static_cast<size_t>(p + pp) * B * B + tid + k * kCayleyThreads] : 0.f;
+        for (int v = 0; v < V; ++v) {
+          acc[v] = make_float4(acc[v].x + g0[v].x, acc[v].y + g0[v].y, acc[v].z + g0[v].z, acc[v].w + g0[v].w);
+          acc[v] = make_float4(acc[v].x + g1[v].x, acc[v].y + g1[v].y, acc[v].z + g1[v].z, acc[v].w + g1[v].w);
+        }
+      }
 #pragma unroll
-      for (int pp = 0; pp < 4; ++pp)
+      for (int v = 0; v < V; ++v) {
+        const int idx = (t + v * NT) * 4;
+        const int i = idx / B, j0 = idx % B;
+        const float e[4] = {rv[v].x + (i == j0 ? 1.f : 0.f), rv[v].y + (i == j0 + 1 ? 1.f : 0.f),
+                            rv[v].z + (i == j0 + 2 ? 1.f : 0.f), rv[v].w + (i == j0 + 3 ? 1.f : 0.f)};
+        *reinterpret_cast<float4*>(Tt + i * LD + j0) = make_float4(e[0], e[1], e[2], e[3]);
 #pragma unroll
-        for (int k = 0; k < EPT; ++k) acc[k] += t[pp][k];
-    }
-#pragma unroll
-    for (int k = 0; k < EPT; ++k) {
-      const int idx = tid + k * kCayleyThreads;
-      const int i = idx / B, j = idx % B;
-      T[j * LD + i] = rv[k] + (i == j ? 1.f : 0.f);
-      Gs[i * LD + j] = acc[k];
-    }
-    __syncthreads();
-    float o[TI][TI];
-#pragma unroll
-    for (int x = 0; x < TI; ++x)
-#pragma unroll
-      for (int y = 0; y < TI; ++y) o[x][y] = 0.f;
-#pragma unroll 4
-    for (int l = 0; l < B; ++l) {  // U = T G
-      float tv[TI], gv[TI];
-#pragma unroll
-      for (int x = 0; x < TI; ++x) tv[x] = T[(ti + x) * LD + l];
-#pragma unroll
-      for (int y = 0; y < TI; ++y) gv[y] = Gs[l * LD + tj + y];
-#pragma unroll
-      for (int x = 0; x < TI; ++x)
-#pragma unroll
-        for (int y = 0; y < TI; ++y) o[x][y] = fmaf(tv[x], gv[y], o[x][y]);
-    }
-#pragma unroll
-    for (int x = 0; x < TI; ++x)
-#pragma unroll
-      for (int y = 0; y < TI; ++y) U[(ti + x) * LD + tj + y] = o[x][y];
-    __syncthreads();
-#pragma unroll
-    for (int x = 0; x < TI; ++x)
-#pragma unroll
-      for (int y = 0; y < TI; ++y) o[x][y] = 0.f;
-#pragma unroll 4
-    for (int l = 0; l < B; ++l) {  // 2D = U T
-      float uv[TI], tv[TI];
-#pragma unroll
-      for (int x = 0; x < TI; ++x) uv[x] = U[(ti + x) * LD + l];
-#pragma unroll
-      for (int y = 0; y < TI; ++y) tv[y] = T[l * LD + tj + y];
-#pragma unroll
-      for (int x = 0; x < TI; ++x)
-#pragma unroll
-        for (int y = 0; y < TI; ++y) o[x][y] = fmaf(uv[x], tv[y], o[x][y]);
-    }
-#pragma unroll
-    for (int x = 0; x < TI; ++x)
-#pragma unroll
-      for (int y = 0; y < TI; ++y) Gs[(ti + x) * LD + tj + y] = o[x][y];
-    __syncthreads();
-    float* out = dQ + static_cast<size_t>(blk) * (B * (B - 1) / 2);
-    for (int idx = tid; idx < B * B; idx += kCayleyThreads) {
-      const int i = idx / B, j = idx % B;
-      if (i < j) out[tri_index(i, j, B)] = 0.5f * (Gs[i * LD + j] - Gs[j * LD + i]);
+        for (int c = 0; c < 4; ++c) T[(j0 + c) * LD + i] = e[c];
+        *reinterpret_cast<float4*>(Gs + i * LD + j0) = acc[v];
+      }
     }
     __syncthreads();
+    float o[4][4];
+    if (act) {  // M = T G
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+#pragma unroll
+        for (int y = 0; y < 4; ++y) o[x][y] = 0.f;
+#pragma unroll 8
+      for (int l = 0; l < B; ++l) {
+        const float4 tv = *reinterpret_cast<const float4*>(Tt + l * LD + ti);  // T[ti + x][l]
+        const float4 gv = *reinterpret_cast<const float4*>(Gs + l * LD + tj);  // G[l][tj + y]
+        const float a4[4] = {tv.x, tv.y, tv.z, tv.w}, b4[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+#pragma unroll
+          for (int y = 0; y < 4; ++y) o[x][y] = fmaf(a4[x], b4[y], o[x][y]);
+      }
+#pragma unroll
+      for (int y = 0; y < 4; ++y)
+        *reinterpret_cast<float4*>(Mt + (tj + y) * LD + ti) = make_float4(o[0][y], o[1][y], o[2][y], o[3][y]);
+    }
+    __syncthreads();
+    if (act) {  // 2D = M T, over G's rows (G is no longer read)
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+#pragma unroll
+        for (int y = 0; y < 4; ++y) o[x][y] = 0.f;
+#pragma unroll 8
+      for (int l = 0; l < B; ++l) {
+        const float4 mv = *reinterpret_cast<const float4*>(Mt + l * LD + ti);  // M[ti + x][l]
+        const float4 tv = *reinterpret_cast<const float4*>(T + l * LD + tj);   // T[l][tj + y]
+        const float a4[4] = {mv.x, mv.y, mv.z, mv.w}, b4[4] = {tv.x, tv.y, tv.z, tv.w};
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+#pragma unroll
+          for (int y = 0; y < 4; ++y) o[x][y] = fmaf(a4[x], b4[y], o[x][y]);
+      }
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+        *reinterpret_cast<float4*>(Gs + (ti + x) * LD + tj) = make_float4(o[x][0], o[x][1], o[x][2], o[x][3]);
+    }
+    __syncthreads();
+    if (act) {
+      float* out = dQ + static_cast<size_t>(blk) * (B * (B - 1) / 2);
+      for (int idx = t; idx < B * B; idx += NT) {
+        const int i = idx / B, j = idx % B;
+        if (i < j) out[tri_index(i, j, B)] = 0.5f * (Gs[i * LD + j] - Gs[j * LD + i]);
+      }
+    }
   }
 }
 

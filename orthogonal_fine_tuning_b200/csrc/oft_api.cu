@@ -360,8 +360,9 @@ int launch_cayley(const uint16_t* Q, int nblocks, int b, float* R, const int* ac
 
 int launch_cayley_bwd(const float* R, const float* G, int nparts, int nblocks, int b, float* dQ, cudaStream_t st,
                       const int* map = nullptr, const int* n_map = nullptr, int per = 1) {
-  const size_t smem = 3ull * b * (b + 1) * sizeof(float);
-  const int grid = std::min(nblocks, sm_count() * 8);
+  const size_t smem = b == 16 ? CayleyBwdCfg<16>::SMEM : (b == 32 ? CayleyBwdCfg<32>::SMEM : CayleyBwdCfg<64>::SMEM);
+  const int bpc = b == 16 ? CayleyBwdCfg<16>::BPC : (b == 32 ? CayleyBwdCfg<32>::BPC : CayleyBwdCfg<64>::BPC);
+  const int grid = std::min((nblocks + bpc - 1) / bpc, sm_count() * 3);
   if (b == 16) OFT_CUDA(cudaFuncSetAttribute(cayley_bwd_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   if (b == 32) OFT_CUDA(cudaFuncSetAttribute(cayley_bwd_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   if (b == 64) OFT_CUDA(cudaFuncSetAttribute(cayley_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));

@@ -390,18 +390,19 @@ __global__ void __launch_bounds__(TPR * B) cayley_fwd_split_kernel(const uint16_
 // sums laid out [nblocks][nparts][b][b], summed in part order (deterministic).
 // With a map (the MoE's active experts), only the blocks map[i] * per + r for
 // i < *n_map and r < per are computed; the others are left as they are.
-// Each thread owns a 4 x 4 tile of the two b x b products, so a CTA works on
-// kCayleyThreads / (b/4)^2 blocks at once (16, 4, 1 for b = 16, 32, 64).  Per block
+// Each thread owns a 4 x 4 tile of the two b x b products, so a CTA of blockDim.x
+// threads works on blockDim.x / (b/4)^2 blocks at once (up to 16, 4, 1 for b = 16,
+// 32, 64; the host takes fewer when the launch has few blocks).  Per block
 // the shared memory holds I + R, its transpose T, G (later 2D) and (T G)^T, rows
 // padded to b + 4 floats, so that both operands of every product step are float4
 // reads: 2 vector loads per 16 FMAs.
 template <int B>
 struct CayleyBwdCfg {
   static constexpr int NT = (B / 4) * (B / 4);        // threads per block
-  static constexpr int BPC = kCayleyThreads / NT;     // blocks per CTA
+  static constexpr int BPC = kCayleyThreads / NT;     // most blocks per CTA
   static constexpr int LD = B + 4;
   static constexpr int SZ = B * LD;                   // floats per array
-  static constexpr size_t SMEM = sizeof(float) * BPC * 4 * SZ;
+  static constexpr size_t SMEM_PER_BLOCK = sizeof(float) * 4 * SZ;
 };
 
 template <int B>
@@ -411,7 +412,8 @@ __global__ void __launch_bounds__(kCayleyThreads) cayley_bwd_kernel(const float*
                                                                     const int* __restrict__ map,
                                                                     const int* __restrict__ n_map, int per) {
   using C = CayleyBwdCfg<B>;
-  constexpr int NT = C::NT, BPC = C::BPC, LD = C::LD, SZ = C::SZ;
+  constexpr int NT = C::NT, LD = C::LD, SZ = C::SZ;
+  const int BPC = blockDim.x / NT;
   constexpr int V = B * B / 4 / NT;  // float4s of a block per thread (4)
   extern __shared__ float4 cbw_smem[];
   const int sub = threadIdx.x / NT, t = threadIdx.x % NT;

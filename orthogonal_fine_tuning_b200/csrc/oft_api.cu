@@ -360,16 +360,23 @@ int launch_cayley(const uint16_t* Q, int nblocks, int b, float* R, const int* ac
 
 int launch_cayley_bwd(const float* R, const float* G, int nparts, int nblocks, int b, float* dQ, cudaStream_t st,
                       const int* map = nullptr, const int* n_map = nullptr, int per = 1) {
-  const size_t smem = b == 16 ? CayleyBwdCfg<16>::SMEM : (b == 32 ? CayleyBwdCfg<32>::SMEM : CayleyBwdCfg<64>::SMEM);
-  const int bpc = b == 16 ? CayleyBwdCfg<16>::BPC : (b == 32 ? CayleyBwdCfg<32>::BPC : CayleyBwdCfg<64>::BPC);
-  const int grid = std::min((nblocks + bpc - 1) / bpc, sm_count() * 3);
+  // blocks per CTA: as many as fit (up to 256 threads), but no fewer CTAs than about
+  // two per SM while the launch has the blocks for it
+  const int nt = (b / 4) * (b / 4);
+  const int bpc_max = kCayleyThreads / nt;
+  int bpc = 1;
+  while (bpc * 2 <= bpc_max && 1ll * nblocks >= 2ll * bpc * 2 * sm_count()) bpc *= 2;
+  const size_t smem = static_cast<size_t>(bpc) * (b == 16 ? CayleyBwdCfg<16>::SMEM_PER_BLOCK
+                                                          : (b == 32 ? CayleyBwdCfg<32>::SMEM_PER_BLOCK
+                                                                     : CayleyBwdCfg<64>::SMEM_PER_BLOCK));
+  const int grid = static_cast<int>(std::min<long long>((nblocks + bpc - 1) / bpc, sm_count() * 3ll * (bpc_max / bpc)));
   if (b == 16) OFT_CUDA(cudaFuncSetAttribute(cayley_bwd_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   if (b == 32) OFT_CUDA(cudaFuncSetAttribute(cayley_bwd_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   if (b == 64) OFT_CUDA(cudaFuncSetAttribute(cayley_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   ProfScope ps(OFT_K_CAYLEY, st);
-  if (b == 16) OFT_CUDA(launch_pdl(cayley_bwd_kernel<16>, grid, kCayleyThreads, smem, st, R, G, nparts, nblocks, dQ, map, n_map, per));
-  if (b == 32) OFT_CUDA(launch_pdl(cayley_bwd_kernel<32>, grid, kCayleyThreads, smem, st, R, G, nparts, nblocks, dQ, map, n_map, per));
-  if (b == 64) OFT_CUDA(launch_pdl(cayley_bwd_kernel<64>, grid, kCayleyThreads, smem, st, R, G, nparts, nblocks, dQ, map, n_map, per));
+  if (b == 16) OFT_CUDA(launch_pdl(cayley_bwd_kernel<16>, grid, bpc * nt, smem, st, R, G, nparts, nblocks, dQ, map, n_map, per));
+  if (b == 32) OFT_CUDA(launch_pdl(cayley_bwd_kernel<32>, grid, bpc * nt, smem, st, R, G, nparts, nblocks, dQ, map, n_map, per));
+  if (b == 64) OFT_CUDA(launch_pdl(cayley_bwd_kernel<64>, grid, bpc * nt, smem, st, R, G, nparts, nblocks, dQ, map, n_map, per));
   OFT_LAUNCHED("cayley_bwd_kernel");
   return OFT_OK;
 }

@@ -161,12 +161,16 @@ __global__ void __launch_bounds__(256) moe_combine_bwd_kernel(const float* __res
                           __uint_as_float(xq.z << 16), __uint_as_float(xq.z & 0xFFFF0000u),
                           __uint_as_float(xq.w << 16), __uint_as_float(xq.w & 0xFFFF0000u)};
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      float4 ua[kMaxTopK], ub[kMaxTopK];  // every slot's loads in flight before the first FMA
 #pragma unroll
       for (int s = 0; s < kMaxTopK; ++s) {
-        if (s >= k) break;
-        const float4 a = *reinterpret_cast<const float4*>(U + static_cast<size_t>(pos[s]) * K + c);
-        const float4 b = *reinterpret_cast<const float4*>(U + static_cast<size_t>(pos[s]) * K + c + 4);
-        const float u[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        ua[s] = s < k ? *reinterpret_cast<const float4*>(U + static_cast<size_t>(pos[s]) * K + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+        ub[s] = s < k ? *reinterpret_cast<const float4*>(U + static_cast<size_t>(pos[s]) * K + c + 4)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int s = 0; s < kMaxTopK; ++s) {
+        const float u[8] = {ua[s].x, ua[s].y, ua[s].z, ua[s].w, ub[s].x, ub[s].y, ub[s].z, ub[s].w};
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           acc[e] = fmaf(ws[s], u[e], acc[e]);

@@ -53,18 +53,23 @@ __global__ void __launch_bounds__(256) moe_gather_dy_kernel(const uint16_t* __re
 
 // Transposed chunk dequant: buf[slot][p][k][j] = deq(W_e)[p * n + j][k] for the
 // experts of chunk `chunk_idx` (INT4 bank), bit-exact like every other decode.
-// grid = (ceil(K / 256), ceil(2n / 64), chunk slots): a CTA walks a 64-row x
-// 256-column strip as four 64 x 64 tiles, with the next tile's codes and scales
-// already loaded into registers while the current one is transposed.  A tile goes
-// through shared memory as 32-bit words (two k per word, rows padded to 33
-// words), so neither side has bank conflicts; the code reads and the bf16 writes
-// are contiguous.  Requires n % 8 == 0 (8 consecutive rows never straddle gate / up).
-constexpr int kDqtStrip = 4;  // 64 x 64 tiles per CTA along K
+// The transpose happens in registers: lane (ro, kw) of a warp decodes the 8 code
+// words of rows 8 ro .. 8 ro + 7 at word kw of the warp's 64-column block (64
+// elements), then packs each k's 8 row values into one 16-byte store with byte
+// permutes.  Per warp that is 32 rows x 64 columns; for a fixed row the 8 lanes of one
+// ro read 32 contiguous bytes of codes, and for a fixed k the 4 lanes of one kw write
+// 64 contiguous bytes.  A CTA's 8 warps take 8 consecutive column blocks of the same
+// 32 rows.  Requires n % 8 == 0 (8 consecutive rows never straddle gate / up).
+constexpr int kDqtRows = 32;    // rows per CTA
+constexpr int kDqtCols = 512;   // columns (k) per CTA: 8 warps x 64
+
+inline dim3 dqt_grid(int K, int N, int chunk) {
+  return dim3((K + kDqtCols - 1) / kDqtCols, (N + kDqtRows - 1) / kDqtRows, chunk);
+}
 
 __global__ void __launch_bounds__(256) moe_chunk_dequant_t_kernel(WeightView bank, const int* __restrict__ chunk_table,
                                                                   int chunk_idx, int chunk, int n,
                                                                   uint16_t* __restrict__ buf) {
-  __shared__ uint32_t tile[64][33];  // [row n][k pair]
   const int slot = blockIdx.z;
   const int e = chunk_table[chunk_idx * chunk + slot];
   if (e < 0) return;
@@ -72,51 +77,29 @@ __global__ void __launch_bounds__(256) moe_chunk_dequant_t_kernel(WeightView ban
   const uint16_t* scales = reinterpret_cast<const uint16_t*>(static_cast<const uint8_t*>(bank.scales) +
                                                              static_cast<long long>(e) * bank.scales_expert_stride);
   const int N = bank.N, K = bank.K, G = bank.group;
-  const int n0 = blockIdx.y * 64;
-  const int lane = threadIdx.x & 31;
-  // this thread's two decode items of a tile: row r, k = 8c .. 8c+7 (it = tid, tid + 256)
-  uint32_t word[2];
-  uint16_t sc[2];
-  auto fetch = [&](int k0) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ro = lane >> 3, kw = lane & 7;
+  const int row0 = blockIdx.y * kDqtRows + ro * 8;           // this lane's 8 rows
+  const int k = blockIdx.x * kDqtCols + warp * 64 + kw * 8;  // and 8 columns
+  if (row0 >= N || k >= K) return;                          // N % 8 == 0, K % 8 == 0: whole octets
+  uint32_t w[8];
+  uint16_t sc[8];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int it = threadIdx.x + 256 * h;
-      const int row = n0 + (it >> 3), k = k0 + (it & 7) * 8;
-      const bool ok = row < N && k < K;
-      word[h] = ok ? *reinterpret_cast<const uint32_t*>(codes + static_cast<size_t>(row) * (K / 2) + k / 2) : 0u;
-      sc[h] = ok ? scales[static_cast<size_t>(k / G) * N + row] : uint16_t(0);
-    }
-  };
-  fetch(blockIdx.x * 64 * kDqtStrip);
-  for (int t = 0; t < kDqtStrip; ++t) {
-    const int k0 = (blockIdx.x * kDqtStrip + t) * 64;
-    if (k0 >= K) break;
+  for (int m = 0; m < 8; ++m) {
+    w[m] = __ldg(reinterpret_cast<const uint32_t*>(codes + static_cast<size_t>(row0 + m) * (K / 2) + k / 2));
+    sc[m] = __ldg(scales + static_cast<size_t>(k / G) * N + row0 + m);
+  }
+  uint32_t v[8][4];  // v[m][q]: row row0 + m, columns k + 2q (low half) and k + 2q + 1
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int it = threadIdx.x + 256 * h;
-      uint32_t v[4];
-      dq::int4x8(word[h], dq::bf2_splat(sc[h]), v);
+  for (int m = 0; m < 8; ++m) dq::int4x8(w[m], dq::bf2_splat(sc[m]), v[m]);
+  const int p = row0 / n, j = row0 - p * n;
+  uint16_t* dst = buf + ((static_cast<size_t>(slot) * 2 + p) * K + k) * n + j;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) tile[it >> 3][(it & 7) * 4 + i] = v[i];
-    }
-    __syncthreads();
-    if (t + 1 < kDqtStrip && k0 + 64 < K) fetch(k0 + 64);
-    for (int it = threadIdx.x; it < 512; it += 256) {
-      const int q = it >> 5;
-      const int r = (lane & 7) + 8 * (q & 7);  // k row
-      const int c = (lane >> 3) + 4 * (q >> 3);  // 8 consecutive n
-      const int k = k0 + r, row = n0 + c * 8;
-      if (k >= K || row >= N) continue;
-      const int p = row / n, j = row - p * n;
-      const int sh = (r & 1) * 16;
-      uint32_t v[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        v[i] = ((tile[c * 8 + 2 * i][r >> 1] >> sh) & 0xFFFFu) | (((tile[c * 8 + 2 * i + 1][r >> 1] >> sh) & 0xFFFFu) << 16);
-      *reinterpret_cast<uint4*>(buf + ((static_cast<size_t>(slot) * 2 + p) * K + k) * n + j) =
-          make_uint4(v[0], v[1], v[2], v[3]);
-    }
-    __syncthreads();
+  for (int i = 0; i < 8; ++i) {  // column k + i: rows row0 .. row0 + 7
+    const uint32_t sel = (i & 1) ? 0x7632u : 0x5410u;
+    *reinterpret_cast<uint4*>(dst + static_cast<size_t>(i) * n) =
+        make_uint4(__byte_perm(v[0][i >> 1], v[1][i >> 1], sel), __byte_perm(v[2][i >> 1], v[3][i >> 1], sel),
+                   __byte_perm(v[4][i >> 1], v[5][i >> 1], sel), __byte_perm(v[6][i >> 1], v[7][i >> 1], sel));
   }
 }
 

@@ -2003,7 +2003,7 @@ int moe_chunked_oft_bwd(const uint16_t* dY, const uint16_t* X, int T, const floa
     if (c >= 2) OFT_CUDA(cudaStreamWaitEvent(sp->side, sp->gemm_done[h], 0));
     {
       ProfScope ps(OFT_K_DEQUANT, sp->side);
-      moe_chunk_dequant_t_kernel<<<dim3((K + 64 * kDqtStrip - 1) / (64 * kDqtStrip), (N + 63) / 64, chunk), 256, 0,
+      moe_chunk_dequant_t_kernel<<<dqt_grid(K, N, chunk), 256, 0,
                                    sp->side>>>(bank, table, c, chunk,
                                                                                                   n_proj, bufc);
       OFT_LAUNCHED("moe_chunk_dequant_t_kernel");
@@ -2063,7 +2063,7 @@ extern "C" int oft_moe_chunk_dequant(const oft_weight* bank, const int32_t* chun
     OFT_LAUNCHED("moe_chunk_dequant_kernel");
   } else {
     if (N % 16 != 0) return fail(OFT_ERR_UNSUPPORTED, "the transposed chunk needs d_out (gate+up) % 16 == 0");
-    moe_chunk_dequant_t_kernel<<<dim3((K + 64 * kDqtStrip - 1) / (64 * kDqtStrip), (N + 63) / 64, chunk), 256, 0, st>>>(
+    moe_chunk_dequant_t_kernel<<<dqt_grid(K, N, chunk), 256, 0, st>>>(
         v, chunk_table, chunk_idx, chunk, N / 2, out);
     OFT_LAUNCHED("moe_chunk_dequant_t_kernel");
   }

@@ -100,62 +100,37 @@ __global__ void __launch_bounds__(256) dequant_rows_kernel(WeightView w, uint16_
   }
 }
 
-// out[k][n] = deq(W)[n][k]: 64 x 64 tiles transposed through shared memory as
-// 32-bit words (two k per word, rows padded to 33 words), so neither the decode
-// side nor the transposed side has bank conflicts; each warp stores 64-byte runs of
-// 8 k-rows.  A CTA walks a strip of kDeqTStrip tiles along K with every code and
-// scale load of the strip issued before the first decode.
-// grid = (ceil(K / (64 * kDeqTStrip)), ceil(N / 64)).
-constexpr int kDeqTStrip = 4;
+// out[k][n] = deq(W)[n][k], transposed in registers: lane (ro, kw) of a warp decodes
+// the 8-element units of rows 8 ro .. 8 ro + 7 at unit kw of the warp's 64-column
+// block, then packs each column's 8 row values into one 16-byte store with byte
+// permutes.  Per warp that is 32 rows x 64 columns; for a fixed row the 8 lanes of one
+// ro read contiguous codes, and for a fixed column the 4 lanes of one kw write 64
+// contiguous bytes.  A CTA's 8 warps take 8 consecutive column blocks of the same 32
+// rows.  N % 8 == 0 (sub-projection sizes are multiples of 8) and K % 32 == 0, so
+// every octet is whole.
+constexpr int kDeqTRows = 32;    // rows per CTA
+constexpr int kDeqTCols = 512;   // columns (k) per CTA: 8 warps x 64
 
 __global__ void __launch_bounds__(256) dequant_transposed_kernel(WeightView w, uint16_t* __restrict__ out) {
-  __shared__ uint32_t tile[64][33];  // [row n][k pair]
   pdl_wait();
-  const int n0 = blockIdx.y * 64;
-  const int kb = blockIdx.x * 64 * kDeqTStrip;
-  Raw8 raw[kDeqTStrip][2];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ro = lane >> 3, kw = lane & 7;
+  const int row0 = blockIdx.y * kDeqTRows + ro * 8;          // this lane's 8 rows
+  const int k = blockIdx.x * kDeqTCols + warp * 64 + kw * 8;  // and 8 columns
+  if (row0 >= w.N || k >= w.K) return;
+  Raw8 raw[8];
 #pragma unroll
-  for (int t = 0; t < kDeqTStrip; ++t)
+  for (int m = 0; m < 8; ++m) raw[m] = load8(w, w.codes, w.scales, row0 + m, k);
+  uint32_t v[8][4];  // v[m][q]: row row0 + m, columns k + 2q (low half) and k + 2q + 1
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int it = threadIdx.x + 256 * h;
-      const int n = n0 + (it >> 3), k = kb + t * 64 + (it & 7) * 8;
-      raw[t][h] = (n < w.N && k < w.K) ? load8(w, w.codes, w.scales, n, k) : Raw8{0u, 0u, 0u};
-    }
-  const int lane = threadIdx.x & 31;
+  for (int m = 0; m < 8; ++m) decode8(w.fmt, raw[m], v[m]);
+  uint16_t* dst = out + static_cast<size_t>(k) * w.N + row0;
 #pragma unroll
-  for (int t = 0; t < kDeqTStrip; ++t) {
-    const int k0 = kb + t * 64;
-    if (k0 >= w.K) break;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int it = threadIdx.x + 256 * h;
-      const int r = it >> 3, c = it & 7;  // row n0 + r, k = k0 + 8c .. +7
-      uint32_t v[4] = {0, 0, 0, 0};
-      if (n0 + r < w.N && k0 + c * 8 < w.K) decode8(w.fmt, raw[t][h], v);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) tile[r][c * 4 + i] = v[i];
-    }
-    __syncthreads();
-    for (int it = threadIdx.x; it < 512; it += 256) {
-      const int q = it >> 5;
-      const int r = (lane & 7) + 8 * (q & 7);    // k row
-      const int c = (lane >> 3) + 4 * (q >> 3);  // 8 consecutive n
-      const int k = k0 + r, n = n0 + c * 8;
-      if (k >= w.K || n >= w.N) continue;
-      const int sh = (r & 1) * 16;
-      uint32_t v[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        v[i] = ((tile[c * 8 + 2 * i][r >> 1] >> sh) & 0xFFFFu) | (((tile[c * 8 + 2 * i + 1][r >> 1] >> sh) & 0xFFFFu) << 16);
-      if (n + 8 <= w.N) {
-        *reinterpret_cast<uint4*>(out + static_cast<size_t>(k) * w.N + n) = make_uint4(v[0], v[1], v[2], v[3]);
-      } else {
-        for (int i = 0; i < 8 && n + i < w.N; ++i)
-          out[static_cast<size_t>(k) * w.N + n + i] = static_cast<uint16_t>((v[i / 2] >> (16 * (i & 1))) & 0xFFFFu);
-      }
-    }
-    __syncthreads();  // the tile is free for the next
+  for (int i = 0; i < 8; ++i) {  // column k + i: rows row0 .. row0 + 7
+    const uint32_t sel = (i & 1) ? 0x7632u : 0x5410u;
+    *reinterpret_cast<uint4*>(dst + static_cast<size_t>(i) * w.N) =
+        make_uint4(__byte_perm(v[0][i >> 1], v[1][i >> 1], sel), __byte_perm(v[2][i >> 1], v[3][i >> 1], sel),
+                   __byte_perm(v[4][i >> 1], v[5][i >> 1], sel), __byte_perm(v[6][i >> 1], v[7][i >> 1], sel));
   }
 }
 

@@ -324,7 +324,7 @@ int launch_dequant(const WeightView& v, uint16_t* out, bool transpose, cudaStrea
     OFT_CUDA(launch_pdl(dequant_rows_kernel, grid, 256, 0, st, v, out));
     OFT_LAUNCHED("dequant_rows_kernel");
   } else {
-    dim3 grid((v.K + 64 * kDeqTStrip - 1) / (64 * kDeqTStrip), (v.N + 63) / 64);
+    dim3 grid((v.K + kDeqTCols - 1) / kDeqTCols, (v.N + kDeqTRows - 1) / kDeqTRows);
     ProfScope ps(OFT_K_DEQUANT, st);
     OFT_CUDA(launch_pdl(dequant_transposed_kernel, grid, 256, 0, st, v, out));
     OFT_LAUNCHED("dequant_transposed_kernel");

@@ -293,25 +293,25 @@ __global__ void __launch_bounds__(CayleyFwdCfg<B>::THREADS, CayleyFwdCfg<B>::MIN
 }
 
 // Forward for launches of a few hundred blocks (b = 32, 64), where each block's
-// serial pivot chain sets the time: TPR threads per row, each holding a 1/TPR
-// slice of the row's sliding window over the uneliminated columns of A and of the
-// right-hand side, so every pivot costs each thread 1/TPR of the loads and FMAs.
-// Per pivot, one shuffle brings the row's pivot-column element (held by the
-// group's first thread) to the others, and one carries the element that crosses
-// from each slice to the previous one when the window shifts.  Same sweep as the one-thread-per-row kernel: the
-// pivot row is published through double-buffered shared memory, rows are never
-// normalised during the sweep, and each row divides by its own pivot at the end.
+// serial pivot chain sets the time: the in-place inversion of the many-block form
+// (R = 2 (I - Q)^-1 - I, one uniform update per pivot), with each row split over TPR
+// threads that hold H = B / TPR consecutive columns each, so a pivot costs each
+// thread H FMAs and H / 4 vector loads.  The row's pivot-column element comes from
+// the thread holding it by one shuffle; the pivot row's TPR threads publish it
+// through double-buffered shared memory (one barrier per pivot).  The pivot loop is
+// unrolled, so every register index is static.
 template <int B, int TPR>
-__global__ void __launch_bounds__(TPR * B) cayley_fwd_split_kernel(const uint16_t* __restrict__ Q, int nblocks,
-                                                                 float* __restrict__ R,
-                                                                 const int* __restrict__ active_list,
-                                                                 const int* __restrict__ n_active,
-                                                                 int blocks_per_expert, long long lo_off) {
+__global__ void __launch_bounds__(TPR * B) cayley_fwd_inv_split_kernel(const uint16_t* __restrict__ Q, int nblocks,
+                                                                     float* __restrict__ R,
+                                                                     const int* __restrict__ active_list,
+                                                                     const int* __restrict__ n_active,
+                                                                     int blocks_per_expert, long long lo_off) {
   constexpr int H = B / TPR;  // columns per thread
-  static_assert(H % 4 == 0 && (TPR & (TPR - 1)) == 0, "slices of whole float4s");
-  __shared__ __align__(16) float piv[2][2 * B + 4];
+  static_assert(H % 4 == 0 && (TPR & (TPR - 1)) == 0 && 32 % TPR == 0, "slices of whole float4s");
+  __shared__ __align__(16) float piv[2][B + 4];  // pivot row, then its reciprocal
   __shared__ __align__(16) uint16_t qsh[B * (B - 1) / 2];
   const int r = threadIdx.x / TPR, h = threadIdx.x % TPR;
+  const int lane0 = (threadIdx.x & 31) & ~(TPR - 1);  // this row's first lane in the warp
   const unsigned full = 0xFFFFFFFFu;
   pdl_wait();
   const int total = active_list != nullptr ? min(nblocks, *n_active * blocks_per_expert) : nblocks;
@@ -321,69 +321,60 @@ __global__ void __launch_bounds__(TPR * B) cayley_fwd_split_kernel(const uint16_
     __syncthreads();  // the previous block is done with qsh and piv
     stage_q<B>(Q + static_cast<size_t>(blk) * (B * (B - 1) / 2), qsh, threadIdx.x, TPR * B);
     __syncthreads();
-    const uint16_t* q = qsh;
-    float a[H], rhs[H];
+    float a[H];
 #pragma unroll
     for (int k = 0; k < H; ++k) {
       const int j = h * H + k;
       float v = 0.f;
       if (j != r) {
-        const float t = bf16_bits_to_f32(q[j > r ? tri_index(r, j, B) : tri_index(j, r, B)]);
+        const float t = bf16_bits_to_f32(qsh[j > r ? tri_index(r, j, B) : tri_index(j, r, B)]);
         v = j > r ? t : -t;  // Q[r][j]
       }
-      const float d = (j == r) ? 1.f : 0.f;
-      a[k] = d - v;
-      rhs[k] = d + v;
+      a[k] = (j == r ? 1.f : 0.f) - v;
     }
-    float my_inv = 1.f;
-#pragma unroll 1
-    for (int c = 0; c < B; ++c) {
-      float* pr = piv[c & 1];
-      // the row's pivot-column element A[r][c] is the first thread's a[0]
-      const float arc = __shfl_sync(full, a[0], threadIdx.x & ~(TPR - 1));
-      if (r == c) {
-        if (h == 0) pr[2 * B] = __frcp_rn(a[0]);  // >= 1 in exact arithmetic; correctly rounded
 #pragma unroll
-        for (int k = 0; k < H; k += 4) {
+    for (int c = 0; c < B; ++c) {
+      const int owner = c / H, kc = c % H;
+      float* pr = piv[c & 1];
+      const float arc = __shfl_sync(full, a[kc], lane0 + owner);  // A[r][c]
+      if (r == c) {
+#pragma unroll
+        for (int k = 0; k < H; k += 4)
           *reinterpret_cast<float4*>(pr + h * H + k) = make_float4(a[k], a[k + 1], a[k + 2], a[k + 3]);
-          *reinterpret_cast<float4*>(pr + B + h * H + k) = make_float4(rhs[k], rhs[k + 1], rhs[k + 2], rhs[k + 3]);
-        }
+        if (h == owner) pr[B] = __frcp_rn(arc);  // correctly rounded; A[c][c] >= 1 in exact arithmetic
       }
       __syncthreads();
-      const float inv = pr[2 * B];
-      if (r == c) my_inv = inv;
-      const float f = (r == c) ? 0.f : arc * inv;
+      const float pinv = pr[B];
+      const float f = (arc - (r == c ? 1.f : 0.f)) * pinv;
 #pragma unroll
       for (int k = 0; k < H; k += 4) {
         const float4 v = *reinterpret_cast<const float4*>(pr + h * H + k);
-        const float4 w = *reinterpret_cast<const float4*>(pr + B + h * H + k);
         a[k] = fmaf(-f, v.x, a[k]);
         a[k + 1] = fmaf(-f, v.y, a[k + 1]);
         a[k + 2] = fmaf(-f, v.z, a[k + 2]);
         a[k + 3] = fmaf(-f, v.w, a[k + 3]);
-        rhs[k] = fmaf(-f, w.x, rhs[k]);
-        rhs[k + 1] = fmaf(-f, w.y, rhs[k + 1]);
-        rhs[k + 2] = fmaf(-f, w.z, rhs[k + 2]);
-        rhs[k + 3] = fmaf(-f, w.w, rhs[k + 3]);
       }
-      // drop column c: the window moves one column right across the pair
-      const float nxt = __shfl_down_sync(full, a[0], 1);  // the next slice's first element
-#pragma unroll
-      for (int k = 0; k < H - 1; ++k) a[k] = a[k + 1];
-      a[H - 1] = h < TPR - 1 ? nxt : 0.f;
+      if (h == owner) a[kc] = (r == c) ? pinv : -f;  // column c of the inverse
     }
     if (lo_off > 0) {
 #pragma unroll
-      for (int k = 0; k < H; ++k) store_r_hl_t(R, lo_off, blk, B, r, h * H + k, rhs[k] * my_inv);
+      for (int k = 0; k < H; ++k) {
+        const int j = h * H + k;
+        store_r_hl_t(R, lo_off, blk, B, r, j, 2.f * a[k] - (j == r ? 1.f : 0.f));
+      }
     } else {
       float* out = R + (static_cast<size_t>(blk) * B + r) * B + h * H;
 #pragma unroll
-      for (int k = 0; k < H; k += 4)
+      for (int k = 0; k < H; k += 4) {
+        const int j = h * H + k;
         *reinterpret_cast<float4*>(out + k) =
-            make_float4(rhs[k] * my_inv, rhs[k + 1] * my_inv, rhs[k + 2] * my_inv, rhs[k + 3] * my_inv);
+            make_float4(2.f * a[k] - (j == r ? 1.f : 0.f), 2.f * a[k + 1] - (j + 1 == r ? 1.f : 0.f),
+                        2.f * a[k + 2] - (j + 2 == r ? 1.f : 0.f), 2.f * a[k + 3] - (j + 3 == r ? 1.f : 0.f));
+      }
     }
   }
 }
+
 
 // dQ[blk] = pack(D - D^T), D = 1/2 (I+R)^T G (I+R)^T.
 // G is read either directly ([nblocks][b][b], nparts = 1) or as `nparts` partial

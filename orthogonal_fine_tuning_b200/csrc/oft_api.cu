@@ -349,10 +349,10 @@ int launch_cayley(const uint16_t* Q, int nblocks, int b, float* R, const int* ac
     if (b == 64) OFT_CUDA(launch_pdl(cayley_fwd_kernel<64, true>, grid, 64, 0, st, Q, nblocks, R, al, n_active, blocks_per_expert, lo_off));
   } else {
     if (b == 16) OFT_CUDA(launch_pdl(cayley_fwd_kernel<16, false>, grid, 32, 0, st, Q, nblocks, R, al, n_active, blocks_per_expert, lo_off));
-    // few blocks: the per-block pivot chain is the time, so two threads share each row
-    const int sgrid = std::max(1, std::min(nblocks, sm_count() * 16));
-    if (b == 32) OFT_CUDA(launch_pdl(cayley_fwd_split_kernel<32, 2>, sgrid, 64, 0, st, Q, nblocks, R, al, n_active, blocks_per_expert, lo_off));
-    if (b == 64) OFT_CUDA(launch_pdl(cayley_fwd_split_kernel<64, 2>, sgrid, 128, 0, st, Q, nblocks, R, al, n_active, blocks_per_expert, lo_off));
+    // few blocks: the per-block pivot chain is the time, so four threads share each row
+    const int sgrid = std::max(1, std::min(nblocks, sm_count() * 8));
+    if (b == 32) OFT_CUDA(launch_pdl(cayley_fwd_inv_split_kernel<32, 4>, sgrid, 128, 0, st, Q, nblocks, R, al, n_active, blocks_per_expert, lo_off));
+    if (b == 64) OFT_CUDA(launch_pdl(cayley_fwd_inv_split_kernel<64, 4>, sgrid, 256, 0, st, Q, nblocks, R, al, n_active, blocks_per_expert, lo_off));
   }
   OFT_LAUNCHED("cayley_fwd_kernel");
   return OFT_OK;

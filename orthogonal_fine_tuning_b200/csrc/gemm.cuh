@@ -242,7 +242,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) gemm_bf16_kernel(const __grid_
   float* s_epi = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(sg) + kGroupBytes);  // [4 warps][32][EPI_LD]
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  if (p.use_moe) pdl_wait();  // the prologue reads the device-built routing tables
+  if (p.use_moe) {
+    pdl_wait();  // the prologue reads the device-built routing tables
+    // a chunk past the active experts (they fill the chunks in order) has no tiles:
+    // leave before the barriers and the TMEM allocation
+    if (p.moe.chunk_table[p.moe.chunk_idx * p.moe.chunk] < 0) return;
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {

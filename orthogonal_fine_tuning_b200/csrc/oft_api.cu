@@ -417,7 +417,7 @@ int launch_rotate_fwd(const uint16_t* X, int M, int K, int P, int b, const float
   }
   const int grid = std::min(sm_count(), prm.groups * prm.tiles_m);
   ProfScope ps(OFT_K_ROTATE, st);
-  OFT_CUDA(launch_pdl(rtc::rot_fwd_tc_kernel, grid, rtc::NUM_THREADS, rtc::kFwdSmem, st, prm));
+  OFT_CUDA(launch_pdl(rtc::rot_fwd_tc_kernel, grid, rtc::FWD_THREADS, rtc::kFwdSmem, st, prm));
   OFT_LAUNCHED("rot_fwd_tc_kernel");
   return OFT_OK;
 }

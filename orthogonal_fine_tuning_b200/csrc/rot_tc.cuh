@@ -75,29 +75,38 @@ constexpr int FWD_A_BYTES = TM * 64 * 2;           // 16 KB
 constexpr int FWD_BP_BYTES = 64 * 64 * 2;          // one 64x64 bf16 tile
 constexpr int FWD_OUT_BYTES = 32 * 64 * 2;           // one staged 32-token x 64-column bf16 box
 constexpr int FWD_OUT_SLOTS = 2;                     // per epilogue warp
-constexpr size_t kFwdSmem = 1024 + A_STAGES * FWD_A_BYTES + 2 * MAX_P * FWD_BP_BYTES + 4 * FWD_OUT_SLOTS * FWD_OUT_BYTES + 256;
+constexpr int FWD_EPI_WARPS = 8;                     // two per TMEM lane quarter, splits shared by parity
+constexpr int FWD_THREADS = 64 + 32 * FWD_EPI_WARPS;
+constexpr size_t kFwdSmem =
+    1024 + A_STAGES * FWD_A_BYTES + 2 * MAX_P * FWD_BP_BYTES + FWD_EPI_WARPS * FWD_OUT_SLOTS * FWD_OUT_BYTES + 256;
 
 // Named barrier over the 128 builder/epilogue threads (warps 2..5).
 __device__ __forceinline__ void builders_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
+// Named barrier over the forward rotation's FWD_EPI_WARPS epilogue warps.
+__device__ __forceinline__ void fwd_epi_sync() { asm volatile("bar.sync 2, %0;" ::"n"(32 * FWD_EPI_WARPS) : "memory"); }
+
 // B[r = p*64 + c][i] = R_p[i][c] restricted to group g (block-diagonal), split
-// hi/lo (with p.transpose: B[r = p*64 + i][c] = R_p[i][c], i.e. R_p^T).  Zero the tiles, then stream each diagonal R block in with coalesced
-// float4 loads (eight in flight per thread) and scatter it transposed.
+// hi/lo (with p.transpose: B[r = p*64 + i][c] = R_p[i][c], i.e. R_p^T), by the
+// forward's epilogue threads (tid < 32 * FWD_EPI_WARPS).  Zero the tiles, then stream
+// each diagonal R block in with coalesced float4 loads (eight in flight per thread)
+// and scatter it transposed.
 __device__ void build_fwd_b(const FwdParams& p, int g, uint8_t* sBhi, uint8_t* sBlo, int tid) {
+  constexpr int NT = 32 * FWD_EPI_WARPS;
   const int b = p.b;
-  for (int v = tid; v < p.P * FWD_BP_BYTES / 16; v += 128) {
+  for (int v = tid; v < p.P * FWD_BP_BYTES / 16; v += NT) {
     reinterpret_cast<uint4*>(sBhi)[v] = make_uint4(0, 0, 0, 0);
     reinterpret_cast<uint4*>(sBlo)[v] = make_uint4(0, 0, 0, 0);
   }
-  builders_sync();
+  fwd_epi_sync();
   const int per_split = 16 * b;             // float4s of the group's diagonal blocks: (64/b) * b * b / 4
   const int total = p.P * per_split;
-  for (int base = 0; base < total; base += 128 * 8) {
+  for (int base = 0; base < total; base += NT * 8) {
     float4 v[8];
     int meta[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
-      const int f = base + u * 128 + tid;
+      const int f = base + u * NT + tid;
       meta[u] = -1;
       v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (f < total) {
@@ -129,14 +138,14 @@ __device__ void build_fwd_b(const FwdParams& p, int g, uint8_t* sBhi, uint8_t* s
   }
 }
 
-__global__ void __launch_bounds__(NUM_THREADS, 1) rot_fwd_tc_kernel(const __grid_constant__ FwdParams p) {
+__global__ void __launch_bounds__(FWD_THREADS, 1) rot_fwd_tc_kernel(const __grid_constant__ FwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sBhi = sA + A_STAGES * FWD_A_BYTES;
   uint8_t* sBlo = sBhi + MAX_P * FWD_BP_BYTES;
   uint8_t* sOut = sBlo + MAX_P * FWD_BP_BYTES;  // 1024-byte aligned: the store boxes are 128B-swizzled
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + 4 * FWD_OUT_SLOTS * FWD_OUT_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + FWD_EPI_WARPS * FWD_OUT_SLOTS * FWD_OUT_BYTES);
   uint64_t* full = bars;
   uint64_t* empty = bars + A_STAGES;
   uint64_t* acc_full = bars + 2 * A_STAGES;
@@ -154,9 +163,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) rot_fwd_tc_kernel(const __grid
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 128);
+      mbar_init(&acc_empty[a], 32 * FWD_EPI_WARPS);
     }
-    mbar_init(b_full, 128);
+    mbar_init(b_full, 32 * FWD_EPI_WARPS);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -235,7 +244,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) rot_fwd_tc_kernel(const __grid
       gemm_drain_wait(drain, 0);
     }
   } else {
-    const int q = warp & 3, tid = threadIdx.x - 64;
+    const int q = warp & 3, tid = threadIdx.x - 64, ew = warp - 2;
+    const int half = ew / 4;  // splits half, half + 2, ... of every unit
     int acc = 0, cur_g = -1, out_slot = 0;
     uint32_t acc_ph = 0;
     for (int u = ubeg; u < uend; ++u) {
@@ -251,8 +261,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) rot_fwd_tc_kernel(const __grid
       // Each warp owns 32 tokens: per split, its 32 x 64 bf16 block is staged in a
       // 128B-swizzled slot (row = token, lane-private, conflict-free) and leaves by one
       // TMA store, which clips tokens past M and columns past K.
-      for (int sp = 0; sp < p.P; ++sp) {
-        uint8_t* slot = sOut + (q * FWD_OUT_SLOTS + out_slot) * FWD_OUT_BYTES;
+      for (int sp = half; sp < p.P; sp += 2) {
+        uint8_t* slot = sOut + (ew * FWD_OUT_SLOTS + out_slot) * FWD_OUT_BYTES;
         if (lane == 0) bulk_wait_read<FWD_OUT_SLOTS - 1>();  // the store that last read this slot is done
         __syncwarp();
 #pragma unroll 1

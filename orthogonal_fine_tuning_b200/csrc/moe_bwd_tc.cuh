@@ -7,11 +7,10 @@
 // "对低精度 MoE 模型的专门优化"; the OFT backward itself is the standard one):
 //
 //   moe_rotb_tc_kernel: U[pos] = sum_p D_p[pos] R_e,p^T        (blockwise; R as tf32 hi + lo)
-//                       dwp[pos][blk] = <U[pos, blk], X[t, blk]>   (partial of dw_tk)
 //   moe_grad_tc_kernel: G_e,p,blk = sum over e's positions of (w_pos X[t, blk])^T D_p[pos, blk]
 //
 // followed by the Cayley backward of every active expert's G (cayley_bwd_kernel
-// with an expert map).  t = bucket[pos] / top_k is the routed token, w_pos its
+// with an expert map); dw_tk = <U[pos], X[t]> is formed by the combine pass over U.  t = bucket[pos] / top_k is the routed token, w_pos its
 // gating weight.
 //
 // Units are (active expert, column group), taken heaviest expert first and dealt

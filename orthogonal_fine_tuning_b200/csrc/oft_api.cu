@@ -2016,9 +2016,9 @@ int moe_chunked_oft_bwd(const uint16_t* dY, const uint16_t* X, int T, const floa
     if (int rc = launch_gemm(prm, 0, st)) return rc;
     OFT_CUDA(cudaEventRecord(sp->gemm_done[h], st));
   }
-  // 4. per (active expert, column group): rows rotated back with the dw partials, the
-  //    expert's adapter gradient (into the chunk buffers, free after the last GEMM), and
-  //    the Cayley backward of the active experts' blocks
+  // 4. per (active expert, column group): rows rotated back, the expert's adapter
+  //    gradient (into the chunk buffers, free after the last GEMM), and the Cayley
+  //    backward of the active experts' blocks
   if (int rc = launch_moe_bwd_tc(D, X, K, TK, E, b, row_t, row_w, offsets, order, n_active, Rex, U,
                                  reinterpret_cast<float*>(buf), dQ, st))
     return rc;

@@ -10,8 +10,8 @@
 //   moe_grad_tc_kernel: G_e,p,blk = sum over e's positions of (w_pos X[t, blk])^T D_p[pos, blk]
 //
 // followed by the Cayley backward of every active expert's G (cayley_bwd_kernel
-// with an expert map); dw_tk = <U[pos], X[t]> is formed by the combine pass over U.  t = bucket[pos] / top_k is the routed token, w_pos its
-// gating weight.
+// with an expert map); dw_tk = <U[pos], X[t]> is formed by the combine pass over U.
+// t = bucket[pos] / top_k is the routed token, w_pos its gating weight.
 //
 // Units are (active expert, column group), taken heaviest expert first and dealt
 // round-robin to the CTAs, so each CTA's share is within one unit of the mean; a

@@ -38,3 +38,21 @@ def test_traffic_entries_are_keyed_by_source_hash():
             assert bench.gemm_traffic(kernel, workload) == (nbytes if current else None)
     # the dense default path's kernel has counters for the fused-QKV workload
     assert bench.gemm_traffic("gemm_bf16_pair_kernel", "c1") is not None
+
+
+def test_reference_arm_reports_the_workloads_config(monkeypatch):
+    """The reference arm times a bounded token sample of the workload, but its line
+    carries the workload's own config, the one our arm reports (token counts included);
+    the sample is described under cpu_baseline.  (The oracle step is replaced by a fixed
+    time here: only the reporting is under test.)"""
+    import argparse
+    monkeypatch.setattr(bench, "oracle_linear_step", lambda case, tokens, backward: 100.0)
+    args = argparse.Namespace(workload="c1", steps=1, warmup=3, moe="chunked", moe_backward=False,
+                              moe_layer=False, weight_side=False)
+    line = bench.run_reference(args, 0, 1)
+    spec = bench.linear_spec("c1")
+    assert line["impl"] == "reference"
+    assert line["config"] == bench.workload_config("c1", spec.M, 1, spec.backward, args)
+    assert line["config"]["tokens_per_gpu"] == spec.M
+    assert str(spec.M) in line["cpu_baseline"]["sample"]
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]

@@ -492,7 +492,7 @@ int launch_grad(const uint16_t* X, const float* dXr, int M, int K, int P, int b,
   if (int rc = set_smem(rtc::grad_tc_kernel, rtc::kGradSmem)) return rc;
   const int grid = std::min(sm_count(), prm.groups * prm.chunks);
   ProfScope ps(OFT_K_GRAD, st);
-  OFT_CUDA(launch_pdl(rtc::grad_tc_kernel, grid, rtc::NUM_THREADS, rtc::kGradSmem, st, prm));
+  OFT_CUDA(launch_pdl(rtc::grad_tc_kernel, grid, rtc::GR_THREADS, rtc::kGradSmem, st, prm));
   OFT_LAUNCHED("grad_tc_kernel");
   return OFT_OK;
 }

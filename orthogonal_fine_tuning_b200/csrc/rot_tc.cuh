@@ -546,9 +546,11 @@ constexpr int GR_X_BYTES = 4 * 16384;   // 128 tokens x 128 columns fp32, MN-maj
 constexpr int GR_XS_BYTES = 2 * 16384;  // the same tile as staged by TMA: bf16, two 64-column boxes
 constexpr int GR_B_BYTES = 4 * 16384;   // one dX' tile, same layout as the fp32 X tile
 constexpr int GR_STAGES = 2;
+constexpr int GR_BUILD_WARPS = 8;  // X-tile conversion and epilogue: two warps per TMEM lane quarter
+constexpr int GR_THREADS = 64 + 32 * GR_BUILD_WARPS;
 constexpr size_t kGradSmem = 1024 + GR_X_BYTES + GR_XS_BYTES + GR_STAGES * GR_B_BYTES + 256;
 
-__global__ void __launch_bounds__(NUM_THREADS, 1) grad_tc_kernel(const __grid_constant__ GradParams p) {
+__global__ void __launch_bounds__(GR_THREADS, 1) grad_tc_kernel(const __grid_constant__ GradParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sX = smem;
@@ -573,12 +575,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grad_tc_kernel(const __grid_co
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(x_full, 128);
+    mbar_init(x_full, 32 * GR_BUILD_WARPS);
     mbar_init(x_empty, 1);
     mbar_init(xs_full, 1);
-    mbar_init(xs_empty, 128);
+    mbar_init(xs_empty, 32 * GR_BUILD_WARPS);
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 128);
+    mbar_init(acc_empty, 32 * GR_BUILD_WARPS);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -689,6 +691,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grad_tc_kernel(const __grid_co
     }
   } else {
     const int q = warp & 3, tid = threadIdx.x - 64;
+    const int half = (warp - 2) / 4;  // sub-projections half, half + 2, ... in the epilogue
     uint32_t x_ph = 0, xs_ph = 0, acc_ph = 0;
     const int b = p.b;
     for (int u = ubeg; u < uend; ++u) {
@@ -709,8 +712,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grad_tc_kernel(const __grid_co
         xs_ph ^= 1;
         // staged X tile (bf16, K-major 128B-swizzled) -> fp32, MN-major, 128B rows with 32-byte atoms
 #pragma unroll 4
-        for (int it = 0; it < 16; ++it) {
-          const int k = tid + 128 * it;
+        for (int it = 0; it < 2048 / (32 * GR_BUILD_WARPS); ++it) {
+          const int k = tid + 32 * GR_BUILD_WARPS * it;
           const int t = k >> 4, ci = k & 15;
           const uint4 v = *reinterpret_cast<const uint4*>(sXs + (ci >> 3) * 16384 + swz(t, ci & 7));
           uint8_t* base = sX + (ci >> 2) * 16384;
@@ -730,7 +733,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) grad_tc_kernel(const __grid_co
       tc_fence_after();
       // this warp's 32 rows i = 32q + lane of the group's 128 x 128 product
       const int i = q * 32 + lane;
-      for (int sp = 0; sp < p.P; ++sp) {
+      for (int sp = half; sp < p.P; sp += 2) {
         if (b >= 32) {
           const int blk_col0 = ((q * 32) / b) * b;  // first column of this warp's diagonal block
 #pragma unroll 1
